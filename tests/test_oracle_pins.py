@@ -1,0 +1,424 @@
+"""Pins for the fp64 CPU oracle.
+
+Each test checks the oracle against something other than itself: numbers the
+pages print for a worked example (tests/golden/page_examples.json), closed
+forms, invariants, library routines (scipy.linalg.hadamard, numpy matmul,
+numpy/torch float conversions, numpy complex arithmetic, numpy QR), or brute
+force on tiny inputs. No GPU is needed.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import synthetic
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_examples.json")
+
+
+@pytest.fixture(scope="module")
+def pages():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def bf16(x):
+    return synthetic.to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+# --------------------------------------------------------------------------
+# Hadamard matrices -- "Rotations: QuaRot, SpinQuant and incoherence",
+# section "Hadamard matrices" (Sylvester recursion, H_n / sqrt(n) orthogonal).
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16, 64, 256, 1024, 4096])
+def test_sylvester_matches_scipy_and_is_orthogonal(orc, n):
+    H = orc.sylvester_matrix(n).astype(np.float64)  # small integers: fp64 products are exact
+    assert np.array_equal(H, scipy.linalg.hadamard(n))
+    assert np.array_equal(H @ H.T, n * np.eye(n))
+    assert np.array_equal(H, H.T)
+
+
+@pytest.mark.parametrize("n", [2, 8, 64, 256])
+def test_normalised_hadamard_is_an_involution(orc, n):
+    Hn = orc.sylvester_matrix(n).astype(np.float64) / math.sqrt(n)
+    assert np.max(np.abs(Hn @ Hn - np.eye(n))) < 1e-15 * n
+
+
+def test_entry_closed_form_matches_recursion(orc):
+    n = 1024
+    H = orc.sylvester_matrix(n)
+    rng = np.random.default_rng(0)
+    for i, j in rng.integers(0, n, size=(2000, 2)):
+        assert orc.hadamard_entry(int(i), int(j)) == H[i, j]
+
+
+def test_kronecker_factorisation_128x128_is_16384(orc):
+    """H_128 (x) H_128 = H_16384 entrywise on sampled entries (Kronecker products)."""
+    H128 = orc.sylvester_matrix(128).astype(np.int64)
+    rows = np.random.default_rng(1).integers(0, 16384, size=24)
+    ref = scipy.linalg.hadamard(16384, dtype=np.int8)[rows].astype(np.int64)  # library construction
+    for r, i in enumerate(rows):
+        kron_row = np.kron(H128[i // 128], H128[i % 128])
+        assert np.array_equal(kron_row, ref[r])
+        cols = np.random.default_rng(int(i)).integers(0, 16384, size=64)
+        for j in cols:
+            assert orc.hadamard_entry(int(i), int(j)) == ref[r, j]
+
+
+# --------------------------------------------------------------------------
+# The fast transform equals the explicit matrix product -- "Rotations: ...",
+# section "Why it's free" (O(d log d) transform with no matrix multiply).
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16, 32, 64])
+def test_fwht_equals_brute_force_matmul(orc, n):
+    rng = np.random.default_rng(n)
+    H = scipy.linalg.hadamard(n).astype(np.float64)
+    xi = rng.integers(-1000, 1000, size=n).astype(np.float64)
+    assert np.array_equal(orc.fwht(xi), H @ xi)  # integers: bit-exact
+    assert np.array_equal(orc.wht_explicit(xi), H @ xi)
+    xg = rng.standard_normal(n)
+    assert np.max(np.abs(orc.fwht(xg) - H @ xg)) <= 1e-12 * max(1.0, np.abs(xg).sum())
+    assert np.max(np.abs(orc.wht_explicit(xg) - H @ xg)) <= 1e-12 * max(1.0, np.abs(xg).sum())
+
+
+@pytest.mark.parametrize("k", [7, 10, 12])
+def test_fwht_equals_explicit_at_larger_sizes(orc, k):
+    n = 1 << k
+    x = np.random.default_rng(k).standard_normal(n)
+    y_fast = orc.rotate(x, method=orc.METHOD_FWHT)
+    y_slow = orc.rotate(x, method=orc.METHOD_EXPLICIT)
+    assert np.max(np.abs(y_fast - y_slow)) < 1e-12 * np.linalg.norm(x)
+
+
+def test_fwht_sampled_outputs_at_32768(orc):
+    """Sampled outputs of the n = 2^15 transform against rows of scipy's matrix."""
+    n = 1 << 15
+    x = np.random.default_rng(15).standard_normal(n)
+    y = orc.rotate(x)
+    for i in (0, 1, 12345, 32767):
+        # the row of H_32768, built from library matrices by the Kronecker factorisation
+        row = np.kron(scipy.linalg.hadamard(256)[i // 128], scipy.linalg.hadamard(128)[i % 128])
+        assert abs(y[i] - row @ x / math.sqrt(n)) < 1e-11 * np.linalg.norm(x)
+
+
+def test_rotation_with_diagonal(orc):
+    n = 256
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal(n)
+    words = synthetic.sign_bits(n, 3)
+    d = synthetic.sign_vector(words, n)
+    y = orc.rotate(x, signs=words)
+    ref = scipy.linalg.hadamard(n) @ (d * x) / math.sqrt(n)
+    assert np.max(np.abs(y - ref)) < 1e-13
+
+
+def test_involution_and_parseval(orc):
+    x = np.random.default_rng(3).standard_normal(4096)
+    y = orc.rotate(x)
+    assert abs(np.linalg.norm(y) - np.linalg.norm(x)) < 1e-12 * np.linalg.norm(x)
+    assert np.max(np.abs(orc.rotate(y) - x)) < 1e-13
+
+
+# --------------------------------------------------------------------------
+# Norm example and RMSNorm invariance -- "SpinQuant, when rotations are worth
+# learning", section "The math, slowly"; "Rotations: ...", "Computational
+# invariance".
+# --------------------------------------------------------------------------
+def test_norm_example(orc, pages):
+    g = pages["norm_example"]
+    h = np.array(g["h"])
+    R90 = np.array([[0.0, -1.0], [1.0, 0.0]])
+    assert np.array_equal(R90 @ h, np.array(g["rotated_90"]))
+    assert np.linalg.norm(h) == g["length"] == np.linalg.norm(R90 @ h)
+    # the normalised H_2 is a rotation-reflection: length stays 5
+    assert abs(np.linalg.norm(orc.rotate(h)) - g["length"]) < 1e-14
+    # RMSNorm commutes with the 90-degree rotation
+    assert np.max(np.abs(orc.rmsnorm(R90 @ h) - R90 @ orc.rmsnorm(h))) < 1e-15
+
+
+@pytest.mark.parametrize("d", [2, 64, 4096])
+@pytest.mark.parametrize("eps", [0.0, 1e-6])
+def test_rmsnorm_commutes_with_random_orthogonal(orc, d, eps):
+    rng = np.random.default_rng(d)
+    Q, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    h = rng.standard_normal(d)
+    assert np.max(np.abs(orc.rmsnorm(Q @ h, eps) - Q @ orc.rmsnorm(h, eps))) < 1e-12
+    if d >= 4:  # and with the oracle's own normalised Hadamard
+        assert np.max(np.abs(orc.rmsnorm(orc.rotate(h), eps) - orc.rotate(orc.rmsnorm(h, eps)))) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# 4-bit steps printed on the pages.
+# --------------------------------------------------------------------------
+def test_widget_step(orc, pages):
+    """'Try it' widget: 16 values, outlier 24 -> step 3.43; values below half a
+    step (12/7) round to 0."""
+    g = pages["widget_step"]
+    rng = np.random.default_rng(24)
+    vals = np.clip(rng.standard_normal(g["n"]) * 0.7, -0.99, 0.99).astype(np.float32)
+    vals[5] = g["outlier"]
+    r = orc.r4_row(bf16(vals), clip=1.0, no_rotate=True)
+    assert round(r["scale64"], g["decimals"]) == g["step_printed"]
+    assert r["scale64"] == pytest.approx(24.0 / 7.0, rel=1e-15)
+    ordinary = np.delete(np.arange(g["n"]), 5)
+    assert np.all(r["codes"][ordinary] == 0)  # every |v| < 12/7 -> 0
+    assert r["codes"][5] == 7
+    # a value just above half a step does survive
+    v2 = vals.copy()
+    v2[0] = 1.75  # > 12/7 = 1.714..., exact in bf16
+    assert orc.r4_row(bf16(v2), clip=1.0, no_rotate=True)["codes"][0] == 1
+
+
+def test_widget_direction_rotation_lowers_error(orc):
+    """The widget reports 0.882 vs 0.304 (inputs not printed: parity of those two
+    numbers is unpinned); the direction -- rotating first lowers the error
+    several-fold -- is checked on seeded 16-value vectors with outlier 24."""
+    ratios = []
+    for seed in range(20):
+        rng = np.random.default_rng(100 + seed)
+        v = np.clip(rng.standard_normal(16), -2, 2).astype(np.float32)
+        v[rng.integers(16)] = 24.0
+        xb = bf16(v)
+        x = synthetic.bf16_bits_to_f32(xb).astype(np.float64)
+        d = orc.r4_row(xb, 1.0, no_rotate=True)
+        xd = orc.dequant_inverse_row(d["packed"], 16, 0, d["scale64"], no_rotate=True)
+        r = orc.r4_row(xb, 1.0)
+        xr = orc.dequant_inverse_row(r["packed"], 16, 0, r["scale64"])
+        ratios.append(orc.mse(xr, x) / orc.mse(xd, x))
+    assert np.median(ratios) < 0.5
+
+
+def test_hidden_state_outlier_spreads(orc, pages):
+    """4096-dim one-hot outlier of 60 spreads to 60/64 = 0.9375 everywhere; the
+    direct step is 60/7 (printed 8.6); after rotation every code is +-7."""
+    g = pages["hidden_state_outlier"]
+    n = g["n"]
+    for j in (0, 1, 777, 4095):
+        x = np.zeros(n, dtype=np.float32)
+        x[j] = g["outlier"]
+        xb = bf16(x)
+        r = orc.r4_row(xb, 1.0)
+        assert np.all(np.abs(r["y"]) == 0.9375)
+        col = scipy.linalg.hadamard(n)[:, j]
+        assert np.array_equal(np.sign(r["y"]), col)
+        assert round(float(np.abs(r["y"]).max()), g["spread_decimals"]) == g["spread_printed"]
+        assert r["scale64"] == pytest.approx(0.9375 / 7, rel=1e-15)
+        assert np.array_equal(r["codes"], 7 * col)
+        d = orc.r4_row(xb, 1.0, no_rotate=True)
+        assert round(d["scale64"], g["direct_step_decimals"]) == g["direct_step_printed"]
+        assert d["scale64"] == pytest.approx(60 / 7, rel=1e-15)
+
+
+def test_outlier_curse_step(orc, pages):
+    g = pages["outlier_curse"]
+    s, pre, codes = orc.quant_sym_int4(np.array(g["values"]), 1.0)
+    assert round(s, g["decimals"]) == g["scale_printed"]
+    assert s == pytest.approx(184.5 / 7, rel=1e-15)
+    assert codes[0] == 0 and codes[1] == g["int4_max"]
+    assert np.all(codes >= g["int4_min"]) and np.all(codes <= g["int4_max"])
+
+
+# --------------------------------------------------------------------------
+# Quantiser details: ties to even, clamping, degenerate rows, packing.
+# --------------------------------------------------------------------------
+def test_symmetric_ties_round_to_even(orc):
+    y = np.array([7.0, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.5, 4.5, -3.5, 5.5, 6.5])
+    s, pre, codes = orc.quant_sym_int4(y, 1.0)
+    assert s == 1.0
+    assert np.array_equal(codes, np.round(y).astype(np.int8))  # numpy rounds half to even
+    assert list(codes[1:4]) == [0, 2, 2]
+
+
+def test_symmetric_clamp(orc):
+    s, pre, codes = orc.quant_sym_int4(np.array([7.0, -7.0, 3.0, -3.2]), 0.5)
+    assert s == 0.5
+    assert list(codes) == [7, -8, 6, -6]
+
+
+def test_degenerate_zero_row(orc):
+    r = orc.r4_row(np.zeros(128, dtype=np.uint16), 1.0)
+    assert r["scale64"] == 1e-8 and np.all(r["codes"] == 0) and np.all(r["packed"] == 0)
+    assert r["scale32"] == np.float32(1e-8)
+
+
+def test_nibble_packing_layout(orc):
+    assert list(orc.pack_nibbles([1, -1, 7, -8])) == [0xF1, 0x87]
+    assert list(orc.pack_nibbles([0, 15, 3, 12])) == [0xF0, 0xC3]
+    codes = np.random.default_rng(0).integers(-8, 8, size=256)
+    assert np.array_equal(orc.unpack_nibbles(orc.pack_nibbles(codes), 256, True), codes)
+    ucodes = np.random.default_rng(1).integers(0, 16, size=256)
+    assert np.array_equal(orc.unpack_nibbles(orc.pack_nibbles(ucodes), 256, False), ucodes)
+
+
+def test_asymmetric_hand_cases(orc):
+    ramp = np.arange(128, dtype=np.float64)
+    codes, s16, z16, pre = orc.quant_asym_int4(ramp, 0.95)
+    assert s16 == 0x4806  # fp16(120.65 / 15 = 8.0433) = 8.046875
+    assert z16 == 0
+    s = 8.046875
+    assert np.array_equal(codes, np.clip(np.round(ramp / s), 0, 15).astype(np.uint8))
+    assert codes[4] == 0 and codes[5] == 1 and codes[127] == 15
+
+    sh = ramp - 64.0
+    codes, s16, z16, pre = orc.quant_asym_int4(sh, 0.95)
+    assert s16 == 0x4806  # range 0.95*63 + 0.95*64 = 120.65 again
+    assert orc.f16_to_f64([z16])[0] == 8.0  # rne(60.8 / 8.046875 = 7.556)
+    assert np.array_equal(codes, np.clip(np.round(sh / s) + 8, 0, 15).astype(np.uint8))
+
+    codes, s16, z16, pre = orc.quant_asym_int4(np.zeros(128), 0.95)
+    assert s16 == 0x3C00 and z16 == 0 and np.all(codes == 0)
+
+
+def test_asymmetric_dequant_error_bound(orc):
+    rng = np.random.default_rng(5)
+    for _ in range(50):
+        x = rng.standard_normal(128) * rng.uniform(0.1, 10) + rng.uniform(-3, 3)
+        codes, s16, z16, pre = orc.quant_asym_int4(x, 1.0)
+        s = orc.f16_to_f64([s16])[0]
+        z = orc.f16_to_f64([z16])[0]
+        deq = orc.dequant_inverse_row(orc.pack_nibbles(codes), 128, 1, s, z, no_rotate=True)
+        # inside the clipped range every value is within half a step (+ fp16 scale slack)
+        assert np.max(np.abs(deq - x)) <= 0.5 * s * 1.02 + abs(z - (-min(x.min(), 0) / s)) * s
+
+
+# --------------------------------------------------------------------------
+# Storage converters: hand-listed bit patterns and library conversions.
+# --------------------------------------------------------------------------
+def test_bf16_converter(orc):
+    cases = [(1.0, 0x3F80), (-2.0, 0xC000), (60.0, 0x4270), (1 + 2 ** -8, 0x3F80),
+             (1 + 3 * 2 ** -8, 0x3F82), (3.4e38, 0x7F80), (2.0 ** -133, 0x0001),
+             (2.0 ** -134, 0x0000), (0.0, 0x0000), (-0.0, 0x8000)]
+    for v, b in cases:
+        assert orc.f64_to_bf16([v])[0] == b, v
+    assert orc.f64_to_bf16([float("nan")])[0] & 0x7F80 == 0x7F80
+    rng = np.random.default_rng(0)
+    f = (rng.standard_normal(4000) * np.exp(rng.uniform(-60, 60, 4000))).astype(np.float32)
+    ref = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(orc.f64_to_bf16(f.astype(np.float64)), ref)
+    assert np.array_equal(orc.bf16_to_f64(ref), torch.from_numpy(ref.view(np.int16)).view(torch.bfloat16).double().numpy())
+
+
+def test_f16_converter(orc):
+    cases = [(1.0, 0x3C00), (65504.0, 0x7BFF), (65520.0, 0x7C00), (2.0 ** -24, 0x0001),
+             (2.0 ** -25, 0x0000), (1.0 / 3.0, 0x3555), (-8.046875, 0xC806), (2.0 ** -14, 0x0400)]
+    for v, b in cases:
+        assert orc.f64_to_f16([v])[0] == b, v
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal(4000) * np.exp(rng.uniform(-20, 12, 4000))
+    with np.errstate(over="ignore"):
+        ref = x.astype(np.float16).view(np.uint16)  # numpy: correctly rounded double -> half
+    assert np.array_equal(orc.f64_to_f16(x), ref)
+    assert np.array_equal(orc.f16_to_f64(ref), ref.view(np.float16).astype(np.float64))
+
+
+# --------------------------------------------------------------------------
+# RoPE and R3 -- "SpinQuant, when rotations are worth learning", section "Four
+# rotation sites" (R3 after RoPE, exact by construction); "SpinQuant Guide",
+# "RoPE Compatibility with 4-Bit KV Caching" (2-D coordinate pairs).
+# --------------------------------------------------------------------------
+def test_rope_matches_complex_formulation(orc):
+    d, theta = 128, 10000.0
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal(d)
+    for pos in (0, 1, 17, 4095):
+        p = np.arange(d // 2)
+        z = (x[: d // 2] + 1j * x[d // 2:]) * np.exp(1j * pos * theta ** (-2.0 * p / d))
+        ref = np.concatenate([z.real, z.imag])
+        assert np.max(np.abs(orc.rope_half(x, pos, theta) - ref)) < 1e-12
+    assert np.array_equal(orc.rope_half(x, 0, theta), x)
+
+
+def test_rope_relative_position(orc):
+    rng = np.random.default_rng(10)
+    q, k = rng.standard_normal(128), rng.standard_normal(128)
+    a = orc.rope_half(q, 5, 1e4) @ orc.rope_half(k, 2, 1e4)
+    b = orc.rope_half(q, 1003, 1e4) @ orc.rope_half(k, 1000, 1e4)
+    assert abs(a - b) < 1e-10
+
+
+def test_r3_preserves_attention_scores(orc):
+    rng = np.random.default_rng(11)
+    q, k = rng.standard_normal(128), rng.standard_normal(128)
+    assert abs(orc.rotate(q) @ orc.rotate(k) - q @ k) < 1e-12
+
+
+def test_r3_token_composition(orc):
+    """r3_token = RoPE -> H/sqrt(d) -> bf16 for Q; RoPE -> H -> asym INT4 for K;
+    asym INT4 on raw V; checked against the building blocks and numpy."""
+    rng = np.random.default_rng(12)
+    q = bf16(rng.standard_normal((4, 128)).astype(np.float32))
+    k = bf16(rng.standard_normal((2, 128)).astype(np.float32))
+    v = bf16(rng.standard_normal((2, 128)).astype(np.float32))
+    out = orc.r3_token(q, k, v, pos=37, theta=1e4, clip=0.95)
+    H = scipy.linalg.hadamard(128) / math.sqrt(128)
+    for h in range(4):
+        ref = H @ orc.rope_half(synthetic.bf16_bits_to_f32(q[h]).astype(np.float64), 37, 1e4)
+        assert np.max(np.abs(out["q_f64"][h] - ref)) < 1e-12
+        assert np.array_equal(out["q_bf16"][h], orc.f64_to_bf16(ref))
+    for h in range(2):
+        kr = H @ orc.rope_half(synthetic.bf16_bits_to_f32(k[h]).astype(np.float64), 37, 1e4)
+        codes, s16, z16, _ = orc.quant_asym_int4(kr, 0.95)
+        assert np.array_equal(out["k_packed"][h], orc.pack_nibbles(codes))
+        assert out["k_s"][h] == s16 and out["k_z"][h] == z16
+        codes, s16, z16, _ = orc.quant_asym_int4(synthetic.bf16_bits_to_f32(v[h]).astype(np.float64), 0.95)
+        assert np.array_equal(out["v_packed"][h], orc.pack_nibbles(codes))
+
+
+# --------------------------------------------------------------------------
+# Round trip and error model -- "Rotations: ...", widget "Try it" (rotate ->
+# quantize -> rotate back); "SpinQuant Guide", "Quantization Noise Reduction
+# Analysis" (error ~ d * step^2 / 12).
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("with_signs", [False, True])
+def test_round_trip_error_equals_rotated_domain_error(orc, with_signs):
+    n = 1024
+    rng = np.random.default_rng(20)
+    xb = bf16(rng.standard_normal(n).astype(np.float32))
+    x = synthetic.bf16_bits_to_f32(xb).astype(np.float64)
+    signs = synthetic.sign_bits(n, 4) if with_signs else None
+    r = orc.r4_row(xb, 1.0, signs=signs)
+    xh = orc.dequant_inverse_row(r["packed"], n, 0, r["scale64"], signs=signs)
+    err_x = np.linalg.norm(xh - x)
+    err_y = np.linalg.norm(r["codes"] * r["scale64"] - r["y"])
+    assert abs(err_x - err_y) < 1e-12 * np.linalg.norm(x)  # orthogonality
+    assert err_y <= math.sqrt(n) * r["scale64"] / 2  # no clamping at clip = 1
+
+
+def test_error_model_step_squared_over_twelve(orc):
+    n = 4096
+    rng = np.random.default_rng(21)
+    ratios = []
+    for _ in range(8):
+        xb = bf16(rng.standard_normal(n).astype(np.float32))
+        r = orc.r4_row(xb, 1.0)
+        err = np.mean((r["codes"] * r["scale64"] - r["y"]) ** 2)
+        ratios.append(err / (r["scale64"] ** 2 / 12))
+    assert 0.8 < np.mean(ratios) < 1.2
+
+
+def test_config1_direct_closed_form(orc):
+    """Tiny workload, direct quantisation: channel 7 (60.0) sets the step 60/7, its
+    code is 7, and every |x| < 30/7 maps to 0, so the direct MSE is the mean of
+    x^2 over the other channels."""
+    xb = synthetic.tiny()
+    x = synthetic.bf16_bits_to_f32(xb).astype(np.float64)
+    assert np.all(np.abs(np.delete(x, 7, axis=1)) < 30 / 7)
+    for t in range(0, 64, 9):
+        d = orc.r4_row(xb[t], 1.0, no_rotate=True)
+        assert d["scale64"] == pytest.approx(60 / 7, rel=1e-15)
+        assert d["codes"][7] == 7 and np.all(np.delete(d["codes"], 7) == 0)
+        xd = orc.dequant_inverse_row(d["packed"], 256, 0, d["scale64"], no_rotate=True)
+        closed = np.sum(np.delete(x[t], 7) ** 2) / 256
+        assert orc.mse(xd, x[t]) == pytest.approx(closed, rel=1e-12)
+
+
+def test_r4_rows_matches_single_rows(orc):
+    xb = synthetic.sweep(8, tokens=6)
+    packed, scales = orc.r4_rows(xb, 0.9, signs=synthetic.sign_bits(256, 1))
+    for t in range(6):
+        r = orc.r4_row(xb[t], 0.9, signs=synthetic.sign_bits(256, 1))
+        assert np.array_equal(r["packed"], packed[t]) and r["scale32"] == scales[t]
