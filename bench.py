@@ -1,0 +1,380 @@
+"""Benchmark of the fused online-Hadamard + INT4 path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl spin|reference] [--workload NAME]
+
+A step is one pass of the R4 hot path (bf16 load, +-1 diagonal, Walsh-Hadamard
+transform, per-token max, scale, round, clamp, nibble pack, store) over one
+batch of the default workload: 8192 tokens x n = 16384, SwiGLU-like bf16
+input with 0.1 % outlier channels, seeded +-1 diagonal, clip 0.9. Inputs are
+synthetic and seeded (synthetic/), generated on the host and resident in HBM
+before timing; the input (268 MB) is larger than L2 (126 MB) and two input and
+output sets alternate between steps.
+
+With N > 1 (torchrun, one process per GPU) every rank processes its own batch
+(weak scaling, no data exchange: tokens are independent); the elapsed time is
+the maximum over ranks and the value counts all ranks' tokens.
+
+Printed as one JSON line on rank 0. `value` is the algorithmic HBM throughput
+(bytes the method must move: bf16 in, packed codes and fp32 scales out) in
+GB/s; tokens/s and the fraction of the measured HBM copy bandwidth are in the
+same line. `--impl reference` times the fp64 CPU oracle on the host cores on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused Hadamard+INT4-quant HBM GB/s (% of B200 peak) and tokens/s at n=16384"
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def algorithmic_bytes_r4(tokens: int, n: int) -> int:
+    """bf16 in (2n) + packed codes out (n/2) + fp32 scale out (4), per token."""
+    return tokens * (2 * n + n // 2 + 4)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "online_hadamard_rotation_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.startswith("k1_") or name == "spin_tile.cuh":
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
+    the current kernel source; None otherwise."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f).get(kernel)
+    if not d or d.get("source_digest") != kernel_source_digest():
+        return None
+    return d.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    smax.append(float(p[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, p[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+def make_workload(name: str, rank: int):
+    import synthetic
+    if name == "r4_prefill":
+        bits, signs, _ = synthetic.r4_prefill(seed=1 + rank)
+        return dict(kind="r4", bits=bits, signs=signs, clip=0.9,
+                    desc={"workload": "R4 prefill: 4x2048 tokens x n=16384 bf16, SwiGLU-like, 0.1% channels x100, "
+                                      "seeded +-1 diagonal, H_16384 = H_128 (x) H_128, clip 0.9",
+                          "tokens": int(bits.shape[0]), "n": int(bits.shape[1])})
+    if name.startswith("decode"):
+        n = int(name[len("decode"):] or 16384)
+        bits = synthetic.decode(32, n, seed=3 + rank)
+        return dict(kind="r4", bits=bits, signs=None, clip=1.0,
+                    desc={"workload": f"decode: 32 tokens x n={n} Student-t(3), one channel x200 per row, clip 1.0",
+                          "tokens": 32, "n": n})
+    if name.startswith("sweep"):
+        k = int(name[len("sweep"):])
+        bits = synthetic.sweep(k, seed=4 + k + 100 * rank)
+        return dict(kind="r4", bits=bits, signs=None, clip=1.0,
+                    desc={"workload": f"sweep: n=2^{k}, 1 GiB bf16 input, N(0,1) with 0.1% channels x100, clip 1.0",
+                          "tokens": int(bits.shape[0]), "n": 1 << k})
+    if name == "r3_kv":
+        q, k, v, pos = synthetic.r3_kv(seed=2 + rank)
+        return dict(kind="r3", q=q, k=k, v=v, pos=pos, clip=0.95,
+                    desc={"workload": "R3+KV: batch 4 x seq 4096, 32 q / 8 kv heads, head_dim 128, RoPE theta 1e4, "
+                                      "asym INT4 KV cache, clip 0.95", "tokens": 4 * 4096})
+    raise SystemExit(f"unknown workload {name}")
+
+
+def r3_bytes(tokens, hq=32, hkv=8, d=128):
+    return tokens * (2 * hq * d * 2 + 2 * hkv * d * 2 + 2 * hkv * d // 2 + 4 * hkv * 2 + 4)
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 CPU oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, wl):
+    import oracle
+    oracle.lib()
+    if wl["kind"] != "r4":
+        raise SystemExit("the reference arm times the R4 workloads")
+    bits, n = wl["bits"], wl["bits"].shape[1]
+    sample = min(bits.shape[0], max(8, (1 << 22) // n))  # about 0.1-0.2 s of oracle work per step
+    rows = bits[:sample]
+    for _ in range(args.warmup):
+        oracle.r4_rows(rows[:1], wl["clip"], wl["signs"])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.r4_rows(rows, wl["clip"], wl["signs"])
+    dt = time.perf_counter() - t0
+    tok_s = args.steps * sample / dt
+    gbs = algorithmic_bytes_r4(sample, n) * args.steps / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "tokens_per_s": tok_s,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(wl["desc"], parallelism="host cpu, 1 thread"),
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"first {sample} of {bits.shape[0]} tokens per step, fp64 fast transform"},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="spin", choices=["spin", "reference"])
+    ap.add_argument("--workload", default="r4_prefill")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        run_reference(args, make_workload(args.workload, 0))
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    import online_hadamard_rotation_b200 as spin
+    from online_hadamard_rotation_b200 import build
+    build.build()
+    spin.lib()
+
+    wl = make_workload(args.workload, rank)
+    stream = torch.cuda.Stream(dev)
+    if wl["kind"] == "r4":
+        bits, n = wl["bits"], wl["bits"].shape[1]
+        tokens = bits.shape[0]
+        host = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        sets = []
+        for _ in range(2):
+            sets.append(dict(x=host.to(dev), q=torch.empty((tokens, n // 2), dtype=torch.uint8, device=dev),
+                             s=torch.empty((tokens,), dtype=torch.float32, device=dev)))
+        signs = (torch.from_numpy(wl["signs"].view(np.int32)).to(dev) if wl["signs"] is not None else None)
+        step_bytes = algorithmic_bytes_r4(tokens, n)
+
+        def step(i):
+            b = sets[i & 1]
+            spin.hadamard_quant_int4(b["x"], wl["clip"], signs, out=b["q"], scales=b["s"], stream=stream)
+    else:
+        q, k, v, pos = wl["q"], wl["k"], wl["v"], wl["pos"]
+        B, S, hq, d = q.shape
+        hkv = k.shape[2]
+        tokens = B * S
+        sets = []
+        for _ in range(2):
+            sets.append(dict(q=torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).to(dev),
+                             k=torch.from_numpy(k.view(np.int16)).view(torch.bfloat16).to(dev),
+                             v=torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).to(dev),
+                             pos=torch.from_numpy(pos).to(dev), qo=torch.empty((B, S, hq, d), dtype=torch.bfloat16,
+                                                                               device=dev),
+                             cache=spin.alloc_kv_cache(B, hkv, S, d, device=dev)))
+        step_bytes = r3_bytes(tokens, hq, hkv, d)
+
+        def step(i):
+            b = sets[i & 1]
+            spin.rope_hadamard_kvquant(b["q"], b["k"], b["v"], b["pos"], b["cache"], clip=wl["clip"], q_out=b["qo"],
+                                       stream=stream)
+
+    torch.cuda.synchronize()
+    for i in range(args.warmup):
+        step(i)
+    stream.synchronize()
+
+    # ---- device-timed region: inputs resident in HBM
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        ev1.synchronize()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    ms_per_step = ms / args.steps
+    gbs = world * step_bytes * args.steps / (ms / 1e3) / 1e9
+    tok_s = world * tokens * args.steps / (ms / 1e3)
+
+    # ---- end to end through the public API from pinned host memory
+    e2e = None
+    if wl["kind"] == "r4":
+        q_host = torch.empty((tokens, n // 2), dtype=torch.uint8).pin_memory()
+        s_host = torch.empty((tokens,), dtype=torch.float32).pin_memory()
+        b = sets[0]
+        e2e_steps = max(3, args.steps // 5)
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                b["x"].copy_(host, non_blocking=True)
+                spin.hadamard_quant_int4(b["x"], wl["clip"], signs, out=b["q"], scales=b["s"], stream=stream)
+                q_host.copy_(b["q"], non_blocking=True)
+                s_host.copy_(b["s"], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        ev0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        ev1.record(stream)
+        ev1.synchronize()
+        ems = ev0.elapsed_time(ev1)
+        if world > 1:
+            t = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * step_bytes * e2e_steps / (ems / 1e3) / 1e9, "unit": "GB/s",
+               "tokens_per_s": world * tokens * e2e_steps / (ems / 1e3),
+               "h2d_bytes_per_step": int(host.numel() * 2), "d2h_bytes_per_step": int(q_host.numel() + 4 * tokens),
+               "steps": e2e_steps}
+
+    peak, peak_kind = measured_peaks()
+    kname = "k1_rotate_quant_int4" if wl["kind"] == "r4" else "k2_rope_hadamard_kvquant"
+    traffic = recorded_traffic(f"{kname}:{args.workload}")
+    per_gpu_gbs = step_bytes / (ms_per_step / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": per_gpu_gbs, "peak": peak, "unit": "GB/s",
+                "frac": per_gpu_gbs / peak, "traffic": traffic, "kernel": kname,
+                "algorithmic_bytes_per_launch": step_bytes,
+                "peak_source": f"{peak_kind} hbm_gbs (STREAM-style copy)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and wl["kind"] == "r4":
+        import oracle
+        oracle.lib()
+        bits = wl["bits"]
+        sample = bits.shape[0] if bits.shape[1] >= 4096 else min(bits.shape[0], 65536)
+        t0 = time.perf_counter()
+        oracle.r4_rows(bits[:sample], wl["clip"], wl["signs"])
+        dt = time.perf_counter() - t0
+        cpu = {"value": algorithmic_bytes_r4(sample, bits.shape[1]) / dt / 1e9, "unit": "GB/s", "cores": 1,
+               "kind": "oracle", "tokens_per_s": sample / dt,
+               "sample": f"{sample} of {bits.shape[0]} tokens, one pass, fp64 fast transform, 1 thread"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": gbs, "unit": "GB/s", "tokens_per_s": tok_s,
+                "pct_of_hbm_peak": 100.0 * per_gpu_gbs / peak, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": dict(wl["desc"], parallelism=f"dp{world}" if world > 1 else "single GPU",
+                               l2="inputs larger than L2 (268 MB bf16 input vs 126 MB L2); two buffer sets alternate"
+                               if args.workload == "r4_prefill" else "two buffer sets alternate"),
+                "gpu_launches": args.steps, "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu,
+                "clocks": clocks.summary()}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

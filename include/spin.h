@@ -1,0 +1,199 @@
+/*
+ * spin.h -- C ABI of libspin.so: SpinQuant's online Hadamard rotations (R3 and
+ * R4) fused with the low-bit quantisers that follow them, for NVIDIA B200
+ * (sm_100a).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  * Pointers are device pointers the caller owns (allocated by any means).
+ *    The library allocates, frees and synchronises nothing; it never blocks.
+ *  * Each call validates its arguments on the host, then enqueues its kernels
+ *    on `stream` (a cudaStream_t; NULL is the legacy default stream) and
+ *    returns. A non-SPIN_OK status means nothing was enqueued, except
+ *    SPIN_ERR_CUDA, which reports a failed launch (spin_last_cuda_error()
+ *    returns the cudaError_t value). Faults inside a kernel surface later, at
+ *    the caller's next synchronisation, as with any CUDA launch.
+ *  * tokens/rows == 0 is a successful no-op.
+ *  * bfloat16 and float16 buffers are passed as `void*` holding the 16-bit
+ *    patterns, so this header needs no CUDA header.
+ *  * Input and output buffers must not overlap unless a parameter says so.
+ *  * Calls on the same stream are ordered; calls that run concurrently on
+ *    different streams may share inputs but not outputs.
+ *
+ * Quantised layout (all entry points)
+ * -----------------------------------
+ *  Two 4-bit codes per byte: element 2j in the low nibble of byte j,
+ *  element 2j+1 in the high nibble. Symmetric codes are 4-bit two's
+ *  complement in [-8, 7]; asymmetric codes are unsigned in [0, 15].
+ *
+ * Sources are cited by page title and section:
+ *  "SpinQuant, when rotations are worth learning" -- section "Four rotation
+ *    sites, two of them free" (R3 on Q and K after RoPE, R4 on the
+ *    down-projection input), section "Paper vs. code" (K-cache quantisation
+ *    needs a power-of-two head dim because R3 uses the fast transform).
+ *  "Rotations: QuaRot, SpinQuant and incoherence" -- section "Hadamard
+ *    matrices" (Sylvester H_n; (1/sqrt n) H_n orthogonal; randomised
+ *    (1/sqrt n) H_n diag(+-1); Kronecker products), section "Why it's free"
+ *    (O(d log d) transform), widget "Try it" (rotate, quantize, rotate back).
+ *  "SpinQuant Guide: Learned Rotations for 4-Bit LLMs" -- section "The Outlier
+ *    Curse" (INT4 range [-8, 7], step = max|x| / 7), section "End-to-End
+ *    Implementation" (step clamped below at 1e-8; dequant = code * step),
+ *    section "RoPE Compatibility with 4-Bit KV Caching" (RoPE rotates 2-D
+ *    pairs; KV cache stored as 4-bit).
+ */
+#ifndef SPIN_H_
+#define SPIN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *spin_stream_t;
+
+typedef enum spin_status_t {
+  SPIN_OK = 0,
+  SPIN_ERR_INVALID_ARG = 1,      /* null pointer, bad count, clip outside (0, 1], ... */
+  SPIN_ERR_UNSUPPORTED_SIZE = 2, /* n or head_dim not a supported power of two */
+  SPIN_ERR_MISALIGNED = 3,       /* a pointer is not 16-byte aligned */
+  SPIN_ERR_CUDA = 4,             /* a CUDA call or launch failed: see spin_last_cuda_error() */
+  SPIN_ERR_DEVICE = 5            /* the current device is not compute capability 10.0 */
+} spin_status_t;
+
+/* flags */
+#define SPIN_NO_ROTATE 1u /* skip the diagonal and the transform (direct quantisation / identity) */
+
+/* spin_dequant_hadamard_inverse modes */
+#define SPIN_SYM_INT4_F32SCALE 0 /* signed codes, fp32 scale per row: value = code * scale */
+#define SPIN_ASYM_INT4_F16SZ 1   /* unsigned codes, fp16 scale and zero per row: (code - zero) * scale */
+
+/* output dtypes */
+#define SPIN_BF16 0
+#define SPIN_F32 1
+
+/*
+ * R4: rotate the down-projection input and quantise it per token
+ * ("SpinQuant, when rotations are worth learning", "Four rotation sites":
+ * R4 is a fixed Hadamard on the down-projection input; "SpinQuant Guide",
+ * "The Outlier Curse": symmetric INT4 with step max|x| / 7).
+ *
+ * For each of `tokens` rows x (n bfloat16 values, row-major, contiguous):
+ *   y = H_n D x / sqrt(n)     (H_n Sylvester order, D = diag(+-1), D = I if sign_bits == NULL)
+ *   m = max_j |y_j|,  scale = max(clip * m / 7, 1e-8)
+ *   code_j = clamp(round_half_even(y_j / scale), -8, 7)
+ * Arithmetic is fp32 on the device (the transform is exact reassociation of
+ * the same sums; only rounding order differs from an fp64 evaluation).
+ *
+ *  x_bf16      [tokens, n] bf16, 16-byte aligned, read only
+ *  tokens      >= 0
+ *  n           power of two, 128 <= n <= 32768
+ *  clip        0 < clip <= 1 (scale multiplier; codes saturate beyond it)
+ *  q_packed_u8 [tokens, n/2] bytes, 16-byte aligned, written
+ *  scales_f32  [tokens] fp32, 4-byte aligned, written (the step, in y units)
+ *  stream      cudaStream_t
+ * Errors: SPIN_ERR_INVALID_ARG (null pointer with tokens > 0, tokens < 0,
+ * clip outside (0, 1] or NaN), SPIN_ERR_UNSUPPORTED_SIZE (n),
+ * SPIN_ERR_MISALIGNED, SPIN_ERR_DEVICE, SPIN_ERR_CUDA.
+ */
+spin_status_t spin_hadamard_quant_int4(const void *x_bf16, int64_t tokens, int32_t n, float clip,
+                                       uint8_t *q_packed_u8, float *scales_f32,
+                                       spin_stream_t stream);
+
+/*
+ * Superset of spin_hadamard_quant_int4 ("Rotations: QuaRot, SpinQuant and
+ * incoherence", "Hadamard matrices": the randomised transform
+ * (1/sqrt n) H_n diag(+-1)).
+ *  sign_bits  nullable; [n/32] uint32 words, bit j of the mask set means
+ *             d_j = -1. 4-byte aligned.
+ *  flags      0 or SPIN_NO_ROTATE (quantise x directly: no D, no H), used to
+ *             measure the direct-quantisation error.
+ * spin_hadamard_quant_int4(...) == spin_hadamard_quant_int4_ex(..., NULL, 0, ...).
+ */
+spin_status_t spin_hadamard_quant_int4_ex(const void *x_bf16, int64_t tokens, int32_t n,
+                                          float clip, const uint32_t *sign_bits, uint32_t flags,
+                                          uint8_t *q_packed_u8, float *scales_f32,
+                                          spin_stream_t stream);
+
+/*
+ * R3 + INT4 KV cache ("SpinQuant, when rotations are worth learning", "Four
+ * rotation sites": R3 is a fixed Hadamard on queries and keys after RoPE,
+ * there only to make the KV cache quantisable; "SpinQuant Guide", "RoPE
+ * Compatibility with 4-Bit KV Caching": RoPE rotates 2-D coordinate pairs).
+ *
+ * For every token (b, s) and head:
+ *   RoPE (rotate-half pairing): for p < d/2, a = pos[b,s] * theta^(-2p/d),
+ *     (x_p, x_{p+d/2}) <- (x_p cos a - x_{p+d/2} sin a, x_{p+d/2} cos a + x_p sin a)
+ *   Q heads: q_out = bf16(H_d RoPE(q) / sqrt(d))
+ *   K heads: k' = H_d RoPE(k) / sqrt(d), quantised asymmetrically
+ *   V heads: v, quantised asymmetrically (no RoPE, no rotation)
+ * Asymmetric INT4 per (token, kv head) group of d values x:
+ *   lo = min(clip * min x, 0), hi = max(clip * max x, 0)
+ *   scale = fp16((hi - lo) / 15) (round to nearest even); if it is 0: scale = 1, zero = 0
+ *   zero  = clamp(round_half_even(-lo / scale), 0, 15)        (stored as fp16, exact)
+ *   code  = clamp(round_half_even(x / scale) + zero, 0, 15)
+ * The cache slot of token (b, s) is cache_offset + s; `pos` only sets the
+ * RoPE angle.
+ *
+ *  q, k, v      [batch, seq, n_q_heads | n_kv_heads, head_dim] bf16, 16-byte aligned
+ *  pos          [batch, seq] int32 RoPE positions (>= 0)
+ *  theta        RoPE base (> 0), e.g. 10000
+ *  head_dim     128 (power of two; other sizes return SPIN_ERR_UNSUPPORTED_SIZE)
+ *  batch, seq   > 0 (0 is a no-op); n_q_heads, n_kv_heads > 0, n_q_heads % n_kv_heads == 0
+ *  clip         0 < clip <= 1
+ *  q_out        [batch, seq, n_q_heads, head_dim] bf16, 16-byte aligned; may equal q
+ *  k_cache, v_cache  [batch, n_kv_heads, cache_len, head_dim/2] bytes, 16-byte aligned
+ *  k_scale, k_zero, v_scale, v_zero  [batch, n_kv_heads, cache_len] fp16
+ *  cache_len    >= cache_offset + seq;  cache_offset >= 0
+ */
+spin_status_t spin_rope_hadamard_kvquant(const void *q, const void *k, const void *v,
+                                         const int32_t *pos, float theta, int32_t head_dim,
+                                         int32_t batch, int32_t seq, int32_t n_q_heads,
+                                         int32_t n_kv_heads, float clip, void *q_out,
+                                         uint8_t *k_cache, uint8_t *v_cache, void *k_scale,
+                                         void *k_zero, void *v_scale, void *v_zero,
+                                         int32_t cache_len, int32_t cache_offset,
+                                         spin_stream_t stream);
+
+/*
+ * Dequantise and rotate back ("Rotations: QuaRot, SpinQuant and
+ * incoherence", widget "Try it": rotate, quantize, rotate back; "Hadamard
+ * matrices": H_n / sqrt(n) is orthogonal and symmetric, so the inverse of
+ * H_n D / sqrt(n) is D H_n / sqrt(n); "SpinQuant Guide", "End-to-End
+ * Implementation": dequant = code * scale).
+ *
+ * For each of `rows` rows of n codes:
+ *   mode SPIN_SYM_INT4_F32SCALE: v_j = code_j * scale            (scale: fp32 [rows])
+ *   mode SPIN_ASYM_INT4_F16SZ:   v_j = (code_j - zero) * scale   (scale, zero: fp16 [rows])
+ *   out = D H_n v / sqrt(n)   unless flags has SPIN_NO_ROTATE (then out = v)
+ * A KV cache [batch, n_kv_heads, cache_len, head_dim/2] is rows = batch *
+ * n_kv_heads * cache_len rows of n = head_dim (use SPIN_NO_ROTATE for V: R3
+ * rotates K only; RoPE is not undone).
+ *
+ *  codes      [rows, n/2] bytes, 16-byte aligned
+ *  n          power of two, 128 <= n <= 32768
+ *  scale      [rows] fp32 or fp16 by mode; zero [rows] fp16 (asym) or NULL (sym)
+ *  sign_bits  nullable, as in spin_hadamard_quant_int4_ex
+ *  out        [rows, n] bf16 or fp32 (out_dtype), 16-byte aligned
+ */
+spin_status_t spin_dequant_hadamard_inverse(const uint8_t *codes, int64_t rows, int32_t n,
+                                            int32_t mode, const void *scale, const void *zero,
+                                            const uint32_t *sign_bits, uint32_t flags, void *out,
+                                            int32_t out_dtype, spin_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *spin_status_string(spin_status_t status);
+
+/* cudaError_t value of the last failed CUDA call made by this library in the
+ * calling thread (0 if none). */
+int spin_last_cuda_error(void);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int spin_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPIN_H_ */

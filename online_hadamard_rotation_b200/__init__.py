@@ -1,0 +1,217 @@
+"""Python binding for libspin.so: SpinQuant's online Hadamard rotations (R3,
+R4) fused with INT4 quantisation, on NVIDIA B200.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/spin.h. PyTorch supplies device
+memory and streams. The library must be built (``build.py``); importing this
+package without it raises, and there is no CPU fallback.
+
+The functions named ``spin_*`` take raw pointers exactly like the C ABI; the
+other functions take torch tensors and return torch tensors.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+
+import torch
+
+__all__ = [
+    "lib", "SpinError", "hadamard_quant_int4", "hadamard_quant_int4_host", "rope_hadamard_kvquant",
+    "dequant_hadamard_inverse", "alloc_kv_cache", "NO_ROTATE", "SYM_INT4_F32SCALE", "ASYM_INT4_F16SZ",
+    "BF16", "F32", "HEADER", "LIB_PATH", "exported_symbols",
+]
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libspin.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "spin.h")
+
+NO_ROTATE = 1
+SYM_INT4_F32SCALE = 0
+ASYM_INT4_F16SZ = 1
+BF16 = 0
+F32 = 1
+
+_STATUS = {0: "SPIN_OK", 1: "SPIN_ERR_INVALID_ARG", 2: "SPIN_ERR_UNSUPPORTED_SIZE",
+           3: "SPIN_ERR_MISALIGNED", 4: "SPIN_ERR_CUDA", 5: "SPIN_ERR_DEVICE"}
+
+
+class SpinError(RuntimeError):
+    def __init__(self, fn: str, status: int, cuda_error: int = 0):
+        self.status = status
+        self.cuda_error = cuda_error
+        msg = f"{fn} returned {_STATUS.get(status, status)}"
+        if status == 4:
+            msg += f" (cudaError {cuda_error})"
+        super().__init__(msg)
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load libspin.so from this package directory (raises if it is not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python online_hadamard_rotation_b200/build.py` (there is no CPU fallback)")
+    L = C.CDLL(LIB_PATH)
+    vp, i64, i32, u32, f32 = C.c_void_p, C.c_int64, C.c_int32, C.c_uint32, C.c_float
+    L.spin_hadamard_quant_int4.argtypes = [vp, i64, i32, f32, vp, vp, vp]
+    L.spin_hadamard_quant_int4_ex.argtypes = [vp, i64, i32, f32, vp, u32, vp, vp, vp]
+    L.spin_rope_hadamard_kvquant.argtypes = [vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, f32, vp, vp, vp,
+                                             vp, vp, vp, vp, i32, i32, vp]
+    L.spin_dequant_hadamard_inverse.argtypes = [vp, i64, i32, i32, vp, vp, vp, u32, vp, i32, vp]
+    for name in ("spin_hadamard_quant_int4", "spin_hadamard_quant_int4_ex", "spin_rope_hadamard_kvquant",
+                 "spin_dequant_hadamard_inverse"):
+        getattr(L, name).restype = C.c_int
+    L.spin_status_string.argtypes = [C.c_int]
+    L.spin_status_string.restype = C.c_char_p
+    L.spin_last_cuda_error.restype = C.c_int
+    L.spin_version.restype = C.c_int
+    _lib = L
+    return L
+
+
+def exported_symbols() -> list[str]:
+    """Function names declared in include/spin.h."""
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(spin_\w+)\s*\(", text, flags=re.M)))
+
+
+# ------------------------------------------------------------------ raw C ABI (pointers)
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise SpinError(fn, status, lib().spin_last_cuda_error())
+
+
+def spin_hadamard_quant_int4(x_bf16, tokens, n, clip, q_packed_u8, scales_f32, stream) -> int:
+    return lib().spin_hadamard_quant_int4(x_bf16, tokens, n, clip, q_packed_u8, scales_f32, stream)
+
+
+def spin_hadamard_quant_int4_ex(x_bf16, tokens, n, clip, sign_bits, flags, q_packed_u8, scales_f32,
+                                stream) -> int:
+    return lib().spin_hadamard_quant_int4_ex(x_bf16, tokens, n, clip, sign_bits, flags, q_packed_u8,
+                                             scales_f32, stream)
+
+
+def spin_rope_hadamard_kvquant(*args) -> int:
+    return lib().spin_rope_hadamard_kvquant(*args)
+
+
+def spin_dequant_hadamard_inverse(*args) -> int:
+    return lib().spin_dequant_hadamard_inverse(*args)
+
+
+# ------------------------------------------------------------------ torch-level helpers
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype, device=None):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+
+
+def hadamard_quant_int4(x: torch.Tensor, clip: float = 1.0, signs: torch.Tensor | None = None,
+                        no_rotate: bool = False, out: torch.Tensor | None = None,
+                        scales: torch.Tensor | None = None, stream=None):
+    """R4: x [tokens, n] bf16 (CUDA) -> (codes [tokens, n/2] uint8, scales [tokens] fp32)."""
+    _need(x, "x", torch.bfloat16)
+    tokens, n = x.shape
+    if out is None:
+        out = torch.empty((tokens, n // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((tokens,), dtype=torch.float32, device=x.device)
+    if signs is not None:
+        _need(signs, "signs", torch.int32, x.device)
+    st = spin_hadamard_quant_int4_ex(_ptr(x), tokens, n, float(clip), _ptr(signs), NO_ROTATE if no_rotate else 0,
+                                     _ptr(out), _ptr(scales), _stream(stream))
+    _check("spin_hadamard_quant_int4_ex", st)
+    return out, scales
+
+
+def hadamard_quant_int4_host(x_host: torch.Tensor, clip: float = 1.0, signs: torch.Tensor | None = None,
+                             device=None, stream=None, buffers=None):
+    """End-to-end R4 from host memory: copy x (pinned, bf16) to the device, run
+    the kernel, copy codes and scales back into pinned host tensors. Returns
+    (codes_host, scales_host); synchronises the stream before returning."""
+    device = torch.device(device or "cuda")
+    tokens, n = x_host.shape
+    if buffers is None:
+        buffers = dict(
+            x=torch.empty((tokens, n), dtype=torch.bfloat16, device=device),
+            q=torch.empty((tokens, n // 2), dtype=torch.uint8, device=device),
+            s=torch.empty((tokens,), dtype=torch.float32, device=device),
+            q_host=torch.empty((tokens, n // 2), dtype=torch.uint8, pin_memory=True),
+            s_host=torch.empty((tokens,), dtype=torch.float32, pin_memory=True))
+    s = stream or torch.cuda.current_stream(device)
+    with torch.cuda.stream(s):
+        buffers["x"].copy_(x_host, non_blocking=True)
+        hadamard_quant_int4(buffers["x"], clip, signs, out=buffers["q"], scales=buffers["s"], stream=s)
+        buffers["q_host"].copy_(buffers["q"], non_blocking=True)
+        buffers["s_host"].copy_(buffers["s"], non_blocking=True)
+    s.synchronize()
+    return buffers["q_host"], buffers["s_host"]
+
+
+def alloc_kv_cache(batch: int, n_kv_heads: int, cache_len: int, head_dim: int = 128, device="cuda"):
+    """Caller-owned INT4 KV cache buffers in the layout the kernel writes."""
+    return dict(
+        k_cache=torch.zeros((batch, n_kv_heads, cache_len, head_dim // 2), dtype=torch.uint8, device=device),
+        v_cache=torch.zeros((batch, n_kv_heads, cache_len, head_dim // 2), dtype=torch.uint8, device=device),
+        k_scale=torch.zeros((batch, n_kv_heads, cache_len), dtype=torch.float16, device=device),
+        k_zero=torch.zeros((batch, n_kv_heads, cache_len), dtype=torch.float16, device=device),
+        v_scale=torch.zeros((batch, n_kv_heads, cache_len), dtype=torch.float16, device=device),
+        v_zero=torch.zeros((batch, n_kv_heads, cache_len), dtype=torch.float16, device=device))
+
+
+def rope_hadamard_kvquant(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos: torch.Tensor,
+                          cache: dict, theta: float = 10000.0, clip: float = 1.0, cache_offset: int = 0,
+                          q_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """R3 + INT4 KV: q [B,S,hq,d], k/v [B,S,hkv,d] bf16, pos [B,S] int32.
+    Writes the cache dict (see alloc_kv_cache) and returns rotated Q (bf16)."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16)
+    _need(pos, "pos", torch.int32)
+    B, S, hq, d = q.shape
+    hkv = k.shape[2]
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    cache_len = cache["k_cache"].shape[2]
+    st = spin_rope_hadamard_kvquant(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(pos), float(theta), d, B, S, hq, hkv, float(clip), _ptr(q_out),
+        _ptr(cache["k_cache"]), _ptr(cache["v_cache"]), _ptr(cache["k_scale"]), _ptr(cache["k_zero"]),
+        _ptr(cache["v_scale"]), _ptr(cache["v_zero"]), cache_len, cache_offset, _stream(stream))
+    _check("spin_rope_hadamard_kvquant", st)
+    return q_out
+
+
+def dequant_hadamard_inverse(codes: torch.Tensor, n: int, scale: torch.Tensor, zero: torch.Tensor | None = None,
+                             mode: int = SYM_INT4_F32SCALE, signs: torch.Tensor | None = None,
+                             no_rotate: bool = False, out_dtype=torch.float32, out: torch.Tensor | None = None,
+                             stream=None) -> torch.Tensor:
+    """codes [..., n/2] uint8 -> out [..., n] (rows = codes.numel() / (n/2))."""
+    _need(codes, "codes", torch.uint8)
+    rows = codes.numel() // (n // 2)
+    if out is None:
+        out = torch.empty(tuple(codes.shape[:-1]) + (n,), dtype=out_dtype, device=codes.device)
+    dt = F32 if out.dtype == torch.float32 else BF16
+    st = spin_dequant_hadamard_inverse(_ptr(codes), rows, n, mode, _ptr(scale), _ptr(zero), _ptr(signs),
+                                       NO_ROTATE if no_rotate else 0, _ptr(out), dt, _stream(stream))
+    _check("spin_dequant_hadamard_inverse", st)
+    return out

@@ -1,0 +1,314 @@
+// k2_rope_kv.cu -- R3 and the INT4 KV cache on CUDA cores.
+//
+// "SpinQuant, when rotations are worth learning", section "Four rotation
+// sites": R3 is a fixed Hadamard applied to queries and keys after RoPE, there
+// to make the KV cache quantisable; section "Paper vs. code": the K cache path
+// needs a power-of-two head dim, since R3 is the fast transform.
+// "SpinQuant Guide: Learned Rotations for 4-Bit LLMs", section "RoPE
+// Compatibility with 4-Bit KV Caching": RoPE rotates 2-D coordinate pairs and
+// the KV cache is stored as 4-bit integers.
+//
+// One thread owns one head vector (d = 128 values) end to end, so RoPE's pair
+// partners (p, p + 64), all seven butterfly stages and the group min/max are
+// in its registers. Head vectors reach shared memory through 16-byte
+// cp.async copies that are coalesced in global memory; inside a 256-byte smem
+// row the 16-byte chunk c sits at c ^ (row & 7), so eight threads reading
+// chunk c of eight consecutive rows hit eight different bank groups. The
+// copies for the next group of tokens are in flight while the current group
+// is computed (two buffers).
+//
+// Q: out = bf16(H RoPE(q) / sqrt(d)), written back into the smem row and then
+// copied out with coalesced 16-byte stores. K: H RoPE(k) / sqrt(d), V: v, each
+// quantised asymmetrically per (token, kv head) group and written straight to
+// its cache row (64 bytes) with fp16 scale and zero.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "spin_launch.h"
+#include "spin_tile.cuh"
+
+namespace spin {
+namespace {
+
+constexpr int kD = 128;          // head dim handled by this kernel
+constexpr int kRowBytes = kD * 2;
+constexpr float kMagic = 12582912.0f;
+
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// byte offset of 16-byte chunk c of smem row r
+__device__ __forceinline__ uint32_t chunk_off(uint32_t r, uint32_t c) {
+  return r * kRowBytes + ((c ^ (r & 7u)) << 4);
+}
+
+// 7 butterfly stages of H_128 over the register index.
+__device__ __forceinline__ void fwht128(float (&x)[kD]) {
+#pragma unroll
+  for (int i = 0; i < kD; i += 2) {
+    const float a = x[i], b = x[i + 1];
+    x[i] = a + b;
+    x[i + 1] = a - b;
+  }
+#pragma unroll
+  for (int h = 2; h < kD; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < kD; i += 2) {
+      if (i & h) continue;
+      bfly2(x[i], x[i + 1], x[i + h], x[i + h + 1]);
+    }
+  }
+}
+
+// Asymmetric INT4 of one group of 128 values; writes 64 bytes of codes and the
+// fp16 scale and zero.
+__device__ __forceinline__ void quant_asym_store(const float (&x)[kD], float clip, uint8_t *codes_dst,
+                                                 __half *scale_dst, __half *zero_dst) {
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < kD; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+  const float lo = fminf(clip * mn, 0.f), hi = fmaxf(clip * mx, 0.f);
+  __half s16 = __float2half_rn((hi - lo) / 15.0f);
+  float s = __half2float(s16), z = 0.f;
+  if (s == 0.f) {
+    s16 = __float2half_rn(1.0f);
+    s = 1.0f;
+  } else {
+    z = fminf(fmaxf(rintf(-lo / s), 0.f), 15.f);
+  }
+  const float c15 = (1.0f / s) / 15.0f, z15 = z / 15.0f;
+  uint32_t words[16];
+#pragma unroll
+  for (int w = 0; w < 16; ++w) {
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      b[i] = __float_as_uint(fmaf(fma_sat(x[8 * w + i], c15, z15), 15.0f, kMagic));
+    const uint32_t e = __byte_perm(__byte_perm(b[0], b[2], 0x0040), __byte_perm(b[4], b[6], 0x0040), 0x5410);
+    const uint32_t o = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
+    words[w] = e | (o << 4);
+  }
+  uint4 *dst = reinterpret_cast<uint4 *>(codes_dst);
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    __stcs(dst + k, make_uint4(words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]));
+  *scale_dst = s16;
+  *zero_dst = __float2half_rn(z);
+}
+
+struct K2Args {
+  const uint16_t *q, *k, *v;
+  const int32_t *pos;
+  uint16_t *q_out;
+  uint8_t *k_cache, *v_cache;
+  __half *k_scale, *k_zero, *v_scale, *v_zero;
+  int64_t ntok;  // batch * seq
+  int seq, hq, hkv, tok_per_group, cache_len, cache_offset;
+  float clip, inv_sqrt_d;
+  double theta;
+};
+
+__global__ void __launch_bounds__(256) k2_rope_hadamard_kvquant(K2Args a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int rows_tok = a.hq + 2 * a.hkv;
+  const int G = a.tok_per_group;
+  const int rows = G * rows_tok;
+  uint8_t *stage[2] = {smem, smem + (size_t)rows * kRowBytes};
+  float2 *table[2];
+  table[0] = reinterpret_cast<float2 *>(smem + 2 * (size_t)rows * kRowBytes);
+  table[1] = table[0] + G * (kD / 2);
+  double *inv_freq = reinterpret_cast<double *>(table[1] + G * (kD / 2));
+
+  const int t = threadIdx.x, nt = blockDim.x;
+  const int64_t ngroups = (a.ntok + G - 1) / G;
+
+  for (int p = t; p < kD / 2; p += nt) inv_freq[p] = pow(a.theta, -2.0 * p / (double)kD);
+  __syncthreads();
+
+  // Issue the copies of group g into buffer b and fill its RoPE table.
+  auto prefetch = [&](int64_t g, int b) {
+    const int64_t tok0 = g * G;
+    const int ntk = (int)((a.ntok - tok0) < G ? (a.ntok - tok0) : G);
+    // Q rows [0, ntk*hq), then K rows, then V rows (token-major inside each)
+    const int nq = ntk * a.hq, nk = ntk * a.hkv;
+    const int chunks = (nq + 2 * nk) * (kRowBytes / 16);
+    for (int i = t; i < chunks; i += nt) {
+      const int r = i >> 4, c = i & 15;
+      const uint16_t *src;
+      int sr;
+      if (r < nq) {
+        src = a.q + (tok0 * a.hq + r) * kD;
+        sr = r;
+      } else if (r < nq + nk) {
+        src = a.k + (tok0 * a.hkv + (r - nq)) * kD;
+        sr = G * a.hq + (r - nq);
+      } else {
+        src = a.v + (tok0 * a.hkv + (r - nq - nk)) * kD;
+        sr = G * (a.hq + a.hkv) + (r - nq - nk);
+      }
+      cp_async16(stage[b] + chunk_off(sr, c), src + c * 8);
+    }
+    cp_async_commit();
+    for (int i = t; i < ntk * (kD / 2); i += nt) {
+      const int tk = i / (kD / 2), p = i % (kD / 2);
+      const double ang = (double)a.pos[tok0 + tk] * inv_freq[p];
+      double sn, cs;
+      sincos(ang, &sn, &cs);
+      table[b][tk * (kD / 2) + p] = make_float2((float)cs, (float)sn);
+    }
+  };
+
+  int64_t g = blockIdx.x;
+  int buf = 0;
+  if (g < ngroups) prefetch(g, 0);
+  for (; g < ngroups; g += gridDim.x, buf ^= 1) {
+    __syncthreads();  // every thread is done with the buffer the next copies overwrite
+    const int64_t gn = g + gridDim.x;
+    if (gn < ngroups) prefetch(gn, buf ^ 1);
+    else cp_async_commit();  // keep the group count uniform
+    cp_async_wait_1();
+    __syncthreads();
+
+    const int64_t tok0 = g * G;
+    const int ntk = (int)((a.ntok - tok0) < G ? (a.ntok - tok0) : G);
+    uint8_t *sb = stage[buf];
+    const float2 *tb = table[buf];
+
+    for (int r = t; r < rows; r += nt) {
+      int kind, tk, h;
+      if (r < G * a.hq) {
+        kind = 0; tk = r / a.hq; h = r % a.hq;
+      } else if (r < G * (a.hq + a.hkv)) {
+        // thread order (head, token) so neighbouring threads write neighbouring cache slots
+        const int i = r - G * a.hq;
+        kind = 1; h = i / G; tk = i % G;
+      } else {
+        const int i = r - G * (a.hq + a.hkv);
+        kind = 2; h = i / G; tk = i % G;
+      }
+      if (tk >= ntk) continue;
+      const int sr = kind == 0 ? tk * a.hq + h : G * a.hq + (kind == 2 ? G * a.hkv : 0) + tk * a.hkv + h;
+      float x[kD];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(sb + chunk_off(sr, c));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          x[8 * c + 2 * k] = bf16lo(ww[k]);
+          x[8 * c + 2 * k + 1] = bf16hi(ww[k]);
+        }
+      }
+      const int64_t tok = tok0 + tk;
+      if (kind != 2) {
+        const float2 *cs = tb + tk * (kD / 2);
+#pragma unroll
+        for (int p = 0; p < kD / 2; ++p) {
+          const float2 e = cs[p];
+          const float x0 = x[p], x1 = x[p + kD / 2];
+          x[p] = fmaf(x0, e.x, -x1 * e.y);
+          x[p + kD / 2] = fmaf(x1, e.x, x0 * e.y);
+        }
+        fwht128(x);
+#pragma unroll
+        for (int i = 0; i < kD; ++i) x[i] *= a.inv_sqrt_d;
+      }
+      if (kind == 0) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const uint4 w = make_uint4(pack_bf16x2(x[8 * c], x[8 * c + 1]), pack_bf16x2(x[8 * c + 2], x[8 * c + 3]),
+                                     pack_bf16x2(x[8 * c + 4], x[8 * c + 5]),
+                                     pack_bf16x2(x[8 * c + 6], x[8 * c + 7]));
+          *reinterpret_cast<uint4 *>(sb + chunk_off(sr, c)) = w;
+        }
+      } else {
+        const int64_t b = tok / a.seq, s = tok % a.seq;
+        const int64_t crow = (b * a.hkv + h) * (int64_t)a.cache_len + a.cache_offset + s;
+        if (kind == 1)
+          quant_asym_store(x, a.clip, a.k_cache + crow * (kD / 2), a.k_scale + crow, a.k_zero + crow);
+        else
+          quant_asym_store(x, a.clip, a.v_cache + crow * (kD / 2), a.v_scale + crow, a.v_zero + crow);
+      }
+    }
+    __syncthreads();
+    // rotated Q rows: smem -> q_out, coalesced
+    const int qchunks = ntk * a.hq * 16;
+    uint4 *qo = reinterpret_cast<uint4 *>(a.q_out + tok0 * a.hq * kD);
+    for (int i = t; i < qchunks; i += nt) {
+      const int r = i >> 4, c = i & 15;
+      __stcs(qo + i, *reinterpret_cast<const uint4 *>(sb + chunk_off(r, c)));
+    }
+  }
+  cp_async_wait_1();
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+}  // namespace
+
+cudaError_t launch_rope_hadamard_kvquant(const void *q, const void *k, const void *v,
+                                         const int32_t *pos, float theta, int batch, int seq,
+                                         int n_q_heads, int n_kv_heads, float clip, void *q_out,
+                                         uint8_t *k_cache, uint8_t *v_cache, void *k_scale,
+                                         void *k_zero, void *v_scale, void *v_zero, int cache_len,
+                                         int cache_offset, cudaStream_t stream) {
+  const int rows_tok = n_q_heads + 2 * n_kv_heads;
+  int G = 1;
+  while (G < 8 && 2 * G * rows_tok <= 256) G *= 2;  // tokens per group: at most 256 head vectors
+  const int rows = G * rows_tok;
+  int threads = rows < 256 ? ((rows + 31) / 32) * 32 : 256;
+  const size_t smem = 2 * (size_t)rows * kRowBytes + 2 * (size_t)G * (kD / 2) * sizeof(float2) +
+                      (kD / 2) * sizeof(double);
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  int slots = 0;
+  cudaError_t err =
+      resident_slots(reinterpret_cast<const void *>(k2_rope_hadamard_kvquant), threads, (int)smem, &slots);
+  if (err != cudaSuccess) return err;
+  K2Args a;
+  a.q = static_cast<const uint16_t *>(q);
+  a.k = static_cast<const uint16_t *>(k);
+  a.v = static_cast<const uint16_t *>(v);
+  a.pos = pos;
+  a.q_out = static_cast<uint16_t *>(q_out);
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.k_scale = static_cast<__half *>(k_scale);
+  a.k_zero = static_cast<__half *>(k_zero);
+  a.v_scale = static_cast<__half *>(v_scale);
+  a.v_zero = static_cast<__half *>(v_zero);
+  a.ntok = (int64_t)batch * seq;
+  a.seq = seq;
+  a.hq = n_q_heads;
+  a.hkv = n_kv_heads;
+  a.tok_per_group = G;
+  a.cache_len = cache_len;
+  a.cache_offset = cache_offset;
+  a.clip = clip;
+  a.inv_sqrt_d = (float)(1.0 / std::sqrt((double)kD));
+  a.theta = (double)theta;
+  const int64_t ngroups = (a.ntok + G - 1) / G;
+  const int64_t grid = ngroups < slots ? ngroups : slots;
+  k2_rope_hadamard_kvquant<<<(unsigned)grid, threads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace spin

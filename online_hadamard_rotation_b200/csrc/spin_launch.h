@@ -1,0 +1,32 @@
+// spin_launch.h -- host-side launchers behind the C ABI (internal header).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace spin {
+
+constexpr uint32_t kNoRotate = 1u;  // same value as SPIN_NO_ROTATE
+
+// Number of blocks of `kernel` that are resident on the current device at once
+// (SM count x blocks per SM), with the dynamic shared-memory opt-in applied.
+// Cached per kernel and device after the first call.
+cudaError_t resident_slots(const void *kernel, int threads, int dyn_smem, int *slots);
+
+cudaError_t launch_rotate_quant_int4(const void *x, int64_t tokens, int log_n, float clip,
+                                     const uint32_t *signs, uint32_t flags, uint8_t *q, float *scales,
+                                     cudaStream_t stream);
+
+cudaError_t launch_dequant_inverse(const uint8_t *codes, int64_t rows, int log_n, int mode,
+                                   const void *scale, const void *zero, const uint32_t *signs,
+                                   uint32_t flags, void *out, int out_dtype, cudaStream_t stream);
+
+cudaError_t launch_rope_hadamard_kvquant(const void *q, const void *k, const void *v,
+                                         const int32_t *pos, float theta, int batch, int seq,
+                                         int n_q_heads, int n_kv_heads, float clip, void *q_out,
+                                         uint8_t *k_cache, uint8_t *v_cache, void *k_scale,
+                                         void *k_zero, void *v_scale, void *v_zero, int cache_len,
+                                         int cache_offset, cudaStream_t stream);
+
+}  // namespace spin

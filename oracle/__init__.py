@@ -59,6 +59,8 @@ def lib():
     L.orc_quant_sym_int4.restype = C.c_double
     L.orc_quant_asym_int4.argtypes = [_dp, C.c_int, C.c_double, vp, _u8p,
                                       C.POINTER(C.c_uint16), C.POINTER(C.c_uint16)]
+    L.orc_asym_unrounded_scale.argtypes = [_dp, C.c_int, C.c_double]
+    L.orc_asym_unrounded_scale.restype = C.c_double
     L.orc_pack_nibbles.argtypes = [_i32p, C.c_int, _u8p]
     L.orc_unpack_nibbles.argtypes = [_u8p, C.c_int, C.c_int, _i32p]
     L.orc_r4_row.argtypes = [_u16p, C.c_int, C.c_double, vp, C.c_uint32, C.c_int,
@@ -179,6 +181,11 @@ def quant_asym_int4(x, clip):
     z16 = C.c_uint16()
     lib().orc_quant_asym_int4(x, x.size, float(clip), _ptr(pre), codes, C.byref(s16), C.byref(z16))
     return codes, int(s16.value), int(z16.value), pre
+
+
+def asym_unrounded_scale(x, clip) -> float:
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    return lib().orc_asym_unrounded_scale(x, x.size, float(clip))
 
 
 def pack_nibbles(codes) -> np.ndarray:

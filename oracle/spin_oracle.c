@@ -247,6 +247,17 @@ void orc_quant_asym_int4(const double *x, int n, double clip, double *pre, uint8
   *z16 = orc_f64_to_f16(z);
 }
 
+/* The asymmetric step before its rounding to fp16, (hi - lo) / 15 (used to
+ * recognise steps that sit on an fp16 rounding boundary). */
+double orc_asym_unrounded_scale(const double *x, int n, double clip) {
+  double mn = x[0], mx = x[0];
+  for (int j = 1; j < n; j++) {
+    mn = fmin(mn, x[j]);
+    mx = fmax(mx, x[j]);
+  }
+  return (fmax(clip * mx, 0.0) - fmin(clip * mn, 0.0)) / 15.0;
+}
+
 /* Two codes per byte: element 2j in the low nibble, element 2j+1 in the high
  * nibble, each as a 4-bit two's-complement (signed) or plain (unsigned) field. */
 void orc_pack_nibbles(const int32_t *codes, int n, uint8_t *packed) {

@@ -18,3 +18,16 @@ def orc():
     import oracle
     oracle.lib()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def spin_gpu():
+    """The CUDA library on a B200. Fails (does not skip) when CUDA is absent, so
+    a GPU run can never pass on a fallback."""
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from online_hadamard_rotation_b200 import build
+    build.build()
+    import online_hadamard_rotation_b200 as spin
+    spin.lib()
+    return spin

@@ -1,0 +1,109 @@
+"""C ABI checks that need no GPU: the library builds and loads, exports every
+function include/spin.h declares, and rejects bad arguments on the host before
+touching the device."""
+import ctypes as C
+import subprocess
+
+import pytest
+
+import online_hadamard_rotation_b200 as spin
+
+
+@pytest.fixture(scope="module")
+def L():
+    from online_hadamard_rotation_b200 import build
+    build.build()
+    return spin.lib()
+
+
+def test_header_declares_the_entry_points():
+    names = spin.exported_symbols()
+    for fn in ("spin_hadamard_quant_int4", "spin_hadamard_quant_int4_ex", "spin_rope_hadamard_kvquant",
+               "spin_dequant_hadamard_inverse", "spin_status_string", "spin_last_cuda_error", "spin_version"):
+        assert fn in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", spin.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    defined = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for fn in spin.exported_symbols():
+        assert fn in defined, fn
+        assert getattr(L, fn) is not None
+
+
+def test_status_strings_and_version(L):
+    assert L.spin_status_string(0) == b"SPIN_OK"
+    assert L.spin_status_string(2) == b"SPIN_ERR_UNSUPPORTED_SIZE"
+    assert L.spin_version() == 100
+    assert L.spin_last_cuda_error() == 0
+
+
+FAKE = 0x10000  # a 16-byte-aligned address that is never dereferenced by these calls
+
+
+@pytest.mark.parametrize("n", [0, 64, 100, 129, 65536, -128])
+def test_r4_rejects_sizes(L, n):
+    assert L.spin_hadamard_quant_int4(FAKE, 4, n, 1.0, FAKE, FAKE, None) == 2
+
+
+@pytest.mark.parametrize("clip", [0.0, -0.5, 1.5, float("nan")])
+def test_r4_rejects_clip(L, clip):
+    assert L.spin_hadamard_quant_int4(FAKE, 4, 256, clip, FAKE, FAKE, None) == 1
+
+
+def test_r4_argument_checks(L):
+    assert L.spin_hadamard_quant_int4(FAKE, -1, 256, 1.0, FAKE, FAKE, None) == 1
+    assert L.spin_hadamard_quant_int4(None, 0, 256, 1.0, None, None, None) == 0  # empty: no-op
+    assert L.spin_hadamard_quant_int4(None, 4, 256, 1.0, FAKE, FAKE, None) == 1
+    assert L.spin_hadamard_quant_int4(FAKE + 2, 4, 256, 1.0, FAKE, FAKE, None) == 3
+    assert L.spin_hadamard_quant_int4(FAKE, 4, 256, 1.0, FAKE + 8, FAKE, None) == 3
+    assert L.spin_hadamard_quant_int4(FAKE, 4, 256, 1.0, FAKE, FAKE + 1, None) == 3
+    assert L.spin_hadamard_quant_int4_ex(FAKE, 4, 256, 1.0, FAKE + 2, 0, FAKE, FAKE, None) == 3
+    assert L.spin_hadamard_quant_int4_ex(FAKE, 4, 256, 1.0, None, 2, FAKE, FAKE, None) == 1
+
+
+def _r3(L, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, pos=FAKE, theta=1e4, head_dim=128, batch=2, seq=8, hq=32, hkv=8, clip=0.95,
+             q_out=FAKE, kc=FAKE, vc=FAKE, ks=FAKE, kz=FAKE, vs=FAKE, vz=FAKE, cache_len=16, cache_offset=0)
+    a.update(kw)
+    return L.spin_rope_hadamard_kvquant(a["q"], a["k"], a["v"], a["pos"], a["theta"], a["head_dim"], a["batch"],
+                                        a["seq"], a["hq"], a["hkv"], a["clip"], a["q_out"], a["kc"], a["vc"],
+                                        a["ks"], a["kz"], a["vs"], a["vz"], a["cache_len"], a["cache_offset"],
+                                        None)
+
+
+def test_r3_argument_checks(L):
+    assert _r3(L, head_dim=64) == 2
+    assert _r3(L, head_dim=96) == 2
+    assert _r3(L, hq=30) == 1  # not a multiple of hkv
+    assert _r3(L, cache_len=7) == 1
+    assert _r3(L, cache_offset=-1) == 1
+    assert _r3(L, theta=0.0) == 1
+    assert _r3(L, clip=0.0) == 1
+    assert _r3(L, batch=0, q=None) == 0
+    assert _r3(L, seq=0) == 0
+    assert _r3(L, v=None) == 1
+    assert _r3(L, q_out=FAKE + 4) == 3
+    assert _r3(L, ks=FAKE + 1) == 3
+    assert _r3(L, hq=400, hkv=40) == 2
+
+
+def test_dequant_argument_checks(L):
+    f = L.spin_dequant_hadamard_inverse
+    assert f(FAKE, 4, 200, 0, FAKE, None, None, 0, FAKE, 0, None) == 2
+    assert f(FAKE, 4, 256, 2, FAKE, None, None, 0, FAKE, 0, None) == 1
+    assert f(FAKE, 4, 256, 0, FAKE, None, None, 0, FAKE, 3, None) == 1
+    assert f(FAKE, 4, 256, 1, FAKE, None, None, 0, FAKE, 0, None) == 1  # asym needs zero
+    assert f(FAKE, -1, 256, 0, FAKE, None, None, 0, FAKE, 0, None) == 1
+    assert f(None, 0, 256, 0, None, None, None, 0, None, 0, None) == 0
+    assert f(FAKE + 8, 4, 256, 0, FAKE, None, None, 0, FAKE, 0, None) == 3
+    assert f(FAKE, 4, 256, 0, FAKE + 2, None, None, 0, FAKE, 0, None) == 3
+    assert f(FAKE, 4, 256, 1, FAKE + 2, FAKE + 1, None, 0, FAKE, 0, None) == 3
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(spin, "_lib", None)
+    monkeypatch.setattr(spin, "LIB_PATH", str(tmp_path / "libspin.so"))
+    with pytest.raises(ImportError):
+        spin.lib()
