@@ -253,9 +253,10 @@ def main():
         signs = (torch.from_numpy(wl["signs"].view(np.int32)).to(dev) if wl["signs"] is not None else None)
         step_bytes = algorithmic_bytes_r4(tokens, n)
 
-        def step(i):
+        def step(i, cores_only=False):
             b = sets[i & 1]
-            spin.hadamard_quant_int4(b["x"], wl["clip"], signs, out=b["q"], scales=b["s"], stream=stream)
+            spin.hadamard_quant_int4(b["x"], wl["clip"], signs, out=b["q"], scales=b["s"], stream=stream,
+                                     cuda_cores_only=cores_only)
     else:
         q, k, v, pos = wl["q"], wl["k"], wl["v"], wl["pos"]
         B, S, hq, d = q.shape
@@ -271,7 +272,7 @@ def main():
                              cache=spin.alloc_kv_cache(B, hkv, S, d, device=dev)))
         step_bytes = r3_bytes(tokens, hq, hkv, d)
 
-        def step(i):
+        def step(i, cores_only=False):
             b = sets[i & 1]
             spin.rope_hadamard_kvquant(b["q"], b["k"], b["v"], b["pos"], b["cache"], clip=wl["clip"], q_out=b["qo"],
                                        stream=stream)
@@ -338,8 +339,26 @@ def main():
                "h2d_bytes_per_step": int(host.numel() * 2), "d2h_bytes_per_step": int(q_host.numel() + 4 * tokens),
                "steps": e2e_steps}
 
+    # ---- the same steps on the all-CUDA-core kernel, for comparison (not the headline)
+    cores = None
+    if wl["kind"] == "r4" and n == 16384:
+        for i in range(args.warmup):
+            step(i, True)
+        stream.synchronize()
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i, True)
+        ev1.record(stream)
+        ev1.synchronize()
+        cms = ev0.elapsed_time(ev1) / args.steps
+        cores = {"kernel": "k1_rotate_quant_int4 (all butterflies on CUDA cores)", "ms_per_step": cms,
+                 "achieved_gbs": step_bytes / (cms / 1e3) / 1e9}
+
     peak, peak_kind = measured_peaks()
-    kname = "k1_rotate_quant_int4" if wl["kind"] == "r4" else "k2_rope_hadamard_kvquant"
+    if wl["kind"] == "r4":
+        kname = "k1_tc_rotate_quant_16384" if n == 16384 else "k1_rotate_quant_int4"
+    else:
+        kname = "k2_rope_hadamard_kvquant"
     traffic = recorded_traffic(f"{kname}:{args.workload}")
     per_gpu_gbs = step_bytes / (ms_per_step / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": per_gpu_gbs, "peak": peak, "unit": "GB/s",
@@ -369,6 +388,7 @@ def main():
                                l2="inputs larger than L2 (268 MB bf16 input vs 126 MB L2); two buffer sets alternate"
                                if args.workload == "r4_prefill" else "two buffer sets alternate"),
                 "gpu_launches": args.steps, "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu,
+                "cuda_core_kernel": cores,
                 "clocks": clocks.summary()}
         print(json.dumps(line), flush=True)
     if world > 1:

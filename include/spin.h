@@ -63,7 +63,8 @@ typedef enum spin_status_t {
 } spin_status_t;
 
 /* flags */
-#define SPIN_NO_ROTATE 1u /* skip the diagonal and the transform (direct quantisation / identity) */
+#define SPIN_NO_ROTATE 1u       /* skip the diagonal and the transform (direct quantisation / identity) */
+#define SPIN_CUDA_CORES_ONLY 2u /* R4: use the CUDA-core kernel even where the tensor-core kernel applies */
 
 /* spin_dequant_hadamard_inverse modes */
 #define SPIN_SYM_INT4_F32SCALE 0 /* signed codes, fp32 scale per row: value = code * scale */
@@ -107,8 +108,15 @@ spin_status_t spin_hadamard_quant_int4(const void *x_bf16, int64_t tokens, int32
  * (1/sqrt n) H_n diag(+-1)).
  *  sign_bits  nullable; [n/32] uint32 words, bit j of the mask set means
  *             d_j = -1. 4-byte aligned.
- *  flags      0 or SPIN_NO_ROTATE (quantise x directly: no D, no H), used to
- *             measure the direct-quantisation error.
+ *  flags      bitwise OR of
+ *             SPIN_NO_ROTATE: quantise x directly (no D, no H), used to
+ *               measure the direct-quantisation error;
+ *             SPIN_CUDA_CORES_ONLY: at n = 16384 the first H_128 Kronecker
+ *               factor normally runs on the tensor cores (exact +-1 x bf16
+ *               products, fp32 accumulation); this bit selects the kernel that
+ *               runs every butterfly on the CUDA cores instead. Both give the
+ *               same codes up to the rounding-tie band and the same steps to
+ *               fp32 accumulation order.
  * spin_hadamard_quant_int4(...) == spin_hadamard_quant_int4_ex(..., NULL, 0, ...).
  */
 spin_status_t spin_hadamard_quant_int4_ex(const void *x_bf16, int64_t tokens, int32_t n,
@@ -181,6 +189,16 @@ spin_status_t spin_dequant_hadamard_inverse(const uint8_t *codes, int64_t rows, 
                                             int32_t mode, const void *scale, const void *zero,
                                             const uint32_t *sign_bits, uint32_t flags, void *out,
                                             int32_t out_dtype, spin_stream_t stream);
+
+/*
+ * Device status word of the current device: nonzero once a kernel of this
+ * library gave up on an internal wait (a pipeline barrier that did not
+ * complete within about two seconds); that kernel then stopped early and its
+ * outputs are incomplete. Copies the word to *status and, if reset != 0,
+ * clears it. Synchronous: it waits for work on the legacy default stream.
+ * Errors: SPIN_ERR_INVALID_ARG (status NULL), SPIN_ERR_CUDA.
+ */
+spin_status_t spin_device_status(uint32_t *status, int reset);
 
 /* Human-readable name of a status code (static storage). */
 const char *spin_status_string(spin_status_t status);

@@ -74,7 +74,11 @@ cudaError_t resident_slots(const void *kernel, int threads, int dyn_smem, int *s
   if (!opted_in[std::make_pair(kernel, dev)]) {
     int optin = 0;
     if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin)) != cudaSuccess)
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess) return e;
+    const int dyn_max = optin - (int)fa.sharedSizeBytes;  // static + dynamic must fit the opt-in limit
+    if (dyn_smem > dyn_max) return cudaErrorInvalidConfiguration;
+    if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max)) != cudaSuccess)
       return e;
     opted_in[std::make_pair(kernel, dev)] = true;
   }
@@ -100,7 +104,8 @@ spin_status_t spin_hadamard_quant_int4_ex(const void *x_bf16, int64_t tokens, in
                                           spin_stream_t stream) {
   const int log_n = log2_pow2(n);
   if (log_n < 7 || log_n > 15) return SPIN_ERR_UNSUPPORTED_SIZE;
-  if (tokens < 0 || !valid_clip(clip) || (flags & ~SPIN_NO_ROTATE) != 0) return SPIN_ERR_INVALID_ARG;
+  if (tokens < 0 || !valid_clip(clip) || (flags & ~(SPIN_NO_ROTATE | SPIN_CUDA_CORES_ONLY)) != 0)
+    return SPIN_ERR_INVALID_ARG;
   if (tokens == 0) return SPIN_OK;
   if (!x_bf16 || !q_packed_u8 || !scales_f32) return SPIN_ERR_INVALID_ARG;
   if (tokens > (INT64_MAX >> 16)) return SPIN_ERR_INVALID_ARG;
@@ -179,6 +184,14 @@ const char *spin_status_string(spin_status_t status) {
 }
 
 int spin_last_cuda_error(void) { return g_last_cuda_error; }
+
+spin_status_t spin_device_status(uint32_t *status, int reset) {
+  if (!status) return SPIN_ERR_INVALID_ARG;
+  unsigned int v = 0;
+  spin_status_t st = cuda_status(read_device_status(&v, reset != 0));
+  *status = v;
+  return st;
+}
 
 int spin_version(void) { return 100; }
 

@@ -1,0 +1,374 @@
+// k1_tc.cu -- R4 at n = 16384 with the first Kronecker factor on the tensor
+// cores.
+//
+// "Rotations: QuaRot, SpinQuant and incoherence", section "Hadamard matrices":
+// H_16384 = H_128 (x) H_128 (Kronecker product of Sylvester matrices), and the
+// randomised transform (1/sqrt n) H_n diag(+-1). "SpinQuant, when rotations are
+// worth learning", section "Four rotation sites": R4 is the fixed Hadamard on
+// the down-projection input. "SpinQuant Guide", section "The Outlier Curse":
+// symmetric INT4, step max|y| / 7.
+//
+// A token row x (16384 bf16) is the 128 x 128 matrix X[a][b] with element
+// index e = 128 a + b. Then H_16384 x = vec(H_128 X H_128):
+//   1. tcgen05.mma computes Y = H_128 X (contraction over a) for two tokens at
+//      once (M = 128, N = 256, K = 128, bf16 in, fp32 accumulate in TMEM). H is
+//      exactly +-1 and X is exactly bf16, so every product is exact and only the
+//      fp32 accumulation rounds.
+//   2. Each epilogue thread owns one row a' of Y (one TMEM lane), loads its 128
+//      values and runs the seven butterfly stages of the second factor (over b)
+//      in registers, then the per-token max, the step, the INT4 codes and the
+//      nibble packing; the 64 bytes of row a' are contiguous in the output.
+//
+// Roles (384 threads, one CTA per SM, persistent over token pairs):
+//   warp 0      TMA producer: four 16 KiB tiles (two tokens x two 64-column
+//               halves, 128-byte swizzle) per pair into a two-stage ring
+//   warp 1      TMEM owner and MMA issuer (8 MMAs of K = 16 per pair)
+//   warps 2-3   +-1 diagonal: XOR of the bf16 sign bits in shared memory
+//   warps 4-7   epilogue for the first token of each pair (TMEM columns 0-127)
+//   warps 8-11  epilogue for the second token (columns 128-255)
+// TMEM holds two 256-column accumulators, so the MMA of pair i + 1 overlaps the
+// epilogue of pair i. Every mbarrier wait is bounded by a clock budget; on
+// expiry the CTA records a status, drains its copies and MMAs, frees TMEM and
+// returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "spin_launch.h"
+#include "spin_tile.cuh"
+#include "tc_ptx.cuh"
+
+namespace spin {
+
+// Nonzero once a tensor-core kernel gave up on a wait (see spin_device_status).
+__device__ unsigned int g_device_status = 0u;
+
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kStages = 2;
+constexpr uint32_t kTileBytes = 16384;              // [128 rows][64 bf16]
+constexpr uint32_t kPairBytes = 4 * kTileBytes;     // two tokens
+constexpr uint32_t kOffH = 0;                       // A operand: H_128, K-major, 2 x 16 KiB
+constexpr uint32_t kOffX = 32768;                   // ring of kStages x 64 KiB
+constexpr uint32_t kOffMask = kOffX + kStages * kPairBytes;  // sign pattern of one token, 32 KiB
+constexpr uint32_t kOffOut = kOffMask + 32768;      // two 8 KiB output staging buffers
+constexpr uint32_t kOffBar = kOffOut + 2 * 8192;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
+constexpr long long kTimeoutCycles = 4000000000LL;     // about two seconds
+
+struct Shared {
+  uint64_t full[kStages], sgn[kStages], empty[kStages], tfull[2], tempty[2], drain;
+  uint32_t tmem_base;
+  int abort;
+  int dec[3];
+  float wmax[2][4];
+};
+
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, Shared &S, bool honor_abort) {
+  if (tc::mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    if (honor_abort && *reinterpret_cast<volatile int *>(&S.abort)) return false;
+    if (clock64() - t0 > kTimeoutCycles) {
+      *reinterpret_cast<volatile int *>(&S.abort) = 1;
+      atomicOr(&g_device_status, 1u);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack8(const uint32_t (&b)[8]) {
+  const uint32_t e = __byte_perm(__byte_perm(b[0], b[2], 0x0040), __byte_perm(b[4], b[6], 0x0040), 0x5410);
+  const uint32_t o = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
+  return (e | (o << 4)) ^ 0x88888888u;
+}
+
+// byte offset of 16-byte chunk `ch` (0..7) of row `r` in a 128-byte-swizzled [rows][128 B] tile
+__device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t ch) { return r * 128u + ((ch ^ (r & 7u)) << 4); }
+
+template <bool SIGNS>
+__global__ void __launch_bounds__(kThreads, 1)
+    k1_tc_rotate_quant_16384(const __grid_constant__ CUtensorMap xmap, int64_t tokens, float clip,
+                             float inv_sqrt_n, const uint32_t *__restrict__ signs, uint8_t *__restrict__ q,
+                             float *__restrict__ scales) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Shared &S = *reinterpret_cast<Shared *>(smem + kOffBar);
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
+  const int64_t npairs = (tokens + 1) >> 1;
+
+  // ------------------------------------------------------------ setup
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&S.full[s], 1);
+      tc::mbar_init(&S.sgn[s], 1);
+      tc::mbar_init(&S.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(&S.tfull[a], 1);
+      tc::mbar_init(&S.tempty[a], 256);
+    }
+    tc::mbar_init(&S.drain, 1);
+    S.abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (threadIdx.x == 32) tc::prefetch_tensormap(&xmap);
+  // H_128 as the A operand: K-major, two K blocks of [128 rows m][64 k], 128-byte swizzle.
+  for (uint32_t c = threadIdx.x; c < 2048; c += kThreads) {
+    const uint32_t kb = c >> 10, m = (c >> 3) & 127u, ch = c & 7u;
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t k0 = kb * 64 + ch * 8 + 2 * j;
+      const uint32_t lo = (__popc(m & k0) & 1) ? 0xBF80u : 0x3F80u;
+      const uint32_t hi = (__popc(m & (k0 + 1)) & 1) ? 0xBF80u : 0x3F80u;
+      w[j] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4 *>(smem + kOffH + kb * 16384 + sw128(m, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if constexpr (SIGNS) {
+    // sign bits of one token in the swizzled tile layout: [half][128 rows a][8 chunks]
+    for (uint32_t c = threadIdx.x; c < 2048; c += kThreads) {
+      const uint32_t h = c >> 10, a = (c >> 3) & 127u, ch = c & 7u;
+      const uint32_t e = a * 128u + h * 64u + ch * 8u;
+      const uint32_t byte = (__ldg(signs + (e >> 5)) >> (e & 31u)) & 0xFFu;
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) w[j] = (((byte >> (2 * j)) & 1u) << 15) | (((byte >> (2 * j + 1)) & 1u) << 31);
+      *reinterpret_cast<uint4 *>(smem + kOffMask + h * kTileBytes + sw128(a, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  tc::fence_proxy_async_smem();
+  if (warp == 1) {
+    tc::tmem_alloc(&S.tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  // ------------------------------------------------------------ roles
+  if (warp == 0) {
+    if (lane == 0) {
+      int64_t last[kStages] = {-1, -1};
+      for (int64_t i = 0;; ++i) {
+        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+        if (p >= npairs) break;
+        const int st = (int)(i & 1);
+        if (!wait_bounded(&S.empty[st], (uint32_t)((i >> 1) & 1) ^ 1u, S, true)) break;
+        const int nvalid = (2 * p + 1 < tokens) ? 2 : 1;
+        tc::mbar_arrive_expect_tx(&S.full[st], (uint32_t)nvalid * 2u * kTileBytes);
+        uint8_t *dst = smem + kOffX + st * kPairBytes;
+        for (int j = 0; j < 2 * nvalid; ++j)
+          tc::tma_load_2d(dst + j * kTileBytes, &xmap, &S.full[st], (j & 1) * 64, (int)((2 * p + (j >> 1)) * 128));
+        last[st] = i;
+      }
+      // every issued copy has landed before the CTA can leave
+      for (int s = 0; s < kStages; ++s)
+        if (last[s] >= 0) wait_bounded(&S.full[s], (uint32_t)((last[s] >> 1) & 1), S, false);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16(128, 256, true);
+      const uint32_t sH = tc::smem_u32(smem + kOffH), sX = tc::smem_u32(smem + kOffX);
+      for (int64_t i = 0;; ++i) {
+        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+        if (p >= npairs) break;
+        const int st = (int)(i & 1), acc = (int)(i & 1);
+        if (!wait_bounded(SIGNS ? &S.sgn[st] : &S.full[st], (uint32_t)((i >> 1) & 1), S, true)) break;
+        if (!wait_bounded(&S.tempty[acc], (uint32_t)((i >> 1) & 1) ^ 1u, S, true)) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
+          const uint64_t bd = tc::smem_desc(sX + st * kPairBytes + s * 2048, kTileBytes, 1024);
+          tc::umma_bf16(tmem + acc * 256, ad, bd, idesc, s > 0 ? 1u : 0u);
+        }
+        tc::umma_commit(&S.empty[st]);
+        tc::umma_commit(&S.tfull[acc]);
+      }
+    }
+  } else if (warp < 4) {
+    if constexpr (SIGNS) {
+      const uint32_t ts = threadIdx.x - 64;  // 0..63
+      for (int64_t i = 0;; ++i) {
+        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+        if (p >= npairs) break;
+        const int st = (int)(i & 1);
+        if (ts == 0) S.dec[2] = wait_bounded(&S.full[st], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+        tc::named_sync(3, 64);
+        if (!S.dec[2]) break;
+        uint4 *X = reinterpret_cast<uint4 *>(smem + kOffX + st * kPairBytes);
+        const uint4 *M = reinterpret_cast<const uint4 *>(smem + kOffMask);
+#pragma unroll 4
+        for (uint32_t c = ts; c < kPairBytes / 16; c += 64) {
+          uint4 x = X[c];
+          const uint4 m = M[c & 2047u];
+          x.x ^= m.x;
+          x.y ^= m.y;
+          x.z ^= m.z;
+          x.w ^= m.w;
+          X[c] = x;
+        }
+        tc::fence_proxy_async_smem();
+        tc::named_sync(3, 64);
+        if (ts == 0) tc::mbar_arrive(&S.sgn[st]);
+      }
+    }
+  } else {
+    // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1)
+    const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
+    const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
+    uint8_t *stg = smem + kOffOut + g * 8192;
+    for (int64_t i = 0;; ++i) {
+      const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+      if (p >= npairs) break;
+      const int acc = (int)(i & 1);
+      if (tg == 0) S.dec[g] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+      tc::named_sync(1 + g, 128);
+      if (!S.dec[g]) break;
+      tc::tc_fence_after();
+      float v[kRegs];
+      {
+        uint32_t r[kRegs];
+        const uint32_t taddr = tmem + ((wq * 32u) << 16) + (uint32_t)acc * 256u + g * 128u;
+        tc::tmem_ld32(taddr, r);
+        tc::tmem_ld32(taddr + 32, r + 32);
+        tc::tmem_ld32(taddr + 64, r + 64);
+        tc::tmem_ld32(taddr + 96, r + 96);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < kRegs; ++k) v[k] = __uint_as_float(r[k]);
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&S.tempty[acc]);
+      // second Kronecker factor: H_128 over b, in registers
+      stage<0>(v);
+      stage<1>(v);
+      stage<2>(v);
+      stage<3>(v);
+      stage<4>(v);
+      stage<5>(v);
+      stage<6>(v);
+      float m = 0.f;
+#pragma unroll
+      for (int k = 0; k < kRegs; ++k) m = fmaxf(m, fabsf(v[k]));
+      const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
+      if (lane == 0) S.wmax[g][wq] = __uint_as_float(wm);
+      if (tg == 0) tc::bulk_wait_read0();  // the previous store has finished reading the staging buffer
+      tc::named_sync(1 + g, 128);
+      const float mu = fmaxf(fmaxf(S.wmax[g][0], S.wmax[g][1]), fmaxf(S.wmax[g][2], S.wmax[g][3]));
+      const float s = fmaxf(clip * (mu * inv_sqrt_n) / 7.0f, 1e-8f);
+      const float c15 = (inv_sqrt_n / s) / 15.0f;
+      constexpr float k815 = 8.0f / 15.0f;
+      constexpr float kMagic = 12582912.0f;
+#pragma unroll
+      for (int w4 = 0; w4 < 4; ++w4) {
+        uint32_t words[4];
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+          uint32_t b[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            b[k] = __float_as_uint(fmaf(fma_sat(v[32 * w4 + 8 * wi + k], c15, k815), 15.0f, kMagic));
+          words[wi] = pack8(b);
+        }
+        *reinterpret_cast<uint4 *>(stg + row * 64 + w4 * 16) = make_uint4(words[0], words[1], words[2], words[3]);
+      }
+      tc::fence_proxy_async_smem();
+      tc::named_sync(1 + g, 128);
+      const int64_t token = 2 * p + g;
+      if (tg == 0 && token < tokens) {
+        tc::bulk_store(q + token * 8192, stg, 8192);
+        tc::bulk_commit();
+        scales[token] = s;
+      }
+    }
+    if (tg == 0) tc::bulk_wait0();
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0) {
+      tc::umma_commit(&S.drain);  // arrives once every MMA this thread issued is complete
+      wait_bounded(&S.drain, 0, S, false);
+    }
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+template <bool SIGNS>
+cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
+                      cudaStream_t stream) {
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {128, (cuuint64_t)tokens * 128};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  auto kern = k1_tc_rotate_quant_16384<SIGNS>;
+  int slots = 0;
+  cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreads, (int)kSmemBytes, &slots);
+  if (err != cudaSuccess) return err;
+  const int64_t npairs = (tokens + 1) / 2;
+  const int64_t grid = npairs < slots ? npairs : slots;
+  const float inv_sqrt_n = (float)(1.0 / 128.0);
+  kern<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(map, tokens, clip, inv_sqrt_n, signs, q, scales);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags) {
+  return log_n == 14 && !(flags & kNoRotate) && tokens > 0 && tokens * 128 < (int64_t(1) << 31);
+}
+
+cudaError_t launch_rotate_quant_int4_tc(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q,
+                                        float *scales, cudaStream_t stream) {
+  if (signs) return launch_tc<true>(x, tokens, clip, signs, q, scales, stream);
+  return launch_tc<false>(x, tokens, clip, nullptr, q, scales, stream);
+}
+
+cudaError_t read_device_status(unsigned int *status, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(status, g_device_status, sizeof(unsigned int));
+  if (e != cudaSuccess || !reset) return e;
+  const unsigned int zero = 0u;
+  return cudaMemcpyToSymbol(g_device_status, &zero, sizeof(unsigned int));
+}
+
+}  // namespace spin

@@ -7,7 +7,8 @@
 
 namespace spin {
 
-constexpr uint32_t kNoRotate = 1u;  // same value as SPIN_NO_ROTATE
+constexpr uint32_t kNoRotate = 1u;        // same value as SPIN_NO_ROTATE
+constexpr uint32_t kCudaCoresOnly = 2u;   // same value as SPIN_CUDA_CORES_ONLY
 
 // Number of blocks of `kernel` that are resident on the current device at once
 // (SM count x blocks per SM), with the dynamic shared-memory opt-in applied.
@@ -17,6 +18,14 @@ cudaError_t resident_slots(const void *kernel, int threads, int dyn_smem, int *s
 cudaError_t launch_rotate_quant_int4(const void *x, int64_t tokens, int log_n, float clip,
                                      const uint32_t *signs, uint32_t flags, uint8_t *q, float *scales,
                                      cudaStream_t stream);
+
+// Tensor-core R4 kernel (n = 16384): availability and launcher.
+bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags);
+cudaError_t launch_rotate_quant_int4_tc(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q,
+                                        float *scales, cudaStream_t stream);
+
+// Device status word set by kernels whose bounded waits ran out.
+cudaError_t read_device_status(unsigned int *status, bool reset);
 
 cudaError_t launch_dequant_inverse(const uint8_t *codes, int64_t rows, int log_n, int mode,
                                    const void *scale, const void *zero, const uint32_t *signs,

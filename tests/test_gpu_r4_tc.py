@@ -1,0 +1,77 @@
+"""The tensor-core R4 kernel (n = 16384: first H_128 Kronecker factor on
+tcgen05, second on CUDA cores) vs the fp64 oracle, and vs the all-CUDA-core
+kernel selected with SPIN_CUDA_CORES_ONLY."""
+import numpy as np
+import pytest
+import torch
+
+import synthetic
+from tests import parity
+from tests.gpu_util import to_dev_bf16, to_dev_signs
+
+pytestmark = pytest.mark.gpu
+
+N = 16384
+
+
+def run(spin, bits, clip, signs, cores_only=False):
+    q, s = spin.hadamard_quant_int4(to_dev_bf16(bits), clip, to_dev_signs(signs), cuda_cores_only=cores_only)
+    torch.cuda.synchronize()
+    return q.cpu().numpy(), s.cpu().numpy()
+
+
+@pytest.mark.parametrize("tokens", [1, 2, 3, 16, 149, 300])
+@pytest.mark.parametrize("clip,with_signs", [(1.0, False), (0.9, True)])
+def test_tc_vs_oracle(spin_gpu, orc, tokens, clip, with_signs):
+    bits = synthetic.r4_prefill(tokens=tokens, seed=50 + tokens)[0]
+    signs = synthetic.sign_bits(N, 101) if with_signs else None
+    q, s = run(spin_gpu, bits, clip, signs)
+    codes = parity.unpack_signed(q, N)
+    for t in range(tokens):
+        r = orc.r4_row(bits[t], clip, signs=signs)
+        parity.check_rel([s[t]], [r["scale64"]], 1e-5, f"scale row {t}")
+        parity.check_codes(codes[t], r["codes"], r["pre"], f"codes row {t}")
+    assert spin_gpu.device_status() == 0
+
+
+def test_tc_matches_cuda_core_kernel(spin_gpu, orc):
+    bits, signs, _ = synthetic.r4_prefill(tokens=512, seed=9)
+    q1, s1 = run(spin_gpu, bits, 0.9, signs)
+    q2, s2 = run(spin_gpu, bits, 0.9, signs, cores_only=True)
+    parity.check_rel(s1, s2, 1e-5, "tc vs cuda-core scales")
+    c1, c2 = parity.unpack_signed(q1, N), parity.unpack_signed(q2, N)
+    diff = np.nonzero((c1 != c2).any(axis=1))[0]
+    for t in diff[:16]:  # any difference must be a rounding tie of the exact value
+        r = orc.r4_row(bits[t], 0.9, signs=signs)
+        parity.check_codes(c1[t], r["codes"], r["pre"], f"tc row {t}")
+        parity.check_codes(c2[t], r["codes"], r["pre"], f"cuda-core row {t}")
+    assert (c1 != c2).mean() < 1e-4
+
+
+def test_tc_special_rows(spin_gpu, orc):
+    rows = [np.zeros(N, np.float32), np.full(N, 1.0, np.float32)]
+    for j in (0, 1, 127, 128, 8191, N - 1):
+        r = np.zeros(N, np.float32)
+        r[j] = 60.0
+        rows.append(r)
+    rows.append(np.where(np.arange(N) % 3 == 0, 3.0e4, -2.0e4).astype(np.float32))
+    bits = synthetic.to_bf16_bits(np.stack(rows))
+    q, s = run(spin_gpu, bits, 1.0, None)
+    codes = parity.unpack_signed(q, N)
+    for t in range(len(rows)):
+        r = orc.r4_row(bits[t], 1.0)
+        parity.check_rel([s[t]], [r["scale64"]], 1e-5, f"scale row {t}")
+        parity.check_codes(codes[t], r["codes"], r["pre"], f"codes row {t}")
+    assert np.all(codes[0] == 0) and s[0] == np.float32(1e-8)
+    for t in range(2, 8):
+        assert np.all(np.abs(codes[t]) == 7)
+
+
+def test_tc_leaves_tail_untouched(spin_gpu):
+    bits = synthetic.r4_prefill(tokens=5, seed=3)[0]
+    out = torch.full((8, N // 2), 0xA5, dtype=torch.uint8, device="cuda")
+    sc = torch.full((8,), -1.0, dtype=torch.float32, device="cuda")
+    spin_gpu.hadamard_quant_int4(to_dev_bf16(bits), 1.0, out=out[:5], scales=sc[:5])
+    torch.cuda.synchronize()
+    assert torch.all(out[5:] == 0xA5) and torch.all(sc[5:] == -1.0)
+    assert torch.all(sc[:5] > 0)
