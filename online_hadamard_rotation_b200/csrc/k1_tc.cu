@@ -21,13 +21,15 @@
 //
 // Roles (384 threads, one CTA per SM, persistent over token pairs):
 //   warp 0      TMA producer: four 16 KiB tiles (two tokens x two 64-column
-//               halves, 128-byte swizzle) per pair into a two-stage ring
+//               halves, 128-byte swizzle) per pair into a three-stage ring
 //   warp 1      TMEM owner and MMA issuer (8 MMAs of K = 16 per pair)
-//   warps 2-3   +-1 diagonal: XOR of the bf16 sign bits in shared memory
+//   warps 2-3   +-1 diagonal: XOR of the bf16 sign bits in shared memory, with
+//               each thread's sign words held in registers
 //   warps 4-7   epilogue for the first token of each pair (TMEM columns 0-127)
 //   warps 8-11  epilogue for the second token (columns 128-255)
 // TMEM holds two 256-column accumulators, so the MMA of pair i + 1 overlaps the
-// epilogue of pair i. Every mbarrier wait is bounded by a clock budget; on
+// epilogue of pair i. Each epilogue thread writes its 64 code bytes straight
+// to global memory (four 16-byte streaming stores). Every mbarrier wait is bounded by a clock budget; on
 // expiry the CTA records a status, drains its copies and MMAs, frees TMEM and
 // returns.
 #include <cuda.h>
@@ -50,14 +52,12 @@ __device__ unsigned int g_device_status = 0u;
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr uint32_t kTileBytes = 16384;              // [128 rows][64 bf16]
 constexpr uint32_t kPairBytes = 4 * kTileBytes;     // two tokens
 constexpr uint32_t kOffH = 0;                       // A operand: H_128, K-major, 2 x 16 KiB
 constexpr uint32_t kOffX = 32768;                   // ring of kStages x 64 KiB
-constexpr uint32_t kOffMask = kOffX + kStages * kPairBytes;  // sign pattern of one token, 32 KiB
-constexpr uint32_t kOffOut = kOffMask + 32768;      // two 8 KiB output staging buffers
-constexpr uint32_t kOffBar = kOffOut + 2 * 8192;
+constexpr uint32_t kOffBar = kOffX + kStages * kPairBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
 constexpr long long kTimeoutCycles = 4000000000LL;     // about two seconds
 
@@ -66,7 +66,7 @@ struct Shared {
   uint32_t tmem_base;
   int abort;
   int dec[3];
-  float wmax[2][4];
+  float wmax[2][2][4];  // [warpgroup][pair parity][warp]
 };
 
 __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, Shared &S, bool honor_abort) {
@@ -86,6 +86,12 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, Sha
 __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   float r;
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
 
@@ -138,18 +144,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     *reinterpret_cast<uint4 *>(smem + kOffH + kb * 16384 + sw128(m, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  if constexpr (SIGNS) {
-    // sign bits of one token in the swizzled tile layout: [half][128 rows a][8 chunks]
-    for (uint32_t c = threadIdx.x; c < 2048; c += kThreads) {
-      const uint32_t h = c >> 10, a = (c >> 3) & 127u, ch = c & 7u;
-      const uint32_t e = a * 128u + h * 64u + ch * 8u;
-      const uint32_t byte = (__ldg(signs + (e >> 5)) >> (e & 31u)) & 0xFFu;
-      uint32_t w[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) w[j] = (((byte >> (2 * j)) & 1u) << 15) | (((byte >> (2 * j + 1)) & 1u) << 31);
-      *reinterpret_cast<uint4 *>(smem + kOffMask + h * kTileBytes + sw128(a, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  }
   tc::fence_proxy_async_smem();
   if (warp == 1) {
     tc::tmem_alloc(&S.tmem_base, 512);
@@ -163,12 +157,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------ roles
   if (warp == 0) {
     if (lane == 0) {
-      int64_t last[kStages] = {-1, -1};
+      int64_t last[kStages] = {-1, -1, -1};
       for (int64_t i = 0;; ++i) {
         const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
         if (p >= npairs) break;
-        const int st = (int)(i & 1);
-        if (!wait_bounded(&S.empty[st], (uint32_t)((i >> 1) & 1) ^ 1u, S, true)) break;
+        const int st = (int)(i % kStages);
+        if (!wait_bounded(&S.empty[st], (uint32_t)((i / kStages) & 1) ^ 1u, S, true)) break;
         const int nvalid = (2 * p + 1 < tokens) ? 2 : 1;
         tc::mbar_arrive_expect_tx(&S.full[st], (uint32_t)nvalid * 2u * kTileBytes);
         uint8_t *dst = smem + kOffX + st * kPairBytes;
@@ -178,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every issued copy has landed before the CTA can leave
       for (int s = 0; s < kStages; ++s)
-        if (last[s] >= 0) wait_bounded(&S.full[s], (uint32_t)((last[s] >> 1) & 1), S, false);
+        if (last[s] >= 0) wait_bounded(&S.full[s], (uint32_t)((last[s] / kStages) & 1), S, false);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -187,8 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t i = 0;; ++i) {
         const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
         if (p >= npairs) break;
-        const int st = (int)(i & 1), acc = (int)(i & 1);
-        if (!wait_bounded(SIGNS ? &S.sgn[st] : &S.full[st], (uint32_t)((i >> 1) & 1), S, true)) break;
+        const int st = (int)(i % kStages), acc = (int)(i & 1);
+        if (!wait_bounded(SIGNS ? &S.sgn[st] : &S.full[st], (uint32_t)((i / kStages) & 1), S, true)) break;
         if (!wait_bounded(&S.tempty[acc], (uint32_t)((i >> 1) & 1) ^ 1u, S, true)) break;
         tc::tc_fence_after();
 #pragma unroll
@@ -203,25 +197,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 4) {
     if constexpr (SIGNS) {
+      // Thread ts flips the signs of chunks ts + 64 j of each pair's 64 KiB.
+      // Those chunks sit at 32 distinct positions of a token tile; their sign
+      // words stay in registers for the whole kernel.
       const uint32_t ts = threadIdx.x - 64;  // 0..63
+      uint4 mk[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const uint32_t pos = ts + 64u * k;  // 16-byte chunk index inside one token's 32 KiB
+        const uint32_t h = pos >> 10, a = (pos >> 3) & 127u, ch = (pos & 7u) ^ (a & 7u);
+        const uint32_t e = a * 128u + h * 64u + ch * 8u;
+        const uint32_t byte = (__ldg(signs + (e >> 5)) >> (e & 31u)) & 0xFFu;
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = (((byte >> (2 * j)) & 1u) << 15) | (((byte >> (2 * j + 1)) & 1u) << 31);
+        mk[k] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
       for (int64_t i = 0;; ++i) {
         const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
         if (p >= npairs) break;
-        const int st = (int)(i & 1);
-        if (ts == 0) S.dec[2] = wait_bounded(&S.full[st], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+        const int st = (int)(i % kStages);
+        if (ts == 0) S.dec[2] = wait_bounded(&S.full[st], (uint32_t)((i / kStages) & 1), S, true) ? 1 : 0;
         tc::named_sync(3, 64);
         if (!S.dec[2]) break;
-        uint4 *X = reinterpret_cast<uint4 *>(smem + kOffX + st * kPairBytes);
-        const uint4 *M = reinterpret_cast<const uint4 *>(smem + kOffMask);
-#pragma unroll 4
-        for (uint32_t c = ts; c < kPairBytes / 16; c += 64) {
-          uint4 x = X[c];
-          const uint4 m = M[c & 2047u];
-          x.x ^= m.x;
-          x.y ^= m.y;
-          x.z ^= m.z;
-          x.w ^= m.w;
-          X[c] = x;
+        uint4 *X = reinterpret_cast<uint4 *>(smem + kOffX + st * kPairBytes) + ts;
+#pragma unroll
+        for (int j0 = 0; j0 < 64; j0 += 4) {
+          uint4 x[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) x[u] = X[64 * (j0 + u)];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint4 m = mk[(j0 + u) & 31];
+            X[64 * (j0 + u)] = make_uint4(x[u].x ^ m.x, x[u].y ^ m.y, x[u].z ^ m.z, x[u].w ^ m.w);
+          }
         }
         tc::fence_proxy_async_smem();
         tc::named_sync(3, 64);
@@ -232,7 +241,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1)
     const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
     const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
-    uint8_t *stg = smem + kOffOut + g * 8192;
     for (int64_t i = 0;; ++i) {
       const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
       if (p >= npairs) break;
@@ -263,41 +271,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       stage<4>(v);
       stage<5>(v);
       stage<6>(v);
-      float m = 0.f;
+      // per-token max |u|: a tree of three-input maxima, then the warp, then the warpgroup
+      float mx[16];
 #pragma unroll
-      for (int k = 0; k < kRegs; ++k) m = fmaxf(m, fabsf(v[k]));
+      for (int k = 0; k < 16; ++k) mx[k] = fmaxf(fabsf(v[8 * k]), fabsf(v[8 * k + 1]));
+#pragma unroll
+      for (int j = 2; j < 8; j += 2)
+#pragma unroll
+        for (int k = 0; k < 16; ++k) mx[k] = fmax3(mx[k], fabsf(v[8 * k + j]), fabsf(v[8 * k + j + 1]));
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], mx[k + 8]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], mx[k + 4]);
+      const float m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
-      if (lane == 0) S.wmax[g][wq] = __uint_as_float(wm);
-      if (tg == 0) tc::bulk_wait_read0();  // the previous store has finished reading the staging buffer
+      if (lane == 0) S.wmax[g][i & 1][wq] = __uint_as_float(wm);
       tc::named_sync(1 + g, 128);
-      const float mu = fmaxf(fmaxf(S.wmax[g][0], S.wmax[g][1]), fmaxf(S.wmax[g][2], S.wmax[g][3]));
+      const float *wmx = S.wmax[g][i & 1];
+      const float mu = fmaxf(fmaxf(wmx[0], wmx[1]), fmaxf(wmx[2], wmx[3]));
       const float s = fmaxf(clip * (mu * inv_sqrt_n) / 7.0f, 1e-8f);
       const float c15 = (inv_sqrt_n / s) / 15.0f;
       constexpr float k815 = 8.0f / 15.0f;
       constexpr float kMagic = 12582912.0f;
-#pragma unroll
-      for (int w4 = 0; w4 < 4; ++w4) {
-        uint32_t words[4];
-#pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
-          uint32_t b[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            b[k] = __float_as_uint(fmaf(fma_sat(v[32 * w4 + 8 * wi + k], c15, k815), 15.0f, kMagic));
-          words[wi] = pack8(b);
-        }
-        *reinterpret_cast<uint4 *>(stg + row * 64 + w4 * 16) = make_uint4(words[0], words[1], words[2], words[3]);
-      }
-      tc::fence_proxy_async_smem();
-      tc::named_sync(1 + g, 128);
       const int64_t token = 2 * p + g;
-      if (tg == 0 && token < tokens) {
-        tc::bulk_store(q + token * 8192, stg, 8192);
-        tc::bulk_commit();
-        scales[token] = s;
+      if (token < tokens) {
+        uint4 *dst = reinterpret_cast<uint4 *>(q + token * 8192 + row * 64);
+#pragma unroll
+        for (int w4 = 0; w4 < 4; ++w4) {
+          uint32_t words[4];
+#pragma unroll
+          for (int wi = 0; wi < 4; ++wi) {
+            uint32_t b[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              b[k] = __float_as_uint(fmaf(fma_sat(v[32 * w4 + 8 * wi + k], c15, k815), 15.0f, kMagic));
+            words[wi] = pack8(b);
+          }
+          __stcs(dst + w4, make_uint4(words[0], words[1], words[2], words[3]));
+        }
+        if (tg == 0) scales[token] = s;
       }
     }
-    if (tg == 0) tc::bulk_wait0();
   }
 
   // ------------------------------------------------------------ teardown
