@@ -27,6 +27,9 @@
 //               each thread's sign words held in registers
 //   warps 4-7   epilogue for the first token of each pair (TMEM columns 0-127)
 //   warps 8-11  epilogue for the second token (columns 128-255)
+// The launch allows programmatic dependent launch: the prologue of a kernel
+// may overlap the tail of the previous one in the stream, and no global memory
+// is read or written before griddepcontrol.wait returns.
 // TMEM holds two 256-column accumulators, so the MMA of pair i + 1 overlaps the
 // epilogue of pair i. Each epilogue thread writes its 64 code bytes straight
 // to global memory (four 16-byte streaming stores). Every mbarrier wait is bounded by a clock budget; on
@@ -89,6 +92,21 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   return r;
 }
 
+// (r0, r1) = bit patterns of fma(a0, 15, 1.5 * 2^23), fma(a1, 15, 1.5 * 2^23): one packed
+// f32x2 FMA rounds two scaled codes to integers (ties to even) in their low mantissa bits.
+__device__ __forceinline__ void round15_x2(float a0, float a1, uint32_t &r0, uint32_t &r1) {
+  uint64_t A, R;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(R) : "l"(A), "l"(0x4170000041700000ull), "l"(0x4B4000004B400000ull));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(R));
+}
+
+__device__ __forceinline__ void st_v8_cs(void *p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -104,7 +122,7 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&b)[8]) {
 // byte offset of 16-byte chunk `ch` (0..7) of row `r` in a 128-byte-swizzled [rows][128 B] tile
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t ch) { return r * 128u + ((ch ^ (r & 7u)) << 4); }
 
-template <bool SIGNS>
+template <bool SIGNS, bool STORE32>
 __global__ void __launch_bounds__(kThreads, 1)
     k1_tc_rotate_quant_16384(const __grid_constant__ CUtensorMap xmap, int64_t tokens, float clip,
                              float inv_sqrt_n, const uint32_t *__restrict__ signs, uint8_t *__restrict__ q,
@@ -116,6 +134,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t npairs = (tokens + 1) >> 1;
 
   // ------------------------------------------------------------ setup
+  // Global memory is touched only after the grids this one depends on have
+  // finished (programmatic dependent launch lets this prologue overlap their tail).
+  tc::grid_dep_wait();
+  int64_t first_issued = 0;  // loads the producer issues before the setup barrier
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&S.full[s], 1);
@@ -129,8 +151,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&S.drain, 1);
     S.abort = 0;
     tc::fence_barrier_init();
+    tc::prefetch_tensormap(&xmap);
+    // The first kStages pairs need no free slot: start their copies now, so the
+    // DRAM latency overlaps the rest of the setup.
+    for (int64_t i = 0; i < kStages; ++i) {
+      const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+      if (p >= npairs) break;
+      const int nvalid = (2 * p + 1 < tokens) ? 2 : 1;
+      tc::mbar_arrive_expect_tx(&S.full[i], (uint32_t)nvalid * 2u * kTileBytes);
+      uint8_t *dst = smem + kOffX + i * kPairBytes;
+      for (int j = 0; j < 2 * nvalid; ++j)
+        tc::tma_load_2d(dst + j * kTileBytes, &xmap, &S.full[i], (j & 1) * 64, (int)((2 * p + (j >> 1)) * 128));
+      first_issued = i + 1;
+    }
   }
-  if (threadIdx.x == 32) tc::prefetch_tensormap(&xmap);
+  tc::grid_dep_launch();
   // H_128 as the A operand: K-major, two K blocks of [128 rows m][64 k], 128-byte swizzle.
   for (uint32_t c = threadIdx.x; c < 2048; c += kThreads) {
     const uint32_t kb = c >> 10, m = (c >> 3) & 127u, ch = c & 7u;
@@ -158,7 +193,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       int64_t last[kStages] = {-1, -1, -1};
-      for (int64_t i = 0;; ++i) {
+      for (int64_t i = 0; i < first_issued; ++i) last[i] = i;
+      for (int64_t i = first_issued;; ++i) {
         const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
         if (p >= npairs) break;
         const int st = (int)(i % kStages);
@@ -290,24 +326,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float *wmx = S.wmax[g][i & 1];
       const float mu = fmaxf(fmaxf(wmx[0], wmx[1]), fmaxf(wmx[2], wmx[3]));
       const float s = fmaxf(clip * (mu * inv_sqrt_n) / 7.0f, 1e-8f);
-      const float c15 = (inv_sqrt_n / s) / 15.0f;
+      const float c15 = (inv_sqrt_n / 15.0f) / s;
       constexpr float k815 = 8.0f / 15.0f;
-      constexpr float kMagic = 12582912.0f;
       const int64_t token = 2 * p + g;
       if (token < tokens) {
-        uint4 *dst = reinterpret_cast<uint4 *>(q + token * 8192 + row * 64);
+        uint8_t *dst = q + token * 8192 + row * 64;
 #pragma unroll
-        for (int w4 = 0; w4 < 4; ++w4) {
-          uint32_t words[4];
+        for (int w8 = 0; w8 < 2; ++w8) {
+          uint32_t words[8];
 #pragma unroll
-          for (int wi = 0; wi < 4; ++wi) {
+          for (int wi = 0; wi < 8; ++wi) {
             uint32_t b[8];
+            float t[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              b[k] = __float_as_uint(fmaf(fma_sat(v[32 * w4 + 8 * wi + k], c15, k815), 15.0f, kMagic));
+            for (int k = 0; k < 8; ++k) t[k] = fma_sat(v[64 * w8 + 8 * wi + k], c15, k815);
+#pragma unroll
+            for (int k = 0; k < 8; k += 2) round15_x2(t[k], t[k + 1], b[k], b[k + 1]);
             words[wi] = pack8(b);
           }
-          __stcs(dst + w4, make_uint4(words[0], words[1], words[2], words[3]));
+          if constexpr (STORE32) {
+            st_v8_cs(dst + 32 * w8, words);
+          } else {
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * w8);
+            __stcs(d4, make_uint4(words[0], words[1], words[2], words[3]));
+            __stcs(d4 + 1, make_uint4(words[4], words[5], words[6], words[7]));
+          }
         }
         if (tg == 0) scales[token] = s;
       }
@@ -341,7 +384,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <bool SIGNS>
+template <bool SIGNS, bool STORE32>
 cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
                       cudaStream_t stream) {
   auto fn = encode_fn();
@@ -355,15 +398,24 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto kern = k1_tc_rotate_quant_16384<SIGNS>;
+  auto kern = k1_tc_rotate_quant_16384<SIGNS, STORE32>;
   int slots = 0;
   cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreads, (int)kSmemBytes, &slots);
   if (err != cudaSuccess) return err;
   const int64_t npairs = (tokens + 1) / 2;
   const int64_t grid = npairs < slots ? npairs : slots;
   const float inv_sqrt_n = (float)(1.0 / 128.0);
-  kern<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(map, tokens, clip, inv_sqrt_n, signs, q, scales);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, map, tokens, clip, inv_sqrt_n, signs, q, scales);
 }
 
 }  // namespace
@@ -374,8 +426,13 @@ bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags) {
 
 cudaError_t launch_rotate_quant_int4_tc(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q,
                                         float *scales, cudaStream_t stream) {
-  if (signs) return launch_tc<true>(x, tokens, clip, signs, q, scales, stream);
-  return launch_tc<false>(x, tokens, clip, nullptr, q, scales, stream);
+  const bool a32 = (reinterpret_cast<uintptr_t>(q) & 31u) == 0;  // 32-byte stores need 32-byte alignment
+  if (signs) {
+    return a32 ? launch_tc<true, true>(x, tokens, clip, signs, q, scales, stream)
+               : launch_tc<true, false>(x, tokens, clip, signs, q, scales, stream);
+  }
+  return a32 ? launch_tc<false, true>(x, tokens, clip, nullptr, q, scales, stream)
+             : launch_tc<false, false>(x, tokens, clip, nullptr, q, scales, stream);
 }
 
 cudaError_t read_device_status(unsigned int *status, bool reset) {
