@@ -341,7 +341,7 @@ def main():
 
     # ---- the same steps on the all-CUDA-core kernel, for comparison (not the headline)
     cores = None
-    if wl["kind"] == "r4" and n == 16384:
+    if wl["kind"] == "r4" and n in (4096, 8192, 16384):
         for i in range(args.warmup):
             step(i, True)
         stream.synchronize()
@@ -356,7 +356,7 @@ def main():
 
     peak, peak_kind = measured_peaks()
     if wl["kind"] == "r4":
-        kname = "k1_tc_rotate_quant_16384" if n == 16384 else "k1_rotate_quant_int4"
+        kname = "k1_tc_rotate_quant" if n in (4096, 8192, 16384) else "k1_rotate_quant_int4"
     else:
         kname = "k2_rope_hadamard_kvquant"
     traffic = recorded_traffic(f"{kname}:{args.workload}")

@@ -208,7 +208,7 @@ cudaError_t launch_rotate_quant_int4(const void *x, int64_t tokens, int log_n, f
                                      const uint32_t *signs, uint32_t flags, uint8_t *q, float *scales,
                                      cudaStream_t stream) {
   if (!(flags & kCudaCoresOnly) && tc_rotate_quant_supported(log_n, tokens, flags))
-    return launch_rotate_quant_int4_tc(x, tokens, clip, signs, q, scales, stream);
+    return launch_rotate_quant_int4_tc(log_n, x, tokens, clip, signs, q, scales, stream);
   flags &= ~kCudaCoresOnly;
   switch (log_n) {
     case 7: return launch_n<7>(x, tokens, clip, signs, flags, q, scales, stream);

@@ -1,40 +1,40 @@
-// k1_tc.cu -- R4 at n = 16384 with the first Kronecker factor on the tensor
-// cores.
+// k1_tc.cu -- R4 for n = 4096, 8192 and 16384 with the first Kronecker factor
+// on the tensor cores.
 //
 // "Rotations: QuaRot, SpinQuant and incoherence", section "Hadamard matrices":
-// H_16384 = H_128 (x) H_128 (Kronecker product of Sylvester matrices), and the
-// randomised transform (1/sqrt n) H_n diag(+-1). "SpinQuant, when rotations are
-// worth learning", section "Four rotation sites": R4 is the fixed Hadamard on
-// the down-projection input. "SpinQuant Guide", section "The Outlier Curse":
-// symmetric INT4, step max|y| / 7.
+// the Sylvester H_n is a Kronecker product of smaller Sylvester matrices, and
+// the randomised transform is (1/sqrt n) H_n diag(+-1). "SpinQuant, when
+// rotations are worth learning", section "Four rotation sites": R4 is the fixed
+// Hadamard on the down-projection input. "SpinQuant Guide", section "The
+// Outlier Curse": symmetric INT4, step max|y| / 7.
 //
-// A token row x (16384 bf16) is the 128 x 128 matrix X[a][b] with element
-// index e = 128 a + b. Then H_16384 x = vec(H_128 X H_128):
-//   1. tcgen05.mma computes Y = H_128 X (contraction over a) for two tokens at
-//      once (M = 128, N = 256, K = 128, bf16 in, fp32 accumulate in TMEM). H is
-//      exactly +-1 and X is exactly bf16, so every product is exact and only the
-//      fp32 accumulation rounds.
-//   2. Each epilogue thread owns one row a' of Y (one TMEM lane), loads its 128
-//      values and runs the seven butterfly stages of the second factor (over b)
-//      in registers, then the per-token max, the step, the INT4 codes and the
-//      nibble packing; the 64 bytes of row a' are contiguous in the output.
+// A token row x of n = 128 B bf16 values is the 128 x B matrix X[a][b], with
+// element index e = B a + b (B = 32, 64, 128). Then H_n x = vec(H_128 X H_B):
+//   1. tcgen05.mma computes Y = H_128 X (contraction over a) for 256 / B tokens
+//      at once (M = 128, N = 256, K = 128, bf16 in, fp32 accumulate in TMEM).
+//      H is exactly +-1 and X is exactly bf16, so every product is exact and
+//      only the fp32 accumulation rounds.
+//   2. Each epilogue thread owns one row a' of Y (one TMEM lane) over 128
+//      columns, i.e. 128 / B token segments of B values; it runs the log2(B)
+//      butterfly stages of the second factor in registers, then each token's
+//      max, step, INT4 codes and nibble packing. Row a' of a token is B / 2
+//      contiguous code bytes.
 //
-// Roles (384 threads, one CTA per SM, persistent over token pairs):
-//   warp 0      TMA producer: four 16 KiB tiles (two tokens x two 64-column
-//               halves, 128-byte swizzle) per pair into a three-stage ring
-//   warp 1      TMEM owner and MMA issuer (8 MMAs of K = 16 per pair)
+// Roles (384 threads, one CTA per SM, persistent over groups of 256 / B tokens):
+//   warp 0      TMA producer: 64 KiB per group (boxes of [128 rows][min(B, 64)]
+//               bf16 with 64- or 128-byte swizzle) into a three-stage ring
+//   warp 1      TMEM owner and MMA issuer (8 MMAs of K = 16 per group)
 //   warps 2-3   +-1 diagonal: XOR of the bf16 sign bits in shared memory, with
 //               each thread's sign words held in registers
-//   warps 4-7   epilogue for the first token of each pair (TMEM columns 0-127)
-//   warps 8-11  epilogue for the second token (columns 128-255)
-// The launch allows programmatic dependent launch: the prologue of a kernel
-// may overlap the tail of the previous one in the stream, and no global memory
-// is read or written before griddepcontrol.wait returns.
-// TMEM holds two 256-column accumulators, so the MMA of pair i + 1 overlaps the
-// epilogue of pair i. Each epilogue thread writes its 64 code bytes straight
-// to global memory (four 16-byte streaming stores). Every mbarrier wait is bounded by a clock budget; on
-// expiry the CTA records a status, drains its copies and MMAs, frees TMEM and
-// returns.
+//   warps 4-7   epilogue for TMEM columns 0-127 of each group
+//   warps 8-11  epilogue for columns 128-255
+// TMEM holds two 256-column accumulators, so the MMA of group i + 1 overlaps
+// the epilogue of group i. Each epilogue thread stores its code bytes straight
+// to global memory. The launch allows programmatic dependent launch: the
+// prologue may overlap the tail of the previous kernel in the stream, and no
+// global memory is read or written before griddepcontrol.wait returns. Every
+// mbarrier wait is bounded by a clock budget; on expiry the CTA records a
+// status, drains its copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -56,21 +56,39 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kStages = 3;
-constexpr uint32_t kTileBytes = 16384;              // [128 rows][64 bf16]
-constexpr uint32_t kPairBytes = 4 * kTileBytes;     // two tokens
-constexpr uint32_t kOffH = 0;                       // A operand: H_128, K-major, 2 x 16 KiB
-constexpr uint32_t kOffX = 32768;                   // ring of kStages x 64 KiB
-constexpr uint32_t kOffBar = kOffX + kStages * kPairBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
+constexpr uint32_t kGroupBytes = 65536;            // one MMA group: 128 rows x 256 columns of bf16
+constexpr uint32_t kOffH = 0;                      // A operand: H_128, K-major, 2 x 16 KiB
+constexpr uint32_t kOffX = 32768;                  // ring of kStages x 64 KiB
+constexpr uint32_t kOffBar = kOffX + kStages * kGroupBytes;
+constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;  // + alignment slack
 constexpr long long kTimeoutCycles = 4000000000LL;     // about two seconds
+
+// Shape constants for n = 2^LOGN.
+template <int LOGN>
+struct Shape {
+  static constexpr int B = 1 << (LOGN - 7);        // columns per row (second factor size)
+  static constexpr int LOGB = LOGN - 7;
+  static constexpr int TOK = 256 / B;               // tokens per MMA group
+  static constexpr int SEG = 128 / B;               // token segments per epilogue thread
+  static constexpr int BOXW = B < 64 ? B : 64;      // TMA box width (columns)
+  static constexpr int ROWB = BOXW * 2;             // bytes per smem tile row (64 or 128)
+  static constexpr int BPT = B / BOXW;              // boxes per token
+  static constexpr uint32_t BOXBYTES = 128u * ROWB; // bytes per box
+  static constexpr int CPR = ROWB / 16;             // 16-byte chunks per tile row
+  static constexpr uint32_t LAYOUT = ROWB == 128 ? 2u : 4u;  // UMMA swizzle: 128 B or 64 B
+  static constexpr uint32_t TOKBYTES = kGroupBytes / TOK;
+  static constexpr int NPOS = (int)(TOKBYTES / 16 / 64);  // sign positions per sign thread
+  static_assert(LOGN >= 12 && LOGN <= 14, "tensor-core R4 covers n = 4096 .. 16384");
+};
 
 struct Shared {
   uint64_t full[kStages], sgn[kStages], empty[kStages], tfull[2], tempty[2], drain;
   uint32_t tmem_base;
   int abort;
   int dec[3];
-  float wmax[2][2][4];  // [warpgroup][pair parity][warp]
+  float wmax[2][2][4][4];  // [warpgroup][group parity][warp][token segment]
 };
+static_assert(sizeof(Shared) <= 512, "barrier area");
 
 __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, Shared &S, bool honor_abort) {
   if (tc::mbar_try_wait(bar, parity)) return true;
@@ -101,7 +119,7 @@ __device__ __forceinline__ void round15_x2(float a0, float a1, uint32_t &r0, uin
   asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(R));
 }
 
-__device__ __forceinline__ void st_v8_cs(void *p, const uint32_t (&w)[8]) {
+__device__ __forceinline__ void st_v8_cs(void *p, const uint32_t *w) {
   asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
                "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
                : "memory");
@@ -122,22 +140,36 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&b)[8]) {
 // byte offset of 16-byte chunk `ch` (0..7) of row `r` in a 128-byte-swizzled [rows][128 B] tile
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t ch) { return r * 128u + ((ch ^ (r & 7u)) << 4); }
 
-template <bool SIGNS, bool STORE32>
+// Issue the TMA copies of group p (tokens p * TOK ...) into `dst`.
+template <int LOGN>
+__device__ __forceinline__ void load_group(uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int64_t p,
+                                           int64_t tokens) {
+  using SH = Shape<LOGN>;
+  const int64_t t0 = p * SH::TOK;
+  const int nvalid = (int)((tokens - t0) < SH::TOK ? (tokens - t0) : SH::TOK);
+  tc::mbar_arrive_expect_tx(bar, (uint32_t)nvalid * SH::TOKBYTES);
+  for (int t = 0; t < nvalid; ++t)
+    for (int j = 0; j < SH::BPT; ++j)
+      tc::tma_load_2d(dst + (t * SH::BPT + j) * SH::BOXBYTES, map, bar, j * SH::BOXW, (int)((t0 + t) * 128));
+}
+
+template <int LOGN, bool SIGNS, bool STORE32>
 __global__ void __launch_bounds__(kThreads, 1)
-    k1_tc_rotate_quant_16384(const __grid_constant__ CUtensorMap xmap, int64_t tokens, float clip,
-                             float inv_sqrt_n, const uint32_t *__restrict__ signs, uint8_t *__restrict__ q,
-                             float *__restrict__ scales) {
+    k1_tc_rotate_quant(const __grid_constant__ CUtensorMap xmap, int64_t tokens, float clip, float inv_sqrt_n,
+                       const uint32_t *__restrict__ signs, uint8_t *__restrict__ q, float *__restrict__ scales) {
+  using SH = Shape<LOGN>;
+  constexpr int B = SH::B, SEG = SH::SEG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Shared &S = *reinterpret_cast<Shared *>(smem + kOffBar);
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
-  const int64_t npairs = (tokens + 1) >> 1;
+  const int64_t ngroups = (tokens + SH::TOK - 1) / SH::TOK;
 
   // ------------------------------------------------------------ setup
   // Global memory is touched only after the grids this one depends on have
   // finished (programmatic dependent launch lets this prologue overlap their tail).
   tc::grid_dep_wait();
-  int64_t first_issued = 0;  // loads the producer issues before the setup barrier
+  int64_t first_issued = 0;  // groups the producer issues before the setup barrier
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&S.full[s], 1);
@@ -152,16 +184,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     S.abort = 0;
     tc::fence_barrier_init();
     tc::prefetch_tensormap(&xmap);
-    // The first kStages pairs need no free slot: start their copies now, so the
+    // The first kStages groups need no free slot: start their copies now, so the
     // DRAM latency overlaps the rest of the setup.
     for (int64_t i = 0; i < kStages; ++i) {
       const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
-      if (p >= npairs) break;
-      const int nvalid = (2 * p + 1 < tokens) ? 2 : 1;
-      tc::mbar_arrive_expect_tx(&S.full[i], (uint32_t)nvalid * 2u * kTileBytes);
-      uint8_t *dst = smem + kOffX + i * kPairBytes;
-      for (int j = 0; j < 2 * nvalid; ++j)
-        tc::tma_load_2d(dst + j * kTileBytes, &xmap, &S.full[i], (j & 1) * 64, (int)((2 * p + (j >> 1)) * 128));
+      if (p >= ngroups) break;
+      load_group<LOGN>(smem + kOffX + i * kGroupBytes, &xmap, &S.full[i], p, tokens);
       first_issued = i + 1;
     }
   }
@@ -196,14 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t i = 0; i < first_issued; ++i) last[i] = i;
       for (int64_t i = first_issued;; ++i) {
         const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
-        if (p >= npairs) break;
+        if (p >= ngroups) break;
         const int st = (int)(i % kStages);
         if (!wait_bounded(&S.empty[st], (uint32_t)((i / kStages) & 1) ^ 1u, S, true)) break;
-        const int nvalid = (2 * p + 1 < tokens) ? 2 : 1;
-        tc::mbar_arrive_expect_tx(&S.full[st], (uint32_t)nvalid * 2u * kTileBytes);
-        uint8_t *dst = smem + kOffX + st * kPairBytes;
-        for (int j = 0; j < 2 * nvalid; ++j)
-          tc::tma_load_2d(dst + j * kTileBytes, &xmap, &S.full[st], (j & 1) * 64, (int)((2 * p + (j >> 1)) * 128));
+        load_group<LOGN>(smem + kOffX + st * kGroupBytes, &xmap, &S.full[st], p, tokens);
         last[st] = i;
       }
       // every issued copy has landed before the CTA can leave
@@ -216,15 +240,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sH = tc::smem_u32(smem + kOffH), sX = tc::smem_u32(smem + kOffX);
       for (int64_t i = 0;; ++i) {
         const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
-        if (p >= npairs) break;
+        if (p >= ngroups) break;
         const int st = (int)(i % kStages), acc = (int)(i & 1);
         if (!wait_bounded(SIGNS ? &S.sgn[st] : &S.full[st], (uint32_t)((i / kStages) & 1), S, true)) break;
         if (!wait_bounded(&S.tempty[acc], (uint32_t)((i >> 1) & 1) ^ 1u, S, true)) break;
         tc::tc_fence_after();
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
+          // A: 16 columns k of H per step. B: rows a = 16 s .. 16 s + 15 of every box
+          // (MN-major: boxes of BOXW columns BOXBYTES apart, 8-row groups 8 ROWB apart).
           const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::smem_desc(sX + st * kPairBytes + s * 2048, kTileBytes, 1024);
+          uint64_t bd = tc::smem_desc(sX + st * kGroupBytes + s * 16 * SH::ROWB, SH::BOXBYTES, 8 * SH::ROWB);
+          bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
           tc::umma_bf16(tmem + acc * 256, ad, bd, idesc, s > 0 ? 1u : 0u);
         }
         tc::umma_commit(&S.empty[st]);
@@ -233,16 +260,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 4) {
     if constexpr (SIGNS) {
-      // Thread ts flips the signs of chunks ts + 64 j of each pair's 64 KiB.
-      // Those chunks sit at 32 distinct positions of a token tile; their sign
-      // words stay in registers for the whole kernel.
+      // Thread ts flips the signs of chunks ts + 64 j of each group's 64 KiB.
+      // Those chunks sit at NPOS distinct positions of a token's tile; their
+      // sign words stay in registers for the whole kernel.
+      constexpr int NPOS = SH::NPOS;
       const uint32_t ts = threadIdx.x - 64;  // 0..63
-      uint4 mk[32];
+      uint4 mk[NPOS];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const uint32_t pos = ts + 64u * k;  // 16-byte chunk index inside one token's 32 KiB
-        const uint32_t h = pos >> 10, a = (pos >> 3) & 127u, ch = (pos & 7u) ^ (a & 7u);
-        const uint32_t e = a * 128u + h * 64u + ch * 8u;
+      for (int k = 0; k < NPOS; ++k) {
+        const uint32_t pos = ts + 64u * k;  // 16-byte chunk index inside one token's tile
+        const uint32_t box = pos / (SH::BOXBYTES / 16), inbox = pos % (SH::BOXBYTES / 16);
+        const uint32_t a = inbox / SH::CPR, pc = inbox % SH::CPR;
+        const uint32_t ch = SH::ROWB == 128 ? (pc ^ (a & 7u)) : (pc ^ ((a >> 1) & 3u));
+        const uint32_t e = a * B + box * SH::BOXW + ch * 8u;
         const uint32_t byte = (__ldg(signs + (e >> 5)) >> (e & 31u)) & 0xFFu;
         uint32_t w[4];
 #pragma unroll
@@ -251,12 +281,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int64_t i = 0;; ++i) {
         const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
-        if (p >= npairs) break;
+        if (p >= ngroups) break;
         const int st = (int)(i % kStages);
         if (ts == 0) S.dec[2] = wait_bounded(&S.full[st], (uint32_t)((i / kStages) & 1), S, true) ? 1 : 0;
         tc::named_sync(3, 64);
         if (!S.dec[2]) break;
-        uint4 *X = reinterpret_cast<uint4 *>(smem + kOffX + st * kPairBytes) + ts;
+        uint4 *X = reinterpret_cast<uint4 *>(smem + kOffX + st * kGroupBytes) + ts;
 #pragma unroll
         for (int j0 = 0; j0 < 64; j0 += 4) {
           uint4 x[4];
@@ -264,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int u = 0; u < 4; ++u) x[u] = X[64 * (j0 + u)];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const uint4 m = mk[(j0 + u) & 31];
+            const uint4 m = mk[(j0 + u) % NPOS];
             X[64 * (j0 + u)] = make_uint4(x[u].x ^ m.x, x[u].y ^ m.y, x[u].z ^ m.z, x[u].w ^ m.w);
           }
         }
@@ -279,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
     for (int64_t i = 0;; ++i) {
       const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
-      if (p >= npairs) break;
+      if (p >= ngroups) break;
       const int acc = (int)(i & 1);
       if (tg == 0) S.dec[g] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
       tc::named_sync(1 + g, 128);
@@ -299,58 +329,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::tc_fence_before();
       tc::mbar_arrive(&S.tempty[acc]);
-      // second Kronecker factor: H_128 over b, in registers
+      // second Kronecker factor: H_B over b inside each token segment, in registers
       stage<0>(v);
       stage<1>(v);
       stage<2>(v);
       stage<3>(v);
       stage<4>(v);
-      stage<5>(v);
-      stage<6>(v);
-      // per-token max |u|: a tree of three-input maxima, then the warp, then the warpgroup
-      float mx[16];
+      if constexpr (SH::LOGB > 5) stage<5>(v);
+      if constexpr (SH::LOGB > 6) stage<6>(v);
+      // per-token max |u|: a tree of three-input maxima per segment, then the warp, then the warpgroup
 #pragma unroll
-      for (int k = 0; k < 16; ++k) mx[k] = fmaxf(fabsf(v[8 * k]), fabsf(v[8 * k + 1]));
+      for (int sg = 0; sg < SEG; ++sg) {
+        float mx[B / 8];
 #pragma unroll
-      for (int j = 2; j < 8; j += 2)
+        for (int k = 0; k < B / 8; ++k) {
+          const float *w = v + sg * B + 8 * k;
+          mx[k] = fmax3(fmax3(fabsf(w[0]), fabsf(w[1]), fabsf(w[2])), fmax3(fabsf(w[3]), fabsf(w[4]), fabsf(w[5])),
+                        fmaxf(fabsf(w[6]), fabsf(w[7])));
+        }
 #pragma unroll
-        for (int k = 0; k < 16; ++k) mx[k] = fmax3(mx[k], fabsf(v[8 * k + j]), fabsf(v[8 * k + j + 1]));
+        for (int h = B / 16; h >= 1; h >>= 1)
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], mx[k + 8]);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], mx[k + 4]);
-      const float m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
-      if (lane == 0) S.wmax[g][i & 1][wq] = __uint_as_float(wm);
+          for (int k = 0; k < h; ++k) mx[k] = fmaxf(mx[k], mx[k + h]);
+        const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mx[0]));
+        if (lane == 0) S.wmax[g][i & 1][wq][sg] = __uint_as_float(wm);
+      }
       tc::named_sync(1 + g, 128);
-      const float *wmx = S.wmax[g][i & 1];
-      const float mu = fmaxf(fmaxf(wmx[0], wmx[1]), fmaxf(wmx[2], wmx[3]));
-      const float s = fmaxf(clip * (mu * inv_sqrt_n) / 7.0f, 1e-8f);
-      const float c15 = (inv_sqrt_n / 15.0f) / s;
       constexpr float k815 = 8.0f / 15.0f;
-      const int64_t token = 2 * p + g;
-      if (token < tokens) {
-        uint8_t *dst = q + token * 8192 + row * 64;
 #pragma unroll
-        for (int w8 = 0; w8 < 2; ++w8) {
-          uint32_t words[8];
+      for (int sg = 0; sg < SEG; ++sg) {
+        const float mu = fmaxf(fmaxf(S.wmax[g][i & 1][0][sg], S.wmax[g][i & 1][1][sg]),
+                               fmaxf(S.wmax[g][i & 1][2][sg], S.wmax[g][i & 1][3][sg]));
+        const float s = fmaxf(clip * (mu * inv_sqrt_n) / 7.0f, 1e-8f);
+        const float c15 = (inv_sqrt_n / 15.0f) / s;
+        const int64_t token = p * SH::TOK + g * SEG + sg;
+        if (token >= tokens) continue;
+        uint8_t *dst = q + token * (int64_t)(B * 64) + row * (B / 2);
+        uint32_t words[B / 8];
 #pragma unroll
-          for (int wi = 0; wi < 8; ++wi) {
-            uint32_t b[8];
-            float t[8];
+        for (int wi = 0; wi < B / 8; ++wi) {
+          uint32_t b[8];
+          float t[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) t[k] = fma_sat(v[64 * w8 + 8 * wi + k], c15, k815);
+          for (int k = 0; k < 8; ++k) t[k] = fma_sat(v[sg * B + 8 * wi + k], c15, k815);
 #pragma unroll
-            for (int k = 0; k < 8; k += 2) round15_x2(t[k], t[k + 1], b[k], b[k + 1]);
-            words[wi] = pack8(b);
-          }
-          if constexpr (STORE32) {
-            st_v8_cs(dst + 32 * w8, words);
-          } else {
-            uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * w8);
-            __stcs(d4, make_uint4(words[0], words[1], words[2], words[3]));
-            __stcs(d4 + 1, make_uint4(words[4], words[5], words[6], words[7]));
-          }
+          for (int k = 0; k < 8; k += 2) round15_x2(t[k], t[k + 1], b[k], b[k + 1]);
+          words[wi] = pack8(b);
+        }
+        if constexpr (STORE32 && B >= 64) {
+#pragma unroll
+          for (int w8 = 0; w8 < B / 64; ++w8) st_v8_cs(dst + 32 * w8, words + 8 * w8);
+        } else {
+#pragma unroll
+          for (int w4 = 0; w4 < B / 32; ++w4)
+            __stcs(reinterpret_cast<uint4 *>(dst) + w4,
+                   make_uint4(words[4 * w4], words[4 * w4 + 1], words[4 * w4 + 2], words[4 * w4 + 3]));
         }
         if (tg == 0) scales[token] = s;
       }
@@ -384,27 +417,29 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <bool SIGNS, bool STORE32>
+template <int LOGN, bool SIGNS, bool STORE32>
 cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
                       cudaStream_t stream) {
+  using SH = Shape<LOGN>;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap map;
-  const cuuint64_t dims[2] = {128, (cuuint64_t)tokens * 128};
-  const cuuint64_t strides[1] = {256};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint64_t dims[2] = {(cuuint64_t)SH::B, (cuuint64_t)tokens * 128};
+  const cuuint64_t strides[1] = {(cuuint64_t)SH::B * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)SH::BOXW, 128};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  SH::ROWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto kern = k1_tc_rotate_quant_16384<SIGNS, STORE32>;
+  auto kern = k1_tc_rotate_quant<LOGN, SIGNS, STORE32>;
   int slots = 0;
   cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreads, (int)kSmemBytes, &slots);
   if (err != cudaSuccess) return err;
-  const int64_t npairs = (tokens + 1) / 2;
-  const int64_t grid = npairs < slots ? npairs : slots;
-  const float inv_sqrt_n = (float)(1.0 / 128.0);
+  const int64_t ngroups = (tokens + SH::TOK - 1) / SH::TOK;
+  const int64_t grid = ngroups < slots ? ngroups : slots;
+  const float inv_sqrt_n = (float)(1.0 / std::sqrt((double)(1 << LOGN)));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(kThreads);
@@ -418,21 +453,32 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
   return cudaLaunchKernelEx(&cfg, kern, map, tokens, clip, inv_sqrt_n, signs, q, scales);
 }
 
+template <int LOGN>
+cudaError_t launch_n(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
+                     cudaStream_t stream) {
+  const bool a32 = (reinterpret_cast<uintptr_t>(q) & 31u) == 0;  // 32-byte stores need 32-byte alignment
+  if (signs) {
+    return a32 ? launch_tc<LOGN, true, true>(x, tokens, clip, signs, q, scales, stream)
+               : launch_tc<LOGN, true, false>(x, tokens, clip, signs, q, scales, stream);
+  }
+  return a32 ? launch_tc<LOGN, false, true>(x, tokens, clip, nullptr, q, scales, stream)
+             : launch_tc<LOGN, false, false>(x, tokens, clip, nullptr, q, scales, stream);
+}
+
 }  // namespace
 
 bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags) {
-  return log_n == 14 && !(flags & kNoRotate) && tokens > 0 && tokens * 128 < (int64_t(1) << 31);
+  return log_n >= 12 && log_n <= 14 && !(flags & kNoRotate) && tokens > 0 && tokens * 128 < (int64_t(1) << 31);
 }
 
-cudaError_t launch_rotate_quant_int4_tc(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q,
-                                        float *scales, cudaStream_t stream) {
-  const bool a32 = (reinterpret_cast<uintptr_t>(q) & 31u) == 0;  // 32-byte stores need 32-byte alignment
-  if (signs) {
-    return a32 ? launch_tc<true, true>(x, tokens, clip, signs, q, scales, stream)
-               : launch_tc<true, false>(x, tokens, clip, signs, q, scales, stream);
+cudaError_t launch_rotate_quant_int4_tc(int log_n, const void *x, int64_t tokens, float clip, const uint32_t *signs,
+                                        uint8_t *q, float *scales, cudaStream_t stream) {
+  switch (log_n) {
+    case 12: return launch_n<12>(x, tokens, clip, signs, q, scales, stream);
+    case 13: return launch_n<13>(x, tokens, clip, signs, q, scales, stream);
+    case 14: return launch_n<14>(x, tokens, clip, signs, q, scales, stream);
+    default: return cudaErrorInvalidValue;
   }
-  return a32 ? launch_tc<false, true>(x, tokens, clip, nullptr, q, scales, stream)
-             : launch_tc<false, false>(x, tokens, clip, nullptr, q, scales, stream);
 }
 
 cudaError_t read_device_status(unsigned int *status, bool reset) {

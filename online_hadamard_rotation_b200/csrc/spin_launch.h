@@ -19,10 +19,10 @@ cudaError_t launch_rotate_quant_int4(const void *x, int64_t tokens, int log_n, f
                                      const uint32_t *signs, uint32_t flags, uint8_t *q, float *scales,
                                      cudaStream_t stream);
 
-// Tensor-core R4 kernel (n = 16384): availability and launcher.
+// Tensor-core R4 kernel (n = 4096, 8192, 16384): availability and launcher.
 bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags);
-cudaError_t launch_rotate_quant_int4_tc(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q,
-                                        float *scales, cudaStream_t stream);
+cudaError_t launch_rotate_quant_int4_tc(int log_n, const void *x, int64_t tokens, float clip, const uint32_t *signs,
+                                        uint8_t *q, float *scales, cudaStream_t stream);
 
 // Device status word set by kernels whose bounded waits ran out.
 cudaError_t read_device_status(unsigned int *status, bool reset);

@@ -1,6 +1,7 @@
-"""The tensor-core R4 kernel (n = 16384: first H_128 Kronecker factor on
-tcgen05, second on CUDA cores) vs the fp64 oracle, and vs the all-CUDA-core
-kernel selected with SPIN_CUDA_CORES_ONLY."""
+"""The tensor-core R4 kernel (n = 4096, 8192, 16384: first H_128 Kronecker
+factor on tcgen05, second on CUDA cores) vs the fp64 oracle, and vs the
+all-CUDA-core kernel selected with SPIN_CUDA_CORES_ONLY. Token counts leave
+partial MMA groups (8, 4 and 2 tokens per group)."""
 import numpy as np
 import pytest
 import torch
@@ -11,7 +12,7 @@ from tests.gpu_util import to_dev_bf16, to_dev_signs
 
 pytestmark = pytest.mark.gpu
 
-N = 16384
+SIZES = [4096, 8192, 16384]
 
 
 def run(spin, bits, clip, signs, cores_only=False):
@@ -20,10 +21,11 @@ def run(spin, bits, clip, signs, cores_only=False):
     return q.cpu().numpy(), s.cpu().numpy()
 
 
-@pytest.mark.parametrize("tokens", [1, 2, 3, 16, 149, 300])
+@pytest.mark.parametrize("N", SIZES)
+@pytest.mark.parametrize("tokens", [1, 2, 3, 7, 9, 149, 300])
 @pytest.mark.parametrize("clip,with_signs", [(1.0, False), (0.9, True)])
-def test_tc_vs_oracle(spin_gpu, orc, tokens, clip, with_signs):
-    bits = synthetic.r4_prefill(tokens=tokens, seed=50 + tokens)[0]
+def test_tc_vs_oracle(spin_gpu, orc, N, tokens, clip, with_signs):
+    bits = synthetic.r4_prefill(tokens=tokens, n=N, seed=50 + tokens)[0]
     signs = synthetic.sign_bits(N, 101) if with_signs else None
     q, s = run(spin_gpu, bits, clip, signs)
     codes = parity.unpack_signed(q, N)
@@ -34,8 +36,9 @@ def test_tc_vs_oracle(spin_gpu, orc, tokens, clip, with_signs):
     assert spin_gpu.device_status() == 0
 
 
-def test_tc_matches_cuda_core_kernel(spin_gpu, orc):
-    bits, signs, _ = synthetic.r4_prefill(tokens=512, seed=9)
+@pytest.mark.parametrize("N", SIZES)
+def test_tc_matches_cuda_core_kernel(spin_gpu, orc, N):
+    bits, signs, _ = synthetic.r4_prefill(tokens=512, n=N, seed=9)
     q1, s1 = run(spin_gpu, bits, 0.9, signs)
     q2, s2 = run(spin_gpu, bits, 0.9, signs, cores_only=True)
     parity.check_rel(s1, s2, 1e-5, "tc vs cuda-core scales")
@@ -48,9 +51,10 @@ def test_tc_matches_cuda_core_kernel(spin_gpu, orc):
     assert (c1 != c2).mean() < 1e-4
 
 
-def test_tc_special_rows(spin_gpu, orc):
+@pytest.mark.parametrize("N", SIZES)
+def test_tc_special_rows(spin_gpu, orc, N):
     rows = [np.zeros(N, np.float32), np.full(N, 1.0, np.float32)]
-    for j in (0, 1, 127, 128, 8191, N - 1):
+    for j in (0, 1, 127, 128, N // 2 - 1, N - 1):
         r = np.zeros(N, np.float32)
         r[j] = 60.0
         rows.append(r)
@@ -67,8 +71,9 @@ def test_tc_special_rows(spin_gpu, orc):
         assert np.all(np.abs(codes[t]) == 7)
 
 
-def test_tc_leaves_tail_untouched(spin_gpu):
-    bits = synthetic.r4_prefill(tokens=5, seed=3)[0]
+@pytest.mark.parametrize("N", SIZES)
+def test_tc_leaves_tail_untouched(spin_gpu, N):
+    bits = synthetic.r4_prefill(tokens=5, n=N, seed=3)[0]
     out = torch.full((8, N // 2), 0xA5, dtype=torch.uint8, device="cuda")
     sc = torch.full((8,), -1.0, dtype=torch.float32, device="cuda")
     spin_gpu.hadamard_quant_int4(to_dev_bf16(bits), 1.0, out=out[:5], scales=sc[:5])
