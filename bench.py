@@ -60,7 +60,7 @@ def kernel_source_digest() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "online_hadamard_rotation_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.startswith("k1_") or name == "spin_tile.cuh":
+        if name.startswith("k1_") or name in ("spin_tile.cuh", "tc_ptx.cuh"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -139,23 +139,42 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------
-def make_workload(name: str, rank: int):
+def max_over_ranks(value: float, device) -> float:
+    """The largest value over all ranks (elapsed times are reported this way)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(world: int, unit_bytes: int, unit_count: int, steps: int, ms: float):
+    """Whole-job GB/s and units/s: every rank processes `unit_count` units per
+    step (weak scaling); `ms` is the maximum elapsed time over ranks."""
+    sec = ms / 1e3
+    return world * unit_bytes * steps / sec / 1e9, world * unit_count * steps / sec
+
+
+def make_workload(name: str, rank: int, tokens: int | None = None):
+    """The workload one rank processes; every rank draws its own shard (seed + rank)."""
     import synthetic
     if name == "r4_prefill":
-        bits, signs, _ = synthetic.r4_prefill(seed=1 + rank)
+        bits, signs, _ = synthetic.r4_prefill(tokens=tokens or 8192, seed=1 + rank)
         return dict(kind="r4", bits=bits, signs=signs, clip=0.9,
                     desc={"workload": "R4 prefill: 4x2048 tokens x n=16384 bf16, SwiGLU-like, 0.1% channels x100, "
                                       "seeded +-1 diagonal, H_16384 = H_128 (x) H_128, clip 0.9",
                           "tokens": int(bits.shape[0]), "n": int(bits.shape[1])})
     if name.startswith("decode"):
         n = int(name[len("decode"):] or 16384)
-        bits = synthetic.decode(32, n, seed=3 + rank)
+        bits = synthetic.decode(tokens or 32, n, seed=3 + rank)
         return dict(kind="r4", bits=bits, signs=None, clip=1.0,
                     desc={"workload": f"decode: 32 tokens x n={n} Student-t(3), one channel x200 per row, clip 1.0",
-                          "tokens": 32, "n": n})
+                          "tokens": int(bits.shape[0]), "n": n})
     if name.startswith("sweep"):
         k = int(name[len("sweep"):])
-        bits = synthetic.sweep(k, seed=4 + k + 100 * rank)
+        bits = synthetic.sweep(k, tokens=tokens, seed=4 + k + 100 * rank)
         return dict(kind="r4", bits=bits, signs=None, clip=1.0,
                     desc={"workload": f"sweep: n=2^{k}, 1 GiB bf16 input, N(0,1) with 0.1% channels x100, clip 1.0",
                           "tokens": int(bits.shape[0]), "n": 1 << k})
@@ -165,6 +184,13 @@ def make_workload(name: str, rank: int):
                     desc={"workload": "R3+KV: batch 4 x seq 4096, 32 q / 8 kv heads, head_dim 128, RoPE theta 1e4, "
                                       "asym INT4 KV cache, clip 0.95", "tokens": 4 * 4096})
     raise SystemExit(f"unknown workload {name}")
+
+
+def config_for(wl, world: int, workload: str) -> dict:
+    """The `config` object both arms print (same workload, same keys)."""
+    return dict(wl["desc"], parallelism=f"dp{world}" if world > 1 else "single GPU",
+                l2="inputs larger than L2 (268 MB bf16 input vs 126 MB L2); two buffer sets alternate"
+                if workload == "r4_prefill" else "two buffer sets alternate")
 
 
 def r3_bytes(tokens, hq=32, hkv=8, d=128):
@@ -194,9 +220,10 @@ def run_reference(args, wl):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": dict(wl["desc"], parallelism="host cpu, 1 thread"),
+            "config": config_for(wl, args.gpus, args.workload),
             "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"first {sample} of {bits.shape[0]} tokens per step, fp64 fast transform"},
+                             "sample": f"first {sample} of {bits.shape[0]} tokens per step, fp64 fast transform, "
+                                       "1 host thread"},
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -294,15 +321,11 @@ def main():
         ev1.record(stream)
         ev1.synchronize()
     torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     ms_per_step = ms / args.steps
-    gbs = world * step_bytes * args.steps / (ms / 1e3) / 1e9
-    tok_s = world * tokens * args.steps / (ms / 1e3)
+    gbs, tok_s = aggregate(world, step_bytes, tokens, args.steps, ms)
 
     # ---- end to end through the public API from pinned host memory
     e2e = None
@@ -329,13 +352,9 @@ def main():
             e2e_step()
         ev1.record(stream)
         ev1.synchronize()
-        ems = ev0.elapsed_time(ev1)
-        if world > 1:
-            t = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * step_bytes * e2e_steps / (ems / 1e3) / 1e9, "unit": "GB/s",
-               "tokens_per_s": world * tokens * e2e_steps / (ems / 1e3),
+        ems = max_over_ranks(ev0.elapsed_time(ev1), dev)
+        e_gbs, e_tok = aggregate(world, step_bytes, tokens, e2e_steps, ems)
+        e2e = {"value": e_gbs, "unit": "GB/s", "tokens_per_s": e_tok,
                "h2d_bytes_per_step": int(host.numel() * 2), "d2h_bytes_per_step": int(q_host.numel() + 4 * tokens),
                "steps": e2e_steps}
 
@@ -353,6 +372,39 @@ def main():
         cms = ev0.elapsed_time(ev1) / args.steps
         cores = {"kernel": "k1_rotate_quant_int4 (all butterflies on CUDA cores)", "ms_per_step": cms,
                  "achieved_gbs": step_bytes / (cms / 1e3) / 1e9}
+
+    # ---- decode: per-call latency, plain launches and CUDA-graph replay
+    latency = None
+    if args.workload.startswith("decode"):
+        calls = 1000
+        b = sets[0]
+        for _ in range(10):
+            step(0)
+        stream.synchronize()
+        ev0.record(stream)
+        for _ in range(calls):
+            step(0)
+        ev1.record(stream)
+        ev1.synchronize()
+        plain_us = ev0.elapsed_time(ev1) / calls * 1e3
+        graph = torch.cuda.CUDAGraph()
+        per_graph = 100
+        with torch.cuda.graph(graph, stream=stream):
+            for _ in range(per_graph):
+                spin.hadamard_quant_int4(b["x"], wl["clip"], signs, out=b["q"], scales=b["s"],
+                                         stream=torch.cuda.current_stream())
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        ev0.record()
+        for _ in range(calls // per_graph):
+            graph.replay()
+        ev1.record()
+        ev1.synchronize()
+        graph_us = ev0.elapsed_time(ev1) / calls * 1e3
+        del graph
+        latency = {"us_per_call_plain": plain_us, "us_per_call_graph": graph_us, "calls": calls,
+                   "note": "inputs are L2-resident at this size (1.3 MB or less)"}
 
     peak, peak_kind = measured_peaks()
     if wl["kind"] == "r4":
@@ -384,11 +436,9 @@ def main():
                 "pct_of_hbm_peak": 100.0 * per_gpu_gbs / peak, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": dict(wl["desc"], parallelism=f"dp{world}" if world > 1 else "single GPU",
-                               l2="inputs larger than L2 (268 MB bf16 input vs 126 MB L2); two buffer sets alternate"
-                               if args.workload == "r4_prefill" else "two buffer sets alternate"),
+                "config": config_for(wl, world, args.workload),
                 "gpu_launches": args.steps, "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu,
-                "cuda_core_kernel": cores,
+                "cuda_core_kernel": cores, "decode_latency": latency,
                 "clocks": clocks.summary()}
         print(json.dumps(line), flush=True)
     if world > 1:

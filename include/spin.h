@@ -65,6 +65,7 @@ typedef enum spin_status_t {
 /* flags */
 #define SPIN_NO_ROTATE 1u       /* skip the diagonal and the transform (direct quantisation / identity) */
 #define SPIN_CUDA_CORES_ONLY 2u /* R4: use the CUDA-core kernel even where the tensor-core kernel applies */
+#define SPIN_TENSOR_CORES 4u    /* R4: use the tensor-core kernel wherever n allows it, at any batch size */
 
 /* spin_dequant_hadamard_inverse modes */
 #define SPIN_SYM_INT4_F32SCALE 0 /* signed codes, fp32 scale per row: value = code * scale */
@@ -116,7 +117,12 @@ spin_status_t spin_hadamard_quant_int4(const void *x_bf16, int64_t tokens, int32
  *               +-1 x bf16 products, fp32 accumulation); this bit selects the
  *               kernel that runs every butterfly on the CUDA cores instead. Both give the
  *               same codes up to the rounding-tie band and the same steps to
- *               fp32 accumulation order.
+ *               fp32 accumulation order. By default the tensor-core kernel runs
+ *               only when the batch has at least 128 MMA groups (128 x 256 / (n/128)
+ *               tokens), since it pays a per-block setup that small (decode)
+ *               batches do not amortise;
+ *             SPIN_TENSOR_CORES: use the tensor-core kernel wherever n allows,
+ *               whatever the batch size (not with SPIN_CUDA_CORES_ONLY).
  * spin_hadamard_quant_int4(...) == spin_hadamard_quant_int4_ex(..., NULL, 0, ...).
  */
 spin_status_t spin_hadamard_quant_int4_ex(const void *x_bf16, int64_t tokens, int32_t n,
@@ -199,6 +205,17 @@ spin_status_t spin_dequant_hadamard_inverse(const uint8_t *codes, int64_t rows, 
  * Errors: SPIN_ERR_INVALID_ARG (status NULL), SPIN_ERR_CUDA.
  */
 spin_status_t spin_device_status(uint32_t *status, int reset);
+
+/*
+ * Test hook for failure detection (no counterpart on the pages). While
+ * enabled (nonzero), every tensor-core R4 launch withholds the completion
+ * signal of its first MMA group and shortens its wait budget to about a
+ * millisecond, so the bounded waits run out, each block takes its abort path
+ * (drains its copies and MMAs, frees TMEM, returns) and the device status word
+ * becomes nonzero; those launches' outputs are incomplete. Process-wide; call
+ * it with 0 to restore normal operation. Never needed outside tests.
+ */
+void spin_test_stall_tensor_core_waits(int enable);
 
 /* Human-readable name of a status code (static storage). */
 const char *spin_status_string(spin_status_t status);

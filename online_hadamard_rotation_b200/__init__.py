@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "lib", "SpinError", "hadamard_quant_int4", "hadamard_quant_int4_host", "rope_hadamard_kvquant",
     "dequant_hadamard_inverse", "alloc_kv_cache", "NO_ROTATE", "SYM_INT4_F32SCALE", "ASYM_INT4_F16SZ",
-    "BF16", "F32", "HEADER", "LIB_PATH", "exported_symbols", "CUDA_CORES_ONLY", "device_status",
+    "BF16", "F32", "HEADER", "LIB_PATH", "exported_symbols", "CUDA_CORES_ONLY", "TENSOR_CORES", "device_status",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,6 +29,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "spin.h")
 
 NO_ROTATE = 1
 CUDA_CORES_ONLY = 2
+TENSOR_CORES = 4
 SYM_INT4_F32SCALE = 0
 ASYM_INT4_F16SZ = 1
 BF16 = 0
@@ -69,6 +70,8 @@ def lib() -> C.CDLL:
     for name in ("spin_hadamard_quant_int4", "spin_hadamard_quant_int4_ex", "spin_rope_hadamard_kvquant",
                  "spin_dequant_hadamard_inverse"):
         getattr(L, name).restype = C.c_int
+    L.spin_test_stall_tensor_core_waits.argtypes = [C.c_int]
+    L.spin_test_stall_tensor_core_waits.restype = None
     L.spin_device_status.argtypes = [C.POINTER(C.c_uint32), C.c_int]
     L.spin_device_status.restype = C.c_int
     L.spin_status_string.argtypes = [C.c_int]
@@ -130,6 +133,11 @@ def _need(t: torch.Tensor, name: str, dtype, device=None):
         raise ValueError(f"{name} must be on {device}")
 
 
+def test_stall_tensor_core_waits(enable: bool) -> None:
+    """Failure-detection test hook (see spin_test_stall_tensor_core_waits)."""
+    lib().spin_test_stall_tensor_core_waits(1 if enable else 0)
+
+
 def device_status(reset: bool = False) -> int:
     """Device status word (nonzero: a kernel gave up on an internal wait)."""
     v = C.c_uint32(0)
@@ -139,7 +147,8 @@ def device_status(reset: bool = False) -> int:
 
 def hadamard_quant_int4(x: torch.Tensor, clip: float = 1.0, signs: torch.Tensor | None = None,
                         no_rotate: bool = False, out: torch.Tensor | None = None,
-                        scales: torch.Tensor | None = None, stream=None, cuda_cores_only: bool = False):
+                        scales: torch.Tensor | None = None, stream=None, cuda_cores_only: bool = False,
+                        tensor_cores: bool = False):
     """R4: x [tokens, n] bf16 (CUDA) -> (codes [tokens, n/2] uint8, scales [tokens] fp32)."""
     _need(x, "x", torch.bfloat16)
     tokens, n = x.shape
@@ -149,7 +158,8 @@ def hadamard_quant_int4(x: torch.Tensor, clip: float = 1.0, signs: torch.Tensor 
         scales = torch.empty((tokens,), dtype=torch.float32, device=x.device)
     if signs is not None:
         _need(signs, "signs", torch.int32, x.device)
-    flags = (NO_ROTATE if no_rotate else 0) | (CUDA_CORES_ONLY if cuda_cores_only else 0)
+    flags = ((NO_ROTATE if no_rotate else 0) | (CUDA_CORES_ONLY if cuda_cores_only else 0) |
+             (TENSOR_CORES if tensor_cores else 0))
     st = spin_hadamard_quant_int4_ex(_ptr(x), tokens, n, float(clip), _ptr(signs), flags,
                                      _ptr(out), _ptr(scales), _stream(stream))
     _check("spin_hadamard_quant_int4_ex", st)

@@ -104,7 +104,8 @@ spin_status_t spin_hadamard_quant_int4_ex(const void *x_bf16, int64_t tokens, in
                                           spin_stream_t stream) {
   const int log_n = log2_pow2(n);
   if (log_n < 7 || log_n > 15) return SPIN_ERR_UNSUPPORTED_SIZE;
-  if (tokens < 0 || !valid_clip(clip) || (flags & ~(SPIN_NO_ROTATE | SPIN_CUDA_CORES_ONLY)) != 0)
+  if (tokens < 0 || !valid_clip(clip) || (flags & ~(SPIN_NO_ROTATE | SPIN_CUDA_CORES_ONLY | SPIN_TENSOR_CORES)) != 0 ||
+      (flags & SPIN_CUDA_CORES_ONLY && flags & SPIN_TENSOR_CORES))
     return SPIN_ERR_INVALID_ARG;
   if (tokens == 0) return SPIN_OK;
   if (!x_bf16 || !q_packed_u8 || !scales_f32) return SPIN_ERR_INVALID_ARG;
@@ -170,6 +171,8 @@ spin_status_t spin_dequant_hadamard_inverse(const uint8_t *codes, int64_t rows, 
   return cuda_status(launch_dequant_inverse(codes, rows, log_n, mode, scale, zero, sign_bits, flags, out,
                                             out_dtype, reinterpret_cast<cudaStream_t>(stream)));
 }
+
+void spin_test_stall_tensor_core_waits(int enable) { set_stall_test(enable); }
 
 const char *spin_status_string(spin_status_t status) {
   switch (status) {

@@ -209,7 +209,7 @@ cudaError_t launch_rotate_quant_int4(const void *x, int64_t tokens, int log_n, f
                                      cudaStream_t stream) {
   if (!(flags & kCudaCoresOnly) && tc_rotate_quant_supported(log_n, tokens, flags))
     return launch_rotate_quant_int4_tc(log_n, x, tokens, clip, signs, q, scales, stream);
-  flags &= ~kCudaCoresOnly;
+  flags &= ~(kCudaCoresOnly | kTensorCores);
   switch (log_n) {
     case 7: return launch_n<7>(x, tokens, clip, signs, flags, q, scales, stream);
     case 8: return launch_n<8>(x, tokens, clip, signs, flags, q, scales, stream);

@@ -39,6 +39,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -62,6 +63,7 @@ constexpr uint32_t kOffX = 32768;                  // ring of kStages x 64 KiB
 constexpr uint32_t kOffBar = kOffX + kStages * kGroupBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;  // + alignment slack
 constexpr long long kTimeoutCycles = 4000000000LL;     // about two seconds
+constexpr long long kStallTestCycles = 2000000LL;      // about a millisecond, for the stall test hook
 
 // Shape constants for n = 2^LOGN.
 template <int LOGN>
@@ -86,6 +88,7 @@ struct Shared {
   uint32_t tmem_base;
   int abort;
   int dec[3];
+  long long budget;        // clock cycles a wait may take before the CTA gives up
   float wmax[2][2][4][4];  // [warpgroup][group parity][warp][token segment]
 };
 static_assert(sizeof(Shared) <= 512, "barrier area");
@@ -96,7 +99,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, Sha
   while (true) {
     if (tc::mbar_try_wait(bar, parity)) return true;
     if (honor_abort && *reinterpret_cast<volatile int *>(&S.abort)) return false;
-    if (clock64() - t0 > kTimeoutCycles) {
+    if (clock64() - t0 > S.budget) {
       *reinterpret_cast<volatile int *>(&S.abort) = 1;
       atomicOr(&g_device_status, 1u);
       return false;
@@ -156,7 +159,8 @@ __device__ __forceinline__ void load_group(uint8_t *dst, const CUtensorMap *map,
 template <int LOGN, bool SIGNS, bool STORE32>
 __global__ void __launch_bounds__(kThreads, 1)
     k1_tc_rotate_quant(const __grid_constant__ CUtensorMap xmap, int64_t tokens, float clip, float inv_sqrt_n,
-                       const uint32_t *__restrict__ signs, uint8_t *__restrict__ q, float *__restrict__ scales) {
+                       const uint32_t *__restrict__ signs, uint8_t *__restrict__ q, float *__restrict__ scales,
+                       int stall_test) {
   using SH = Shape<LOGN>;
   constexpr int B = SH::B, SEG = SH::SEG;
   extern __shared__ uint8_t smem_raw[];
@@ -182,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc::mbar_init(&S.drain, 1);
     S.abort = 0;
+    S.budget = stall_test ? kStallTestCycles : kTimeoutCycles;
     tc::fence_barrier_init();
     tc::prefetch_tensormap(&xmap);
     // The first kStages groups need no free slot: start their copies now, so the
@@ -255,7 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::umma_bf16(tmem + acc * 256, ad, bd, idesc, s > 0 ? 1u : 0u);
         }
         tc::umma_commit(&S.empty[st]);
-        tc::umma_commit(&S.tfull[acc]);
+        // Stall test hook: withhold the first group's completion signal, so the
+        // epilogue's wait runs out and the CTA takes its abort path.
+        if (!(stall_test && i == 0)) tc::umma_commit(&S.tfull[acc]);
       }
     }
   } else if (warp < 4) {
@@ -419,7 +426,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int LOGN, bool SIGNS, bool STORE32>
 cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, int stall_test) {
   using SH = Shape<LOGN>;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
@@ -450,36 +457,47 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, map, tokens, clip, inv_sqrt_n, signs, q, scales);
+  return cudaLaunchKernelEx(&cfg, kern, map, tokens, clip, inv_sqrt_n, signs, q, scales, stall_test);
 }
 
 template <int LOGN>
 cudaError_t launch_n(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, int stall_test) {
   const bool a32 = (reinterpret_cast<uintptr_t>(q) & 31u) == 0;  // 32-byte stores need 32-byte alignment
   if (signs) {
-    return a32 ? launch_tc<LOGN, true, true>(x, tokens, clip, signs, q, scales, stream)
-               : launch_tc<LOGN, true, false>(x, tokens, clip, signs, q, scales, stream);
+    return a32 ? launch_tc<LOGN, true, true>(x, tokens, clip, signs, q, scales, stream, stall_test)
+               : launch_tc<LOGN, true, false>(x, tokens, clip, signs, q, scales, stream, stall_test);
   }
-  return a32 ? launch_tc<LOGN, false, true>(x, tokens, clip, nullptr, q, scales, stream)
-             : launch_tc<LOGN, false, false>(x, tokens, clip, nullptr, q, scales, stream);
+  return a32 ? launch_tc<LOGN, false, true>(x, tokens, clip, nullptr, q, scales, stream, stall_test)
+             : launch_tc<LOGN, false, false>(x, tokens, clip, nullptr, q, scales, stream, stall_test);
 }
+
+std::atomic<int> g_stall_test{0};
 
 }  // namespace
 
+// The tensor-core kernel pays a per-CTA setup (H tile, TMEM, first copies) that
+// only pays off with at least about one MMA group per SM; smaller batches (decode)
+// go to the CUDA-core kernel, which needs no setup.
 bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags) {
-  return log_n >= 12 && log_n <= 14 && !(flags & kNoRotate) && tokens > 0 && tokens * 128 < (int64_t(1) << 31);
+  if (log_n < 12 || log_n > 14 || (flags & kNoRotate) || tokens <= 0 || tokens * 128 >= (int64_t(1) << 31))
+    return false;
+  const int64_t tok_per_group = int64_t(256) >> (log_n - 7);
+  return (flags & kTensorCores) || tokens >= 128 * tok_per_group;
 }
 
 cudaError_t launch_rotate_quant_int4_tc(int log_n, const void *x, int64_t tokens, float clip, const uint32_t *signs,
                                         uint8_t *q, float *scales, cudaStream_t stream) {
+  const int stall = g_stall_test.load(std::memory_order_relaxed);
   switch (log_n) {
-    case 12: return launch_n<12>(x, tokens, clip, signs, q, scales, stream);
-    case 13: return launch_n<13>(x, tokens, clip, signs, q, scales, stream);
-    case 14: return launch_n<14>(x, tokens, clip, signs, q, scales, stream);
+    case 12: return launch_n<12>(x, tokens, clip, signs, q, scales, stream, stall);
+    case 13: return launch_n<13>(x, tokens, clip, signs, q, scales, stream, stall);
+    case 14: return launch_n<14>(x, tokens, clip, signs, q, scales, stream, stall);
     default: return cudaErrorInvalidValue;
   }
 }
+
+void set_stall_test(int enable) { g_stall_test.store(enable ? 1 : 0, std::memory_order_relaxed); }
 
 cudaError_t read_device_status(unsigned int *status, bool reset) {
   cudaError_t e = cudaMemcpyFromSymbol(status, g_device_status, sizeof(unsigned int));

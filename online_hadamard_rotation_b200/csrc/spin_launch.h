@@ -9,6 +9,7 @@ namespace spin {
 
 constexpr uint32_t kNoRotate = 1u;        // same value as SPIN_NO_ROTATE
 constexpr uint32_t kCudaCoresOnly = 2u;   // same value as SPIN_CUDA_CORES_ONLY
+constexpr uint32_t kTensorCores = 4u;     // same value as SPIN_TENSOR_CORES
 
 // Number of blocks of `kernel` that are resident on the current device at once
 // (SM count x blocks per SM), with the dynamic shared-memory opt-in applied.
@@ -23,6 +24,9 @@ cudaError_t launch_rotate_quant_int4(const void *x, int64_t tokens, int log_n, f
 bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags);
 cudaError_t launch_rotate_quant_int4_tc(int log_n, const void *x, int64_t tokens, float clip, const uint32_t *signs,
                                         uint8_t *q, float *scales, cudaStream_t stream);
+
+// Test hook: make the tensor-core R4 kernel withhold one internal signal.
+void set_stall_test(int enable);
 
 // Device status word set by kernels whose bounded waits ran out.
 cudaError_t read_device_status(unsigned int *status, bool reset);

@@ -60,7 +60,8 @@ def test_r4_argument_checks(L):
     assert L.spin_hadamard_quant_int4(FAKE, 4, 256, 1.0, FAKE + 8, FAKE, None) == 3
     assert L.spin_hadamard_quant_int4(FAKE, 4, 256, 1.0, FAKE, FAKE + 1, None) == 3
     assert L.spin_hadamard_quant_int4_ex(FAKE, 4, 256, 1.0, FAKE + 2, 0, FAKE, FAKE, None) == 3
-    assert L.spin_hadamard_quant_int4_ex(FAKE, 4, 256, 1.0, None, 4, FAKE, FAKE, None) == 1
+    assert L.spin_hadamard_quant_int4_ex(FAKE, 4, 256, 1.0, None, 8, FAKE, FAKE, None) == 1
+    assert L.spin_hadamard_quant_int4_ex(FAKE, 4, 256, 1.0, None, 6, FAKE, FAKE, None) == 1  # both kernel choices
 
 
 def _r3(L, **kw):

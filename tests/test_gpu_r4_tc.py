@@ -16,7 +16,8 @@ SIZES = [4096, 8192, 16384]
 
 
 def run(spin, bits, clip, signs, cores_only=False):
-    q, s = spin.hadamard_quant_int4(to_dev_bf16(bits), clip, to_dev_signs(signs), cuda_cores_only=cores_only)
+    q, s = spin.hadamard_quant_int4(to_dev_bf16(bits), clip, to_dev_signs(signs), cuda_cores_only=cores_only,
+                                    tensor_cores=not cores_only)
     torch.cuda.synchronize()
     return q.cpu().numpy(), s.cpu().numpy()
 
@@ -76,7 +77,7 @@ def test_tc_leaves_tail_untouched(spin_gpu, N):
     bits = synthetic.r4_prefill(tokens=5, n=N, seed=3)[0]
     out = torch.full((8, N // 2), 0xA5, dtype=torch.uint8, device="cuda")
     sc = torch.full((8,), -1.0, dtype=torch.float32, device="cuda")
-    spin_gpu.hadamard_quant_int4(to_dev_bf16(bits), 1.0, out=out[:5], scales=sc[:5])
+    spin_gpu.hadamard_quant_int4(to_dev_bf16(bits), 1.0, out=out[:5], scales=sc[:5], tensor_cores=True)
     torch.cuda.synchronize()
     assert torch.all(out[5:] == 0xA5) and torch.all(sc[5:] == -1.0)
     assert torch.all(sc[:5] > 0)
