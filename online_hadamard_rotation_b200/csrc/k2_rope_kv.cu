@@ -35,7 +35,7 @@ namespace {
 
 constexpr int kD = 128;          // head dim handled by this kernel
 constexpr int kRowBytes = kD * 2;
-constexpr float kMagic = 12582912.0f;
+constexpr double kInvSqrtD = 0.08838834764831845;  // 1/sqrt(128)
 
 __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   float r;
@@ -77,17 +77,51 @@ __device__ __forceinline__ void fwht128(float (&x)[kD]) {
   }
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// (r0, r1) = bit patterns of fma(a, 15, 1.5 * 2^23) for a pair: one packed FMA rounds two
+// scaled codes to integers (ties to even) in their low mantissa bits.
+__device__ __forceinline__ void round15_x2(float a0, float a1, uint32_t &r0, uint32_t &r1) {
+  uint64_t A, R;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(R) : "l"(A), "l"(0x4170000041700000ull), "l"(0x4B4000004B400000ull));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(R));
+}
+
 // Asymmetric INT4 of one group of 128 values; writes 64 bytes of codes and the
 // fp16 scale and zero.
 __device__ __forceinline__ void quant_asym_store(const float (&x)[kD], float clip, uint8_t *codes_dst,
                                                  __half *scale_dst, __half *zero_dst) {
-  float mn = x[0], mx = x[0];
+  float mn[8], mx[8];
 #pragma unroll
-  for (int i = 1; i < kD; ++i) {
-    mn = fminf(mn, x[i]);
-    mx = fmaxf(mx, x[i]);
+  for (int k = 0; k < 8; ++k) {
+    mn[k] = fmin3(x[16 * k], x[16 * k + 1], x[16 * k + 2]);
+    mx[k] = fmax3(x[16 * k], x[16 * k + 1], x[16 * k + 2]);
+#pragma unroll
+    for (int j = 3; j < 15; j += 2) {
+      mn[k] = fmin3(mn[k], x[16 * k + j], x[16 * k + j + 1]);
+      mx[k] = fmax3(mx[k], x[16 * k + j], x[16 * k + j + 1]);
+    }
+    mn[k] = fminf(mn[k], x[16 * k + 15]);
+    mx[k] = fmaxf(mx[k], x[16 * k + 15]);
   }
-  const float lo = fminf(clip * mn, 0.f), hi = fmaxf(clip * mx, 0.f);
+#pragma unroll
+  for (int h = 4; h >= 1; h >>= 1)
+#pragma unroll
+    for (int k = 0; k < h; ++k) {
+      mn[k] = fminf(mn[k], mn[k + h]);
+      mx[k] = fmaxf(mx[k], mx[k + h]);
+    }
+  const float lo = fminf(clip * mn[0], 0.f), hi = fmaxf(clip * mx[0], 0.f);
   __half s16 = __float2half_rn((hi - lo) / 15.0f);
   float s = __half2float(s16), z = 0.f;
   if (s == 0.f) {
@@ -97,21 +131,25 @@ __device__ __forceinline__ void quant_asym_store(const float (&x)[kD], float cli
     z = fminf(fmaxf(rintf(-lo / s), 0.f), 15.f);
   }
   const float c15 = (1.0f / s) / 15.0f, z15 = z / 15.0f;
-  uint32_t words[16];
-#pragma unroll
-  for (int w = 0; w < 16; ++w) {
-    uint32_t b[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      b[i] = __float_as_uint(fmaf(fma_sat(x[8 * w + i], c15, z15), 15.0f, kMagic));
-    const uint32_t e = __byte_perm(__byte_perm(b[0], b[2], 0x0040), __byte_perm(b[4], b[6], 0x0040), 0x5410);
-    const uint32_t o = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
-    words[w] = e | (o << 4);
-  }
   uint4 *dst = reinterpret_cast<uint4 *>(codes_dst);
 #pragma unroll
-  for (int k = 0; k < 4; ++k)
-    __stcs(dst + k, make_uint4(words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]));
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint32_t words[4];
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+      const int w = 4 * q4 + wi;
+      uint32_t b[8];
+      float t[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) t[i] = fma_sat(x[8 * w + i], c15, z15);
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) round15_x2(t[i], t[i + 1], b[i], b[i + 1]);
+      const uint32_t e = __byte_perm(__byte_perm(b[0], b[2], 0x0040), __byte_perm(b[4], b[6], 0x0040), 0x5410);
+      const uint32_t o = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
+      words[wi] = e | (o << 4);
+    }
+    __stcs(dst + q4, make_uint4(words[0], words[1], words[2], words[3]));
+  }
   *scale_dst = s16;
   *zero_dst = __float2half_rn(z);
 }
@@ -128,7 +166,7 @@ struct K2Args {
   double theta;
 };
 
-__global__ void __launch_bounds__(256) k2_rope_hadamard_kvquant(K2Args a) {
+__global__ void __launch_bounds__(192, 2) k2_rope_hadamard_kvquant(K2Args a) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int rows_tok = a.hq + 2 * a.hkv;
   const int G = a.tok_per_group;
@@ -174,7 +212,8 @@ __global__ void __launch_bounds__(256) k2_rope_hadamard_kvquant(K2Args a) {
       const double ang = (double)a.pos[tok0 + tk] * inv_freq[p];
       double sn, cs;
       sincos(ang, &sn, &cs);
-      table[b][tk * (kD / 2) + p] = make_float2((float)cs, (float)sn);
+      // 1/sqrt(d) of the rotation is folded into the angle's cosine and sine
+      table[b][tk * (kD / 2) + p] = make_float2((float)(cs * kInvSqrtD), (float)(sn * kInvSqrtD));
     }
   };
 
@@ -230,8 +269,6 @@ __global__ void __launch_bounds__(256) k2_rope_hadamard_kvquant(K2Args a) {
           x[p + kD / 2] = fmaf(x1, e.x, x0 * e.y);
         }
         fwht128(x);
-#pragma unroll
-        for (int i = 0; i < kD; ++i) x[i] *= a.inv_sqrt_d;
       }
       if (kind == 0) {
 #pragma unroll
@@ -273,9 +310,9 @@ cudaError_t launch_rope_hadamard_kvquant(const void *q, const void *k, const voi
                                          int cache_offset, cudaStream_t stream) {
   const int rows_tok = n_q_heads + 2 * n_kv_heads;
   int G = 1;
-  while (G < 8 && 2 * G * rows_tok <= 256) G *= 2;  // tokens per group: at most 256 head vectors
+  while (G < 8 && 2 * G * rows_tok <= 192) G *= 2;  // tokens per group: at most 192 head vectors
   const int rows = G * rows_tok;
-  int threads = rows < 256 ? ((rows + 31) / 32) * 32 : 256;
+  int threads = rows < 192 ? ((rows + 31) / 32) * 32 : 192;
   const size_t smem = 2 * (size_t)rows * kRowBytes + 2 * (size_t)G * (kD / 2) * sizeof(float2) +
                       (kD / 2) * sizeof(double);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
