@@ -8,17 +8,19 @@
 // Compatibility with 4-Bit KV Caching": RoPE rotates 2-D coordinate pairs and
 // the KV cache is stored as 4-bit integers.
 //
-// One thread owns one head vector (d = 128 values) end to end, so RoPE's pair
-// partners (p, p + 64), all seven butterfly stages and the group min/max are
-// in its registers. Head vectors reach shared memory through 16-byte
+// Two neighbouring threads own one head vector (d = 128 values): thread h of
+// the pair holds elements (p + 32 h, p + 32 h + 64) for p < 32, so RoPE's pair
+// partners (p, p + 64) and six of the seven butterfly stages stay in its
+// registers, and the stage over element bit 5 is one shuffle with the partner
+// lane; the group min/max combine with one more. Head vectors reach shared memory through 16-byte
 // cp.async copies that are coalesced in global memory; inside a 256-byte smem
 // row the 16-byte chunk c sits at c ^ (row & 7), so eight threads reading
 // chunk c of eight consecutive rows hit eight different bank groups. The
 // copies for the next group of tokens are in flight while the current group
 // is computed (two buffers).
 //
-// Q: out = bf16(H RoPE(q) / sqrt(d)), written back into the smem row and then
-// copied out with coalesced 16-byte stores. K: H RoPE(k) / sqrt(d), V: v, each
+// Q: out = bf16(H RoPE(q) / sqrt(d)), stored from registers (each thread writes
+// four 16-byte pieces of its head row). K: H RoPE(k) / sqrt(d), V: v, each
 // quantised asymmetrically per (token, kv head) group and written straight to
 // its cache row (64 bytes) with fp16 scale and zero.
 #include <cuda_fp16.h>
@@ -35,7 +37,11 @@ namespace {
 
 constexpr int kD = 128;          // head dim handled by this kernel
 constexpr int kRowBytes = kD * 2;
-constexpr double kInvSqrtD = 0.08838834764831845;  // 1/sqrt(128)
+constexpr float kInvSqrtDf = 0.0883883476f;         // 1/sqrt(128)
+constexpr int kTabStride = kD / 2 + 2;               // float2 entries per token in the RoPE table
+constexpr double kInv2Pi = 0.15915494309189535;     // 1 / (2 pi)
+constexpr double k2PiHi = 6.283185307179586;        // 2 pi rounded to double
+constexpr double k2PiLo = 2.4492935982947064e-16;   // 2 pi - k2PiHi
 
 __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   float r;
@@ -59,21 +65,32 @@ __device__ __forceinline__ uint32_t chunk_off(uint32_t r, uint32_t c) {
   return r * kRowBytes + ((c ^ (r & 7u)) << 4);
 }
 
-// 7 butterfly stages of H_128 over the register index.
-__device__ __forceinline__ void fwht128(float (&x)[kD]) {
+constexpr int kHalf = 64;  // values per thread
+
+// H_128 on a head vector split over a lane pair. Register j of half h holds
+// element (j & 31) + 32 h + 64 (j >> 5): register bits 0-4 are element bits
+// 0-4, register bit 5 is element bit 6, and element bit 5 is the lane pair.
+__device__ __forceinline__ void fwht128_pair(float (&x)[kHalf], uint32_t h, unsigned pair_mask) {
 #pragma unroll
-  for (int i = 0; i < kD; i += 2) {
+  for (int i = 0; i < kHalf; i += 2) {
     const float a = x[i], b = x[i + 1];
     x[i] = a + b;
     x[i + 1] = a - b;
   }
 #pragma unroll
-  for (int h = 2; h < kD; h <<= 1) {
+  for (int st = 2; st < kHalf; st <<= 1) {
 #pragma unroll
-    for (int i = 0; i < kD; i += 2) {
-      if (i & h) continue;
-      bfly2(x[i], x[i + 1], x[i + h], x[i + h + 1]);
+    for (int i = 0; i < kHalf; i += 2) {
+      if (i & st) continue;
+      bfly2(x[i], x[i + 1], x[i + st], x[i + st + 1]);
     }
+  }
+  // element bit 5: (a, b) -> (a + b, a - b) with a on half 0 and b on half 1
+  const float sgn = h ? -1.0f : 1.0f;
+#pragma unroll
+  for (int i = 0; i < kHalf; ++i) {
+    const float w = __shfl_xor_sync(pair_mask, x[i], 1);
+    x[i] = fmaf(x[i], sgn, w);
   }
 }
 
@@ -97,13 +114,15 @@ __device__ __forceinline__ void round15_x2(float a0, float a1, uint32_t &r0, uin
   asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(R));
 }
 
-// Asymmetric INT4 of one group of 128 values; writes 64 bytes of codes and the
+// Asymmetric INT4 of one group of 128 values held by a lane pair (64 each, in
+// the split of fwht128_pair); each thread writes its 32 code bytes, half 0 the
 // fp16 scale and zero.
-__device__ __forceinline__ void quant_asym_store(const float (&x)[kD], float clip, uint8_t *codes_dst,
-                                                 __half *scale_dst, __half *zero_dst) {
-  float mn[8], mx[8];
+__device__ __forceinline__ void quant_asym_store_pair(const float (&x)[kHalf], float clip, uint32_t h,
+                                                      unsigned pair_mask, uint8_t *codes_row, __half *scale_dst,
+                                                      __half *zero_dst) {
+  float mn[4], mx[4];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
+  for (int k = 0; k < 4; ++k) {
     mn[k] = fmin3(x[16 * k], x[16 * k + 1], x[16 * k + 2]);
     mx[k] = fmax3(x[16 * k], x[16 * k + 1], x[16 * k + 2]);
 #pragma unroll
@@ -114,14 +133,11 @@ __device__ __forceinline__ void quant_asym_store(const float (&x)[kD], float cli
     mn[k] = fminf(mn[k], x[16 * k + 15]);
     mx[k] = fmaxf(mx[k], x[16 * k + 15]);
   }
-#pragma unroll
-  for (int h = 4; h >= 1; h >>= 1)
-#pragma unroll
-    for (int k = 0; k < h; ++k) {
-      mn[k] = fminf(mn[k], mn[k + h]);
-      mx[k] = fmaxf(mx[k], mx[k + h]);
-    }
-  const float lo = fminf(clip * mn[0], 0.f), hi = fmaxf(clip * mx[0], 0.f);
+  float vmn = fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3]));
+  float vmx = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+  vmn = fminf(vmn, __shfl_xor_sync(pair_mask, vmn, 1));
+  vmx = fmaxf(vmx, __shfl_xor_sync(pair_mask, vmx, 1));
+  const float lo = fminf(clip * vmn, 0.f), hi = fmaxf(clip * vmx, 0.f);
   __half s16 = __float2half_rn((hi - lo) / 15.0f);
   float s = __half2float(s16), z = 0.f;
   if (s == 0.f) {
@@ -131,13 +147,12 @@ __device__ __forceinline__ void quant_asym_store(const float (&x)[kD], float cli
     z = fminf(fmaxf(rintf(-lo / s), 0.f), 15.f);
   }
   const float c15 = (1.0f / s) / 15.0f, z15 = z / 15.0f;
-  uint4 *dst = reinterpret_cast<uint4 *>(codes_dst);
 #pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
+  for (int q = 0; q < 2; ++q) {  // registers 32 q .. 32 q + 31 -> code bytes 32 q + 16 h .. + 15
     uint32_t words[4];
 #pragma unroll
     for (int wi = 0; wi < 4; ++wi) {
-      const int w = 4 * q4 + wi;
+      const int w = 4 * q + wi;
       uint32_t b[8];
       float t[8];
 #pragma unroll
@@ -148,10 +163,12 @@ __device__ __forceinline__ void quant_asym_store(const float (&x)[kD], float cli
       const uint32_t o = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
       words[wi] = e | (o << 4);
     }
-    __stcs(dst + q4, make_uint4(words[0], words[1], words[2], words[3]));
+    __stcs(reinterpret_cast<uint4 *>(codes_row + 32 * q + 16 * h), make_uint4(words[0], words[1], words[2], words[3]));
   }
-  *scale_dst = s16;
-  *zero_dst = __float2half_rn(z);
+  if (h == 0) {
+    *scale_dst = s16;
+    *zero_dst = __float2half_rn(z);
+  }
 }
 
 struct K2Args {
@@ -166,7 +183,7 @@ struct K2Args {
   double theta;
 };
 
-__global__ void __launch_bounds__(192, 2) k2_rope_hadamard_kvquant(K2Args a) {
+__global__ void __launch_bounds__(192, 3) k2_rope_hadamard_kvquant(K2Args a) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int rows_tok = a.hq + 2 * a.hkv;
   const int G = a.tok_per_group;
@@ -174,8 +191,8 @@ __global__ void __launch_bounds__(192, 2) k2_rope_hadamard_kvquant(K2Args a) {
   uint8_t *stage[2] = {smem, smem + (size_t)rows * kRowBytes};
   float2 *table[2];
   table[0] = reinterpret_cast<float2 *>(smem + 2 * (size_t)rows * kRowBytes);
-  table[1] = table[0] + G * (kD / 2);
-  double *inv_freq = reinterpret_cast<double *>(table[1] + G * (kD / 2));
+  table[1] = table[0] + G * kTabStride;
+  double *inv_freq = reinterpret_cast<double *>(table[1] + G * kTabStride);
 
   const int t = threadIdx.x, nt = blockDim.x;
   const int64_t ngroups = (a.ntok + G - 1) / G;
@@ -209,11 +226,18 @@ __global__ void __launch_bounds__(192, 2) k2_rope_hadamard_kvquant(K2Args a) {
     cp_async_commit();
     for (int i = t; i < ntk * (kD / 2); i += nt) {
       const int tk = i / (kD / 2), p = i % (kD / 2);
+      // angle pos * theta^(-2p/d) in fp64, reduced to [-pi, pi] by Cody-Waite
+      // (2 pi split into a head and a tail, each multiple subtracted with an FMA),
+      // then the fp32 sine and cosine of the reduced angle
       const double ang = (double)a.pos[tok0 + tk] * inv_freq[p];
-      double sn, cs;
-      sincos(ang, &sn, &cs);
-      // 1/sqrt(d) of the rotation is folded into the angle's cosine and sine
-      table[b][tk * (kD / 2) + p] = make_float2((float)(cs * kInvSqrtD), (float)(sn * kInvSqrtD));
+      const double k = rint(ang * kInv2Pi);
+      const double red = fma(-k, k2PiLo, fma(-k, k2PiHi, ang));
+      float sn, cs;
+      sincosf((float)red, &sn, &cs);
+      // 1/sqrt(d) of the rotation is folded into the angle's cosine and sine. Layout
+      // [token][j][half] (p = 32 half + j) with a padded token stride, so the two
+      // threads of a pair and neighbouring tokens read different banks.
+      table[b][tk * kTabStride + 2 * (p & 31) + (p >> 5)] = make_float2(cs * kInvSqrtDf, sn * kInvSqrtDf);
     }
   };
 
@@ -233,12 +257,15 @@ __global__ void __launch_bounds__(192, 2) k2_rope_hadamard_kvquant(K2Args a) {
     uint8_t *sb = stage[buf];
     const float2 *tb = table[buf];
 
-    for (int r = t; r < rows; r += nt) {
+    for (int rh = t; rh < 2 * rows; rh += nt) {
+      const int r = rh >> 1;
+      const uint32_t hf = (uint32_t)rh & 1u;               // which half of the head vector
+      const unsigned pm = 3u << ((threadIdx.x & 31u) & ~1u);  // this lane pair
       int kind, tk, h;
       if (r < G * a.hq) {
         kind = 0; tk = r / a.hq; h = r % a.hq;
       } else if (r < G * (a.hq + a.hkv)) {
-        // thread order (head, token) so neighbouring threads write neighbouring cache slots
+        // row order (head, token) so neighbouring rows write neighbouring cache slots
         const int i = r - G * a.hq;
         kind = 1; h = i / G; tk = i % G;
       } else {
@@ -247,10 +274,11 @@ __global__ void __launch_bounds__(192, 2) k2_rope_hadamard_kvquant(K2Args a) {
       }
       if (tk >= ntk) continue;
       const int sr = kind == 0 ? tk * a.hq + h : G * a.hq + (kind == 2 ? G * a.hkv : 0) + tk * a.hkv + h;
-      float x[kD];
+      float x[kHalf];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const uint4 w = *reinterpret_cast<const uint4 *>(sb + chunk_off(sr, c));
+      for (int c = 0; c < 8; ++c) {  // chunks 4 hf .. 4 hf + 3 and 8 + 4 hf .. 8 + 4 hf + 3
+        const uint32_t chunk = (c & 3u) + 4u * hf + 8u * (c >> 2);
+        const uint4 w = *reinterpret_cast<const uint4 *>(sb + chunk_off(sr, chunk));
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -260,40 +288,35 @@ __global__ void __launch_bounds__(192, 2) k2_rope_hadamard_kvquant(K2Args a) {
       }
       const int64_t tok = tok0 + tk;
       if (kind != 2) {
-        const float2 *cs = tb + tk * (kD / 2);
+        const float2 *cs = tb + tk * kTabStride + hf;
 #pragma unroll
-        for (int p = 0; p < kD / 2; ++p) {
-          const float2 e = cs[p];
-          const float x0 = x[p], x1 = x[p + kD / 2];
-          x[p] = fmaf(x0, e.x, -x1 * e.y);
-          x[p + kD / 2] = fmaf(x1, e.x, x0 * e.y);
+        for (int j = 0; j < 32; ++j) {  // pair (p, p + 64) with p = 32 hf + j
+          const float2 e = cs[2 * j];
+          const float x0 = x[j], x1 = x[j + 32];
+          x[j] = fmaf(x0, e.x, -x1 * e.y);
+          x[j + 32] = fmaf(x1, e.x, x0 * e.y);
         }
-        fwht128(x);
+        fwht128_pair(x, hf, pm);
       }
       if (kind == 0) {
+        // rotated Q straight to global memory: registers 0-31 are bytes 64 hf .. 64 hf + 63
+        // of the head row, registers 32-63 bytes 128 + 64 hf .. 128 + 64 hf + 63
+        uint4 *qrow = reinterpret_cast<uint4 *>(a.q_out + (tok * a.hq + h) * kD);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint4 w = make_uint4(pack_bf16x2(x[8 * c], x[8 * c + 1]), pack_bf16x2(x[8 * c + 2], x[8 * c + 3]),
-                                     pack_bf16x2(x[8 * c + 4], x[8 * c + 5]),
-                                     pack_bf16x2(x[8 * c + 6], x[8 * c + 7]));
-          *reinterpret_cast<uint4 *>(sb + chunk_off(sr, c)) = w;
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t chunk = (c & 3u) + 4u * hf + 8u * (c >> 2);
+          __stcs(qrow + chunk, make_uint4(pack_bf16x2(x[8 * c], x[8 * c + 1]), pack_bf16x2(x[8 * c + 2], x[8 * c + 3]),
+                                          pack_bf16x2(x[8 * c + 4], x[8 * c + 5]),
+                                          pack_bf16x2(x[8 * c + 6], x[8 * c + 7])));
         }
       } else {
         const int64_t b = tok / a.seq, s = tok % a.seq;
         const int64_t crow = (b * a.hkv + h) * (int64_t)a.cache_len + a.cache_offset + s;
         if (kind == 1)
-          quant_asym_store(x, a.clip, a.k_cache + crow * (kD / 2), a.k_scale + crow, a.k_zero + crow);
+          quant_asym_store_pair(x, a.clip, hf, pm, a.k_cache + crow * (kD / 2), a.k_scale + crow, a.k_zero + crow);
         else
-          quant_asym_store(x, a.clip, a.v_cache + crow * (kD / 2), a.v_scale + crow, a.v_zero + crow);
+          quant_asym_store_pair(x, a.clip, hf, pm, a.v_cache + crow * (kD / 2), a.v_scale + crow, a.v_zero + crow);
       }
-    }
-    __syncthreads();
-    // rotated Q rows: smem -> q_out, coalesced
-    const int qchunks = ntk * a.hq * 16;
-    uint4 *qo = reinterpret_cast<uint4 *>(a.q_out + tok0 * a.hq * kD);
-    for (int i = t; i < qchunks; i += nt) {
-      const int r = i >> 4, c = i & 15;
-      __stcs(qo + i, *reinterpret_cast<const uint4 *>(sb + chunk_off(r, c)));
     }
   }
   cp_async_wait_1();
@@ -310,10 +333,10 @@ cudaError_t launch_rope_hadamard_kvquant(const void *q, const void *k, const voi
                                          int cache_offset, cudaStream_t stream) {
   const int rows_tok = n_q_heads + 2 * n_kv_heads;
   int G = 1;
-  while (G < 8 && 2 * G * rows_tok <= 192) G *= 2;  // tokens per group: at most 192 head vectors
+  while (G < 8 && 2 * G * rows_tok <= 96) G *= 2;  // tokens per group: at most 96 head vectors
   const int rows = G * rows_tok;
-  int threads = rows < 192 ? ((rows + 31) / 32) * 32 : 192;
-  const size_t smem = 2 * (size_t)rows * kRowBytes + 2 * (size_t)G * (kD / 2) * sizeof(float2) +
+  int threads = 2 * rows < 192 ? ((2 * rows + 31) / 32) * 32 : 192;  // two threads per head vector
+  const size_t smem = 2 * (size_t)rows * kRowBytes + 2 * (size_t)G * kTabStride * sizeof(float2) +
                       (kD / 2) * sizeof(double);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   int slots = 0;
