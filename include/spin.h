@@ -154,7 +154,9 @@ spin_status_t spin_hadamard_quant_int4_ex(const void *x_bf16, int64_t tokens, in
  *  pos          [batch, seq] int32 RoPE positions (>= 0)
  *  theta        RoPE base (> 0), e.g. 10000
  *  head_dim     128 (power of two; other sizes return SPIN_ERR_UNSUPPORTED_SIZE)
- *  batch, seq   > 0 (0 is a no-op); n_q_heads, n_kv_heads > 0, n_q_heads % n_kv_heads == 0
+ *  batch, seq   > 0 (0 is a no-op); n_q_heads, n_kv_heads > 0, n_q_heads % n_kv_heads == 0;
+ *               n_q_heads <= 256, n_q_heads + 2 n_kv_heads <= 384 and
+ *               batch * seq * n_q_heads < 2^31, else SPIN_ERR_UNSUPPORTED_SIZE
  *  clip         0 < clip <= 1
  *  q_out        [batch, seq, n_q_heads, head_dim] bf16, 16-byte aligned; may equal q
  *  k_cache, v_cache  [batch, n_kv_heads, cache_len, head_dim/2] bytes, 16-byte aligned

@@ -135,7 +135,7 @@ spin_status_t spin_rope_hadamard_kvquant(const void *q, const void *k, const voi
       !valid_clip(clip) || !(theta > 0.0f) || !std::isfinite(theta) || cache_offset < 0 ||
       (int64_t)cache_len < (int64_t)cache_offset + seq)
     return SPIN_ERR_INVALID_ARG;
-  if (n_q_heads + 2 * n_kv_heads > 440) return SPIN_ERR_UNSUPPORTED_SIZE;  // staging must fit in smem
+  if (!rope_shape_supported(n_q_heads, n_kv_heads, (int64_t)batch * seq)) return SPIN_ERR_UNSUPPORTED_SIZE;
   if (batch == 0 || seq == 0) return SPIN_OK;
   if (!q || !k || !v || !pos || !q_out || !k_cache || !v_cache || !k_scale || !k_zero || !v_scale || !v_zero)
     return SPIN_ERR_INVALID_ARG;
@@ -190,9 +190,10 @@ int spin_last_cuda_error(void) { return g_last_cuda_error; }
 
 spin_status_t spin_device_status(uint32_t *status, int reset) {
   if (!status) return SPIN_ERR_INVALID_ARG;
-  unsigned int v = 0;
+  unsigned int v = 0, w = 0;
   spin_status_t st = cuda_status(read_device_status(&v, reset != 0));
-  *status = v;
+  if (st == SPIN_OK) st = cuda_status(read_rope_status(&w, reset != 0));
+  *status = v | w;
   return st;
 }
 

@@ -1,6 +1,8 @@
 // spin_launch.h -- host-side launchers behind the C ABI (internal header).
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -16,6 +18,9 @@ constexpr uint32_t kTensorCores = 4u;     // same value as SPIN_TENSOR_CORES
 // Cached per kernel and device after the first call.
 cudaError_t resident_slots(const void *kernel, int threads, int dyn_smem, int *slots);
 
+// cuTensorMapEncodeTiled from the driver (null if unavailable), looked up once.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
 cudaError_t launch_rotate_quant_int4(const void *x, int64_t tokens, int log_n, float clip,
                                      const uint32_t *signs, uint32_t flags, uint8_t *q, float *scales,
                                      cudaStream_t stream);
@@ -28,13 +33,18 @@ cudaError_t launch_rotate_quant_int4_tc(int log_n, const void *x, int64_t tokens
 // Test hook: make the tensor-core R4 kernel withhold one internal signal.
 void set_stall_test(int enable);
 
-// Device status word set by kernels whose bounded waits ran out.
+// Device status words set by kernels whose bounded waits ran out (the tensor-core
+// R4 kernel and the R3 kernel each keep one).
 cudaError_t read_device_status(unsigned int *status, bool reset);
+cudaError_t read_rope_status(unsigned int *status, bool reset);
 
 cudaError_t launch_dequant_inverse(const uint8_t *codes, int64_t rows, int log_n, int mode,
                                    const void *scale, const void *zero, const uint32_t *signs,
                                    uint32_t flags, void *out, int out_dtype, cudaStream_t stream);
 
+// Head counts and token counts the R3 kernel takes: n_q_heads <= 256,
+// n_q_heads + 2 n_kv_heads <= 384, batch * seq * n_q_heads < 2^31.
+bool rope_shape_supported(int n_q_heads, int n_kv_heads, int64_t tokens);
 cudaError_t launch_rope_hadamard_kvquant(const void *q, const void *k, const void *v,
                                          const int32_t *pos, float theta, int batch, int seq,
                                          int n_q_heads, int n_kv_heads, float clip, void *q_out,

@@ -88,6 +88,9 @@ def test_r3_argument_checks(L):
     assert _r3(L, q_out=FAKE + 4) == 3
     assert _r3(L, ks=FAKE + 1) == 3
     assert _r3(L, hq=400, hkv=40) == 2
+    assert _r3(L, hq=264, hkv=8) == 2  # more than 256 query heads
+    assert _r3(L, hq=256, hkv=128) == 2  # more than 384 head vectors per token
+    assert _r3(L, batch=1 << 20, seq=1024, cache_len=1024) == 2  # batch * seq * hq >= 2^31
 
 
 def test_dequant_argument_checks(L):

@@ -67,7 +67,8 @@ def compare_tokens(orc, q, k, v, pos, theta, clip, out, cache_offset, tokens):
     return skipped
 
 
-@pytest.mark.parametrize("shape", [(2, 37, 32, 8), (1, 5, 8, 8), (3, 2, 16, 2), (1, 1, 32, 8)])
+@pytest.mark.parametrize("shape", [(2, 37, 32, 8), (1, 5, 8, 8), (3, 2, 16, 2), (1, 1, 32, 8), (1, 9, 20, 10),
+                                   (2, 3, 128, 32), (1, 3, 256, 64), (1, 7, 4, 1)])
 def test_r3_small_shapes(spin_gpu, orc, shape):
     B, S, hq, hkv = shape
     q, k, v, _ = synthetic.r3_kv(B, S, hq, hkv, 128, seed=sum(shape))
