@@ -47,6 +47,18 @@ def algorithmic_bytes_r4(tokens: int, n: int) -> int:
     return tokens * (2 * n + n // 2 + 4)
 
 
+def r4_kernel_name(n: int, tokens: int, has_signs: bool) -> str:
+    """The R4 kernel the library's dispatch picks by default: the tensor-core one for
+    n = 4096 .. 32768 (n = 32768 without a sign diagonal) once the batch has at least
+    128 MMA groups, else the CUDA-core one."""
+    log_n = n.bit_length() - 1
+    if 12 <= log_n <= 15 and not (log_n == 15 and has_signs):
+        tokens_per_group = 1 if log_n == 15 else 256 >> (log_n - 7)
+        if tokens >= 128 * tokens_per_group:
+            return "k1_tc_rotate_quant"
+    return "k1_rotate_quant_int4"
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -360,7 +372,7 @@ def main():
 
     # ---- the same steps on the all-CUDA-core kernel, for comparison (not the headline)
     cores = None
-    if wl["kind"] == "r4" and n in (4096, 8192, 16384):
+    if wl["kind"] == "r4" and r4_kernel_name(n, tokens, wl["signs"] is not None) == "k1_tc_rotate_quant":
         for i in range(args.warmup):
             step(i, True)
         stream.synchronize()
@@ -408,7 +420,7 @@ def main():
 
     peak, peak_kind = measured_peaks()
     if wl["kind"] == "r4":
-        kname = "k1_tc_rotate_quant" if n in (4096, 8192, 16384) else "k1_rotate_quant_int4"
+        kname = r4_kernel_name(n, tokens, wl["signs"] is not None)
     else:
         kname = "k2_rope_hadamard_kvquant"
     traffic = recorded_traffic(f"{kname}:{args.workload}")

@@ -80,6 +80,12 @@ cudaError_t resident_slots(const void *kernel, int threads, int dyn_smem, int *s
     if (dyn_smem > dyn_max) return cudaErrorInvalidConfiguration;
     if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max)) != cudaSuccess)
       return e;
+    // All of the unified L1/shared storage as shared memory, so the blocks per SM
+    // found below are the blocks that become resident at launch (none of these
+    // kernels relies on L1 caching).
+    if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  (int)cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+      return e;
     opted_in[std::make_pair(kernel, dev)] = true;
   }
   int sms = 0, per_sm = 0;

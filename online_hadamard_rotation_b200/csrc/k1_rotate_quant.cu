@@ -207,7 +207,7 @@ cudaError_t launch_n(const void *x, int64_t tokens, float clip, const uint32_t *
 cudaError_t launch_rotate_quant_int4(const void *x, int64_t tokens, int log_n, float clip,
                                      const uint32_t *signs, uint32_t flags, uint8_t *q, float *scales,
                                      cudaStream_t stream) {
-  if (!(flags & kCudaCoresOnly) && tc_rotate_quant_supported(log_n, tokens, flags))
+  if (!(flags & kCudaCoresOnly) && tc_rotate_quant_supported(log_n, tokens, flags, signs != nullptr))
     return launch_rotate_quant_int4_tc(log_n, x, tokens, clip, signs, q, scales, stream);
   flags &= ~(kCudaCoresOnly | kTensorCores);
   switch (log_n) {

@@ -1,5 +1,5 @@
-// k1_tc.cu -- R4 for n = 4096, 8192 and 16384 with the first Kronecker factor
-// on the tensor cores.
+// k1_tc.cu -- R4 for n = 4096 to 32768 with the first Kronecker factor on the
+// tensor cores.
 //
 // "Rotations: QuaRot, SpinQuant and incoherence", section "Hadamard matrices":
 // the Sylvester H_n is a Kronecker product of smaller Sylvester matrices, and
@@ -9,7 +9,8 @@
 // Outlier Curse": symmetric INT4, step max|y| / 7.
 //
 // A token row x of n = 128 B bf16 values is the 128 x B matrix X[a][b], with
-// element index e = B a + b (B = 32, 64, 128). Then H_n x = vec(H_128 X H_B):
+// element index e = B a + b (B = 32, 64, 128; n = 32768 is two such blocks, see
+// Shape). Then H_n x = vec(H_128 X H_B):
 //   1. tcgen05.mma computes Y = H_128 X (contraction over a) for 256 / B tokens
 //      at once (M = 128, N = 256, K = 128, bf16 in, fp32 accumulate in TMEM).
 //      H is exactly +-1 and X is exactly bf16, so every product is exact and
@@ -65,22 +66,31 @@ constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;  // + alignment slack
 constexpr long long kTimeoutCycles = 4000000000LL;     // about two seconds
 constexpr long long kStallTestCycles = 2000000LL;      // about a millisecond, for the stall test hook
 
-// Shape constants for n = 2^LOGN.
+// Shape constants for n = 2^LOGN. For n = 32768 (SPLIT) a token is 256 rows of
+// B = 128 columns: H_n = H_2 (x) H_128 (x) H_128, and the top factor H_2 pairs the row
+// blocks X_0 (rows 0-127) and X_1 (rows 128-255). The group is that one token: the
+// MMA accumulates H_128 X_0 + H_128 X_1 into TMEM columns 0-127 and H_128 X_0 -
+// H_128 X_1 (negated A) into columns 128-255, so epilogue warpgroup g holds output
+// rows 128 g + a' and the token's max spans both warpgroups.
 template <int LOGN>
 struct Shape {
-  static constexpr int B = 1 << (LOGN - 7);        // columns per row (second factor size)
-  static constexpr int LOGB = LOGN - 7;
-  static constexpr int TOK = 256 / B;               // tokens per MMA group
-  static constexpr int SEG = 128 / B;               // token segments per epilogue thread
+  static constexpr bool SPLIT = LOGN == 15;
+  static constexpr int B = SPLIT ? 128 : 1 << (LOGN - 7);  // columns per row (last factor size)
+  static constexpr int LOGB = SPLIT ? 7 : LOGN - 7;
+  static constexpr int ROWS = SPLIT ? 256 : 128;    // rows per token
+  static constexpr int TOK = SPLIT ? 1 : 256 / B;   // tokens per MMA group
+  static constexpr int SEG = SPLIT ? 1 : 128 / B;   // token segments per epilogue thread
   static constexpr int BOXW = B < 64 ? B : 64;      // TMA box width (columns)
   static constexpr int ROWB = BOXW * 2;             // bytes per smem tile row (64 or 128)
-  static constexpr int BPT = B / BOXW;              // boxes per token
+  static constexpr int CBOX = B / BOXW;             // column boxes per 128-row block
+  static constexpr int BPT = CBOX * ROWS / 128;     // boxes per token
   static constexpr uint32_t BOXBYTES = 128u * ROWB; // bytes per box
   static constexpr int CPR = ROWB / 16;             // 16-byte chunks per tile row
   static constexpr uint32_t LAYOUT = ROWB == 128 ? 2u : 4u;  // UMMA swizzle: 128 B or 64 B
   static constexpr uint32_t TOKBYTES = kGroupBytes / TOK;
   static constexpr int NPOS = (int)(TOKBYTES / 16 / 64);  // sign positions per sign thread
-  static_assert(LOGN >= 12 && LOGN <= 14, "tensor-core R4 covers n = 4096 .. 16384");
+  static constexpr int64_t OUTB = (int64_t(1) << LOGN) / 2;  // code bytes per token
+  static_assert(LOGN >= 12 && LOGN <= 15, "tensor-core R4 covers n = 4096 .. 32768");
 };
 
 struct Shared {
@@ -153,7 +163,8 @@ __device__ __forceinline__ void load_group(uint8_t *dst, const CUtensorMap *map,
   tc::mbar_arrive_expect_tx(bar, (uint32_t)nvalid * SH::TOKBYTES);
   for (int t = 0; t < nvalid; ++t)
     for (int j = 0; j < SH::BPT; ++j)
-      tc::tma_load_2d(dst + (t * SH::BPT + j) * SH::BOXBYTES, map, bar, j * SH::BOXW, (int)((t0 + t) * 128));
+      tc::tma_load_2d(dst + (t * SH::BPT + j) * SH::BOXBYTES, map, bar, (j % SH::CBOX) * SH::BOXW,
+                      (int)((t0 + t) * SH::ROWS + (j / SH::CBOX) * 128));
 }
 
 template <int LOGN, bool SIGNS, bool STORE32>
@@ -163,6 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        int stall_test) {
   using SH = Shape<LOGN>;
   constexpr int B = SH::B, SEG = SH::SEG;
+  static_assert(!(SIGNS && SH::SPLIT), "the sign masks of n = 32768 do not fit in registers");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Shared &S = *reinterpret_cast<Shared *>(smem + kOffBar);
@@ -241,7 +253,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = tc::idesc_bf16(128, 256, true);
+      constexpr uint32_t idesc = tc::idesc_bf16(128, SH::SPLIT ? 128 : 256, true);
+      constexpr uint32_t idesc_neg = idesc | (1u << 13);  // negate A
       const uint32_t sH = tc::smem_u32(smem + kOffH), sX = tc::smem_u32(smem + kOffX);
       for (int64_t i = 0;; ++i) {
         const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
@@ -250,14 +263,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_bounded(SIGNS ? &S.sgn[st] : &S.full[st], (uint32_t)((i / kStages) & 1), S, true)) break;
         if (!wait_bounded(&S.tempty[acc], (uint32_t)((i >> 1) & 1) ^ 1u, S, true)) break;
         tc::tc_fence_after();
+        if constexpr (SH::SPLIT) {
+          // columns 128 u + b: sum over row blocks v of (-1)^(u v) H_128 X_v
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          // A: 16 columns k of H per step. B: rows a = 16 s .. 16 s + 15 of every box
-          // (MN-major: boxes of BOXW columns BOXBYTES apart, 8-row groups 8 ROWB apart).
-          const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-          uint64_t bd = tc::smem_desc(sX + st * kGroupBytes + s * 16 * SH::ROWB, SH::BOXBYTES, 8 * SH::ROWB);
-          bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
-          tc::umma_bf16(tmem + acc * 256, ad, bd, idesc, s > 0 ? 1u : 0u);
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int v = 0; v < 2; ++v)
+#pragma unroll
+              for (int s = 0; s < 8; ++s) {
+                const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
+                uint64_t bd = tc::smem_desc(sX + st * kGroupBytes + v * SH::CBOX * SH::BOXBYTES + s * 16 * SH::ROWB,
+                                            SH::BOXBYTES, 8 * SH::ROWB);
+                bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
+                tc::umma_bf16(tmem + acc * 256 + u * 128, ad, bd, (u & v) ? idesc_neg : idesc,
+                              (v > 0 || s > 0) ? 1u : 0u);
+              }
+        } else {
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            // A: 16 columns k of H per step. B: rows a = 16 s .. 16 s + 15 of every box
+            // (MN-major: boxes of BOXW columns BOXBYTES apart, 8-row groups 8 ROWB apart).
+            const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
+            uint64_t bd = tc::smem_desc(sX + st * kGroupBytes + s * 16 * SH::ROWB, SH::BOXBYTES, 8 * SH::ROWB);
+            bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
+            tc::umma_bf16(tmem + acc * 256, ad, bd, idesc, s > 0 ? 1u : 0u);
+          }
         }
         tc::umma_commit(&S.empty[st]);
         // Stall test hook: withhold the first group's completion signal, so the
@@ -318,9 +348,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
       if (p >= ngroups) break;
       const int acc = (int)(i & 1);
-      if (tg == 0) S.dec[g] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
-      tc::named_sync(1 + g, 128);
-      if (!S.dec[g]) break;
+      if constexpr (SH::SPLIT) {  // one decision for both warpgroups: they meet at barrier 4 below
+        if (threadIdx.x == 128) S.dec[0] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+        tc::named_sync(4, 256);
+        if (!S.dec[0]) break;
+      } else {
+        if (tg == 0) S.dec[g] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+        tc::named_sync(1 + g, 128);
+        if (!S.dec[g]) break;
+      }
       tc::tc_fence_after();
       float v[kRegs];
       {
@@ -361,17 +397,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mx[0]));
         if (lane == 0) S.wmax[g][i & 1][wq][sg] = __uint_as_float(wm);
       }
-      tc::named_sync(1 + g, 128);
+      if constexpr (SH::SPLIT) tc::named_sync(4, 256);
+      else tc::named_sync(1 + g, 128);
       constexpr float k815 = 8.0f / 15.0f;
 #pragma unroll
       for (int sg = 0; sg < SEG; ++sg) {
-        const float mu = fmaxf(fmaxf(S.wmax[g][i & 1][0][sg], S.wmax[g][i & 1][1][sg]),
-                               fmaxf(S.wmax[g][i & 1][2][sg], S.wmax[g][i & 1][3][sg]));
+        float mu = fmaxf(fmaxf(S.wmax[g][i & 1][0][sg], S.wmax[g][i & 1][1][sg]),
+                         fmaxf(S.wmax[g][i & 1][2][sg], S.wmax[g][i & 1][3][sg]));
+        if constexpr (SH::SPLIT)
+          mu = fmaxf(mu, fmaxf(fmaxf(S.wmax[g ^ 1][i & 1][0][0], S.wmax[g ^ 1][i & 1][1][0]),
+                               fmaxf(S.wmax[g ^ 1][i & 1][2][0], S.wmax[g ^ 1][i & 1][3][0])));
         const float s = fmaxf(clip * (mu * inv_sqrt_n) / 7.0f, 1e-8f);
         const float c15 = (inv_sqrt_n / 15.0f) / s;
-        const int64_t token = p * SH::TOK + g * SEG + sg;
+        const int64_t token = SH::SPLIT ? p : p * SH::TOK + g * SEG + sg;
         if (token >= tokens) continue;
-        uint8_t *dst = q + token * (int64_t)(B * 64) + row * (B / 2);
+        const uint32_t orow = SH::SPLIT ? 128u * g + row : row;  // output row of B values
+        uint8_t *dst = q + token * SH::OUTB + orow * (B / 2);
         uint32_t words[B / 8];
 #pragma unroll
         for (int wi = 0; wi < B / 8; ++wi) {
@@ -392,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __stcs(reinterpret_cast<uint4 *>(dst) + w4,
                    make_uint4(words[4 * w4], words[4 * w4 + 1], words[4 * w4 + 2], words[4 * w4 + 3]));
         }
-        if (tg == 0) scales[token] = s;
+        if (tg == 0 && (!SH::SPLIT || g == 0)) scales[token] = s;
       }
     }
   }
@@ -418,7 +459,7 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
   auto fn = tensor_map_encoder();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap map;
-  const cuuint64_t dims[2] = {(cuuint64_t)SH::B, (cuuint64_t)tokens * 128};
+  const cuuint64_t dims[2] = {(cuuint64_t)SH::B, (cuuint64_t)tokens * SH::ROWS};
   const cuuint64_t strides[1] = {(cuuint64_t)SH::B * 2};
   const cuuint32_t box[2] = {(cuuint32_t)SH::BOXW, 128};
   const cuuint32_t estr[2] = {1, 1};
@@ -451,7 +492,9 @@ template <int LOGN>
 cudaError_t launch_n(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
                      cudaStream_t stream, int stall_test) {
   const bool a32 = (reinterpret_cast<uintptr_t>(q) & 31u) == 0;  // 32-byte stores need 32-byte alignment
-  if (signs) {
+  if constexpr (Shape<LOGN>::SPLIT) {
+    if (signs) return cudaErrorInvalidValue;
+  } else if (signs) {
     return a32 ? launch_tc<LOGN, true, true>(x, tokens, clip, signs, q, scales, stream, stall_test)
                : launch_tc<LOGN, true, false>(x, tokens, clip, signs, q, scales, stream, stall_test);
   }
@@ -479,10 +522,12 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // The tensor-core kernel pays a per-CTA setup (H tile, TMEM, first copies) that
 // only pays off with at least about one MMA group per SM; smaller batches (decode)
 // go to the CUDA-core kernel, which needs no setup.
-bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags) {
-  if (log_n < 12 || log_n > 14 || (flags & kNoRotate) || tokens <= 0 || tokens * 128 >= (int64_t(1) << 31))
-    return false;
-  const int64_t tok_per_group = int64_t(256) >> (log_n - 7);
+bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags, bool has_signs) {
+  if (log_n < 12 || log_n > 15 || (flags & kNoRotate) || tokens <= 0) return false;
+  if (log_n == 15 && has_signs) return false;  // its sign masks do not fit the sign warps' registers
+  const int64_t rows_per_token = log_n == 15 ? 256 : 128;
+  if (tokens * rows_per_token >= (int64_t(1) << 31)) return false;
+  const int64_t tok_per_group = log_n == 15 ? 1 : int64_t(256) >> (log_n - 7);
   return (flags & kTensorCores) || tokens >= 128 * tok_per_group;
 }
 
@@ -493,6 +538,7 @@ cudaError_t launch_rotate_quant_int4_tc(int log_n, const void *x, int64_t tokens
     case 12: return launch_n<12>(x, tokens, clip, signs, q, scales, stream, stall);
     case 13: return launch_n<13>(x, tokens, clip, signs, q, scales, stream, stall);
     case 14: return launch_n<14>(x, tokens, clip, signs, q, scales, stream, stall);
+    case 15: return launch_n<15>(x, tokens, clip, signs, q, scales, stream, stall);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -25,8 +25,9 @@ cudaError_t launch_rotate_quant_int4(const void *x, int64_t tokens, int log_n, f
                                      const uint32_t *signs, uint32_t flags, uint8_t *q, float *scales,
                                      cudaStream_t stream);
 
-// Tensor-core R4 kernel (n = 4096, 8192, 16384): availability and launcher.
-bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags);
+// Tensor-core R4 kernel (n = 4096 to 32768; n = 32768 without a sign diagonal):
+// availability and launcher.
+bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags, bool has_signs);
 cudaError_t launch_rotate_quant_int4_tc(int log_n, const void *x, int64_t tokens, float clip, const uint32_t *signs,
                                         uint8_t *q, float *scales, cudaStream_t stream);
 

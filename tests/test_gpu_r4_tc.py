@@ -1,7 +1,8 @@
 """The tensor-core R4 kernel (n = 4096, 8192, 16384: first H_128 Kronecker
-factor on tcgen05, second on CUDA cores) vs the fp64 oracle, and vs the
-all-CUDA-core kernel selected with SPIN_CUDA_CORES_ONLY. Token counts leave
-partial MMA groups (8, 4 and 2 tokens per group)."""
+factor on tcgen05, second on CUDA cores; n = 32768: H_2 and H_128 on tcgen05,
+without a sign diagonal) vs the fp64 oracle, and vs the all-CUDA-core kernel
+selected with SPIN_CUDA_CORES_ONLY. Token counts leave partial MMA groups (8, 4
+and 2 tokens per group). At n = 32768 with sign_bits the CUDA-core kernel runs."""
 import numpy as np
 import pytest
 import torch
@@ -12,7 +13,7 @@ from tests.gpu_util import to_dev_bf16, to_dev_signs
 
 pytestmark = pytest.mark.gpu
 
-SIZES = [4096, 8192, 16384]
+SIZES = [4096, 8192, 16384, 32768]
 
 
 def run(spin, bits, clip, signs, cores_only=False):
@@ -40,6 +41,8 @@ def test_tc_vs_oracle(spin_gpu, orc, N, tokens, clip, with_signs):
 @pytest.mark.parametrize("N", SIZES)
 def test_tc_matches_cuda_core_kernel(spin_gpu, orc, N):
     bits, signs, _ = synthetic.r4_prefill(tokens=512, n=N, seed=9)
+    if N == 32768:
+        signs = None  # the tensor-core kernel takes no diagonal at this size
     q1, s1 = run(spin_gpu, bits, 0.9, signs)
     q2, s2 = run(spin_gpu, bits, 0.9, signs, cores_only=True)
     parity.check_rel(s1, s2, 1e-5, "tc vs cuda-core scales")
