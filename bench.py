@@ -68,24 +68,27 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_digest() -> str:
+def kernel_source_digest(kernel: str) -> str:
+    """Hash of the sources a kernel is built from: the .cu files of its family
+    (k1_, k2_, k3_) and the shared device headers."""
+    family = kernel.split("_")[0] + "_"
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "online_hadamard_rotation_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.startswith("k1_") or name in ("spin_tile.cuh", "tc_ptx.cuh"):
+        if name.startswith(family) or name in ("spin_tile.cuh", "tc_ptx.cuh"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str):
-    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
-    the current kernel source; None otherwise."""
+def recorded_traffic(key: str):
+    """Per-launch DRAM bytes from the committed ncu summary (key "kernel:workload"),
+    if it was taken on the current kernel source; None otherwise."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
-        d = json.load(f).get(kernel)
-    if not d or d.get("source_digest") != kernel_source_digest():
+        d = json.load(f).get(key)
+    if not d or d.get("source_digest") != kernel_source_digest(key.split(":")[0]):
         return None
     return d.get("bytes_per_launch")
 
@@ -385,6 +388,46 @@ def main():
         cores = {"kernel": "k1_rotate_quant_int4 (all butterflies on CUDA cores)", "ms_per_step": cms,
                  "achieved_gbs": step_bytes / (cms / 1e3) / 1e9}
 
+    # ---- bandwidth sweep: the dequantise -> inverse-rotate round trip on this step's
+    # codes (its own kernel, timed alone), and the reconstruction error of the rotated
+    # path against direct quantisation over the whole workload
+    round_trip = None
+    if args.workload.startswith("sweep"):
+        b = sets[0]
+        step(0)
+        xr = torch.empty((tokens, n), dtype=torch.bfloat16, device=dev)
+
+        def inverse(codes, scales, direct=False):
+            spin.dequant_hadamard_inverse(codes, n, scales, no_rotate=direct, out_dtype=torch.bfloat16, out=xr,
+                                          stream=stream)
+
+        for _ in range(args.warmup):
+            inverse(b["q"], b["s"])
+        stream.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            inverse(b["q"], b["s"])
+        ev1.record(stream)
+        ev1.synchronize()
+        rms = max_over_ranks(ev0.elapsed_time(ev1), dev) / args.steps
+        rt_bytes = tokens * (n // 2 + 4 + 2 * n)
+        x32 = b["x"].float()
+        mse = {}
+        for direct in (False, True):
+            q_d = torch.empty_like(b["q"])
+            s_d = torch.empty_like(b["s"])
+            spin.hadamard_quant_int4(b["x"], wl["clip"], None, no_rotate=direct, out=q_d, scales=s_d, stream=stream)
+            inverse(q_d, s_d, direct)
+            stream.synchronize()
+            mse[direct] = float(((xr.float() - x32) ** 2).mean().item())
+            del q_d, s_d
+        del x32, xr
+        rt_gbs = rt_bytes / (rms / 1e3) / 1e9
+        round_trip = {"kernel": "k3_dequant_inverse", "ms_per_step": rms, "achieved_gbs": rt_gbs * world,
+                      "frac": rt_gbs / measured_peaks()[0], "bytes_per_row": n // 2 + 4 + 2 * n,
+                      "out_dtype": "bf16", "mse_rotated": mse[False], "mse_direct": mse[True],
+                      "mse_ratio": mse[False] / mse[True] if mse[True] > 0 else None}
+
     # ---- decode: per-call latency, plain launches and CUDA-graph replay
     latency = None
     if args.workload.startswith("decode"):
@@ -450,7 +493,7 @@ def main():
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": config_for(wl, world, args.workload),
                 "gpu_launches": args.steps, "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu,
-                "cuda_core_kernel": cores, "decode_latency": latency,
+                "cuda_core_kernel": cores, "decode_latency": latency, "round_trip": round_trip,
                 "clocks": clocks.summary()}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -104,10 +104,10 @@ struct Shared {
 static_assert(sizeof(Shared) <= 512, "barrier area");
 
 __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, Shared &S, bool honor_abort) {
-  if (tc::mbar_try_wait(bar, parity)) return true;
+  if (tc::mbar_try_wait_suspend(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (tc::mbar_try_wait(bar, parity)) return true;
+    if (tc::mbar_try_wait_suspend(bar, parity)) return true;
     if (honor_abort && *reinterpret_cast<volatile int *>(&S.abort)) return false;
     if (clock64() - t0 > S.budget) {
       *reinterpret_cast<volatile int *>(&S.abort) = 1;
