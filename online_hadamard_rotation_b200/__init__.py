@@ -225,14 +225,18 @@ def rope_hadamard_kvquant(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos
 def dequant_hadamard_inverse(codes: torch.Tensor, n: int, scale: torch.Tensor, zero: torch.Tensor | None = None,
                              mode: int = SYM_INT4_F32SCALE, signs: torch.Tensor | None = None,
                              no_rotate: bool = False, out_dtype=torch.float32, out: torch.Tensor | None = None,
-                             stream=None) -> torch.Tensor:
-    """codes [..., n/2] uint8 -> out [..., n] (rows = codes.numel() / (n/2))."""
+                             stream=None, cuda_cores_only: bool = False, tensor_cores: bool = False) -> torch.Tensor:
+    """codes [..., n/2] uint8 -> out [..., n] (rows = codes.numel() / (n/2)).
+    cuda_cores_only / tensor_cores select the kernel (SPIN_CUDA_CORES_ONLY /
+    SPIN_TENSOR_CORES); by default the library picks."""
     _need(codes, "codes", torch.uint8)
     rows = codes.numel() // (n // 2)
     if out is None:
         out = torch.empty(tuple(codes.shape[:-1]) + (n,), dtype=out_dtype, device=codes.device)
     dt = F32 if out.dtype == torch.float32 else BF16
+    flags = (NO_ROTATE if no_rotate else 0) | (CUDA_CORES_ONLY if cuda_cores_only else 0) | \
+        (TENSOR_CORES if tensor_cores else 0)
     st = spin_dequant_hadamard_inverse(_ptr(codes), rows, n, mode, _ptr(scale), _ptr(zero), _ptr(signs),
-                                       NO_ROTATE if no_rotate else 0, _ptr(out), dt, _stream(stream))
+                                       flags, _ptr(out), dt, _stream(stream))
     _check("spin_dequant_hadamard_inverse", st)
     return out

@@ -164,7 +164,9 @@ spin_status_t spin_dequant_hadamard_inverse(const uint8_t *codes, int64_t rows, 
   const int log_n = log2_pow2(n);
   if (log_n < 7 || log_n > 15) return SPIN_ERR_UNSUPPORTED_SIZE;
   if (rows < 0 || (mode != SPIN_SYM_INT4_F32SCALE && mode != SPIN_ASYM_INT4_F16SZ) ||
-      (out_dtype != SPIN_BF16 && out_dtype != SPIN_F32) || (flags & ~SPIN_NO_ROTATE) != 0)
+      (out_dtype != SPIN_BF16 && out_dtype != SPIN_F32) ||
+      (flags & ~(SPIN_NO_ROTATE | SPIN_CUDA_CORES_ONLY | SPIN_TENSOR_CORES)) != 0 ||
+      (flags & (SPIN_CUDA_CORES_ONLY | SPIN_TENSOR_CORES)) == (SPIN_CUDA_CORES_ONLY | SPIN_TENSOR_CORES))
     return SPIN_ERR_INVALID_ARG;
   if (rows == 0) return SPIN_OK;
   if (!codes || !scale || !out || (mode == SPIN_ASYM_INT4_F16SZ && !zero)) return SPIN_ERR_INVALID_ARG;
@@ -196,10 +198,11 @@ int spin_last_cuda_error(void) { return g_last_cuda_error; }
 
 spin_status_t spin_device_status(uint32_t *status, int reset) {
   if (!status) return SPIN_ERR_INVALID_ARG;
-  unsigned int v = 0, w = 0;
+  unsigned int v = 0, w = 0, u = 0;
   spin_status_t st = cuda_status(read_device_status(&v, reset != 0));
   if (st == SPIN_OK) st = cuda_status(read_rope_status(&w, reset != 0));
-  *status = v | w;
+  if (st == SPIN_OK) st = cuda_status(read_dequant_status(&u, reset != 0));
+  *status = v | w | u;
   return st;
 }
 

@@ -130,6 +130,9 @@ cudaError_t launch_n(const uint8_t *codes, int64_t rows, int mode, const void *s
 cudaError_t launch_dequant_inverse(const uint8_t *codes, int64_t rows, int log_n, int mode,
                                    const void *scale, const void *zero, const uint32_t *signs,
                                    uint32_t flags, void *out, int out_dtype, cudaStream_t stream) {
+  if (!(flags & kCudaCoresOnly) && tc_dequant_supported(log_n, rows, flags))
+    return launch_dequant_inverse_tc(log_n, codes, rows, mode, scale, zero, signs, out, out_dtype, stream);
+  flags &= ~(kCudaCoresOnly | kTensorCores);
   switch (log_n) {
     case 7: return launch_n<7>(codes, rows, mode, scale, zero, signs, flags, out, out_dtype, stream);
     case 8: return launch_n<8>(codes, rows, mode, scale, zero, signs, flags, out, out_dtype, stream);

@@ -1,0 +1,508 @@
+// k3_tc.cu -- dequantise + inverse rotation for n = 4096 to 32768 with the first
+// Kronecker factor on the tensor cores.
+//
+// "Rotations: QuaRot, SpinQuant and incoherence", widget "Try it": rotate,
+// quantize, rotate back; section "Hadamard matrices": H_n / sqrt(n) is
+// orthogonal and symmetric, so D H_n / sqrt(n) undoes H_n D / sqrt(n), and the
+// Sylvester H_n is a Kronecker product of smaller Sylvester matrices.
+// "SpinQuant Guide: Learned Rotations for 4-Bit LLMs", section "End-to-End
+// Implementation": dequantised value = code * scale.
+//
+// out = D H_n v / sqrt(n) with v = s (c - z): s and z are constant over a row, so
+// out = (s / sqrt(n)) D H_n (c - z), and c - z is a small integer vector. A row of
+// n = 128 B values is the 128 x B matrix C[a][b] (e = B a + b), and
+// H_n (c - z) = vec(H_128 C' H_B):
+//   1. Converter warps expand the packed nibbles of a group (32768 elements:
+//      256 / B rows, or one row at n = 32768) into fp16 integers c - z (exact),
+//      written as the MMA's MN-major B operand with the 64- or 128-byte swizzle.
+//   2. tcgen05.mma (kind::f16, fp16 H = +-1 as the K-major A operand, fp32
+//      accumulate in TMEM) computes H_128 C' exactly: every partial sum is an
+//      integer below 2^24.
+//   3. Each epilogue thread owns one TMEM lane (row a') over 128 columns, runs the
+//      log2(B) butterfly stages of H_B in registers (still exact), multiplies by
+//      s / sqrt(n), flips the signs of D (its row's sign words stay in registers)
+//      and stores bf16 or fp32 straight to the output row.
+// n = 32768 is H_2 (x) H_128 (x) H_128: a row is 256 x 128, the MMA accumulates
+// H_128 C'_0 + H_128 C'_1 and H_128 C'_0 - H_128 C'_1 (negate-A bit) into the two
+// 128-column halves, and epilogue warpgroup g writes output rows 128 g + a'.
+//
+// Roles (384 threads, one CTA per SM, persistent over groups):
+//   warp 0      producer: one bulk copy of the group's 16 KiB of codes into a
+//               three-stage ring
+//   warp 1      TMEM owner and MMA issuer
+//   warps 2-3   converters: codes -> fp16 operand, two-stage ring of 64 KiB
+//   warps 4-11  epilogue, two warpgroups over TMEM columns 0-127 and 128-255
+// Every mbarrier wait is bounded by a clock budget; on expiry the CTA records a
+// status (read by spin_device_status), drains its copies and MMAs, frees TMEM and
+// returns.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "spin_launch.h"
+#include "spin_tile.cuh"
+#include "tc_ptx.cuh"
+
+namespace spin {
+
+// Nonzero once a tensor-core dequantise launch gave up on a wait (see spin_device_status).
+__device__ unsigned int g_dequant_status = 0u;
+
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kCStages = 3;                        // codes ring
+constexpr int kOStages = 2;                        // fp16 operand ring
+constexpr uint32_t kCodeBytes = 16384;             // codes of one group (32768 nibbles)
+constexpr uint32_t kOpBytes = 65536;               // fp16 operand of one group
+constexpr uint32_t kOffH = 0;                      // A operand: H_128 in fp16, K-major, 2 x 16 KiB
+constexpr uint32_t kOffO = 32768;                  // operand ring
+constexpr uint32_t kOffC = kOffO + kOStages * kOpBytes;
+constexpr uint32_t kOffBar = kOffC + kCStages * kCodeBytes;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
+constexpr long long kTimeoutCycles = 4000000000LL;     // about two seconds
+
+template <int LOGN>
+struct Shape {
+  static constexpr bool SPLIT = LOGN == 15;
+  static constexpr int B = SPLIT ? 128 : 1 << (LOGN - 7);  // columns per row
+  static constexpr int LOGB = SPLIT ? 7 : LOGN - 7;
+  static constexpr int ROWS = SPLIT ? 256 : 128;    // matrix rows per token row
+  static constexpr int TOK = SPLIT ? 1 : 256 / B;   // token rows per group
+  static constexpr int SEG = SPLIT ? 1 : 128 / B;   // token rows per epilogue thread
+  static constexpr int BOXW = B < 64 ? B : 64;      // operand tile width (columns)
+  static constexpr int ROWB = BOXW * 2;             // bytes per operand tile row
+  static constexpr int CBOX = B / BOXW;             // column tiles per 128-row block
+  static constexpr int BPT = CBOX * ROWS / 128;     // tiles per token row
+  static constexpr uint32_t BOXBYTES = 128u * ROWB; // bytes per tile
+  static constexpr uint32_t LAYOUT = ROWB == 128 ? 2u : 4u;  // UMMA swizzle: 128 B or 64 B
+  static constexpr int WPT = (1 << LOGN) / 8;       // code words (8 nibbles) per token row
+  static_assert(LOGN >= 12 && LOGN <= 15, "tensor-core dequantise covers n = 4096 .. 32768");
+};
+
+struct Shared {
+  uint64_t cfull[kCStages], cempty[kCStages], ofull[kOStages], oempty[kOStages], tfull[2], tempty[2], drain;
+  uint32_t tmem_base;
+  int abort;
+  int dec[3];
+  long long budget;
+  __half2 zc[8];  // per token row of the group being converted: -(1024 + zero)
+};
+static_assert(sizeof(Shared) <= 256, "barrier area");
+
+// One bulk copy global -> shared that completes `bar`'s transaction count (16-byte
+// aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   tc::smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+               : "memory");
+}
+
+// Instruction descriptor for kind::f16 with fp16 A and B (format 0), fp32 accumulator,
+// A K-major, B MN-major (`b_mn`).
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn) {
+  return (1u << 4) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, Shared &S, bool honor_abort) {
+  if (tc::mbar_try_wait_suspend(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (tc::mbar_try_wait_suspend(bar, parity)) return true;
+    if (honor_abort && *reinterpret_cast<volatile int *>(&S.abort)) return false;
+    if (clock64() - t0 > S.budget) {
+      *reinterpret_cast<volatile int *>(&S.abort) = 1;
+      atomicOr(&g_dequant_status, 1u);
+      return false;
+    }
+  }
+}
+
+// Eight 32-bit words to global memory: one 32-byte streaming store when `wide`
+// (32-byte aligned destination), else two 16-byte ones.
+template <bool WIDE>
+__device__ __forceinline__ void store8(void *p, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t w4,
+                                       uint32_t w5, uint32_t w6, uint32_t w7) {
+  if constexpr (WIDE) {
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w0), "r"(w1),
+                 "r"(w2), "r"(w3), "r"(w4), "r"(w5), "r"(w6), "r"(w7)
+                 : "memory");
+  } else {
+    __stcs(reinterpret_cast<uint4 *>(p), make_uint4(w0, w1, w2, w3));
+    __stcs(reinterpret_cast<uint4 *>(p) + 1, make_uint4(w4, w5, w6, w7));
+  }
+}
+
+// (a0, a1) <- (a0, a1) * (m, m), one packed multiply
+__device__ __forceinline__ void mul2(float &a0, float &a1, float m) {
+  uint64_t A, M, R;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(M) : "f"(m));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(R) : "l"(A), "l"(M));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(R));
+}
+
+// Eight nibbles (element 2j in the low nibble of byte j; unsigned after the caller's
+// sign fix-up) -> four fp16 pairs (u - zc): each half is first 1024 + u (exponent 10,
+// one unit per ulp), then the exact sum with zc = -(1024 + zero).
+__device__ __forceinline__ uint4 expand8(uint32_t w, __half2 zc) {
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+  const uint32_t e0 = __byte_perm(lo, hi, 0x5140), e1 = __byte_perm(lo, hi, 0x7362);  // nibbles 0-3, 4-7
+  uint32_t h[4];
+  h[0] = __byte_perm(e0, 0x64646464u, 0x4140);
+  h[1] = __byte_perm(e0, 0x64646464u, 0x4342);
+  h[2] = __byte_perm(e1, 0x64646464u, 0x4140);
+  h[3] = __byte_perm(e1, 0x64646464u, 0x4342);
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 v = __hadd2(*reinterpret_cast<const __half2 *>(&h[i]), zc);
+    o[i] = *reinterpret_cast<const uint32_t *>(&v);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <int LOGN, bool SIGNS, bool F32, bool STORE32>
+__global__ void __launch_bounds__(kThreads, 1)
+    k3_tc_dequant_inverse(const uint8_t *__restrict__ codes, int64_t rows, float inv_sqrt_n,
+                          const void *__restrict__ scale, const __half *__restrict__ zero,
+                          const uint32_t *__restrict__ signs, void *__restrict__ out, int asym) {
+  using SH = Shape<LOGN>;
+  constexpr int B = SH::B, SEG = SH::SEG;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Shared &S = *reinterpret_cast<Shared *>(smem + kOffBar);
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
+  const int64_t ngroups = (rows + SH::TOK - 1) / SH::TOK;
+
+  // ------------------------------------------------------------ setup
+  tc::grid_dep_wait();
+  int64_t first_issued = 0;
+  auto issue = [&](int64_t i, int64_t p) {  // codes of group p into codes stage i % kCStages
+    const int cs = (int)(i % kCStages);
+    const int64_t t0 = p * SH::TOK;
+    const int nvalid = (int)((rows - t0) < SH::TOK ? (rows - t0) : SH::TOK);
+    const uint32_t bytes = (uint32_t)nvalid * (uint32_t)(SH::WPT * 4);
+    tc::mbar_arrive_expect_tx(&S.cfull[cs], bytes);
+    bulk_load(smem + kOffC + cs * kCodeBytes, codes + t0 * (int64_t)(SH::WPT * 4), bytes, &S.cfull[cs]);
+  };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kCStages; ++s) {
+      tc::mbar_init(&S.cfull[s], 1);
+      tc::mbar_init(&S.cempty[s], 1);
+    }
+    for (int s = 0; s < kOStages; ++s) {
+      tc::mbar_init(&S.ofull[s], 1);
+      tc::mbar_init(&S.oempty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(&S.tfull[a], 1);
+      tc::mbar_init(&S.tempty[a], 256);
+    }
+    tc::mbar_init(&S.drain, 1);
+    S.abort = 0;
+    S.budget = kTimeoutCycles;
+    tc::fence_barrier_init();
+    for (int64_t i = 0; i < kCStages; ++i) {  // the first stages need no free slot
+      const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+      if (p >= ngroups) break;
+      issue(i, p);
+      first_issued = i + 1;
+    }
+  }
+  tc::grid_dep_launch();
+  // H_128 in fp16 as the A operand: K-major, two K blocks of [128 rows m][64 k], 128-byte swizzle.
+  for (uint32_t c = threadIdx.x; c < 2048; c += kThreads) {
+    const uint32_t kb = c >> 10, m = (c >> 3) & 127u, ch = c & 7u;
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t k0 = kb * 64 + ch * 8 + 2 * j;
+      const uint32_t lo = (__popc(m & k0) & 1) ? 0xBC00u : 0x3C00u;
+      const uint32_t hi = (__popc(m & (k0 + 1)) & 1) ? 0xBC00u : 0x3C00u;
+      w[j] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4 *>(smem + kOffH + kb * 16384 + m * 128u + ((ch ^ (m & 7u)) << 4)) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  tc::fence_proxy_async_smem();
+  if (warp == 1) {
+    tc::tmem_alloc(&S.tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  // ------------------------------------------------------------ roles
+  if (warp == 0) {
+    if (lane == 0) {
+      int64_t last[kCStages] = {-1, -1, -1};
+      for (int64_t i = 0; i < first_issued; ++i) last[i] = i;
+      for (int64_t i = first_issued;; ++i) {
+        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+        if (p >= ngroups) break;
+        const int cs = (int)(i % kCStages);
+        if (!wait_bounded(&S.cempty[cs], (uint32_t)((i / kCStages) & 1) ^ 1u, S, true)) break;
+        issue(i, p);
+        last[cs] = i;
+      }
+      // every issued copy has landed before the CTA can leave
+      for (int s = 0; s < kCStages; ++s)
+        if (last[s] >= 0) wait_bounded(&S.cfull[s], (uint32_t)((last[s] / kCStages) & 1), S, false);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(128, SH::SPLIT ? 128 : 256, true);
+      constexpr uint32_t idesc_neg = idesc | (1u << 13);  // negate A
+      const uint32_t sH = tc::smem_u32(smem + kOffH), sO = tc::smem_u32(smem + kOffO);
+      for (int64_t i = 0;; ++i) {
+        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+        if (p >= ngroups) break;
+        const int os = (int)(i % kOStages), acc = (int)(i & 1);
+        if (!wait_bounded(&S.ofull[os], (uint32_t)((i / kOStages) & 1), S, true)) break;
+        if (!wait_bounded(&S.tempty[acc], (uint32_t)((i >> 1) & 1) ^ 1u, S, true)) break;
+        tc::tc_fence_after();
+        if constexpr (SH::SPLIT) {
+          // columns 128 u + b: sum over row blocks v of (-1)^(u v) H_128 C'_v
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int v = 0; v < 2; ++v)
+#pragma unroll
+              for (int s = 0; s < 8; ++s) {
+                const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
+                uint64_t bd = tc::smem_desc(sO + os * kOpBytes + v * SH::CBOX * SH::BOXBYTES + s * 16 * SH::ROWB,
+                                            SH::BOXBYTES, 8 * SH::ROWB);
+                bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
+                tc::umma_bf16(tmem + acc * 256 + u * 128, ad, bd, (u & v) ? idesc_neg : idesc,
+                              (v > 0 || s > 0) ? 1u : 0u);
+              }
+        } else {
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
+            uint64_t bd = tc::smem_desc(sO + os * kOpBytes + s * 16 * SH::ROWB, SH::BOXBYTES, 8 * SH::ROWB);
+            bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
+            tc::umma_bf16(tmem + acc * 256, ad, bd, idesc, s > 0 ? 1u : 0u);
+          }
+        }
+        tc::umma_commit(&S.oempty[os]);
+        tc::umma_commit(&S.tfull[acc]);
+      }
+    }
+  } else if (warp < 4) {
+    // Converters: thread ts expands code words 4 (ts + 64 k) .. + 3, k < 16, of the
+    // group (16-byte loads; 32 consecutive elements of one matrix row).
+    const uint32_t ts = threadIdx.x - 64;  // 0..63
+    for (int64_t i = 0;; ++i) {
+      const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+      if (p >= ngroups) break;
+      const int cs = (int)(i % kCStages), os = (int)(i % kOStages);
+      if (ts < (uint32_t)SH::TOK) {
+        const int64_t row = p * SH::TOK + ts;
+        float z = 8.0f;  // symmetric codes: c + 8 after flipping the nibble's top bit
+        if (asym) z = row < rows ? __half2float(zero[row]) : 0.0f;
+        S.zc[ts] = __float2half2_rn(-(1024.0f + z));
+      }
+      if (ts == 0) {
+        int ok = wait_bounded(&S.cfull[cs], (uint32_t)((i / kCStages) & 1), S, true) ? 1 : 0;
+        if (ok) ok = wait_bounded(&S.oempty[os], (uint32_t)((i / kOStages) & 1) ^ 1u, S, true) ? 1 : 0;
+        S.dec[2] = ok;
+      }
+      tc::named_sync(3, 64);
+      if (!S.dec[2]) break;
+      const uint4 *cw = reinterpret_cast<const uint4 *>(smem + kOffC + cs * kCodeBytes);
+      uint8_t *op = smem + kOffO + os * kOpBytes;
+      const uint32_t flip = asym ? 0u : 0x88888888u;
+#pragma unroll 2
+      for (int k = 0; k < 16; ++k) {
+        const uint32_t q = ts + 64u * k;  // quad of code words
+        uint4 w = cw[q];
+        const uint32_t word0 = 4u * q;
+        const uint32_t t = word0 / SH::WPT;                  // token row in the group
+        const uint32_t e = (word0 % SH::WPT) * 8u;           // first element
+        const uint32_t r = e / B, b = e % B;                 // matrix row and column
+        const uint32_t a = r & 127u, j = (r >> 7) * SH::CBOX + b / SH::BOXW;
+        const uint32_t c0 = (b % SH::BOXW) / 8u;             // first 16-byte chunk in the tile row
+        uint8_t *rowp = op + (t * SH::BPT + j) * SH::BOXBYTES + a * SH::ROWB;
+        const uint32_t sx = SH::ROWB == 128 ? (a & 7u) : ((a >> 1) & 3u);
+        const __half2 zc = S.zc[t];
+        const uint32_t ws[4] = {w.x ^ flip, w.y ^ flip, w.z ^ flip, w.w ^ flip};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4 *>(rowp + (((c0 + u) ^ sx) << 4)) = expand8(ws[u], zc);
+      }
+      tc::fence_proxy_async_smem();
+      tc::named_sync(3, 64);
+      if (ts == 0) {
+        tc::mbar_arrive(&S.cempty[cs]);
+        tc::mbar_arrive(&S.ofull[os]);
+      }
+    }
+  } else {
+    // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1)
+    const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
+    const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
+    const uint32_t orow = SH::SPLIT ? 128u * g + row : row;  // output matrix row
+    uint32_t sw[B / 32];  // this row's sign words (the same for every token row)
+#pragma unroll
+    for (int k = 0; k < B / 32; ++k) sw[k] = SIGNS ? __ldg(signs + (orow * B) / 32 + k) : 0u;
+    for (int64_t i = 0;; ++i) {
+      const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+      if (p >= ngroups) break;
+      const int acc = (int)(i & 1);
+      if (tg == 0) S.dec[g] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+      tc::named_sync(1 + g, 128);
+      if (!S.dec[g]) break;
+      tc::tc_fence_after();
+      float v[kRegs];
+      {
+        uint32_t r[kRegs];
+        const uint32_t taddr = tmem + ((wq * 32u) << 16) + (uint32_t)acc * 256u + g * 128u;
+        tc::tmem_ld32(taddr, r);
+        tc::tmem_ld32(taddr + 32, r + 32);
+        tc::tmem_ld32(taddr + 64, r + 64);
+        tc::tmem_ld32(taddr + 96, r + 96);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < kRegs; ++k) v[k] = __uint_as_float(r[k]);
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&S.tempty[acc]);
+      // second Kronecker factor: H_B over b inside each token row's segment
+      stage<0>(v);
+      stage<1>(v);
+      stage<2>(v);
+      stage<3>(v);
+      stage<4>(v);
+      if constexpr (SH::LOGB > 5) stage<5>(v);
+      if constexpr (SH::LOGB > 6) stage<6>(v);
+#pragma unroll
+      for (int sg = 0; sg < SEG; ++sg) {
+        const int64_t token = SH::SPLIT ? p : p * SH::TOK + g * SEG + sg;
+        if (token >= rows) continue;
+        const float s = asym ? __half2float(static_cast<const __half *>(scale)[token])
+                             : static_cast<const float *>(scale)[token];
+        const float m = s * inv_sqrt_n;
+        float *w = v + sg * B;
+#pragma unroll
+        for (int k = 0; k < B; k += 2) mul2(w[k], w[k + 1], m);
+        if constexpr (SIGNS) {
+#pragma unroll
+          for (int k = 0; k < B; ++k)
+            w[k] = __uint_as_float(__float_as_uint(w[k]) ^ ((sw[k >> 5] >> (k & 31)) << 31));
+        }
+        const int64_t off = token * (int64_t)(B * SH::ROWS) + (int64_t)orow * B;  // first element of the row
+        if constexpr (F32) {
+          float *dst = static_cast<float *>(out) + off;
+#pragma unroll
+          for (int k = 0; k < B; k += 8)
+            store8<STORE32>(dst + k, __float_as_uint(w[k]), __float_as_uint(w[k + 1]), __float_as_uint(w[k + 2]),
+                            __float_as_uint(w[k + 3]), __float_as_uint(w[k + 4]), __float_as_uint(w[k + 5]),
+                            __float_as_uint(w[k + 6]), __float_as_uint(w[k + 7]));
+        } else {
+          uint16_t *dst = static_cast<uint16_t *>(out) + off;
+#pragma unroll
+          for (int k = 0; k < B; k += 16)
+            store8<STORE32>(dst + k, pack_bf16x2(w[k], w[k + 1]), pack_bf16x2(w[k + 2], w[k + 3]),
+                            pack_bf16x2(w[k + 4], w[k + 5]), pack_bf16x2(w[k + 6], w[k + 7]),
+                            pack_bf16x2(w[k + 8], w[k + 9]), pack_bf16x2(w[k + 10], w[k + 11]),
+                            pack_bf16x2(w[k + 12], w[k + 13]), pack_bf16x2(w[k + 14], w[k + 15]));
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0) {
+      tc::umma_commit(&S.drain);  // arrives once every MMA this thread issued is complete
+      wait_bounded(&S.drain, 0, S, false);
+    }
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int LOGN, bool SIGNS, bool F32, bool STORE32>
+cudaError_t launch_tc(const uint8_t *codes, int64_t rows, const void *scale, const void *zero,
+                      const uint32_t *signs, void *out, bool asym, cudaStream_t stream) {
+  using SH = Shape<LOGN>;
+  auto kern = k3_tc_dequant_inverse<LOGN, SIGNS, F32, STORE32>;
+  int slots = 0;
+  cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreads, (int)kSmemBytes, &slots);
+  if (err != cudaSuccess) return err;
+  const int64_t ngroups = (rows + SH::TOK - 1) / SH::TOK;
+  const int64_t grid = ngroups < slots ? ngroups : slots;
+  const float inv_sqrt_n = (float)(1.0 / std::sqrt((double)(1 << LOGN)));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, codes, rows, inv_sqrt_n, scale, static_cast<const __half *>(zero), signs,
+                            out, asym ? 1 : 0);
+}
+
+template <int LOGN, bool SIGNS>
+cudaError_t launch_s(const uint8_t *codes, int64_t rows, const void *scale, const void *zero, const uint32_t *signs,
+                     void *out, bool asym, bool f32, cudaStream_t stream) {
+  const bool a32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;  // 32-byte stores need 32-byte alignment
+  if (f32)
+    return a32 ? launch_tc<LOGN, SIGNS, true, true>(codes, rows, scale, zero, signs, out, asym, stream)
+               : launch_tc<LOGN, SIGNS, true, false>(codes, rows, scale, zero, signs, out, asym, stream);
+  return a32 ? launch_tc<LOGN, SIGNS, false, true>(codes, rows, scale, zero, signs, out, asym, stream)
+             : launch_tc<LOGN, SIGNS, false, false>(codes, rows, scale, zero, signs, out, asym, stream);
+}
+
+template <int LOGN>
+cudaError_t launch_n(const uint8_t *codes, int64_t rows, const void *scale, const void *zero, const uint32_t *signs,
+                     void *out, bool asym, bool f32, cudaStream_t stream) {
+  return signs ? launch_s<LOGN, true>(codes, rows, scale, zero, signs, out, asym, f32, stream)
+               : launch_s<LOGN, false>(codes, rows, scale, zero, nullptr, out, asym, f32, stream);
+}
+
+}  // namespace
+
+bool tc_dequant_supported(int log_n, int64_t rows, uint32_t flags) {
+  if (log_n < 12 || log_n > 15 || (flags & kNoRotate) || rows <= 0) return false;
+  if (rows * (int64_t(1) << log_n) >= (int64_t(1) << 40)) return false;
+  const int64_t rows_per_group = log_n == 15 ? 1 : int64_t(256) >> (log_n - 7);
+  return (flags & kTensorCores) || rows >= 128 * rows_per_group;
+}
+
+cudaError_t launch_dequant_inverse_tc(int log_n, const uint8_t *codes, int64_t rows, int mode, const void *scale,
+                                      const void *zero, const uint32_t *signs, void *out, int out_dtype,
+                                      cudaStream_t stream) {
+  const bool asym = mode == 1, f32 = out_dtype == 1;
+  switch (log_n) {
+    case 12: return launch_n<12>(codes, rows, scale, zero, signs, out, asym, f32, stream);
+    case 13: return launch_n<13>(codes, rows, scale, zero, signs, out, asym, f32, stream);
+    case 14: return launch_n<14>(codes, rows, scale, zero, signs, out, asym, f32, stream);
+    case 15: return launch_n<15>(codes, rows, scale, zero, signs, out, asym, f32, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t read_dequant_status(unsigned int *status, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(status, g_dequant_status, sizeof(unsigned int));
+  if (e != cudaSuccess || !reset) return e;
+  const unsigned int zero = 0u;
+  return cudaMemcpyToSymbol(g_dequant_status, &zero, sizeof(unsigned int));
+}
+
+}  // namespace spin

@@ -35,9 +35,16 @@ cudaError_t launch_rotate_quant_int4_tc(int log_n, const void *x, int64_t tokens
 void set_stall_test(int enable);
 
 // Device status words set by kernels whose bounded waits ran out (the tensor-core
-// R4 kernel and the R3 kernel each keep one).
+// R4 kernel, the R3 kernel and the tensor-core dequantise kernel each keep one).
 cudaError_t read_device_status(unsigned int *status, bool reset);
 cudaError_t read_rope_status(unsigned int *status, bool reset);
+
+// Tensor-core dequantise + inverse kernel (n = 4096 to 32768): availability and launcher.
+bool tc_dequant_supported(int log_n, int64_t rows, uint32_t flags);
+cudaError_t launch_dequant_inverse_tc(int log_n, const uint8_t *codes, int64_t rows, int mode, const void *scale,
+                                      const void *zero, const uint32_t *signs, void *out, int out_dtype,
+                                      cudaStream_t stream);
+cudaError_t read_dequant_status(unsigned int *status, bool reset);
 
 cudaError_t launch_dequant_inverse(const uint8_t *codes, int64_t rows, int log_n, int mode,
                                    const void *scale, const void *zero, const uint32_t *signs,

@@ -104,6 +104,8 @@ def test_dequant_argument_checks(L):
     assert f(FAKE + 8, 4, 256, 0, FAKE, None, None, 0, FAKE, 0, None) == 3
     assert f(FAKE, 4, 256, 0, FAKE + 2, None, None, 0, FAKE, 0, None) == 3
     assert f(FAKE, 4, 256, 1, FAKE + 2, FAKE + 1, None, 0, FAKE, 0, None) == 3
+    assert f(FAKE, 4, 4096, 0, FAKE, None, None, 8, FAKE, 0, None) == 1  # unknown flag
+    assert f(FAKE, 4, 4096, 0, FAKE, None, None, 6, FAKE, 0, None) == 1  # both kernel choices
 
 
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
