@@ -176,7 +176,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int B = SH::B, SEG = SH::SEG;
   static_assert(!(SIGNS && SH::SPLIT), "the sign masks of n = 32768 do not fit in registers");
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, derived from the shared array itself so that accesses
+  // through it stay shared-memory accesses
+  uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   Shared &S = *reinterpret_cast<Shared *>(smem + kOffBar);
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
   const int64_t ngroups = (tokens + SH::TOK - 1) / SH::TOK;

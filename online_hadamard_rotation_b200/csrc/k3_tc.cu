@@ -27,11 +27,11 @@
 // 128-column halves, and epilogue warpgroup g writes output rows 128 g + a'.
 //
 // Roles (384 threads, one CTA per SM, persistent over groups):
-//   warp 0      producer: one bulk copy of the group's 16 KiB of codes into a
-//               three-stage ring
-//   warp 1      TMEM owner and MMA issuer
-//   warps 2-3   converters: codes -> fp16 operand, two-stage ring of 64 KiB
-//   warps 4-11  epilogue, two warpgroups over TMEM columns 0-127 and 128-255
+//   warps 0, 2, 3  converters: codes -> fp16 operand (two-stage ring of 64 KiB);
+//                  thread 0 also issues each group's 16 KiB bulk copy of codes
+//                  into a three-stage ring
+//   warp 1         TMEM owner and MMA issuer
+//   warps 4-11     epilogue, two warpgroups over TMEM columns 0-127 and 128-255
 // Every mbarrier wait is bounded by a clock budget; on expiry the CTA records a
 // status (read by spin_device_status), drains its copies and MMAs, frees TMEM and
 // returns.
@@ -84,7 +84,7 @@ struct Shape {
 };
 
 struct Shared {
-  uint64_t cfull[kCStages], cempty[kCStages], ofull[kOStages], oempty[kOStages], tfull[2], tempty[2], drain;
+  uint64_t cfull[kCStages], ofull[kOStages], oempty[kOStages], tfull[2], tempty[2], drain;
   uint32_t tmem_base;
   int abort;
   int dec[3];
@@ -157,12 +157,10 @@ __device__ __forceinline__ uint4 expand8(uint32_t w, __half2 zc) {
   h[1] = __byte_perm(e0, 0x64646464u, 0x4342);
   h[2] = __byte_perm(e1, 0x64646464u, 0x4140);
   h[3] = __byte_perm(e1, 0x64646464u, 0x4342);
+  const uint32_t z = *reinterpret_cast<const uint32_t *>(&zc);
   uint32_t o[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __half2 v = __hadd2(*reinterpret_cast<const __half2 *>(&h[i]), zc);
-    o[i] = *reinterpret_cast<const uint32_t *>(&v);
-  }
+  for (int i = 0; i < 4; ++i) asm("add.rn.f16x2 %0, %1, %2;" : "=r"(o[i]) : "r"(h[i]), "r"(z));
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
@@ -174,7 +172,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   using SH = Shape<LOGN>;
   constexpr int B = SH::B, SEG = SH::SEG;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, derived from the shared array itself so that accesses
+  // through it stay shared-memory accesses
+  uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   Shared &S = *reinterpret_cast<Shared *>(smem + kOffBar);
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
   const int64_t ngroups = (rows + SH::TOK - 1) / SH::TOK;
@@ -191,10 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bulk_load(smem + kOffC + cs * kCodeBytes, codes + t0 * (int64_t)(SH::WPT * 4), bytes, &S.cfull[cs]);
   };
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kCStages; ++s) {
-      tc::mbar_init(&S.cfull[s], 1);
-      tc::mbar_init(&S.cempty[s], 1);
-    }
+    for (int s = 0; s < kCStages; ++s) tc::mbar_init(&S.cfull[s], 1);
     for (int s = 0; s < kOStages; ++s) {
       tc::mbar_init(&S.ofull[s], 1);
       tc::mbar_init(&S.oempty[s], 1);
@@ -240,23 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = S.tmem_base;
 
   // ------------------------------------------------------------ roles
-  if (warp == 0) {
-    if (lane == 0) {
-      int64_t last[kCStages] = {-1, -1, -1};
-      for (int64_t i = 0; i < first_issued; ++i) last[i] = i;
-      for (int64_t i = first_issued;; ++i) {
-        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
-        if (p >= ngroups) break;
-        const int cs = (int)(i % kCStages);
-        if (!wait_bounded(&S.cempty[cs], (uint32_t)((i / kCStages) & 1) ^ 1u, S, true)) break;
-        issue(i, p);
-        last[cs] = i;
-      }
-      // every issued copy has landed before the CTA can leave
-      for (int s = 0; s < kCStages; ++s)
-        if (last[s] >= 0) wait_bounded(&S.cfull[s], (uint32_t)((last[s] / kCStages) & 1), S, false);
-    }
-  } else if (warp == 1) {
+  if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(128, SH::SPLIT ? 128 : 256, true);
       constexpr uint32_t idesc_neg = idesc | (1u << 13);  // negate A
@@ -297,40 +278,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp < 4) {
-    // Converters: thread ts expands code words 4 (ts + 64 k) .. + 3, k < 16, of the
-    // group (16-byte loads; 32 consecutive elements of one matrix row).
-    const uint32_t ts = threadIdx.x - 64;  // 0..63
+    // Converters (warps 0, 2, 3): converter c expands the quads (four code words, 32
+    // consecutive elements of one matrix row) of slots c, c + 96, ... < 1024 of the
+    // group. A slot's bits are, from the bottom: the half of a 64-column tile row (when
+    // the tile is 64 wide), the row a (7 bits), the column tile, then the token row (or
+    // the 128-row block at n = 32768); so the eight lanes of a 16-byte store phase write
+    // eight different bank groups of the swizzled tiles. Converter 0 (thread 0) also
+    // refills each codes stage with the group kCStages steps ahead as soon as the group
+    // in it has been converted.
+    constexpr uint32_t kConv = 96;
+    const uint32_t cid = warp == 0 ? lane : threadIdx.x - 32;
+    int64_t last[kCStages] = {-1, -1, -1};  // converter 0: last group index issued per stage
+    for (int64_t i = 0; i < first_issued; ++i) last[i] = i;
     for (int64_t i = 0;; ++i) {
       const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
       if (p >= ngroups) break;
       const int cs = (int)(i % kCStages), os = (int)(i % kOStages);
-      if (ts < (uint32_t)SH::TOK) {
-        const int64_t row = p * SH::TOK + ts;
+      if (cid < (uint32_t)SH::TOK) {
+        const int64_t row = p * SH::TOK + cid;
         float z = 8.0f;  // symmetric codes: c + 8 after flipping the nibble's top bit
         if (asym) z = row < rows ? __half2float(zero[row]) : 0.0f;
-        S.zc[ts] = __float2half2_rn(-(1024.0f + z));
+        S.zc[cid] = __float2half2_rn(-(1024.0f + z));
       }
-      if (ts == 0) {
+      if (cid == 0) {
         int ok = wait_bounded(&S.cfull[cs], (uint32_t)((i / kCStages) & 1), S, true) ? 1 : 0;
         if (ok) ok = wait_bounded(&S.oempty[os], (uint32_t)((i / kOStages) & 1) ^ 1u, S, true) ? 1 : 0;
         S.dec[2] = ok;
       }
-      tc::named_sync(3, 64);
+      tc::named_sync(3, kConv);
       if (!S.dec[2]) break;
       const uint4 *cw = reinterpret_cast<const uint4 *>(smem + kOffC + cs * kCodeBytes);
       uint8_t *op = smem + kOffO + os * kOpBytes;
       const uint32_t flip = asym ? 0u : 0x88888888u;
 #pragma unroll 2
-      for (int k = 0; k < 16; ++k) {
-        const uint32_t q = ts + 64u * k;  // quad of code words
-        uint4 w = cw[q];
-        const uint32_t word0 = 4u * q;
-        const uint32_t t = word0 / SH::WPT;                  // token row in the group
-        const uint32_t e = (word0 % SH::WPT) * 8u;           // first element
-        const uint32_t r = e / B, b = e % B;                 // matrix row and column
-        const uint32_t a = r & 127u, j = (r >> 7) * SH::CBOX + b / SH::BOXW;
-        const uint32_t c0 = (b % SH::BOXW) / 8u;             // first 16-byte chunk in the tile row
-        uint8_t *rowp = op + (t * SH::BPT + j) * SH::BOXBYTES + a * SH::ROWB;
+      for (uint32_t q = cid; q < 1024u; q += kConv) {
+        constexpr uint32_t HB = SH::BOXW / 32, LHB = HB == 2 ? 1 : 0;  // quads per tile row
+        const uint32_t h = q & (HB - 1), a = (q >> LHB) & 127u, rest = q >> (LHB + 7);
+        const uint32_t jc = rest % SH::CBOX, blk = rest / SH::CBOX;  // column tile, token row or row block
+        const uint32_t t = SH::SPLIT ? 0u : blk, rb = SH::SPLIT ? blk : 0u;
+        const uint32_t e = B * (128u * rb + a) + SH::BOXW * jc + 32u * h;  // first element in the token row
+        const uint4 w = cw[(t * SH::WPT + e / 8u) / 4u];
+        const uint32_t c0 = 4u * h;                          // first 16-byte chunk in the tile row
+        uint8_t *rowp = op + (t * SH::BPT + rb * SH::CBOX + jc) * SH::BOXBYTES + a * SH::ROWB;
         const uint32_t sx = SH::ROWB == 128 ? (a & 7u) : ((a >> 1) & 3u);
         const __half2 zc = S.zc[t];
         const uint32_t ws[4] = {w.x ^ flip, w.y ^ flip, w.z ^ flip, w.w ^ flip};
@@ -339,12 +328,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4 *>(rowp + (((c0 + u) ^ sx) << 4)) = expand8(ws[u], zc);
       }
       tc::fence_proxy_async_smem();
-      tc::named_sync(3, 64);
-      if (ts == 0) {
-        tc::mbar_arrive(&S.cempty[cs]);
+      tc::named_sync(3, kConv);
+      if (cid == 0) {
         tc::mbar_arrive(&S.ofull[os]);
+        const int64_t inext = i + kCStages, pn = blockIdx.x + inext * (int64_t)gridDim.x;
+        if (pn < ngroups && !*reinterpret_cast<volatile int *>(&S.abort)) {
+          tc::fence_proxy_async_smem();  // every converter's reads of the stage come before the copy
+          issue(inext, pn);
+          last[cs] = inext;
+        }
       }
     }
+    if (cid == 0)  // every issued copy has landed before the CTA can leave
+      for (int s2 = 0; s2 < kCStages; ++s2)
+        if (last[s2] >= 0) wait_bounded(&S.cfull[s2], (uint32_t)((last[s2] / kCStages) & 1), S, false);
   } else {
     // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1)
     const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
@@ -353,9 +350,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t sw[B / 32];  // this row's sign words (the same for every token row)
 #pragma unroll
     for (int k = 0; k < B / 32; ++k) sw[k] = SIGNS ? __ldg(signs + (orow * B) / 32 + k) : 0u;
+    // The row steps of a group are loaded one group ahead, so their DRAM latency hides
+    // behind the previous group's work: raw bits, converted when used.
+    auto load_steps = [&](int64_t pp, uint32_t (&dst)[SEG]) {
+#pragma unroll
+      for (int sg = 0; sg < SEG; ++sg) {
+        const int64_t token = SH::SPLIT ? pp : pp * SH::TOK + g * SEG + sg;
+        dst[sg] = 0u;
+        if (pp < ngroups && token < rows)
+          dst[sg] = asym ? (uint32_t)__ldg(static_cast<const unsigned short *>(scale) + token)
+                         : __float_as_uint(__ldg(static_cast<const float *>(scale) + token));
+      }
+    };
+    uint32_t step_next[SEG];
+    load_steps(blockIdx.x, step_next);
     for (int64_t i = 0;; ++i) {
       const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
       if (p >= ngroups) break;
+      uint32_t step_raw[SEG];
+#pragma unroll
+      for (int sg = 0; sg < SEG; ++sg) step_raw[sg] = step_next[sg];
+      load_steps(p + gridDim.x, step_next);
       const int acc = (int)(i & 1);
       if (tg == 0) S.dec[g] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
       tc::named_sync(1 + g, 128);
@@ -387,33 +402,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int sg = 0; sg < SEG; ++sg) {
         const int64_t token = SH::SPLIT ? p : p * SH::TOK + g * SEG + sg;
         if (token >= rows) continue;
-        const float s = asym ? __half2float(static_cast<const __half *>(scale)[token])
-                             : static_cast<const float *>(scale)[token];
+        const float s = asym ? __half2float(__ushort_as_half((unsigned short)step_raw[sg]))
+                             : __uint_as_float(step_raw[sg]);
         const float m = s * inv_sqrt_n;
-        float *w = v + sg * B;
-#pragma unroll
-        for (int k = 0; k < B; k += 2) mul2(w[k], w[k + 1], m);
-        if constexpr (SIGNS) {
-#pragma unroll
-          for (int k = 0; k < B; ++k)
-            w[k] = __uint_as_float(__float_as_uint(w[k]) ^ ((sw[k >> 5] >> (k & 31)) << 31));
-        }
+        const float *w = v + sg * B;
         const int64_t off = token * (int64_t)(B * SH::ROWS) + (int64_t)orow * B;  // first element of the row
-        if constexpr (F32) {
-          float *dst = static_cast<float *>(out) + off;
+        // one 8 (fp32) or 16 (bf16) element piece at a time: scale, diagonal sign, store
+        constexpr int P = F32 ? 8 : 16;
 #pragma unroll
-          for (int k = 0; k < B; k += 8)
-            store8<STORE32>(dst + k, __float_as_uint(w[k]), __float_as_uint(w[k + 1]), __float_as_uint(w[k + 2]),
-                            __float_as_uint(w[k + 3]), __float_as_uint(w[k + 4]), __float_as_uint(w[k + 5]),
-                            __float_as_uint(w[k + 6]), __float_as_uint(w[k + 7]));
-        } else {
-          uint16_t *dst = static_cast<uint16_t *>(out) + off;
+        for (int k = 0; k < B; k += P) {
+          float o[P];
 #pragma unroll
-          for (int k = 0; k < B; k += 16)
-            store8<STORE32>(dst + k, pack_bf16x2(w[k], w[k + 1]), pack_bf16x2(w[k + 2], w[k + 3]),
-                            pack_bf16x2(w[k + 4], w[k + 5]), pack_bf16x2(w[k + 6], w[k + 7]),
-                            pack_bf16x2(w[k + 8], w[k + 9]), pack_bf16x2(w[k + 10], w[k + 11]),
-                            pack_bf16x2(w[k + 12], w[k + 13]), pack_bf16x2(w[k + 14], w[k + 15]));
+          for (int u = 0; u < P; u += 2) {
+            o[u] = w[k + u];
+            o[u + 1] = w[k + u + 1];
+            mul2(o[u], o[u + 1], m);
+          }
+          if constexpr (SIGNS) {
+            const uint32_t sb = sw[k >> 5] >> (k & 31);
+#pragma unroll
+            for (int u = 0; u < P; ++u) o[u] = __uint_as_float(__float_as_uint(o[u]) ^ (((sb >> u) & 1u) << 31));
+          }
+          if constexpr (F32) {
+            store8<STORE32>(static_cast<float *>(out) + off + k, __float_as_uint(o[0]), __float_as_uint(o[1]),
+                            __float_as_uint(o[2]), __float_as_uint(o[3]), __float_as_uint(o[4]),
+                            __float_as_uint(o[5]), __float_as_uint(o[6]), __float_as_uint(o[7]));
+          } else {
+            store8<STORE32>(static_cast<uint16_t *>(out) + off + k, pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                            pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]), pack_bf16x2(o[8], o[9]),
+                            pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]), pack_bf16x2(o[14], o[15]));
+          }
         }
       }
     }
