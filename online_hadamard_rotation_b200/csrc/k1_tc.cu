@@ -21,7 +21,11 @@
 //      max, step, INT4 codes and nibble packing. Row a' of a token is B / 2
 //      contiguous code bytes.
 //
-// Roles (384 threads, one CTA per SM, persistent over groups of 256 / B tokens):
+// Work: one CTA per group of 256 / B tokens is launched; one CTA fits an SM, and each
+// resident CTA, after its own group, takes over groups of CTAs that have not started
+// yet (cluster launch control `try_cancel`), so the work spreads dynamically over the
+// SMs and the last groups land wherever an SM is free.
+// Roles (384 threads, one CTA per SM, persistent over groups):
 //   warp 0      TMA producer: 64 KiB per group (boxes of [128 rows][min(B, 64)]
 //               bf16 with 64- or 128-byte swizzle) into a three-stage ring
 //   warp 1      TMEM owner and MMA issuer (8 MMAs of K = 16 per group)
@@ -62,7 +66,7 @@ constexpr uint32_t kGroupBytes = 65536;            // one MMA group: 128 rows x 
 constexpr uint32_t kOffH = 0;                      // A operand: H_128, K-major, 2 x 16 KiB
 constexpr uint32_t kOffX = 32768;                  // ring of kStages x 64 KiB
 constexpr uint32_t kOffBar = kOffX + kStages * kGroupBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;  // + alignment slack
+constexpr uint32_t kSmemBytes = kOffBar + 1024 + 1024;  // barrier area + alignment slack
 constexpr long long kTimeoutCycles = 4000000000LL;     // about two seconds
 constexpr long long kStallTestCycles = 2000000LL;      // about a millisecond, for the stall test hook
 
@@ -93,15 +97,47 @@ struct Shape {
   static_assert(LOGN >= 12 && LOGN <= 15, "tensor-core R4 covers n = 4096 .. 32768");
 };
 
+constexpr int kRing = 8;  // group ids in flight between the producer and the epilogue
+
 struct Shared {
-  uint64_t full[kStages], sgn[kStages], empty[kStages], tfull[2], tempty[2], drain;
+  uint4 clc_resp;          // response of the pending work-stealing request
+  uint64_t full[kStages], sgn[kStages], empty[kStages], tfull[2], tempty[2], drain, clc;
+  uint64_t gfull[kRing];   // group id i & 7 written
+  int64_t gid[kRing];      // group of the CTA's i-th step (i & 7), -1 once there is none
+  int64_t egid[2];         // epilogue warpgroup g's current group
   uint32_t tmem_base;
   int abort;
   int dec[3];
   long long budget;        // clock cycles a wait may take before the CTA gives up
   float wmax[2][2][4][4];  // [warpgroup][group parity][warp][token segment]
 };
-static_assert(sizeof(Shared) <= 512, "barrier area");
+static_assert(sizeof(Shared) <= 1024, "barrier area");
+
+// Work stealing by cluster launch control: ask the hardware to cancel a CTA of this
+// grid that has not started yet; its 16-byte response lands in `resp` and completes
+// `bar`. Issued by one thread, never again after a response that cancelled nothing.
+__device__ __forceinline__ void clc_request(uint4 *resp, uint64_t *bar) {
+  tc::mbar_arrive_expect_tx(bar, 16);
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+          tc::smem_u32(resp)),
+      "r"(tc::smem_u32(bar))
+      : "memory");
+}
+// The cancelled CTA's x index, or -1 if the request cancelled nothing.
+__device__ __forceinline__ int64_t clc_result(const uint4 *resp) {
+  uint32_t ok, x;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b128 q;\n\t"
+      "ld.shared.b128 q, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, q;\n\t}"
+      : "=r"(ok), "=r"(x)
+      : "r"(tc::smem_u32(resp))
+      : "memory");
+  return ok ? (int64_t)x : -1;
+}
 
 __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, Shared &S, bool honor_abort) {
   if (tc::mbar_try_wait_suspend(bar, parity)) return true;
@@ -199,18 +235,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&S.tempty[a], 256);
     }
     tc::mbar_init(&S.drain, 1);
+    tc::mbar_init(&S.clc, 1);
+    for (int j = 0; j < kRing; ++j) tc::mbar_init(&S.gfull[j], 1);
     S.abort = 0;
     S.budget = stall_test ? kStallTestCycles : kTimeoutCycles;
     tc::fence_barrier_init();
     tc::prefetch_tensormap(&xmap);
-    // The first kStages groups need no free slot: start their copies now, so the
-    // DRAM latency overlaps the rest of the setup.
-    for (int64_t i = 0; i < kStages; ++i) {
-      const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
-      if (p >= ngroups) break;
-      load_group<LOGN>(smem + kOffX + i * kGroupBytes, &xmap, &S.full[i], p, tokens);
-      first_issued = i + 1;
-    }
+    // The CTA's own group needs no free slot: start its copies now, so the DRAM
+    // latency overlaps the rest of the setup; ask for the next group at once.
+    S.gid[0] = blockIdx.x;
+    tc::mbar_arrive(&S.gfull[0]);
+    load_group<LOGN>(smem + kOffX, &xmap, &S.full[0], blockIdx.x, tokens);
+    first_issued = 1;
+    clc_request(&S.clc_resp, &S.clc);
   }
   tc::grid_dep_launch();
   // H_128 as the A operand: K-major, two K blocks of [128 rows m][64 k], 128-byte swizzle.
@@ -241,17 +278,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int64_t last[kStages] = {-1, -1, -1};
       for (int64_t i = 0; i < first_issued; ++i) last[i] = i;
+      bool pending = true;  // a work-stealing request is in flight
+      uint32_t clc_phase = 0;
       for (int64_t i = first_issued;; ++i) {
-        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
-        if (p >= ngroups) break;
+        // the group of step i: the one the last request cancelled, or none
+        int64_t p = -1;
+        if (pending) {
+          if (!wait_bounded(&S.clc, clc_phase, S, true)) break;
+          clc_phase ^= 1u;
+          p = clc_result(&S.clc_resp);
+          if (p >= ngroups) p = -1;
+          pending = p >= 0;
+          if (pending) clc_request(&S.clc_resp, &S.clc);
+        }
         const int st = (int)(i % kStages);
         if (!wait_bounded(&S.empty[st], (uint32_t)((i / kStages) & 1) ^ 1u, S, true)) break;
+        S.gid[i % kRing] = p;
+        tc::mbar_arrive(&S.gfull[i % kRing]);
+        if (p < 0) {
+          tc::mbar_arrive(&S.full[st]);  // no copies: the sign warps and the MMA read the end mark
+          last[st] = -1;  // its previous copy was consumed before the slot came free
+          break;
+        }
         load_group<LOGN>(smem + kOffX + st * kGroupBytes, &xmap, &S.full[st], p, tokens);
         last[st] = i;
       }
-      // every issued copy has landed before the CTA can leave
+      // every issued copy (and work request) has landed before the CTA can leave
       for (int s = 0; s < kStages; ++s)
         if (last[s] >= 0) wait_bounded(&S.full[s], (uint32_t)((last[s] / kStages) & 1), S, false);
+      if (pending) wait_bounded(&S.clc, clc_phase, S, false);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -259,10 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_neg = idesc | (1u << 13);  // negate A
       const uint32_t sH = tc::smem_u32(smem + kOffH), sX = tc::smem_u32(smem + kOffX);
       for (int64_t i = 0;; ++i) {
-        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
-        if (p >= ngroups) break;
         const int st = (int)(i % kStages), acc = (int)(i & 1);
         if (!wait_bounded(SIGNS ? &S.sgn[st] : &S.full[st], (uint32_t)((i / kStages) & 1), S, true)) break;
+        if (S.gid[i % kRing] < 0) break;
         if (!wait_bounded(&S.tempty[acc], (uint32_t)((i >> 1) & 1) ^ 1u, S, true)) break;
         tc::tc_fence_after();
         if constexpr (SH::SPLIT) {
@@ -319,10 +373,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         mk[k] = make_uint4(w[0], w[1], w[2], w[3]);
       }
       for (int64_t i = 0;; ++i) {
-        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
-        if (p >= ngroups) break;
         const int st = (int)(i % kStages);
-        if (ts == 0) S.dec[2] = wait_bounded(&S.full[st], (uint32_t)((i / kStages) & 1), S, true) ? 1 : 0;
+        if (ts == 0) {
+          int ok = wait_bounded(&S.full[st], (uint32_t)((i / kStages) & 1), S, true) ? 1 : 0;
+          if (ok && S.gid[i % kRing] < 0) {
+            tc::mbar_arrive(&S.sgn[st]);  // pass the end mark on to the MMA
+            ok = 0;
+          }
+          S.dec[2] = ok;
+        }
         tc::named_sync(3, 64);
         if (!S.dec[2]) break;
         uint4 *X = reinterpret_cast<uint4 *>(smem + kOffX + st * kGroupBytes) + ts;
@@ -347,17 +406,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
     const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
     for (int64_t i = 0;; ++i) {
-      const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
-      if (p >= ngroups) break;
       const int acc = (int)(i & 1);
+      // the step's group from the producer's ring, then its accumulator
+      auto decide = [&](int slot) {
+        int ok = wait_bounded(&S.gfull[i % kRing], (uint32_t)((i / kRing) & 1), S, true) ? 1 : 0;
+        const int64_t gp = ok ? S.gid[i % kRing] : -1;
+        if (gp < 0) ok = 0;
+        if (ok) ok = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+        S.egid[slot] = gp;
+        S.dec[slot] = ok;
+      };
+      int64_t p;
       if constexpr (SH::SPLIT) {  // one decision for both warpgroups: they meet at barrier 4 below
-        if (threadIdx.x == 128) S.dec[0] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+        if (threadIdx.x == 128) decide(0);
         tc::named_sync(4, 256);
         if (!S.dec[0]) break;
+        p = S.egid[0];
       } else {
-        if (tg == 0) S.dec[g] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+        if (tg == 0) decide(g);
         tc::named_sync(1 + g, 128);
         if (!S.dec[g]) break;
+        p = S.egid[g];
       }
       tc::tc_fence_after();
       float v[kRegs];
@@ -474,8 +543,9 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
   int slots = 0;
   cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreads, (int)kSmemBytes, &slots);
   if (err != cudaSuccess) return err;
-  const int64_t ngroups = (tokens + SH::TOK - 1) / SH::TOK;
-  const int64_t grid = ngroups < slots ? ngroups : slots;
+  // One CTA per group: the resident ones take the groups of CTAs that have not started
+  // yet (cluster launch control), so the groups spread over the SMs as they free up.
+  const int64_t grid = (tokens + SH::TOK - 1) / SH::TOK;
   const float inv_sqrt_n = (float)(1.0 / std::sqrt((double)(1 << LOGN)));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
