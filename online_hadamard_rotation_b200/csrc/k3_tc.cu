@@ -32,6 +32,7 @@
 //                  into a three-stage ring
 //   warp 1         TMEM owner and MMA issuer
 //   warps 4-11     epilogue, two warpgroups over TMEM columns 0-127 and 128-255
+// (setmaxnreg moves registers from warps 0-3 to the epilogue warpgroups).
 // Every mbarrier wait is bounded by a clock budget; on expiry the CTA records a
 // status (read by spin_device_status), drains its copies and MMAs, frees TMEM and
 // returns.
@@ -64,6 +65,9 @@ constexpr uint32_t kOffC = kOffO + kOStages * kOpBytes;
 constexpr uint32_t kOffBar = kOffC + kCStages * kCodeBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
 constexpr long long kTimeoutCycles = 4000000000LL;     // about two seconds
+constexpr int kLaunchRegs = 168;                       // registers per thread at launch (65536 / 384, rounded)
+constexpr int kRegsLow = 104, kRegsHigh = 200;         // after the split: warps 0-3, warps 4-11
+static_assert(kRegsLow * 128 + kRegsHigh * 256 == kLaunchRegs * kThreads, "register split must add up");
 
 template <int LOGN>
 struct Shape {
@@ -237,6 +241,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = S.tmem_base;
 
   // ------------------------------------------------------------ roles
+  // Registers: warps 0-3 (converters, MMA) need few, the epilogue's 128 values per
+  // thread many. kRegsLow x 128 + kRegsHigh x 256 equals the launch's kLaunchRegs x 384
+  // (the launcher checks the compiled count), so the increase never waits for
+  // registers that are not there.
+  if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow) : "memory");
+  else asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh) : "memory");
   if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(128, SH::SPLIT ? 128 : 256, true);
@@ -456,6 +466,13 @@ cudaError_t launch_tc(const uint8_t *codes, int64_t rows, const void *scale, con
                       const uint32_t *signs, void *out, bool asym, cudaStream_t stream) {
   using SH = Shape<LOGN>;
   auto kern = k3_tc_dequant_inverse<LOGN, SIGNS, F32, STORE32>;
+  static cudaError_t checked = [&] {  // the register split assumes this count at launch
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(kern));
+    if (e != cudaSuccess) return e;
+    return fa.numRegs == kLaunchRegs ? cudaSuccess : cudaErrorInvalidConfiguration;
+  }();
+  if (checked != cudaSuccess) return checked;
   int slots = 0;
   cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreads, (int)kSmemBytes, &slots);
   if (err != cudaSuccess) return err;
