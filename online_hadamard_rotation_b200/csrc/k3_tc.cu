@@ -13,8 +13,10 @@
 // n = 128 B values is the 128 x B matrix C[a][b] (e = B a + b), and
 // H_n (c - z) = vec(H_128 C' H_B):
 //   1. Converter warps expand the packed nibbles of a group (32768 elements:
-//      256 / B rows, or one row at n = 32768) into fp16 integers c - z (exact),
-//      written as the MMA's MN-major B operand with the 64- or 128-byte swizzle.
+//      256 / B rows, or one row at n = 32768) into fp16 integers c - z + 1024 + z'
+//      (exact; the epilogue removes the constant from matrix row 0, the only row
+//      H_128 maps it to), written as the MMA's MN-major B operand with the 64- or
+//      128-byte swizzle.
 //   2. tcgen05.mma (kind::f16, fp16 H = +-1 as the K-major A operand, fp32
 //      accumulate in TMEM) computes H_128 C' exactly: every partial sum is an
 //      integer below 2^24.
@@ -93,7 +95,6 @@ struct Shared {
   int abort;
   int dec[3];
   long long budget;
-  __half2 zc[8];  // per token row of the group being converted: -(1024 + zero)
 };
 static_assert(sizeof(Shared) <= 256, "barrier area");
 
@@ -150,22 +151,14 @@ __device__ __forceinline__ void mul2(float &a0, float &a1, float m) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(R));
 }
 
-// Eight nibbles (element 2j in the low nibble of byte j; unsigned after the caller's
-// sign fix-up) -> four fp16 pairs (u - zc): each half is first 1024 + u (exponent 10,
-// one unit per ulp), then the exact sum with zc = -(1024 + zero).
-__device__ __forceinline__ uint4 expand8(uint32_t w, __half2 zc) {
+// Eight nibbles u (element 2j in the low nibble of byte j; unsigned after the caller's
+// sign fix-up) -> four fp16 pairs 1024 + u: a byte permute puts each nibble under the
+// exponent of 1024 (one unit per ulp). The epilogue removes the constant.
+__device__ __forceinline__ uint4 expand8(uint32_t w) {
   const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
   const uint32_t e0 = __byte_perm(lo, hi, 0x5140), e1 = __byte_perm(lo, hi, 0x7362);  // nibbles 0-3, 4-7
-  uint32_t h[4];
-  h[0] = __byte_perm(e0, 0x64646464u, 0x4140);
-  h[1] = __byte_perm(e0, 0x64646464u, 0x4342);
-  h[2] = __byte_perm(e1, 0x64646464u, 0x4140);
-  h[3] = __byte_perm(e1, 0x64646464u, 0x4342);
-  const uint32_t z = *reinterpret_cast<const uint32_t *>(&zc);
-  uint32_t o[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) asm("add.rn.f16x2 %0, %1, %2;" : "=r"(o[i]) : "r"(h[i]), "r"(z));
-  return make_uint4(o[0], o[1], o[2], o[3]);
+  return make_uint4(__byte_perm(e0, 0x64646464u, 0x4140), __byte_perm(e0, 0x64646464u, 0x4342),
+                    __byte_perm(e1, 0x64646464u, 0x4140), __byte_perm(e1, 0x64646464u, 0x4342));
 }
 
 template <int LOGN, bool SIGNS, bool F32, bool STORE32>
@@ -304,12 +297,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
       if (p >= ngroups) break;
       const int cs = (int)(i % kCStages), os = (int)(i % kOStages);
-      if (cid < (uint32_t)SH::TOK) {
-        const int64_t row = p * SH::TOK + cid;
-        float z = 8.0f;  // symmetric codes: c + 8 after flipping the nibble's top bit
-        if (asym) z = row < rows ? __half2float(zero[row]) : 0.0f;
-        S.zc[cid] = __float2half2_rn(-(1024.0f + z));
-      }
       if (cid == 0) {
         int ok = wait_bounded(&S.cfull[cs], (uint32_t)((i / kCStages) & 1), S, true) ? 1 : 0;
         if (ok) ok = wait_bounded(&S.oempty[os], (uint32_t)((i / kOStages) & 1) ^ 1u, S, true) ? 1 : 0;
@@ -331,11 +318,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t c0 = 4u * h;                          // first 16-byte chunk in the tile row
         uint8_t *rowp = op + (t * SH::BPT + rb * SH::CBOX + jc) * SH::BOXBYTES + a * SH::ROWB;
         const uint32_t sx = SH::ROWB == 128 ? (a & 7u) : ((a >> 1) & 3u);
-        const __half2 zc = S.zc[t];
         const uint32_t ws[4] = {w.x ^ flip, w.y ^ flip, w.z ^ flip, w.w ^ flip};
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          *reinterpret_cast<uint4 *>(rowp + (((c0 + u) ^ sx) << 4)) = expand8(ws[u], zc);
+        for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4 *>(rowp + (((c0 + u) ^ sx) << 4)) = expand8(ws[u]);
       }
       tc::fence_proxy_async_smem();
       tc::named_sync(3, kConv);
@@ -360,15 +345,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t sw[B / 32];  // this row's sign words (the same for every token row)
 #pragma unroll
     for (int k = 0; k < B / 32; ++k) sw[k] = SIGNS ? __ldg(signs + (orow * B) / 32 + k) : 0u;
-    // The row steps of a group are loaded one group ahead, so their DRAM latency hides
-    // behind the previous group's work: raw bits, converted when used.
+    // The row steps (and zero points) of a group are loaded one group ahead, so their
+    // DRAM latency hides behind the previous group's work: raw bits, converted when used
+    // (fp32 step, or fp16 step in the low and fp16 zero in the high half).
     auto load_steps = [&](int64_t pp, uint32_t (&dst)[SEG]) {
 #pragma unroll
       for (int sg = 0; sg < SEG; ++sg) {
         const int64_t token = SH::SPLIT ? pp : pp * SH::TOK + g * SEG + sg;
         dst[sg] = 0u;
         if (pp < ngroups && token < rows)
-          dst[sg] = asym ? (uint32_t)__ldg(static_cast<const unsigned short *>(scale) + token)
+          dst[sg] = asym ? (uint32_t)__ldg(static_cast<const unsigned short *>(scale) + token) |
+                               ((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(zero) + token) << 16)
                          : __float_as_uint(__ldg(static_cast<const float *>(scale) + token));
       }
     };
@@ -400,6 +387,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::tc_fence_before();
       tc::mbar_arrive(&S.tempty[acc]);
+      // The operand carried every value plus 1024 + K (K = 8 for symmetric codes, else
+      // the row's zero point). H_128 of a constant is nonzero only in matrix row 0
+      // (128 times it; twice that in the top half at n = 32768, nothing in the bottom
+      // half), so the thread holding row 0 takes it out before H_B; all exact integers.
+      if (row == 0 && (!SH::SPLIT || g == 0)) {
+#pragma unroll
+        for (int sg = 0; sg < SEG; ++sg) {
+          const float K = asym ? __half2float(__ushort_as_half((unsigned short)(step_raw[sg] >> 16))) : 8.0f;
+          const float corr = (SH::SPLIT ? 256.0f : 128.0f) * (1024.0f + K);
+#pragma unroll
+          for (int k = 0; k < B; ++k) v[sg * B + k] -= corr;
+        }
+      }
       // second Kronecker factor: H_B over b inside each token row's segment
       stage<0>(v);
       stage<1>(v);
