@@ -152,14 +152,20 @@ __device__ __forceinline__ void mul2(float &a0, float &a1, float m) {
 }
 
 // Eight nibbles u (element 2j in the low nibble of byte j; unsigned after the caller's
-// sign fix-up) -> four fp16 pairs 1024 + u: a byte permute puts each nibble under the
-// exponent of 1024 (one unit per ulp). The epilogue removes the constant.
+// sign fix-up) -> eight fp16 values 1024 + u: a byte permute puts each nibble under the
+// exponent of 1024 (one unit per ulp). The epilogue removes the constant. The halves
+// come out in element order 0, 2, 4, 6, 1, 3, 5, 7 (two permutes fewer than natural
+// order): a permutation of the index bits inside each 8-column group, which the
+// butterflies of H_B leave as it is (H is unchanged by a bit permutation applied to
+// row and column indices alike); the epilogue reads element e of a group from column
+// pos8(e).
 __device__ __forceinline__ uint4 expand8(uint32_t w) {
-  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-  const uint32_t e0 = __byte_perm(lo, hi, 0x5140), e1 = __byte_perm(lo, hi, 0x7362);  // nibbles 0-3, 4-7
-  return make_uint4(__byte_perm(e0, 0x64646464u, 0x4140), __byte_perm(e0, 0x64646464u, 0x4342),
-                    __byte_perm(e1, 0x64646464u, 0x4140), __byte_perm(e1, 0x64646464u, 0x4342));
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;  // even, odd elements
+  return make_uint4(__byte_perm(lo, 0x64646464u, 0x4140), __byte_perm(lo, 0x64646464u, 0x4342),
+                    __byte_perm(hi, 0x64646464u, 0x4140), __byte_perm(hi, 0x64646464u, 0x4342));
 }
+// column of element e within an 8-column group, as expand8 lays them out
+__host__ __device__ constexpr int pos8(int e) { return (e >> 1) | ((e & 1) << 2); }
 
 template <int LOGN, bool SIGNS, bool F32, bool STORE32>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -417,15 +423,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m = s * inv_sqrt_n;
         const float *w = v + sg * B;
         const int64_t off = token * (int64_t)(B * SH::ROWS) + (int64_t)orow * B;  // first element of the row
-        // one 8 (fp32) or 16 (bf16) element piece at a time: scale, diagonal sign, store
+        // one 8 (fp32) or 16 (bf16) element piece at a time, in element order: scale,
+        // diagonal sign, store
         constexpr int P = F32 ? 8 : 16;
 #pragma unroll
         for (int k = 0; k < B; k += P) {
           float o[P];
 #pragma unroll
           for (int u = 0; u < P; u += 2) {
-            o[u] = w[k + u];
-            o[u + 1] = w[k + u + 1];
+            o[u] = w[k + (u & ~7) + pos8(u & 7)];
+            o[u + 1] = w[k + (u & ~7) + pos8((u + 1) & 7)];
             mul2(o[u], o[u + 1], m);
           }
           if constexpr (SIGNS) {
