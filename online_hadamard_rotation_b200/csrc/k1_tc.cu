@@ -139,7 +139,8 @@ __device__ __forceinline__ int64_t clc_result(const uint4 *resp) {
   return ok ? (int64_t)x : -1;
 }
 
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, Shared &S, bool honor_abort) {
+template <class SS>
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, SS &S, bool honor_abort) {
   if (tc::mbar_try_wait_suspend(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
@@ -574,6 +575,334 @@ cudaError_t launch_n(const void *x, int64_t tokens, float clip, const uint32_t *
              : launch_tc<LOGN, false, false>(x, tokens, clip, nullptr, q, scales, stream, stall_test);
 }
 
+
+// ============================================================================ n = 128, 256
+// Tokens as the MMA's M. A token row of n = 128 V (V = 1, 2) is V chunks x_v of 128
+// and H_n D x = [sum_v (-1)^(u v) H_128 D_v x_v]_u. The MMA computes, for 128 tokens
+// at once, Y_v[t][a'] = sum_a X_v[t][a] B_v[a][a'] with A = X_v (K-major, as TMA loads
+// it) and B_v = D_v H_128 (the diagonal folded into the constant operand, so it costs
+// nothing per token); at n = 256 the epilogue forms the halves Y_0 + Y_1 and Y_0 - Y_1.
+// Each epilogue thread owns one token (one TMEM lane): max, step and codes with no
+// butterflies and no cross-thread reduction.
+//   warp 0      TMA producer: four [128 token][64 element] boxes per group (64 KiB)
+//   warp 1      TMEM owner and MMA issuer; two accumulators of 256 columns
+//   warps 2-9   epilogue, two warpgroups: n = 128, warpgroup g takes token tile g of
+//               every group; n = 256, warpgroup g takes the groups on accumulator g
+//               and reads it twice (maximum first, codes second)
+constexpr int kThreadsS = 320;
+
+template <int NB>
+struct SmallLayout {
+  static constexpr int kStages = NB == 2 ? 2 : 3;
+  static constexpr uint32_t kOffB = 0;  // B operand(s): 32 KiB each
+  static constexpr uint32_t kOffX = 32768u * NB;
+  static constexpr uint32_t kOffBar = kOffX + kStages * kGroupBytes;
+  static constexpr uint32_t kSmemBytes = kOffBar + 1024 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
+
+template <int ST>
+struct SharedS {
+  uint64_t full[ST], empty[ST], tfull[2], tempty[2], drain;
+  uint32_t tmem_base;
+  int abort;
+  int dec[2];
+  long long budget;
+};
+
+// 8 consecutive outputs t[0..7] (already multiplied into the code domain) to one
+// word of 8 nibbles
+__device__ __forceinline__ uint32_t codes8(const float *v, float c15) {
+  constexpr float k815 = 8.0f / 15.0f;
+  uint32_t b[8];
+  float t[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) t[k] = fma_sat(v[k], c15, k815);
+#pragma unroll
+  for (int k = 0; k < 8; k += 2) round15_x2(t[k], t[k + 1], b[k], b[k + 1]);
+  return pack8(b);
+}
+
+__device__ __forceinline__ float absmax32(const uint32_t *r, float m) {
+#pragma unroll
+  for (int k = 0; k < 32; ++k) m = fmaxf(m, fabsf(__uint_as_float(r[k])));
+  return m;
+}
+
+template <int V, bool SIGNS, bool STORE32>
+__global__ void __launch_bounds__(kThreadsS, 1)
+    k1_tcs_rotate_quant(const __grid_constant__ CUtensorMap xmap, int64_t tokens, float clip, float inv_sqrt_n,
+                        const uint32_t *__restrict__ signs, uint8_t *__restrict__ q, float *__restrict__ scales) {
+  constexpr int TOKG = 256 / V;  // tokens per group
+  constexpr int NB = (SIGNS && V == 2) ? 2 : 1;
+  using L = SmallLayout<NB>;
+  constexpr int ST = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  SharedS<ST> &S = *reinterpret_cast<SharedS<ST> *>(smem + L::kOffBar);
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
+  const int64_t ngroups = (tokens + TOKG - 1) / TOKG;
+  auto issue = [&](int st, int64_t p) {  // four boxes of group p into stage st
+    tc::mbar_arrive_expect_tx(&S.full[st], kGroupBytes);
+    uint8_t *dst = smem + L::kOffX + st * kGroupBytes;
+#pragma unroll
+    for (int b4 = 0; b4 < 4; ++b4) {  // box b4 = 2 t + (k >= 64): operand t, K half
+      const int x = V == 1 ? 64 * (b4 & 1) : 64 * b4;
+      const int y = (int)(p * TOKG) + (V == 1 ? 128 * (b4 >> 1) : 0);
+      tc::tma_load_2d(dst + b4 * 16384, &xmap, &S.full[st], x, y);
+    }
+  };
+
+  tc::grid_dep_wait();
+  int first_issued = 0;
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < ST; ++s2) {
+      tc::mbar_init(&S.full[s2], 1);
+      tc::mbar_init(&S.empty[s2], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(&S.tfull[a], 1);
+      tc::mbar_init(&S.tempty[a], V == 1 ? 256 : 128);
+    }
+    tc::mbar_init(&S.drain, 1);
+    S.abort = 0;
+    S.budget = kTimeoutCycles;
+    tc::fence_barrier_init();
+    tc::prefetch_tensormap(&xmap);
+    for (int i = 0; i < ST; ++i) {
+      const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+      if (p >= ngroups) break;
+      issue(i, p);
+      first_issued = i + 1;
+    }
+  }
+  tc::grid_dep_launch();
+  // B_v = D_v H_128 as the K-major B operand [n = a'][k = a]: entry d_v[a] H[a'][a]
+  for (uint32_t c = threadIdx.x; c < 2048u * NB; c += kThreadsS) {
+    const uint32_t v = c >> 11, kb = (c >> 10) & 1u, m = (c >> 3) & 127u, ch = c & 7u;
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t k0 = kb * 64 + ch * 8 + 2 * j;
+      uint32_t lo = (__popc(m & k0) & 1) ? 0xBF80u : 0x3F80u;
+      uint32_t hi = (__popc(m & (k0 + 1)) & 1) ? 0xBF80u : 0x3F80u;
+      if constexpr (SIGNS) {
+        const uint32_t e0 = 128u * v + k0;
+        lo ^= ((__ldg(signs + (e0 >> 5)) >> (e0 & 31u)) & 1u) << 15;
+        hi ^= ((__ldg(signs + ((e0 + 1) >> 5)) >> ((e0 + 1) & 31u)) & 1u) << 15;
+      }
+      w[j] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4 *>(smem + L::kOffB + v * 32768u + kb * 16384u + sw128(m, ch)) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  tc::fence_proxy_async_smem();
+  if (warp == 1) {
+    tc::tmem_alloc(&S.tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int64_t last[ST];
+      for (int s2 = 0; s2 < ST; ++s2) last[s2] = s2 < first_issued ? s2 : -1;
+      for (int64_t i = first_issued;; ++i) {
+        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+        if (p >= ngroups) break;
+        const int st = (int)(i % ST);
+        if (!wait_bounded(&S.empty[st], (uint32_t)((i / ST) & 1) ^ 1u, S, true)) break;
+        issue(st, p);
+        last[st] = i;
+      }
+      for (int s2 = 0; s2 < ST; ++s2)
+        if (last[s2] >= 0) wait_bounded(&S.full[s2], (uint32_t)((last[s2] / ST) & 1), S, false);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16(128, 128, false);  // A and B K-major
+      const uint32_t sB = tc::smem_u32(smem + L::kOffB), sX = tc::smem_u32(smem + L::kOffX);
+      for (int64_t i = 0;; ++i) {
+        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+        if (p >= ngroups) break;
+        const int st = (int)(i % ST), acc = (int)(i & 1);
+        if (!wait_bounded(&S.full[st], (uint32_t)((i / ST) & 1), S, true)) break;
+        if (!wait_bounded(&S.tempty[acc], (uint32_t)((i >> 1) & 1) ^ 1u, S, true)) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int t = 0; t < 2; ++t)  // V = 1: token tile t; V = 2: input chunk t
+#pragma unroll
+          for (int s2 = 0; s2 < 8; ++s2) {
+            const uint32_t xa = sX + st * kGroupBytes + (2 * t + (s2 >> 2)) * 16384 + (s2 & 3) * 32;
+            const uint32_t ba = sB + (NB == 2 ? t * 32768 : 0) + (s2 >> 2) * 16384 + (s2 & 3) * 32;
+            tc::umma_bf16(tmem + acc * 256 + t * 128, tc::smem_desc(xa, 16, 1024), tc::smem_desc(ba, 16, 1024),
+                          idesc, s2 > 0 ? 1u : 0u);
+          }
+        tc::umma_commit(&S.empty[st]);
+        tc::umma_commit(&S.tfull[acc]);
+      }
+    }
+  } else {
+    const uint32_t g = (warp - 2) >> 2, tg = threadIdx.x - 64 - 128 * g;
+    const uint32_t row = (warp & 3u) * 32 + lane;
+    const uint32_t lane_base = tmem + (((warp & 3u) * 32u) << 16);
+    for (int64_t i = (V == 1 ? 0 : g);; i += (V == 1 ? 1 : 2)) {
+      const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+      if (p >= ngroups) break;
+      const int acc = (int)(i & 1);
+      if (tg == 0) S.dec[g] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+      tc::named_sync(1 + g, 128);
+      if (!S.dec[g]) break;
+      tc::tc_fence_after();
+      const int64_t token = p * TOKG + (V == 1 ? 128 * g : 0) + row;
+      const bool live = token < tokens;
+      uint8_t *dst = q + token * (int64_t)(64 * V);
+      float s;
+      if constexpr (V == 1) {
+        uint32_t r[128];
+        const uint32_t taddr = lane_base + (uint32_t)acc * 256u + g * 128u;
+        tc::tmem_ld32(taddr, r);
+        tc::tmem_ld32(taddr + 32, r + 32);
+        tc::tmem_ld32(taddr + 64, r + 64);
+        tc::tmem_ld32(taddr + 96, r + 96);
+        tc::tmem_wait_ld();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&S.tempty[acc]);
+        float mu = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mu = absmax32(r + 32 * c, mu);
+        s = fmaxf(clip * (mu * inv_sqrt_n) / 7.0f, 1e-8f);
+        const float c15 = (inv_sqrt_n / 15.0f) / s;
+        uint32_t words[16];
+#pragma unroll
+        for (int wi = 0; wi < 16; ++wi) {
+          float f[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(r[8 * wi + k]);
+          words[wi] = codes8(f, c15);
+        }
+        if (live) {
+#pragma unroll
+          for (int w8 = 0; w8 < 2; ++w8) {
+            if constexpr (STORE32) {
+              st_v8_cs(dst + 32 * w8, words + 8 * w8);
+            } else {
+              __stcs(reinterpret_cast<uint4 *>(dst + 32 * w8),
+                     make_uint4(words[8 * w8], words[8 * w8 + 1], words[8 * w8 + 2], words[8 * w8 + 3]));
+              __stcs(reinterpret_cast<uint4 *>(dst + 32 * w8) + 1,
+                     make_uint4(words[8 * w8 + 4], words[8 * w8 + 5], words[8 * w8 + 6], words[8 * w8 + 7]));
+            }
+          }
+        }
+      } else {
+        const uint32_t taddr = lane_base + (uint32_t)acc * 256u;
+        float mu = 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {  // pass 1: |Y0 + Y1| and |Y0 - Y1|
+          uint32_t a[32], b[32];
+          tc::tmem_ld32(taddr + 32 * c, a);
+          tc::tmem_ld32(taddr + 128 + 32 * c, b);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float y0 = __uint_as_float(a[k]), y1 = __uint_as_float(b[k]);
+            mu = fmax3(mu, fabsf(y0 + y1), fabsf(y0 - y1));
+          }
+        }
+        s = fmaxf(clip * (mu * inv_sqrt_n) / 7.0f, 1e-8f);
+        const float c15 = (inv_sqrt_n / 15.0f) / s;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {  // pass 2: codes of outputs 32c.. of both halves
+          uint32_t a[32], b[32], w0[4], w1[4];
+          tc::tmem_ld32(taddr + 32 * c, a);
+          tc::tmem_ld32(taddr + 128 + 32 * c, b);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int wi = 0; wi < 4; ++wi) {
+            float f0[8], f1[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float y0 = __uint_as_float(a[8 * wi + k]), y1 = __uint_as_float(b[8 * wi + k]);
+              f0[k] = y0 + y1;
+              f1[k] = y0 - y1;
+            }
+            w0[wi] = codes8(f0, c15);
+            w1[wi] = codes8(f1, c15);
+          }
+          if (live) {
+            __stcs(reinterpret_cast<uint4 *>(dst + 16 * c), make_uint4(w0[0], w0[1], w0[2], w0[3]));
+            __stcs(reinterpret_cast<uint4 *>(dst + 64 + 16 * c), make_uint4(w1[0], w1[1], w1[2], w1[3]));
+          }
+        }
+        tc::tc_fence_before();
+        tc::mbar_arrive(&S.tempty[acc]);
+      }
+      if (live) scales[token] = s;
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0) {
+      tc::umma_commit(&S.drain);
+      wait_bounded(&S.drain, 0, S, false);
+    }
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int V, bool SIGNS, bool STORE32>
+cudaError_t launch_tcs(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
+                       cudaStream_t stream) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)(128 * V), (cuuint64_t)tokens};
+  const cuuint64_t strides[1] = {(cuuint64_t)(256 * V)};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  auto kern = k1_tcs_rotate_quant<V, SIGNS, STORE32>;
+  constexpr uint32_t smem_bytes = SmallLayout<(SIGNS && V == 2) ? 2 : 1>::kSmemBytes;
+  int slots = 0;
+  cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreadsS, (int)smem_bytes, &slots);
+  if (err != cudaSuccess) return err;
+  const int64_t ngroups = (tokens + 256 / V - 1) / (256 / V);
+  const int64_t grid = ngroups < slots ? ngroups : slots;
+  const float inv_sqrt_n = (float)(1.0 / std::sqrt((double)(128 * V)));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreadsS);
+  cfg.dynamicSmemBytes = smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, map, tokens, clip, inv_sqrt_n, signs, q, scales);
+}
+
+template <int V>
+cudaError_t launch_small(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
+                         cudaStream_t stream) {
+  const bool a32 = V == 1 && (reinterpret_cast<uintptr_t>(q) & 31u) == 0;  // n = 256 stores 16 B pieces
+  if (signs)
+    return a32 ? launch_tcs<V, true, V == 1>(x, tokens, clip, signs, q, scales, stream)
+               : launch_tcs<V, true, false>(x, tokens, clip, signs, q, scales, stream);
+  return a32 ? launch_tcs<V, false, V == 1>(x, tokens, clip, nullptr, q, scales, stream)
+             : launch_tcs<V, false, false>(x, tokens, clip, nullptr, q, scales, stream);
+}
+
 std::atomic<int> g_stall_test{0};
 
 }  // namespace
@@ -595,7 +924,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // only pays off with at least about one MMA group per SM; smaller batches (decode)
 // go to the CUDA-core kernel, which needs no setup.
 bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags, bool has_signs) {
-  if (log_n < 12 || log_n > 15 || (flags & kNoRotate) || tokens <= 0) return false;
+  if ((flags & kNoRotate) || tokens <= 0) return false;
+  if (log_n == 7 || log_n == 8) {  // tokens as M: 256 / V tokens per group
+    if (tokens >= (int64_t(1) << 31)) return false;
+    const int64_t tok_per_group = log_n == 7 ? 256 : 128;
+    return (flags & kTensorCores) || tokens >= 128 * tok_per_group;
+  }
+  if (log_n < 12 || log_n > 15) return false;
   if (log_n == 15 && has_signs) return false;  // its sign masks do not fit the sign warps' registers
   const int64_t rows_per_token = log_n == 15 ? 256 : 128;
   if (tokens * rows_per_token >= (int64_t(1) << 31)) return false;
@@ -607,6 +942,8 @@ cudaError_t launch_rotate_quant_int4_tc(int log_n, const void *x, int64_t tokens
                                         uint8_t *q, float *scales, cudaStream_t stream) {
   const int stall = g_stall_test.load(std::memory_order_relaxed);
   switch (log_n) {
+    case 7: return launch_small<1>(x, tokens, clip, signs, q, scales, stream);
+    case 8: return launch_small<2>(x, tokens, clip, signs, q, scales, stream);
     case 12: return launch_n<12>(x, tokens, clip, signs, q, scales, stream, stall);
     case 13: return launch_n<13>(x, tokens, clip, signs, q, scales, stream, stall);
     case 14: return launch_n<14>(x, tokens, clip, signs, q, scales, stream, stall);

@@ -1,8 +1,12 @@
-"""The tensor-core R4 kernel (n = 4096, 8192, 16384: first H_128 Kronecker
-factor on tcgen05, second on CUDA cores; n = 32768: H_2 and H_128 on tcgen05,
-without a sign diagonal) vs the fp64 oracle, and vs the all-CUDA-core kernel
-selected with SPIN_CUDA_CORES_ONLY. Token counts leave partial MMA groups (8, 4
-and 2 tokens per group). At n = 32768 with sign_bits the CUDA-core kernel runs."""
+"""The tensor-core R4 kernels vs the fp64 oracle, and vs the all-CUDA-core kernel
+selected with SPIN_CUDA_CORES_ONLY:
+  n = 128, 256: tokens as the MMA's M (128 tokens per MMA, the diagonal folded
+    into the constant operand, H_2 of n = 256 in the epilogue);
+  n = 4096, 8192, 16384: first H_128 Kronecker factor on tcgen05, second on CUDA
+    cores; n = 32768: H_2 and H_128 on tcgen05, without a sign diagonal.
+Token counts leave partial MMA groups (256 / 128 tokens per group at n = 128 /
+256; 8, 4 and 2 at the large sizes). At n = 32768 with sign_bits the CUDA-core
+kernel runs."""
 import numpy as np
 import pytest
 import torch
@@ -13,7 +17,7 @@ from tests.gpu_util import to_dev_bf16, to_dev_signs
 
 pytestmark = pytest.mark.gpu
 
-SIZES = [4096, 8192, 16384, 32768]
+SIZES = [128, 256, 4096, 8192, 16384, 32768]
 
 
 def run(spin, bits, clip, signs, cores_only=False):
@@ -58,7 +62,7 @@ def test_tc_matches_cuda_core_kernel(spin_gpu, orc, N):
 @pytest.mark.parametrize("N", SIZES)
 def test_tc_special_rows(spin_gpu, orc, N):
     rows = [np.zeros(N, np.float32), np.full(N, 1.0, np.float32)]
-    for j in (0, 1, 127, 128, N // 2 - 1, N - 1):
+    for j in sorted({0, 1, 127, 128 % N, N // 2 - 1, N - 1}):
         r = np.zeros(N, np.float32)
         r[j] = 60.0
         rows.append(r)
@@ -71,7 +75,7 @@ def test_tc_special_rows(spin_gpu, orc, N):
         parity.check_rel([s[t]], [r["scale64"]], 1e-5, f"scale row {t}")
         parity.check_codes(codes[t], r["codes"], r["pre"], f"codes row {t}")
     assert np.all(codes[0] == 0) and s[0] == np.float32(1e-8)
-    for t in range(2, 8):
+    for t in range(2, len(rows) - 1):
         assert np.all(np.abs(codes[t]) == 7)
 
 
@@ -84,3 +88,26 @@ def test_tc_leaves_tail_untouched(spin_gpu, N):
     torch.cuda.synchronize()
     assert torch.all(out[5:] == 0xA5) and torch.all(sc[5:] == -1.0)
     assert torch.all(sc[:5] > 0)
+
+
+@pytest.mark.parametrize("N,tokens", [(128, 149 * 256 + 77), (256, 149 * 128 + 77)])
+@pytest.mark.parametrize("with_signs", [False, True])
+def test_tc_small_n_many_groups(spin_gpu, orc, N, tokens, with_signs):
+    """More MMA groups than resident blocks, so every block loops over several
+    groups and both accumulators and every ring stage turn over."""
+    bits, signs, _ = synthetic.r4_prefill(tokens=tokens, n=N, seed=17)
+    if not with_signs:
+        signs = None
+    q1, s1 = run(spin_gpu, bits, 0.9, signs)
+    q2, s2 = run(spin_gpu, bits, 0.9, signs, cores_only=True)
+    parity.check_rel(s1, s2, 1e-5, "tc vs cuda-core scales")
+    c1, c2 = parity.unpack_signed(q1, N), parity.unpack_signed(q2, N)
+    rng = np.random.default_rng(N)
+    sample = np.concatenate([rng.choice(tokens, 48, replace=False), [0, tokens - 1],
+                             np.nonzero((c1 != c2).any(axis=1))[0][:16]])
+    for t in sample:
+        r = orc.r4_row(bits[t], 0.9, signs=signs)
+        parity.check_rel([s1[t]], [r["scale64"]], 1e-5, f"scale row {t}")
+        parity.check_codes(c1[t], r["codes"], r["pre"], f"tc row {t}")
+    assert (c1 != c2).mean() < 1e-4
+    assert spin_gpu.device_status() == 0
