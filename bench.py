@@ -61,6 +61,18 @@ def r4_kernel_name(n: int, tokens: int, has_signs: bool) -> str:
     return "k1_rotate_quant_int4"
 
 
+def k3_kernel_name(n: int, rows: int) -> str:
+    """The dequantise + inverse kernel the library's dispatch picks by default: a
+    tensor-core one for n = 128, 256 and 4096 .. 32768 once the batch has at least
+    128 MMA groups, else the CUDA-core one."""
+    log_n = n.bit_length() - 1
+    if log_n in (7, 8) and rows >= 128 * 128:
+        return "k3_tcs_dequant_inverse"
+    if 12 <= log_n <= 15 and rows >= 128 * (1 if log_n == 15 else 256 >> (log_n - 7)):
+        return "k3_tc_dequant_inverse"
+    return "k3_dequant_inverse"
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -425,7 +437,7 @@ def main():
             del q_d, s_d
         del x32, xr
         rt_gbs = rt_bytes / (rms / 1e3) / 1e9
-        round_trip = {"kernel": "k3_dequant_inverse", "ms_per_step": rms, "achieved_gbs": rt_gbs * world,
+        round_trip = {"kernel": k3_kernel_name(n, tokens), "ms_per_step": rms, "achieved_gbs": rt_gbs * world,
                       "frac": rt_gbs / measured_peaks()[0], "bytes_per_row": n // 2 + 4 + 2 * n,
                       "out_dtype": "bf16", "mse_rotated": mse[False], "mse_direct": mse[True],
                       "mse_ratio": mse[False] / mse[True] if mse[True] > 0 else None}

@@ -195,14 +195,17 @@ spin_status_t spin_rope_hadamard_kvquant(const void *q, const void *k, const voi
  *  scale      [rows] fp32 or fp16 by mode; zero [rows] fp16 (asym) or NULL (sym)
  *  sign_bits  nullable, as in spin_hadamard_quant_int4_ex
  *  flags      bitwise OR of SPIN_NO_ROTATE and at most one of
- *             SPIN_CUDA_CORES_ONLY: at n = 4096 .. 32768 the first H_128
- *               Kronecker factor normally runs on the tensor cores (the codes
- *               minus the zero point are exact fp16 integers and so is every
- *               sum); this bit selects the kernel that runs every butterfly on
- *               the CUDA cores instead. By default the tensor-core kernel runs
- *               only from 128 MMA groups (128 x max(1, 256 / (n/128)) rows) up;
+ *             SPIN_CUDA_CORES_ONLY: at n = 128 and 256 the transform, and at
+ *               n = 4096 .. 32768 its first H_128 Kronecker factor, normally
+ *               run on the tensor cores (the codes minus the zero point are
+ *               exact fp16 integers and so is every sum, so both kernels give
+ *               the same bits); this bit selects the kernel that runs every
+ *               butterfly on the CUDA cores instead. By default the tensor-core
+ *               kernel runs only from 128 MMA groups up (128 rows per group at
+ *               n = 128 and 256, 128 x max(1, 256 / (n/128)) rows from 4096);
  *             SPIN_TENSOR_CORES: use the tensor-core kernel wherever n allows
- *               (n >= 4096, not with SPIN_NO_ROTATE), whatever the row count.
+ *               (n = 128, 256 or n >= 4096, not with SPIN_NO_ROTATE), whatever
+ *               the row count.
  *             Other bits: SPIN_ERR_INVALID_ARG.
  *  out        [rows, n] bf16 or fp32 (out_dtype), 16-byte aligned
  */

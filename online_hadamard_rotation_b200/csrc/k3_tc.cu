@@ -113,7 +113,8 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn) {
   return (1u << 4) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, Shared &S, bool honor_abort) {
+template <class SS>
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, SS &S, bool honor_abort) {
   if (tc::mbar_try_wait_suspend(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
@@ -518,12 +519,357 @@ cudaError_t launch_n(const uint8_t *codes, int64_t rows, const void *scale, cons
                : launch_s<LOGN, false>(codes, rows, scale, zero, nullptr, out, asym, f32, stream);
 }
 
+
+// ============================================================================ n = 128, 256
+// Tokens as the MMA's M. A row of n = 128 V (V = 1, 2) is V chunks c_v of 128
+// codes, and H_n (c - z) = [sum_v (-1)^(u v) H_128 (c_v - z)]_u. For 128 rows at
+// once the MMA computes Y_v[t][a'] = sum_a C'_v[t][a] H[a'][a] with A = C'_v (the
+// rows' fp16 integers 1024 + u, K-major) and B = H_128 (K-major, fp16 +-1, built
+// once). The constant 1024 + K of every element lands only in column 0 of each
+// Y_v (128 times it), which the epilogue takes out; at n = 256 it then forms
+// Y_0 + Y_1 and Y_0 - Y_1. Each epilogue thread owns one row (one TMEM lane) and
+// writes it in element order: scale, diagonal sign, store.
+//   warp 0      bulk copies of each group's codes (128 rows) into a codes ring
+//   warp 1      TMEM owner and MMA issuer; two accumulators of 128 V columns
+//   warps 2-5   converters: codes -> fp16 operand ring (two stages)
+//   warps 6-9   epilogue
+constexpr int kThreadsS = 320;
+
+template <int V>
+struct SmallLayout {
+  static constexpr int kCS = V == 1 ? 4 : 3;              // codes stages
+  static constexpr int kAS = 2;                           // operand stages
+  static constexpr uint32_t kCodeBytes = 8192u * V;       // 128 rows of codes
+  static constexpr uint32_t kOpBytes = 32768u * V;        // 128 rows of fp16 operand
+  static constexpr uint32_t kOffB = 0;                    // H_128, fp16, K-major, 2 x 16 KiB
+  static constexpr uint32_t kOffC = 32768;
+  static constexpr uint32_t kOffA = kOffC + kCS * kCodeBytes;
+  static constexpr uint32_t kOffBar = kOffA + kAS * kOpBytes;
+  static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
+
+template <int CS, int AS>
+struct SharedS {
+  uint64_t cfull[CS], cempty[CS], afull[AS], aempty[AS], tfull[2], tempty[2], drain;
+  uint32_t tmem_base;
+  int abort;
+  int dec[2];
+  long long budget;
+};
+
+template <int V, bool SIGNS, bool F32, bool STORE32>
+__global__ void __launch_bounds__(kThreadsS, 1)
+    k3_tcs_dequant_inverse(const uint8_t *__restrict__ codes, int64_t rows, float inv_sqrt_n,
+                           const void *__restrict__ scale, const __half *__restrict__ zero,
+                           const uint32_t *__restrict__ signs, void *__restrict__ out, int asym) {
+  using L = SmallLayout<V>;
+  constexpr int CS = L::kCS, AS = L::kAS;
+  constexpr int N = 128 * V;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  SharedS<CS, AS> &S = *reinterpret_cast<SharedS<CS, AS> *>(smem + L::kOffBar);
+  static_assert(sizeof(SharedS<CS, AS>) <= 256, "barrier area");
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
+  const int64_t ngroups = (rows + 127) / 128;
+  auto issue = [&](int cs, int64_t p) {  // codes of group p into codes stage cs
+    const int64_t t0 = p * 128;
+    const uint32_t nvalid = (uint32_t)((rows - t0) < 128 ? (rows - t0) : 128);
+    const uint32_t bytes = nvalid * (uint32_t)(N / 2);
+    tc::mbar_arrive_expect_tx(&S.cfull[cs], bytes);
+    bulk_load(smem + L::kOffC + cs * L::kCodeBytes, codes + t0 * (int64_t)(N / 2), bytes, &S.cfull[cs]);
+  };
+
+  tc::grid_dep_wait();
+  int first_issued = 0;
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < CS; ++s2) {
+      tc::mbar_init(&S.cfull[s2], 1);
+      tc::mbar_init(&S.cempty[s2], 128);
+    }
+    for (int s2 = 0; s2 < AS; ++s2) {
+      tc::mbar_init(&S.afull[s2], 128);
+      tc::mbar_init(&S.aempty[s2], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(&S.tfull[a], 1);
+      tc::mbar_init(&S.tempty[a], 128);
+    }
+    tc::mbar_init(&S.drain, 1);
+    S.abort = 0;
+    S.budget = kTimeoutCycles;
+    tc::fence_barrier_init();
+    for (int i = 0; i < CS; ++i) {  // the first stages need no free slot
+      const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+      if (p >= ngroups) break;
+      issue(i, p);
+      first_issued = i + 1;
+    }
+  }
+  tc::grid_dep_launch();
+  // H_128 in fp16 as the B operand [n = a'][k = a], K-major, two K blocks of 64 with
+  // the 128-byte swizzle; physical K position p of an 8-column group holds element
+  // e = 2 (p & 3) + (p >> 2), the order expand8 writes the codes in.
+  for (uint32_t c = threadIdx.x; c < 2048; c += kThreadsS) {
+    const uint32_t kb = c >> 10, m = (c >> 3) & 127u, ch = c & 7u;
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t p0 = 2 * j, p1 = 2 * j + 1;
+      const uint32_t k0 = kb * 64 + ch * 8 + 2 * (p0 & 3u) + (p0 >> 2);
+      const uint32_t k1 = kb * 64 + ch * 8 + 2 * (p1 & 3u) + (p1 >> 2);
+      const uint32_t lo = (__popc(m & k0) & 1) ? 0xBC00u : 0x3C00u;
+      const uint32_t hi = (__popc(m & k1) & 1) ? 0xBC00u : 0x3C00u;
+      w[j] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4 *>(smem + L::kOffB + kb * 16384 + m * 128u + ((ch ^ (m & 7u)) << 4)) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  tc::fence_proxy_async_smem();
+  if (warp == 1) {
+    tc::tmem_alloc(&S.tmem_base, 256 * V);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int64_t last[CS];
+      for (int s2 = 0; s2 < CS; ++s2) last[s2] = s2 < first_issued ? s2 : -1;
+      for (int64_t i = first_issued;; ++i) {
+        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+        if (p >= ngroups) break;
+        const int cs = (int)(i % CS);
+        if (!wait_bounded(&S.cempty[cs], (uint32_t)((i / CS) & 1) ^ 1u, S, true)) break;
+        tc::fence_proxy_async_smem();  // the converters' reads of the stage come before the copy
+        issue(cs, p);
+        last[cs] = i;
+      }
+      for (int s2 = 0; s2 < CS; ++s2)  // every issued copy has landed before the CTA can leave
+        if (last[s2] >= 0) wait_bounded(&S.cfull[s2], (uint32_t)((last[s2] / CS) & 1), S, false);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(128, 128, false);  // A and B K-major
+      const uint32_t sB = tc::smem_u32(smem + L::kOffB), sA = tc::smem_u32(smem + L::kOffA);
+      for (int64_t i = 0;; ++i) {
+        const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+        if (p >= ngroups) break;
+        const int as = (int)(i % AS), acc = (int)(i & 1);
+        if (!wait_bounded(&S.afull[as], (uint32_t)((i / AS) & 1), S, true)) break;
+        if (!wait_bounded(&S.tempty[acc], (uint32_t)((i >> 1) & 1) ^ 1u, S, true)) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+#pragma unroll
+          for (int s2 = 0; s2 < 8; ++s2) {
+            const uint32_t aa = sA + as * L::kOpBytes + v * 32768 + (s2 >> 2) * 16384 + (s2 & 3) * 32;
+            const uint32_t ba = sB + (s2 >> 2) * 16384 + (s2 & 3) * 32;
+            tc::umma_bf16(tmem + acc * (128 * V) + v * 128, tc::smem_desc(aa, 16, 1024),
+                          tc::smem_desc(ba, 16, 1024), idesc, s2 > 0 ? 1u : 0u);
+          }
+        tc::umma_commit(&S.aempty[as]);
+        tc::umma_commit(&S.tfull[acc]);
+      }
+    }
+  } else if (warp < 6) {
+    // Converters. One 16-byte read covers 32 consecutive codes of a row: the read
+    // phases take 128 contiguous bytes. Lane (row t, chunk v, quarter qd) writes the
+    // four 8-code groups of its quarter in the order j ^ (qd & 2) ^ v, so the eight
+    // lanes of a 16-byte store phase hit eight different bank groups of the swizzled
+    // rows.
+    const uint32_t cid = threadIdx.x - 64, cw = cid >> 5;
+    const uint32_t flip = asym ? 0u : 0x88888888u;
+    for (int64_t i = 0;; ++i) {
+      const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+      if (p >= ngroups) break;
+      const int cs = (int)(i % CS), as = (int)(i % AS);
+      if (cid == 0) {
+        int ok = wait_bounded(&S.cfull[cs], (uint32_t)((i / CS) & 1), S, true) ? 1 : 0;
+        if (ok) ok = wait_bounded(&S.aempty[as], (uint32_t)((i / AS) & 1) ^ 1u, S, true) ? 1 : 0;
+        S.dec[0] = ok;
+      }
+      tc::named_sync(1, 128);
+      if (!S.dec[0]) break;
+      const uint8_t *cb = smem + L::kOffC + cs * L::kCodeBytes;
+      uint8_t *ab = smem + L::kOffA + as * L::kOpBytes;
+      constexpr int RPI = 32 / (4 * V);  // rows per warp and iteration
+#pragma unroll 2
+      for (int it = 0; it < 128 / (4 * RPI); ++it) {
+        const uint32_t t = (uint32_t)(it * 4 + cw) * RPI + (lane / (4 * V));
+        const uint32_t u = lane & (4 * V - 1), v = u >> 2, qd = u & 3u;
+        const uint4 w = *reinterpret_cast<const uint4 *>(cb + t * (N / 2) + u * 16);
+        const uint32_t ws[4] = {w.x ^ flip, w.y ^ flip, w.z ^ flip, w.w ^ flip};
+        uint8_t *rowp = ab + v * 32768 + (qd >> 1) * 16384 + t * 128;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t jj = (uint32_t)j ^ (qd & 2u) ^ v;
+          const uint32_t word = (jj & 2u) ? ((jj & 1u) ? ws[3] : ws[2]) : ((jj & 1u) ? ws[1] : ws[0]);
+          const uint32_t ch = (qd & 1u) * 4u + jj;
+          *reinterpret_cast<uint4 *>(rowp + ((ch ^ (t & 7u)) << 4)) = expand8(word);
+        }
+      }
+      tc::mbar_arrive(&S.cempty[cs]);
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&S.afull[as]);
+    }
+  } else {
+    const uint32_t tg = threadIdx.x - 192;
+    const uint32_t row = (warp & 3u) * 32 + lane;
+    const uint32_t lane_base = tmem + (((warp & 3u) * 32u) << 16);
+    uint32_t sw[N / 32];  // the diagonal's sign words, the same for every row
+#pragma unroll
+    for (int k = 0; k < N / 32; ++k) sw[k] = SIGNS ? __ldg(signs + k) : 0u;
+    // a row's step (fp32; or fp16 step | fp16 zero << 16), loaded one group ahead
+    auto load_step = [&](int64_t pp) -> uint32_t {
+      const int64_t token = pp * 128 + row;
+      if (pp >= ngroups || token >= rows) return 0u;
+      return asym ? (uint32_t)__ldg(static_cast<const unsigned short *>(scale) + token) |
+                        ((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(zero) + token) << 16)
+                  : __float_as_uint(__ldg(static_cast<const float *>(scale) + token));
+    };
+    uint32_t step_next = load_step(blockIdx.x);
+    for (int64_t i = 0;; ++i) {
+      const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
+      if (p >= ngroups) break;
+      const uint32_t step_raw = step_next;
+      step_next = load_step(p + gridDim.x);
+      const int acc = (int)(i & 1);
+      if (tg == 0) S.dec[1] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+      tc::named_sync(2, 128);
+      if (!S.dec[1]) break;
+      tc::tc_fence_after();
+      const int64_t token = p * 128 + row;
+      const bool live = token < rows;
+      const float s = asym ? __half2float(__ushort_as_half((unsigned short)step_raw)) : __uint_as_float(step_raw);
+      const float K = asym ? __half2float(__ushort_as_half((unsigned short)(step_raw >> 16))) : 8.0f;
+      const float corr = 128.0f * (1024.0f + K);  // H_128 of the constant: column 0 only
+      const float m = s * inv_sqrt_n;
+      const uint32_t taddr = lane_base + (uint32_t)acc * (128u * V);
+      const int64_t off = token * (int64_t)N;
+      // 32 outputs (elements e0 ..) of this row: scale, sign, store
+      auto emit = [&](float (&o)[32], int e0) {
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) mul2(o[k], o[k + 1], m);
+        if constexpr (SIGNS) {
+          const uint32_t sb = sw[e0 >> 5];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __uint_as_float(__float_as_uint(o[k]) ^ (((sb >> k) & 1u) << 31));
+        }
+        if (!live) return;
+        if constexpr (F32) {
+          float *dst = static_cast<float *>(out) + off + e0;
+#pragma unroll
+          for (int k = 0; k < 32; k += 8)
+            store8<STORE32>(dst + k, __float_as_uint(o[k]), __float_as_uint(o[k + 1]), __float_as_uint(o[k + 2]),
+                            __float_as_uint(o[k + 3]), __float_as_uint(o[k + 4]), __float_as_uint(o[k + 5]),
+                            __float_as_uint(o[k + 6]), __float_as_uint(o[k + 7]));
+        } else {
+          uint16_t *dst = static_cast<uint16_t *>(out) + off + e0;
+#pragma unroll
+          for (int k = 0; k < 32; k += 16)
+            store8<STORE32>(dst + k, pack_bf16x2(o[k], o[k + 1]), pack_bf16x2(o[k + 2], o[k + 3]),
+                            pack_bf16x2(o[k + 4], o[k + 5]), pack_bf16x2(o[k + 6], o[k + 7]),
+                            pack_bf16x2(o[k + 8], o[k + 9]), pack_bf16x2(o[k + 10], o[k + 11]),
+                            pack_bf16x2(o[k + 12], o[k + 13]), pack_bf16x2(o[k + 14], o[k + 15]));
+        }
+      };
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        if constexpr (V == 1) {
+          uint32_t r[32];
+          tc::tmem_ld32(taddr + 32 * c, r);
+          tc::tmem_wait_ld();
+          float o[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __uint_as_float(r[k]);
+          if (c == 0) o[0] -= corr;
+          emit(o, 32 * c);
+        } else {
+          uint32_t a[32], b[32];
+          tc::tmem_ld32(taddr + 32 * c, a);
+          tc::tmem_ld32(taddr + 128 + 32 * c, b);
+          tc::tmem_wait_ld();
+          float o0[32], o1[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            float y0 = __uint_as_float(a[k]), y1 = __uint_as_float(b[k]);
+            if (k == 0 && c == 0) {
+              y0 -= corr;
+              y1 -= corr;
+            }
+            o0[k] = y0 + y1;
+            o1[k] = y0 - y1;
+          }
+          emit(o0, 32 * c);
+          emit(o1, 128 + 32 * c);
+        }
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&S.tempty[acc]);
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0) {
+      tc::umma_commit(&S.drain);
+      wait_bounded(&S.drain, 0, S, false);
+    }
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 256 * V);
+  }
+}
+
+template <int V, bool SIGNS, bool F32, bool STORE32>
+cudaError_t launch_tcs(const uint8_t *codes, int64_t rows, const void *scale, const void *zero,
+                       const uint32_t *signs, void *out, bool asym, cudaStream_t stream) {
+  auto kern = k3_tcs_dequant_inverse<V, SIGNS, F32, STORE32>;
+  constexpr uint32_t smem_bytes = SmallLayout<V>::kSmemBytes;
+  int slots = 0;
+  cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreadsS, (int)smem_bytes, &slots);
+  if (err != cudaSuccess) return err;
+  const int64_t ngroups = (rows + 127) / 128;
+  const int64_t grid = ngroups < slots ? ngroups : slots;
+  const float inv_sqrt_n = (float)(1.0 / std::sqrt((double)(128 * V)));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreadsS);
+  cfg.dynamicSmemBytes = smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, codes, rows, inv_sqrt_n, scale, static_cast<const __half *>(zero), signs,
+                            out, asym ? 1 : 0);
+}
+
+template <int V>
+cudaError_t launch_small(const uint8_t *codes, int64_t rows, const void *scale, const void *zero,
+                         const uint32_t *signs, void *out, bool asym, bool f32, cudaStream_t stream) {
+  const bool a32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;  // 32-byte stores need 32-byte alignment
+#define SPIN_TCS(S_, F_) \
+  (a32 ? launch_tcs<V, S_, F_, true>(codes, rows, scale, zero, signs, out, asym, stream) \
+       : launch_tcs<V, S_, F_, false>(codes, rows, scale, zero, signs, out, asym, stream))
+  if (signs) return f32 ? SPIN_TCS(true, true) : SPIN_TCS(true, false);
+  return f32 ? SPIN_TCS(false, true) : SPIN_TCS(false, false);
+#undef SPIN_TCS
+}
+
 }  // namespace
 
 bool tc_dequant_supported(int log_n, int64_t rows, uint32_t flags) {
-  if (log_n < 12 || log_n > 15 || (flags & kNoRotate) || rows <= 0) return false;
+  if ((flags & kNoRotate) || rows <= 0) return false;
+  if (!(log_n == 7 || log_n == 8 || (log_n >= 12 && log_n <= 15))) return false;
   if (rows * (int64_t(1) << log_n) >= (int64_t(1) << 40)) return false;
-  const int64_t rows_per_group = log_n == 15 ? 1 : int64_t(256) >> (log_n - 7);
+  const int64_t rows_per_group = log_n <= 8 ? 128 : log_n == 15 ? 1 : int64_t(256) >> (log_n - 7);
   return (flags & kTensorCores) || rows >= 128 * rows_per_group;
 }
 
@@ -532,6 +878,8 @@ cudaError_t launch_dequant_inverse_tc(int log_n, const uint8_t *codes, int64_t r
                                       cudaStream_t stream) {
   const bool asym = mode == 1, f32 = out_dtype == 1;
   switch (log_n) {
+    case 7: return launch_small<1>(codes, rows, scale, zero, signs, out, asym, f32, stream);
+    case 8: return launch_small<2>(codes, rows, scale, zero, signs, out, asym, f32, stream);
     case 12: return launch_n<12>(codes, rows, scale, zero, signs, out, asym, f32, stream);
     case 13: return launch_n<13>(codes, rows, scale, zero, signs, out, asym, f32, stream);
     case 14: return launch_n<14>(codes, rows, scale, zero, signs, out, asym, f32, stream);

@@ -1,9 +1,11 @@
-"""The tensor-core dequantise + inverse kernel (n = 4096 .. 32768: codes expanded
-to exact fp16 integers, first H_128 factor on tcgen05, second in registers) vs
-the fp64 oracle, and vs the all-CUDA-core kernel selected with
-SPIN_CUDA_CORES_ONLY. Both kernels transform exact integers and scale once at
-the end, so their outputs must agree bit for bit. Row counts leave partial MMA
-groups (8, 4, 2 and 1 rows per group)."""
+"""The tensor-core dequantise + inverse kernels vs the fp64 oracle, and vs the
+all-CUDA-core kernel selected with SPIN_CUDA_CORES_ONLY. Codes are expanded to
+exact fp16 integers; at n = 128 and 256 the rows are the MMA's M against a
+constant H_128 (H_2 of n = 256 in the epilogue), at n = 4096 .. 32768 the first
+H_128 factor runs on tcgen05 and the second in registers. Both kernels transform
+exact integers and scale once at the end, so their outputs must agree bit for
+bit. Row counts leave partial MMA groups (128 rows per group at n = 128 and 256;
+8, 4, 2 and 1 from 4096)."""
 import numpy as np
 import pytest
 import torch
@@ -14,7 +16,7 @@ from tests.gpu_util import to_dev_signs
 
 pytestmark = pytest.mark.gpu
 
-SIZES = [4096, 8192, 16384, 32768]
+SIZES = [128, 256, 4096, 8192, 16384, 32768]
 
 
 def inverse(spin, packed, n, scale, zero, mode, signs, out_dtype, cores_only=False):
@@ -38,7 +40,7 @@ def sym_rows(orc, n, rows, seed, signs):
 
 
 @pytest.mark.parametrize("n", SIZES)
-@pytest.mark.parametrize("rows", [1, 3, 9, 37])
+@pytest.mark.parametrize("rows", [1, 3, 9, 37, 300])
 @pytest.mark.parametrize("with_signs", [False, True])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_tc_sym_vs_oracle(spin_gpu, orc, n, rows, with_signs, out_dtype):
@@ -79,7 +81,7 @@ def test_tc_asym_vs_oracle(spin_gpu, orc, n, out_dtype):
 @pytest.mark.parametrize("n", SIZES)
 @pytest.mark.parametrize("with_signs", [False, True])
 def test_tc_matches_cuda_core_kernel(spin_gpu, orc, n, with_signs):
-    rows = max(64, (1 << 21) // n)
+    rows = max(64, (1 << 21) // n) + 77
     rng = np.random.default_rng(n + 1)
     packed = rng.integers(0, 256, size=(rows, n // 2), dtype=np.uint8)
     scales = rng.uniform(0.001, 2.0, rows).astype(np.float32)
@@ -102,3 +104,33 @@ def test_tc_leaves_tail_untouched(spin_gpu, orc, n):
     assert torch.all(out[rows:] == -7.0)
     ref = np.stack([orc.dequant_inverse_row(packed[t], n, 0, float(scales[t])) for t in range(rows)])
     parity.check_f32_rows(out[:rows].cpu().numpy().astype(np.float64), ref, f"tc inverse n={n} into a slice")
+
+
+@pytest.mark.parametrize("n", [128, 256])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_tc_small_n_many_groups(spin_gpu, orc, n, mode):
+    """More 128-row groups than resident blocks (every block loops, every ring
+    stage and both accumulators turn over), both code modes: bit-exact against
+    the CUDA-core kernel, sampled rows against the oracle."""
+    rows = 149 * 128 * 3 + 45
+    rng = np.random.default_rng(n + mode)
+    packed = rng.integers(0, 256, size=(rows, n // 2), dtype=np.uint8)
+    if mode == 0:
+        scales, zero = rng.uniform(0.001, 2.0, rows).astype(np.float32), None
+    else:
+        scales = orc.f64_to_f16(rng.uniform(0.01, 3.0, rows)).view(np.float16)
+        zero = orc.f64_to_f16(rng.integers(0, 16, rows).astype(np.float64)).view(np.float16)
+    signs = synthetic.sign_bits(n, 5)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        a = inverse(spin_gpu, packed, n, scales, zero, mode, signs, out_dtype)
+        b = inverse(spin_gpu, packed, n, scales, zero, mode, signs, out_dtype, cores_only=True)
+        assert torch.equal(a.view(torch.int16) if out_dtype == torch.bfloat16 else a.view(torch.int32),
+                           b.view(torch.int16) if out_dtype == torch.bfloat16 else b.view(torch.int32))
+    got = a.float().cpu().numpy().astype(np.float64)
+    s = scales.astype(np.float64) if mode == 0 else orc.f16_to_f64(scales.view(np.uint16))
+    z = None if mode == 0 else orc.f16_to_f64(zero.view(np.uint16))
+    for t in list(rng.choice(rows, 24, replace=False)) + [0, rows - 1]:
+        ref = orc.dequant_inverse_row(packed[t], n, mode, float(s[t]), 0.0 if z is None else float(z[t]),
+                                      signs=signs)
+        parity.check_bf16(got[t:t + 1], ref[None, :], f"tc inverse n={n} row {t}")
+    assert spin_gpu.device_status() == 0
