@@ -57,6 +57,11 @@ def lib():
     L.orc_rotate.restype = C.c_int
     L.orc_quant_sym_int4.argtypes = [_dp, C.c_int, C.c_double, vp, _i8p]
     L.orc_quant_sym_int4.restype = C.c_double
+    L.orc_quant_sym_int8.argtypes = [_dp, C.c_int, C.c_double, vp, _i8p]
+    L.orc_quant_sym_int8.restype = C.c_double
+    L.orc_r4_row_int8.argtypes = [_u16p, C.c_int, C.c_double, vp, C.c_uint32, C.c_int, vp, vp, _i8p,
+                                  vp, vp]
+    L.orc_r4_row_int8.restype = C.c_int
     L.orc_quant_asym_int4.argtypes = [_dp, C.c_int, C.c_double, vp, _u8p,
                                       C.POINTER(C.c_uint16), C.POINTER(C.c_uint16)]
     L.orc_asym_unrounded_scale.argtypes = [_dp, C.c_int, C.c_double]
@@ -173,6 +178,14 @@ def quant_sym_int4(y, clip):
     return s, pre, codes
 
 
+def quant_sym_int8(y, clip):
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    pre = np.empty_like(y)
+    codes = np.empty(y.size, dtype=np.int8)
+    s = lib().orc_quant_sym_int8(y, y.size, float(clip), _ptr(pre), codes)
+    return s, pre, codes
+
+
 def quant_asym_int4(x, clip):
     x = np.ascontiguousarray(x, dtype=np.float64)
     pre = np.empty_like(x)
@@ -220,6 +233,23 @@ def r4_row(x_bits, clip, signs=None, no_rotate=False, method=METHOD_FWHT):
         raise ValueError(f"orc_r4_row failed ({rc})")
     return dict(y=y, pre=pre, codes=codes, packed=packed, scale64=s64.value,
                 scale32=np.float32(s32.value))
+
+
+def r4_row_int8(x_bits, clip, signs=None, no_rotate=False, method=METHOD_FWHT):
+    """One token through the R4 path with per-token INT8 codes."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    n = x.size
+    y = np.empty(n, dtype=np.float64)
+    pre = np.empty(n, dtype=np.float64)
+    codes = np.empty(n, dtype=np.int8)
+    s64 = C.c_double()
+    s32 = C.c_float()
+    s = _signs(signs)
+    rc = lib().orc_r4_row_int8(x, n, float(clip), _ptr(s), NO_ROTATE if no_rotate else 0, method,
+                               _ptr(y), _ptr(pre), codes, C.byref(s64), C.byref(s32))
+    if rc:
+        raise ValueError(f"orc_r4_row_int8 failed ({rc})")
+    return dict(y=y, pre=pre, codes=codes, scale64=s64.value, scale32=np.float32(s32.value))
 
 
 def r4_rows(x_bits, clip, signs=None, no_rotate=False):

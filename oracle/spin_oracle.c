@@ -22,7 +22,8 @@
  *        (rotate -> quantize -> rotate back).
  *  [SG]  "SpinQuant Guide: Learned Rotations for 4-Bit LLMs", section "The
  *        Outlier Curse in 4-Bit Weight-Activation Quantization" (INT4 range
- *        [-8, 7], step = max|x| / (2^(b-1) - 1)), section "End-to-End
+ *        [-8, 7], step = max|x| / (2^(b-1) - 1); at b = 8 the per-token INT8
+ *        activations of W4A8), section "End-to-End
  *        Implementation" (scale clamped below at 1e-8, x_dequant = x_quant *
  *        scale), section "RoPE Compatibility with 4-Bit KV Caching" (RoPE
  *        rotates 2-D coordinate pairs; KV cache stored as 4-bit).
@@ -215,6 +216,24 @@ double orc_quant_sym_int4(const double *y, int n, double clip, double *pre, int8
   return s;
 }
 
+/* Symmetric per-token INT8, the same rule at b = 8 bits [SG "The Outlier Curse":
+ * signed b-bit range [-2^(b-1), 2^(b-1) - 1], step = max|x| / (2^(b-1) - 1); the
+ * A8 of the W4A8 decoding figure in "SpinQuant, when rotations are worth
+ * learning", section "Measured effects"]: s = max(clip * max|y| / 127, 1e-8),
+ * q = clamp(rne(y/s), -128, 127). `pre` (nullable) receives y/s. Returns s. */
+double orc_quant_sym_int8(const double *y, int n, double clip, double *pre, int8_t *codes) {
+  double m = 0.0;
+  for (int j = 0; j < n; j++) m = fmax(m, fabs(y[j]));
+  double s = clip * m / 127.0;
+  if (s < 1e-8) s = 1e-8;
+  for (int j = 0; j < n; j++) {
+    double p = y[j] / s;
+    if (pre) pre[j] = p;
+    codes[j] = (int8_t)clampd(nearbyint(p), -128.0, 127.0);
+  }
+  return s;
+}
+
 /* Asymmetric INT4 over one group (reading of "KV cache stored as 4-bit INT4";
  * the pages give no formula): lo = min(clip*min x, 0), hi = max(clip*max x, 0),
  * s = (hi - lo) / 15 rounded to fp16, z = clamp(rne(-lo/s), 0, 15),
@@ -305,6 +324,29 @@ int orc_r4_row(const uint16_t *x, int n, double clip, const uint32_t *signs, uin
   if (scale64) *scale64 = s;
   *scale32 = (float)s;
   free(xd); free(y); free(q); free(q32);
+  return 0;
+}
+
+/* One token row through R4 with per-token INT8 codes (one signed byte per
+ * element). Outputs as in orc_r4_row; codes (n bytes) is required. */
+int orc_r4_row_int8(const uint16_t *x, int n, double clip, const uint32_t *signs, uint32_t flags,
+                    int method, double *y_out, double *pre, int8_t *codes, double *scale64,
+                    float *scale32) {
+  if (!is_pow2(n) || n < 2) return -1;
+  double *xd = (double *)malloc(sizeof(double) * (size_t)n);
+  double *y = (double *)malloc(sizeof(double) * (size_t)n);
+  if (!xd || !y) {
+    free(xd); free(y);
+    return -2;
+  }
+  for (int j = 0; j < n; j++) xd[j] = orc_bf16_to_f64(x[j]);
+  if (flags & ORC_NO_ROTATE) memcpy(y, xd, sizeof(double) * (size_t)n);
+  else orc_rotate(xd, n, signs, method, y);
+  double s = orc_quant_sym_int8(y, n, clip, pre, codes);
+  if (y_out) memcpy(y_out, y, sizeof(double) * (size_t)n);
+  if (scale64) *scale64 = s;
+  *scale32 = (float)s;
+  free(xd); free(y);
   return 0;
 }
 

@@ -422,3 +422,89 @@ def test_r4_rows_matches_single_rows(orc):
     for t in range(6):
         r = orc.r4_row(xb[t], 0.9, signs=synthetic.sign_bits(256, 1))
         assert np.array_equal(r["packed"], packed[t]) and r["scale32"] == scales[t]
+
+
+# --------------------------------------------------------------------------
+# Per-token INT8 (the b = 8 case of "SpinQuant Guide: Learned Rotations for
+# 4-Bit LLMs", section "The Outlier Curse": range [-128, 127], step
+# max|x| / 127).
+# --------------------------------------------------------------------------
+def test_int8_outlier_curse_rule(orc, pages):
+    g = pages["outlier_curse"]
+    v = np.array(g["values"], dtype=np.float64)
+    s, pre, codes = orc.quant_sym_int8(v, 1.0)
+    assert s == pytest.approx(np.max(np.abs(v)) / 127, rel=1e-15)
+    assert codes[np.argmax(np.abs(v))] in (127, -127)
+    s4, _, _ = orc.quant_sym_int4(v, 1.0)
+    assert s * 127 == pytest.approx(s4 * 7, rel=1e-15)  # same max, wider grid
+
+
+def test_int8_ties_round_to_even(orc):
+    y = np.array([127.0, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 100.5, 125.5, -126.5, 63.5, -64.5])
+    s, pre, codes = orc.quant_sym_int8(y, 1.0)
+    assert s == 1.0
+    assert np.array_equal(codes, np.round(y).astype(np.int8))  # numpy rounds half to even
+    assert list(codes[1:4]) == [0, 2, 2] and codes[8] == 126 and codes[9] == -126
+
+
+def test_int8_clamp(orc):
+    s, pre, codes = orc.quant_sym_int8(np.array([127.0, -127.0, 60.0, -64.2, 63.75]), 0.5)
+    assert s == 0.5
+    assert list(codes) == [127, -128, 120, -128, 127]
+
+
+def test_int8_one_hot_rotates_to_full_scale(orc):
+    """H e_j / sqrt(n) has every entry +-1/sqrt(n): at clip 1 every code is +-127,
+    with the signs of row j of the Sylvester matrix."""
+    n = 256
+    H = scipy.linalg.hadamard(n)
+    for j in (0, 5, 200):
+        x = np.zeros(n, np.float32)
+        x[j] = 3.0
+        r = orc.r4_row_int8(bf16(x), 1.0)
+        assert np.array_equal(r["codes"], 127 * H[j])
+        assert r["scale64"] == pytest.approx(3.0 / math.sqrt(n) / 127, rel=1e-15)
+
+
+def test_int8_degenerate_zero_row(orc):
+    r = orc.r4_row_int8(np.zeros(512, dtype=np.uint16), 1.0)
+    assert r["scale64"] == 1e-8 and np.all(r["codes"] == 0) and r["scale32"] == np.float32(1e-8)
+
+
+def test_int8_error_model_and_bound(orc):
+    """At clip 1 nothing clamps, so |code * s - y| <= s/2 element-wise, and for a
+    Gaussian row the rounding error is close to uniform: mean square ~ s^2 / 12."""
+    n = 4096
+    rng = np.random.default_rng(23)
+    ratios = []
+    for _ in range(6):
+        xb = bf16(rng.standard_normal(n).astype(np.float32))
+        r = orc.r4_row_int8(xb, 1.0)
+        e = r["codes"] * r["scale64"] - r["y"]
+        assert np.max(np.abs(e)) <= r["scale64"] / 2 * (1 + 1e-12)
+        ratios.append(np.mean(e ** 2) / (r["scale64"] ** 2 / 12))
+    assert 0.85 < np.mean(ratios) < 1.15
+
+
+def test_int8_diagonal_equals_flipped_input(orc):
+    """D is applied before the transform: signs on the call equal flipping the
+    input's sign bits by hand."""
+    n = 1024
+    xb = synthetic.sweep(10, tokens=1, seed=3)[0]
+    signs = synthetic.sign_bits(n, 9)
+    bits = np.unpackbits(signs.view(np.uint8), bitorder="little")[:n].astype(bool)
+    flipped = np.where(bits, xb ^ np.uint16(0x8000), xb).astype(np.uint16)
+    a = orc.r4_row_int8(xb, 0.9, signs=signs)
+    b = orc.r4_row_int8(flipped, 0.9)
+    assert np.array_equal(a["codes"], b["codes"]) and a["scale64"] == b["scale64"]
+
+
+def test_int8_and_int4_share_the_rotation(orc):
+    """Both quantisers see the same rotated row; the INT8 codes are 127/7 times
+    finer: |codes8 * s8 - y| <= s8 / 2 and |codes4 * s4 - y| <= s4 / 2 (clip 1)."""
+    xb = synthetic.sweep(12, tokens=1, seed=5)[0]
+    r4 = orc.r4_row(xb, 1.0)
+    r8 = orc.r4_row_int8(xb, 1.0)
+    assert np.array_equal(r4["y"], r8["y"])
+    assert r8["scale64"] * 127 == pytest.approx(r4["scale64"] * 7, rel=1e-15)
+    assert np.max(np.abs(r8["codes"] * r8["scale64"] - r8["y"])) <= r8["scale64"] / 2 * (1 + 1e-12)
