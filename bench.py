@@ -42,9 +42,21 @@ FALLBACK_HBM_GBS = 6650.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
-def algorithmic_bytes_r4(tokens: int, n: int) -> int:
-    """bf16 in (2n) + packed codes out (n/2) + fp32 scale out (4), per token."""
-    return tokens * (2 * n + n // 2 + 4)
+def metric_for(wl) -> str:
+    """The headline metric, or its INT8 counterpart for the INT8 workload."""
+    return METRIC.replace("INT4", "INT8") if wl.get("code_bits", 4) == 8 else METRIC
+
+
+def algorithmic_bytes_r4(tokens: int, n: int, code_bits: int = 4) -> int:
+    """bf16 in (2n) + codes out (n/2 packed INT4 or n INT8) + fp32 scale out (4), per token."""
+    return tokens * (2 * n + n * code_bits // 8 + 4)
+
+
+def oracle_r4_rows(oracle, bits, clip, signs, code_bits):
+    """The oracle over rows: its C loop for INT4, one call per row for INT8."""
+    if code_bits == 4:
+        return oracle.r4_rows(bits, clip, signs)
+    return [oracle.r4_row_int8(row, clip, signs=signs) for row in bits]
 
 
 def r4_kernel_name(n: int, tokens: int, has_signs: bool) -> str:
@@ -189,22 +201,24 @@ def aggregate(world: int, unit_bytes: int, unit_count: int, steps: int, ms: floa
 def make_workload(name: str, rank: int, tokens: int | None = None):
     """The workload one rank processes; every rank draws its own shard (seed + rank)."""
     import synthetic
-    if name == "r4_prefill":
+    if name in ("r4_prefill", "r4_prefill_int8"):
         bits, signs, _ = synthetic.r4_prefill(tokens=tokens or 8192, seed=1 + rank)
-        return dict(kind="r4", bits=bits, signs=signs, clip=0.9,
+        code_bits = 8 if name.endswith("int8") else 4
+        return dict(kind="r4", bits=bits, signs=signs, clip=0.9, code_bits=code_bits,
                     desc={"workload": "R4 prefill: 4x2048 tokens x n=16384 bf16, SwiGLU-like, 0.1% channels x100, "
-                                      "seeded +-1 diagonal, H_16384 = H_128 (x) H_128, clip 0.9",
+                                      "seeded +-1 diagonal, H_16384 = H_128 (x) H_128, clip 0.9"
+                                      + (", per-token INT8 codes" if code_bits == 8 else ""),
                           "tokens": int(bits.shape[0]), "n": int(bits.shape[1])})
     if name.startswith("decode"):
         n = int(name[len("decode"):] or 16384)
         bits = synthetic.decode(tokens or 32, n, seed=3 + rank)
-        return dict(kind="r4", bits=bits, signs=None, clip=1.0,
+        return dict(kind="r4", bits=bits, signs=None, clip=1.0, code_bits=4,
                     desc={"workload": f"decode: 32 tokens x n={n} Student-t(3), one channel x200 per row, clip 1.0",
                           "tokens": int(bits.shape[0]), "n": n})
     if name.startswith("sweep"):
         k = int(name[len("sweep"):])
         bits = synthetic.sweep(k, tokens=tokens, seed=4 + k + 100 * rank)
-        return dict(kind="r4", bits=bits, signs=None, clip=1.0,
+        return dict(kind="r4", bits=bits, signs=None, clip=1.0, code_bits=4,
                     desc={"workload": f"sweep: n=2^{k}, 1 GiB bf16 input, N(0,1) with 0.1% channels x100, clip 1.0",
                           "tokens": int(bits.shape[0]), "n": 1 << k})
     if name == "r3_kv":
@@ -219,7 +233,7 @@ def config_for(wl, world: int, workload: str) -> dict:
     """The `config` object both arms print (same workload, same keys)."""
     return dict(wl["desc"], parallelism=f"dp{world}" if world > 1 else "single GPU",
                 l2="inputs larger than L2 (268 MB bf16 input vs 126 MB L2); two buffer sets alternate"
-                if workload == "r4_prefill" else "two buffer sets alternate")
+                if workload.startswith("r4_prefill") else "two buffer sets alternate")
 
 
 def r3_bytes(tokens, hq=32, hkv=8, d=128):
@@ -238,14 +252,14 @@ def run_reference(args, wl):
     sample = min(bits.shape[0], max(8, (1 << 22) // n))  # about 0.1-0.2 s of oracle work per step
     rows = bits[:sample]
     for _ in range(args.warmup):
-        oracle.r4_rows(rows[:1], wl["clip"], wl["signs"])
+        oracle_r4_rows(oracle, rows[:1], wl["clip"], wl["signs"], wl["code_bits"])
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.r4_rows(rows, wl["clip"], wl["signs"])
+        oracle_r4_rows(oracle, rows, wl["clip"], wl["signs"], wl["code_bits"])
     dt = time.perf_counter() - t0
     tok_s = args.steps * sample / dt
-    gbs = algorithmic_bytes_r4(sample, n) * args.steps / dt / 1e9
-    line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "tokens_per_s": tok_s,
+    gbs = algorithmic_bytes_r4(sample, n, wl["code_bits"]) * args.steps / dt / 1e9
+    line = {"impl": "reference", "metric": metric_for(wl), "value": gbs, "unit": "GB/s", "tokens_per_s": tok_s,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -302,17 +316,19 @@ def main():
         bits, n = wl["bits"], wl["bits"].shape[1]
         tokens = bits.shape[0]
         host = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        code_bits = wl["code_bits"]
+        qshape, qtype = ((tokens, n // 2), torch.uint8) if code_bits == 4 else ((tokens, n), torch.int8)
+        quant = spin.hadamard_quant_int4 if code_bits == 4 else spin.hadamard_quant_int8
         sets = []
         for _ in range(2):
-            sets.append(dict(x=host.to(dev), q=torch.empty((tokens, n // 2), dtype=torch.uint8, device=dev),
+            sets.append(dict(x=host.to(dev), q=torch.empty(qshape, dtype=qtype, device=dev),
                              s=torch.empty((tokens,), dtype=torch.float32, device=dev)))
         signs = (torch.from_numpy(wl["signs"].view(np.int32)).to(dev) if wl["signs"] is not None else None)
-        step_bytes = algorithmic_bytes_r4(tokens, n)
+        step_bytes = algorithmic_bytes_r4(tokens, n, code_bits)
 
         def step(i, cores_only=False):
             b = sets[i & 1]
-            spin.hadamard_quant_int4(b["x"], wl["clip"], signs, out=b["q"], scales=b["s"], stream=stream,
-                                     cuda_cores_only=cores_only)
+            quant(b["x"], wl["clip"], signs, out=b["q"], scales=b["s"], stream=stream, cuda_cores_only=cores_only)
     else:
         q, k, v, pos = wl["q"], wl["k"], wl["v"], wl["pos"]
         B, S, hq, d = q.shape
@@ -359,7 +375,7 @@ def main():
     # ---- end to end through the public API from pinned host memory
     e2e = None
     if wl["kind"] == "r4":
-        q_host = torch.empty((tokens, n // 2), dtype=torch.uint8).pin_memory()
+        q_host = torch.empty(qshape, dtype=qtype).pin_memory()
         s_host = torch.empty((tokens,), dtype=torch.float32).pin_memory()
         b = sets[0]
         e2e_steps = max(3, args.steps // 5)
@@ -367,7 +383,7 @@ def main():
         def e2e_step():
             with torch.cuda.stream(stream):
                 b["x"].copy_(host, non_blocking=True)
-                spin.hadamard_quant_int4(b["x"], wl["clip"], signs, out=b["q"], scales=b["s"], stream=stream)
+                quant(b["x"], wl["clip"], signs, out=b["q"], scales=b["s"], stream=stream)
                 q_host.copy_(b["q"], non_blocking=True)
                 s_host.copy_(b["s"], non_blocking=True)
 
@@ -399,7 +415,7 @@ def main():
         ev1.record(stream)
         ev1.synchronize()
         cms = ev0.elapsed_time(ev1) / args.steps
-        cores = {"kernel": "k1_rotate_quant_int4 (all butterflies on CUDA cores)", "ms_per_step": cms,
+        cores = {"kernel": f"k1_rotate_quant_int{code_bits} (all butterflies on CUDA cores)", "ms_per_step": cms,
                  "achieved_gbs": step_bytes / (cms / 1e3) / 1e9}
 
     # ---- bandwidth sweep: the dequantise -> inverse-rotate round trip on this step's
@@ -494,14 +510,15 @@ def main():
         bits = wl["bits"]
         sample = bits.shape[0] if bits.shape[1] >= 4096 else min(bits.shape[0], 65536)
         t0 = time.perf_counter()
-        oracle.r4_rows(bits[:sample], wl["clip"], wl["signs"])
+        oracle_r4_rows(oracle, bits[:sample], wl["clip"], wl["signs"], wl["code_bits"])
         dt = time.perf_counter() - t0
-        cpu = {"value": algorithmic_bytes_r4(sample, bits.shape[1]) / dt / 1e9, "unit": "GB/s", "cores": 1,
+        cpu = {"value": algorithmic_bytes_r4(sample, bits.shape[1], wl["code_bits"]) / dt / 1e9, "unit": "GB/s",
+               "cores": 1,
                "kind": "oracle", "tokens_per_s": sample / dt,
                "sample": f"{sample} of {bits.shape[0]} tokens, one pass, fp64 fast transform, 1 thread"}
 
     if rank == 0:
-        line = {"metric": METRIC, "value": gbs, "unit": "GB/s", "tokens_per_s": tok_s,
+        line = {"metric": metric_for(wl), "value": gbs, "unit": "GB/s", "tokens_per_s": tok_s,
                 "pct_of_hbm_peak": 100.0 * per_gpu_gbs / peak, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic",

@@ -134,6 +134,27 @@ spin_status_t spin_hadamard_quant_int4_ex(const void *x_bf16, int64_t tokens, in
                                           spin_stream_t stream);
 
 /*
+ * R4 with per-token INT8 codes ("SpinQuant Guide: Learned Rotations for 4-Bit
+ * LLMs", section "The Outlier Curse": the symmetric b-bit rule, range
+ * [-2^(b-1), 2^(b-1) - 1] and step max / (2^(b-1) - 1), here at b = 8 -- the
+ * 8-bit activations of the W4A8 decoding figure in "SpinQuant, when rotations
+ * are worth learning", section "Measured effects").
+ * For each of `tokens` rows x:
+ *   y = H_n D x / sqrt(n),  m = max_j |y_j|,  scale = max(clip * m / 127, 1e-8)
+ *   code_j = clamp(round_half_even(y_j / scale), -128, 127)
+ *
+ *  x_bf16, tokens, n, clip, sign_bits, flags, scales_f32, stream: as in
+ *             spin_hadamard_quant_int4_ex (same kernels and dispatch, the same
+ *             SPIN_NO_ROTATE / SPIN_CUDA_CORES_ONLY / SPIN_TENSOR_CORES bits)
+ *  q_i8       [tokens, n] int8 codes (one two's-complement byte per element,
+ *             element j at byte j), 16-byte aligned, written
+ * Errors: as spin_hadamard_quant_int4_ex.
+ */
+spin_status_t spin_hadamard_quant_int8(const void *x_bf16, int64_t tokens, int32_t n, float clip,
+                                       const uint32_t *sign_bits, uint32_t flags, int8_t *q_i8,
+                                       float *scales_f32, spin_stream_t stream);
+
+/*
  * R3 + INT4 KV cache ("SpinQuant, when rotations are worth learning", "Four
  * rotation sites": R3 is a fixed Hadamard on queries and keys after RoPE,
  * there only to make the KV cache quantisable; "SpinQuant Guide", "RoPE

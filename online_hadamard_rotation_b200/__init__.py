@@ -18,7 +18,8 @@ import re
 import torch
 
 __all__ = [
-    "lib", "SpinError", "hadamard_quant_int4", "hadamard_quant_int4_host", "rope_hadamard_kvquant",
+    "lib", "SpinError", "hadamard_quant_int4", "hadamard_quant_int8", "hadamard_quant_int4_host",
+    "rope_hadamard_kvquant",
     "dequant_hadamard_inverse", "alloc_kv_cache", "NO_ROTATE", "SYM_INT4_F32SCALE", "ASYM_INT4_F16SZ",
     "BF16", "F32", "HEADER", "LIB_PATH", "exported_symbols", "CUDA_CORES_ONLY", "TENSOR_CORES", "device_status",
 ]
@@ -66,9 +67,10 @@ def lib() -> C.CDLL:
     L.spin_hadamard_quant_int4_ex.argtypes = [vp, i64, i32, f32, vp, u32, vp, vp, vp]
     L.spin_rope_hadamard_kvquant.argtypes = [vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, f32, vp, vp, vp,
                                              vp, vp, vp, vp, i32, i32, vp]
+    L.spin_hadamard_quant_int8.argtypes = [vp, i64, i32, f32, vp, u32, vp, vp, vp]
     L.spin_dequant_hadamard_inverse.argtypes = [vp, i64, i32, i32, vp, vp, vp, u32, vp, i32, vp]
-    for name in ("spin_hadamard_quant_int4", "spin_hadamard_quant_int4_ex", "spin_rope_hadamard_kvquant",
-                 "spin_dequant_hadamard_inverse"):
+    for name in ("spin_hadamard_quant_int4", "spin_hadamard_quant_int4_ex", "spin_hadamard_quant_int8",
+                 "spin_rope_hadamard_kvquant", "spin_dequant_hadamard_inverse"):
         getattr(L, name).restype = C.c_int
     L.spin_test_stall_tensor_core_waits.argtypes = [C.c_int]
     L.spin_test_stall_tensor_core_waits.restype = None
@@ -103,6 +105,10 @@ def spin_hadamard_quant_int4_ex(x_bf16, tokens, n, clip, sign_bits, flags, q_pac
                                 stream) -> int:
     return lib().spin_hadamard_quant_int4_ex(x_bf16, tokens, n, clip, sign_bits, flags, q_packed_u8,
                                              scales_f32, stream)
+
+
+def spin_hadamard_quant_int8(x_bf16, tokens, n, clip, sign_bits, flags, q_i8, scales_f32, stream) -> int:
+    return lib().spin_hadamard_quant_int8(x_bf16, tokens, n, clip, sign_bits, flags, q_i8, scales_f32, stream)
 
 
 def spin_rope_hadamard_kvquant(*args) -> int:
@@ -163,6 +169,27 @@ def hadamard_quant_int4(x: torch.Tensor, clip: float = 1.0, signs: torch.Tensor 
     st = spin_hadamard_quant_int4_ex(_ptr(x), tokens, n, float(clip), _ptr(signs), flags,
                                      _ptr(out), _ptr(scales), _stream(stream))
     _check("spin_hadamard_quant_int4_ex", st)
+    return out, scales
+
+
+def hadamard_quant_int8(x: torch.Tensor, clip: float = 1.0, signs: torch.Tensor | None = None,
+                        no_rotate: bool = False, out: torch.Tensor | None = None,
+                        scales: torch.Tensor | None = None, stream=None, cuda_cores_only: bool = False,
+                        tensor_cores: bool = False):
+    """R4 with INT8 codes: x [tokens, n] bf16 (CUDA) -> (codes [tokens, n] int8, scales [tokens] fp32)."""
+    _need(x, "x", torch.bfloat16)
+    tokens, n = x.shape
+    if out is None:
+        out = torch.empty((tokens, n), dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty((tokens,), dtype=torch.float32, device=x.device)
+    if signs is not None:
+        _need(signs, "signs", torch.int32, x.device)
+    flags = ((NO_ROTATE if no_rotate else 0) | (CUDA_CORES_ONLY if cuda_cores_only else 0) |
+             (TENSOR_CORES if tensor_cores else 0))
+    st = spin_hadamard_quant_int8(_ptr(x), tokens, n, float(clip), _ptr(signs), flags, _ptr(out), _ptr(scales),
+                                  _stream(stream))
+    _check("spin_hadamard_quant_int8", st)
     return out, scales
 
 

@@ -102,27 +102,40 @@ cudaError_t resident_slots(const void *kernel, int threads, int dyn_smem, int *s
 
 using namespace spin;
 
-extern "C" {
-
-spin_status_t spin_hadamard_quant_int4_ex(const void *x_bf16, int64_t tokens, int32_t n, float clip,
-                                          const uint32_t *sign_bits, uint32_t flags,
-                                          uint8_t *q_packed_u8, float *scales_f32,
-                                          spin_stream_t stream) {
+// R4 with `bits` = 4 or 8: host-side checks, then the launch.
+static spin_status_t hadamard_quant(const void *x_bf16, int64_t tokens, int32_t n, float clip,
+                                    const uint32_t *sign_bits, uint32_t flags, int bits, uint8_t *q,
+                                    float *scales_f32, spin_stream_t stream) {
   const int log_n = log2_pow2(n);
   if (log_n < 7 || log_n > 15) return SPIN_ERR_UNSUPPORTED_SIZE;
   if (tokens < 0 || !valid_clip(clip) || (flags & ~(SPIN_NO_ROTATE | SPIN_CUDA_CORES_ONLY | SPIN_TENSOR_CORES)) != 0 ||
       (flags & SPIN_CUDA_CORES_ONLY && flags & SPIN_TENSOR_CORES))
     return SPIN_ERR_INVALID_ARG;
   if (tokens == 0) return SPIN_OK;
-  if (!x_bf16 || !q_packed_u8 || !scales_f32) return SPIN_ERR_INVALID_ARG;
+  if (!x_bf16 || !q || !scales_f32) return SPIN_ERR_INVALID_ARG;
   if (tokens > (INT64_MAX >> 16)) return SPIN_ERR_INVALID_ARG;
-  if (!aligned(x_bf16, 16) || !aligned(q_packed_u8, 16) || !aligned(scales_f32, 4) ||
-      (sign_bits && !aligned(sign_bits, 4)))
+  if (!aligned(x_bf16, 16) || !aligned(q, 16) || !aligned(scales_f32, 4) || (sign_bits && !aligned(sign_bits, 4)))
     return SPIN_ERR_MISALIGNED;
   spin_status_t st = check_device();
   if (st != SPIN_OK) return st;
-  return cuda_status(launch_rotate_quant_int4(x_bf16, tokens, log_n, clip, sign_bits, flags, q_packed_u8,
-                                              scales_f32, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_rotate_quant(x_bf16, tokens, log_n, clip, sign_bits, flags, bits, q, scales_f32,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+extern "C" {
+
+spin_status_t spin_hadamard_quant_int4_ex(const void *x_bf16, int64_t tokens, int32_t n, float clip,
+                                          const uint32_t *sign_bits, uint32_t flags,
+                                          uint8_t *q_packed_u8, float *scales_f32,
+                                          spin_stream_t stream) {
+  return hadamard_quant(x_bf16, tokens, n, clip, sign_bits, flags, 4, q_packed_u8, scales_f32, stream);
+}
+
+spin_status_t spin_hadamard_quant_int8(const void *x_bf16, int64_t tokens, int32_t n, float clip,
+                                       const uint32_t *sign_bits, uint32_t flags, int8_t *q_i8,
+                                       float *scales_f32, spin_stream_t stream) {
+  return hadamard_quant(x_bf16, tokens, n, clip, sign_bits, flags, 8, reinterpret_cast<uint8_t *>(q_i8),
+                        scales_f32, stream);
 }
 
 spin_status_t spin_hadamard_quant_int4(const void *x_bf16, int64_t tokens, int32_t n, float clip,

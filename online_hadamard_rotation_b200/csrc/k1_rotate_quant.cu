@@ -1,6 +1,7 @@
 // k1_rotate_quant.cu -- R4 on CUDA cores: bf16 rows -> optional +-1 diagonal
 // -> Walsh-Hadamard transform -> per-row max|y| -> symmetric INT4 codes packed
-// two per byte, plus an fp32 step per row, in one pass over memory.
+// two per byte (or INT8 codes, one per byte), plus an fp32 step per row, in one
+// pass over memory.
 //
 // "SpinQuant, when rotations are worth learning", section "Four rotation
 // sites": R4 is a fixed Hadamard on the down-projection input.
@@ -9,14 +10,16 @@
 // outlier channel": per-token 4-bit step max/7.
 // "SpinQuant Guide: Learned Rotations for 4-Bit LLMs", section "The Outlier
 // Curse": INT4 range [-8, 7]; section "End-to-End Implementation": the step is
-// clamped below at 1e-8.
+// clamped below at 1e-8. The same rule at b = 8 bits gives the per-token INT8
+// codes (range [-128, 127], step max / 127).
 //
 // The transform is computed unnormalised (u = H_n D x); the 1/sqrt(n) factor
-// is folded into the step, since the codes do not depend on it:
-//   step = max(clip * max|u| / sqrt(n) / 7, 1e-8),   code = clamp(rne(u / (sqrt(n) * step)), -8, 7).
-// Codes come out of two FMAs: v = sat(u * c/15 + 8/15) clamps to the code
-// range, and fma(v, 15, 1.5 * 2^23) rounds 15 v to the nearest integer (ties to
-// even) in the low mantissa bits, where byte permutes pick them up.
+// is folded into the step, since the codes do not depend on it (Q = 7 or 127):
+//   step = max(clip * max|u| / sqrt(n) / Q, 1e-8),   code = clamp(rne(u / (sqrt(n) * step)), -Q-1, Q).
+// Codes come out of two FMAs: v = sat(u * c/(2Q+1) + (Q+1)/(2Q+1)) clamps to the
+// code range, and fma(v, 2Q+1, 1.5 * 2^23) rounds (2Q+1) v to the nearest
+// integer (ties to even) in the low mantissa bits, where byte permutes pick
+// them up.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -45,11 +48,18 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&b)[8]) {
   return (e | (o << 4)) ^ 0x88888888u;
 }
 
-template <int TB, int LOGN, bool ROTATE, bool SIGNS>
-__global__ void __launch_bounds__(1 << (TB - 7))
-    k1_rotate_quant_int4(const uint4 *__restrict__ x, int64_t tokens, float clip, float inv_sqrt_n,
-                         const uint32_t *__restrict__ signs, uint32_t *__restrict__ q,
-                         float *__restrict__ scales) {
+// 4 biased codes (0..255, in the low byte of each word) -> one word of 4 bytes,
+// code k in byte k, converted to 8-bit two's complement.
+__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410) ^ 0x80808080u;
+}
+
+template <int BITS, int TB, int LOGN, bool ROTATE, bool SIGNS>
+__device__ __forceinline__ void rotate_quant_body(const uint4 *__restrict__ x, int64_t tokens, float clip,
+                                                  float inv_sqrt_n, const uint32_t *__restrict__ signs,
+                                                  uint32_t *__restrict__ q, float *__restrict__ scales) {
+  constexpr float QMAX = BITS == 4 ? 7.0f : 127.0f;   // largest code
+  constexpr float LEVELS = 2.0f * QMAX + 1.0f;        // 15 or 255 steps across the range
   constexpr int ROWS = 1 << (TB - LOGN);  // rows per tile
   constexpr uint32_t NMASK = (1u << LOGN) - 1u;
   using LI = L1<TB>;
@@ -148,16 +158,16 @@ __global__ void __launch_bounds__(1 << (TB - 7))
     __syncthreads();
     if (t < (uint32_t)ROWS) {
       const float m = __uint_as_float(rowmax[t]) * inv_sqrt_n;
-      const float s = fmaxf(clip * m / 7.0f, 1e-8f);
-      rowc15[t] = (inv_sqrt_n / s) / 15.0f;
+      const float s = fmaxf(clip * m / QMAX, 1e-8f);
+      rowc15[t] = (inv_sqrt_n / s) / LEVELS;
       const int64_t row = tile * ROWS + t;
       if (row < tokens) scales[row] = s;
     }
     __syncthreads();
 
     // ---- quantise, pack, store
-    constexpr float k815 = 8.0f / 15.0f;
-    uint32_t *qt = q + tile * (int64_t)(1 << (TB - 3));
+    constexpr float k815 = (QMAX + 1.0f) / LEVELS;  // code 0 sits at (Q + 1) / (2Q + 1)
+    uint32_t *qt = q + tile * (int64_t)(1 << (TB - 3)) * (BITS / 4);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const uint32_t rr = ((((uint32_t)(j >> SH) << SH)) << HB) >> LOGN;
@@ -166,18 +176,40 @@ __global__ void __launch_bounds__(1 << (TB - 7))
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float vv = fma_sat(v[8 * j + i], c15, k815);
-        b[i] = __float_as_uint(fmaf(vv, 15.0f, kMagic));
+        b[i] = __float_as_uint(fmaf(vv, LEVELS, kMagic));
       }
       const uint32_t E = LO::thr(t) | LO::reg(8 * j);
-      if (tile * ROWS + (E >> LOGN) < tokens) __stcs(qt + (E >> 3), pack8(b));
+      if (tile * ROWS + (E >> LOGN) < tokens) {
+        if constexpr (BITS == 4)
+          __stcs(qt + (E >> 3), pack8(b));
+        else
+          __stcs(reinterpret_cast<uint2 *>(qt) + (E >> 3),
+                 make_uint2(pack4(b[0], b[1], b[2], b[3]), pack4(b[4], b[5], b[6], b[7])));
+      }
     }
   }
 }
 
 template <int TB, int LOGN, bool ROTATE, bool SIGNS>
+__global__ void __launch_bounds__(1 << (TB - 7))
+    k1_rotate_quant_int4(const uint4 *__restrict__ x, int64_t tokens, float clip, float inv_sqrt_n,
+                         const uint32_t *__restrict__ signs, uint32_t *__restrict__ q,
+                         float *__restrict__ scales) {
+  rotate_quant_body<4, TB, LOGN, ROTATE, SIGNS>(x, tokens, clip, inv_sqrt_n, signs, q, scales);
+}
+
+template <int TB, int LOGN, bool ROTATE, bool SIGNS>
+__global__ void __launch_bounds__(1 << (TB - 7))
+    k1_rotate_quant_int8(const uint4 *__restrict__ x, int64_t tokens, float clip, float inv_sqrt_n,
+                         const uint32_t *__restrict__ signs, uint32_t *__restrict__ q,
+                         float *__restrict__ scales) {
+  rotate_quant_body<8, TB, LOGN, ROTATE, SIGNS>(x, tokens, clip, inv_sqrt_n, signs, q, scales);
+}
+
+template <int BITS, int TB, int LOGN, bool ROTATE, bool SIGNS>
 cudaError_t launch_one(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q,
                        float *scales, cudaStream_t stream) {
-  auto kern = k1_rotate_quant_int4<TB, LOGN, ROTATE, SIGNS>;
+  auto kern = BITS == 4 ? k1_rotate_quant_int4<TB, LOGN, ROTATE, SIGNS> : k1_rotate_quant_int8<TB, LOGN, ROTATE, SIGNS>;
   constexpr int kThreads = 1 << (TB - 7);
   constexpr int kSmem = (1 << TB) * (int)sizeof(float);
   int slots = 0;
@@ -193,35 +225,43 @@ cudaError_t launch_one(const void *x, int64_t tokens, float clip, const uint32_t
   return cudaGetLastError();
 }
 
-template <int LOGN>
+template <int BITS, int LOGN>
 cudaError_t launch_n(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint32_t flags,
                      uint8_t *q, float *scales, cudaStream_t stream) {
   constexpr int TB = LOGN <= 14 ? 14 : 15;
-  if (flags & kNoRotate) return launch_one<TB, LOGN, false, false>(x, tokens, clip, nullptr, q, scales, stream);
-  if (signs) return launch_one<TB, LOGN, true, true>(x, tokens, clip, signs, q, scales, stream);
-  return launch_one<TB, LOGN, true, false>(x, tokens, clip, nullptr, q, scales, stream);
+  if (flags & kNoRotate)
+    return launch_one<BITS, TB, LOGN, false, false>(x, tokens, clip, nullptr, q, scales, stream);
+  if (signs) return launch_one<BITS, TB, LOGN, true, true>(x, tokens, clip, signs, q, scales, stream);
+  return launch_one<BITS, TB, LOGN, true, false>(x, tokens, clip, nullptr, q, scales, stream);
+}
+
+template <int BITS>
+cudaError_t launch_bits(const void *x, int64_t tokens, int log_n, float clip, const uint32_t *signs,
+                        uint32_t flags, uint8_t *q, float *scales, cudaStream_t stream) {
+  switch (log_n) {
+    case 7: return launch_n<BITS, 7>(x, tokens, clip, signs, flags, q, scales, stream);
+    case 8: return launch_n<BITS, 8>(x, tokens, clip, signs, flags, q, scales, stream);
+    case 9: return launch_n<BITS, 9>(x, tokens, clip, signs, flags, q, scales, stream);
+    case 10: return launch_n<BITS, 10>(x, tokens, clip, signs, flags, q, scales, stream);
+    case 11: return launch_n<BITS, 11>(x, tokens, clip, signs, flags, q, scales, stream);
+    case 12: return launch_n<BITS, 12>(x, tokens, clip, signs, flags, q, scales, stream);
+    case 13: return launch_n<BITS, 13>(x, tokens, clip, signs, flags, q, scales, stream);
+    case 14: return launch_n<BITS, 14>(x, tokens, clip, signs, flags, q, scales, stream);
+    case 15: return launch_n<BITS, 15>(x, tokens, clip, signs, flags, q, scales, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
 
-cudaError_t launch_rotate_quant_int4(const void *x, int64_t tokens, int log_n, float clip,
-                                     const uint32_t *signs, uint32_t flags, uint8_t *q, float *scales,
-                                     cudaStream_t stream) {
+cudaError_t launch_rotate_quant(const void *x, int64_t tokens, int log_n, float clip, const uint32_t *signs,
+                                uint32_t flags, int bits, uint8_t *q, float *scales, cudaStream_t stream) {
+  if (bits != 4 && bits != 8) return cudaErrorInvalidValue;
   if (!(flags & kCudaCoresOnly) && tc_rotate_quant_supported(log_n, tokens, flags, signs != nullptr))
-    return launch_rotate_quant_int4_tc(log_n, x, tokens, clip, signs, q, scales, stream);
+    return launch_rotate_quant_tc(log_n, bits, x, tokens, clip, signs, q, scales, stream);
   flags &= ~(kCudaCoresOnly | kTensorCores);
-  switch (log_n) {
-    case 7: return launch_n<7>(x, tokens, clip, signs, flags, q, scales, stream);
-    case 8: return launch_n<8>(x, tokens, clip, signs, flags, q, scales, stream);
-    case 9: return launch_n<9>(x, tokens, clip, signs, flags, q, scales, stream);
-    case 10: return launch_n<10>(x, tokens, clip, signs, flags, q, scales, stream);
-    case 11: return launch_n<11>(x, tokens, clip, signs, flags, q, scales, stream);
-    case 12: return launch_n<12>(x, tokens, clip, signs, flags, q, scales, stream);
-    case 13: return launch_n<13>(x, tokens, clip, signs, flags, q, scales, stream);
-    case 14: return launch_n<14>(x, tokens, clip, signs, flags, q, scales, stream);
-    case 15: return launch_n<15>(x, tokens, clip, signs, flags, q, scales, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  return bits == 4 ? launch_bits<4>(x, tokens, log_n, clip, signs, flags, q, scales, stream)
+                   : launch_bits<8>(x, tokens, log_n, clip, signs, flags, q, scales, stream);
 }
 
 }  // namespace spin

@@ -169,6 +169,35 @@ __device__ __forceinline__ void round15_x2(float a0, float a1, uint32_t &r0, uin
   asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(R));
 }
 
+// INT8 variant: (r0, r1) = bit patterns of fma(a, 255, 1.5 * 2^23), rounding 255 a to
+// an integer (ties to even) in the low mantissa bits.
+__device__ __forceinline__ void round255_x2(float a0, float a1, uint32_t &r0, uint32_t &r1) {
+  uint64_t A, R;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(R) : "l"(A), "l"(0x437F0000437F0000ull), "l"(0x4B4000004B400000ull));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(R));
+}
+
+// four biased INT8 codes (0..255 in the low byte of each word) -> one word, code k in
+// byte k, converted to two's complement
+__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410) ^ 0x80808080u;
+}
+
+// 8 consecutive values -> two words of INT8 codes (c255 = 1 / (255 step) in the
+// values' scale)
+__device__ __forceinline__ void codes8_int8(const float *v, float c255, uint32_t &w0, uint32_t &w1) {
+  constexpr float k128 = 128.0f / 255.0f;
+  uint32_t b[8];
+  float t[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) t[k] = fma_sat(v[k], c255, k128);
+#pragma unroll
+  for (int k = 0; k < 8; k += 2) round255_x2(t[k], t[k + 1], b[k], b[k + 1]);
+  w0 = pack4(b[0], b[1], b[2], b[3]);
+  w1 = pack4(b[4], b[5], b[6], b[7]);
+}
+
 __device__ __forceinline__ void st_v8_cs(void *p, const uint32_t *w) {
   asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
                "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
@@ -204,7 +233,7 @@ __device__ __forceinline__ void load_group(uint8_t *dst, const CUtensorMap *map,
                       (int)((t0 + t) * SH::ROWS + (j / SH::CBOX) * 128));
 }
 
-template <int LOGN, bool SIGNS, bool STORE32>
+template <int LOGN, bool SIGNS, bool STORE32, int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
     k1_tc_rotate_quant(const __grid_constant__ CUtensorMap xmap, int64_t tokens, float clip, float inv_sqrt_n,
                        const uint32_t *__restrict__ signs, uint8_t *__restrict__ q, float *__restrict__ scales,
@@ -337,93 +366,93 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
         } else {
 #pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            // A: 16 columns k of H per step. B: rows a = 16 s .. 16 s + 15 of every box
-            // (MN-major: boxes of BOXW columns BOXBYTES apart, 8-row groups 8 ROWB apart).
-            const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-            uint64_t bd = tc::smem_desc(sX + st * kGroupBytes + s * 16 * SH::ROWB, SH::BOXBYTES, 8 * SH::ROWB);
-            bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
-            tc::umma_bf16(tmem + acc * 256, ad, bd, idesc, s > 0 ? 1u : 0u);
+            for (int s = 0; s < 8; ++s) {
+              // A: 16 columns k of H per step. B: rows a = 16 s .. 16 s + 15 of every box
+              // (MN-major: boxes of BOXW columns BOXBYTES apart, 8-row groups 8 ROWB apart).
+              const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
+              uint64_t bd = tc::smem_desc(sX + st * kGroupBytes + s * 16 * SH::ROWB, SH::BOXBYTES, 8 * SH::ROWB);
+              bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
+              tc::umma_bf16(tmem + acc * 256, ad, bd, idesc, s > 0 ? 1u : 0u);
+            }
           }
+          tc::umma_commit(&S.empty[st]);
+          // Stall test hook: withhold the first group's completion signal, so the
+          // epilogue's wait runs out and the CTA takes its abort path.
+          if (!(stall_test && i == 0)) tc::umma_commit(&S.tfull[acc]);
         }
-        tc::umma_commit(&S.empty[st]);
-        // Stall test hook: withhold the first group's completion signal, so the
-        // epilogue's wait runs out and the CTA takes its abort path.
-        if (!(stall_test && i == 0)) tc::umma_commit(&S.tfull[acc]);
       }
-    }
-  } else if (warp < 4) {
-    if constexpr (SIGNS) {
-      // Thread ts flips the signs of chunks ts + 64 j of each group's 64 KiB.
-      // Those chunks sit at NPOS distinct positions of a token's tile; their
-      // sign words stay in registers for the whole kernel.
-      constexpr int NPOS = SH::NPOS;
-      const uint32_t ts = threadIdx.x - 64;  // 0..63
-      uint4 mk[NPOS];
+    } else if (warp < 4) {
+      if constexpr (SIGNS) {
+        // Thread ts flips the signs of chunks ts + 64 j of each group's 64 KiB.
+        // Those chunks sit at NPOS distinct positions of a token's tile; their
+        // sign words stay in registers for the whole kernel.
+        constexpr int NPOS = SH::NPOS;
+        const uint32_t ts = threadIdx.x - 64;  // 0..63
+        uint4 mk[NPOS];
 #pragma unroll
-      for (int k = 0; k < NPOS; ++k) {
-        const uint32_t pos = ts + 64u * k;  // 16-byte chunk index inside one token's tile
-        const uint32_t box = pos / (SH::BOXBYTES / 16), inbox = pos % (SH::BOXBYTES / 16);
-        const uint32_t a = inbox / SH::CPR, pc = inbox % SH::CPR;
-        const uint32_t ch = SH::ROWB == 128 ? (pc ^ (a & 7u)) : (pc ^ ((a >> 1) & 3u));
-        const uint32_t e = a * B + box * SH::BOXW + ch * 8u;
-        const uint32_t byte = (__ldg(signs + (e >> 5)) >> (e & 31u)) & 0xFFu;
-        uint32_t w[4];
+        for (int k = 0; k < NPOS; ++k) {
+          const uint32_t pos = ts + 64u * k;  // 16-byte chunk index inside one token's tile
+          const uint32_t box = pos / (SH::BOXBYTES / 16), inbox = pos % (SH::BOXBYTES / 16);
+          const uint32_t a = inbox / SH::CPR, pc = inbox % SH::CPR;
+          const uint32_t ch = SH::ROWB == 128 ? (pc ^ (a & 7u)) : (pc ^ ((a >> 1) & 3u));
+          const uint32_t e = a * B + box * SH::BOXW + ch * 8u;
+          const uint32_t byte = (__ldg(signs + (e >> 5)) >> (e & 31u)) & 0xFFu;
+          uint32_t w[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) w[j] = (((byte >> (2 * j)) & 1u) << 15) | (((byte >> (2 * j + 1)) & 1u) << 31);
-        mk[k] = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int j = 0; j < 4; ++j) w[j] = (((byte >> (2 * j)) & 1u) << 15) | (((byte >> (2 * j + 1)) & 1u) << 31);
+          mk[k] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        for (int64_t i = 0;; ++i) {
+          const int st = (int)(i % kStages);
+          if (ts == 0) {
+            int ok = wait_bounded(&S.full[st], (uint32_t)((i / kStages) & 1), S, true) ? 1 : 0;
+            if (ok && S.gid[i % kRing] < 0) {
+              tc::mbar_arrive(&S.sgn[st]);  // pass the end mark on to the MMA
+              ok = 0;
+            }
+            S.dec[2] = ok;
+          }
+          tc::named_sync(3, 64);
+          if (!S.dec[2]) break;
+          uint4 *X = reinterpret_cast<uint4 *>(smem + kOffX + st * kGroupBytes) + ts;
+#pragma unroll
+          for (int j0 = 0; j0 < 64; j0 += 4) {
+            uint4 x[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) x[u] = X[64 * (j0 + u)];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint4 m = mk[(j0 + u) % NPOS];
+              X[64 * (j0 + u)] = make_uint4(x[u].x ^ m.x, x[u].y ^ m.y, x[u].z ^ m.z, x[u].w ^ m.w);
+            }
+          }
+          tc::fence_proxy_async_smem();
+          tc::named_sync(3, 64);
+          if (ts == 0) tc::mbar_arrive(&S.sgn[st]);
+        }
       }
+    } else {
+      // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1)
+      const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
+      const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
       for (int64_t i = 0;; ++i) {
-        const int st = (int)(i % kStages);
-        if (ts == 0) {
-          int ok = wait_bounded(&S.full[st], (uint32_t)((i / kStages) & 1), S, true) ? 1 : 0;
-          if (ok && S.gid[i % kRing] < 0) {
-            tc::mbar_arrive(&S.sgn[st]);  // pass the end mark on to the MMA
-            ok = 0;
-          }
-          S.dec[2] = ok;
-        }
-        tc::named_sync(3, 64);
-        if (!S.dec[2]) break;
-        uint4 *X = reinterpret_cast<uint4 *>(smem + kOffX + st * kGroupBytes) + ts;
-#pragma unroll
-        for (int j0 = 0; j0 < 64; j0 += 4) {
-          uint4 x[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) x[u] = X[64 * (j0 + u)];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint4 m = mk[(j0 + u) % NPOS];
-            X[64 * (j0 + u)] = make_uint4(x[u].x ^ m.x, x[u].y ^ m.y, x[u].z ^ m.z, x[u].w ^ m.w);
-          }
-        }
-        tc::fence_proxy_async_smem();
-        tc::named_sync(3, 64);
-        if (ts == 0) tc::mbar_arrive(&S.sgn[st]);
-      }
-    }
-  } else {
-    // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1)
-    const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
-    const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
-    for (int64_t i = 0;; ++i) {
-      const int acc = (int)(i & 1);
-      // the step's group from the producer's ring, then its accumulator
-      auto decide = [&](int slot) {
-        int ok = wait_bounded(&S.gfull[i % kRing], (uint32_t)((i / kRing) & 1), S, true) ? 1 : 0;
-        const int64_t gp = ok ? S.gid[i % kRing] : -1;
-        if (gp < 0) ok = 0;
-        if (ok) ok = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
-        S.egid[slot] = gp;
-        S.dec[slot] = ok;
-      };
-      int64_t p;
-      if constexpr (SH::SPLIT) {  // one decision for both warpgroups: they meet at barrier 4 below
-        if (threadIdx.x == 128) decide(0);
-        tc::named_sync(4, 256);
-        if (!S.dec[0]) break;
-        p = S.egid[0];
-      } else {
+        const int acc = (int)(i & 1);
+        // the step's group from the producer's ring, then its accumulator
+        auto decide = [&](int slot) {
+          int ok = wait_bounded(&S.gfull[i % kRing], (uint32_t)((i / kRing) & 1), S, true) ? 1 : 0;
+          const int64_t gp = ok ? S.gid[i % kRing] : -1;
+          if (gp < 0) ok = 0;
+          if (ok) ok = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+          S.egid[slot] = gp;
+          S.dec[slot] = ok;
+        };
+        int64_t p;
+        if constexpr (SH::SPLIT) {  // one decision for both warpgroups: they meet at barrier 4 below
+          if (threadIdx.x == 128) decide(0);
+          tc::named_sync(4, 256);
+          if (!S.dec[0]) break;
+          p = S.egid[0];
+        } else {
         if (tg == 0) decide(g);
         tc::named_sync(1 + g, 128);
         if (!S.dec[g]) break;
@@ -479,31 +508,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (SH::SPLIT)
           mu = fmaxf(mu, fmaxf(fmaxf(S.wmax[g ^ 1][i & 1][0][0], S.wmax[g ^ 1][i & 1][1][0]),
                                fmaxf(S.wmax[g ^ 1][i & 1][2][0], S.wmax[g ^ 1][i & 1][3][0])));
-        const float s = fmaxf(clip * (mu * inv_sqrt_n) / 7.0f, 1e-8f);
-        const float c15 = (inv_sqrt_n / 15.0f) / s;
+        const float s = fmaxf(clip * (mu * inv_sqrt_n) / (BITS == 4 ? 7.0f : 127.0f), 1e-8f);
+        const float c15 = (inv_sqrt_n / (BITS == 4 ? 15.0f : 255.0f)) / s;
         const int64_t token = SH::SPLIT ? p : p * SH::TOK + g * SEG + sg;
         if (token >= tokens) continue;
         const uint32_t orow = SH::SPLIT ? 128u * g + row : row;  // output row of B values
-        uint8_t *dst = q + token * SH::OUTB + orow * (B / 2);
-        uint32_t words[B / 8];
+        uint8_t *dst = q + token * (SH::OUTB * (BITS / 4)) + orow * (B * BITS / 8);
+        if constexpr (BITS == 8) {
+          // one code byte per value: 32 bytes (8 words) at a time
 #pragma unroll
-        for (int wi = 0; wi < B / 8; ++wi) {
-          uint32_t b[8];
-          float t[8];
+          for (int c8 = 0; c8 < B / 32; ++c8) {
+            uint32_t w8[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) t[k] = fma_sat(v[sg * B + 8 * wi + k], c15, k815);
-#pragma unroll
-          for (int k = 0; k < 8; k += 2) round15_x2(t[k], t[k + 1], b[k], b[k + 1]);
-          words[wi] = pack8(b);
-        }
-        if constexpr (STORE32 && B >= 64) {
-#pragma unroll
-          for (int w8 = 0; w8 < B / 64; ++w8) st_v8_cs(dst + 32 * w8, words + 8 * w8);
+            for (int h = 0; h < 4; ++h) codes8_int8(v + sg * B + 32 * c8 + 8 * h, c15, w8[2 * h], w8[2 * h + 1]);
+            if constexpr (STORE32) {
+              st_v8_cs(dst + 32 * c8, w8);
+            } else {
+              __stcs(reinterpret_cast<uint4 *>(dst + 32 * c8), make_uint4(w8[0], w8[1], w8[2], w8[3]));
+              __stcs(reinterpret_cast<uint4 *>(dst + 32 * c8) + 1, make_uint4(w8[4], w8[5], w8[6], w8[7]));
+            }
+          }
         } else {
+          uint32_t words[B / 8];
 #pragma unroll
-          for (int w4 = 0; w4 < B / 32; ++w4)
-            __stcs(reinterpret_cast<uint4 *>(dst) + w4,
-                   make_uint4(words[4 * w4], words[4 * w4 + 1], words[4 * w4 + 2], words[4 * w4 + 3]));
+          for (int wi = 0; wi < B / 8; ++wi) {
+            uint32_t b[8];
+            float t[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t[k] = fma_sat(v[sg * B + 8 * wi + k], c15, k815);
+#pragma unroll
+            for (int k = 0; k < 8; k += 2) round15_x2(t[k], t[k + 1], b[k], b[k + 1]);
+            words[wi] = pack8(b);
+          }
+          if constexpr (STORE32 && B >= 64) {
+#pragma unroll
+            for (int w8 = 0; w8 < B / 64; ++w8) st_v8_cs(dst + 32 * w8, words + 8 * w8);
+          } else {
+#pragma unroll
+            for (int w4 = 0; w4 < B / 32; ++w4)
+              __stcs(reinterpret_cast<uint4 *>(dst) + w4,
+                     make_uint4(words[4 * w4], words[4 * w4 + 1], words[4 * w4 + 2], words[4 * w4 + 3]));
+          }
         }
         if (tg == 0 && (!SH::SPLIT || g == 0)) scales[token] = s;
       }
@@ -524,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int LOGN, bool SIGNS, bool STORE32>
+template <int LOGN, bool SIGNS, bool STORE32, int BITS>
 cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
                       cudaStream_t stream, int stall_test) {
   using SH = Shape<LOGN>;
@@ -540,7 +585,7 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
                   SH::ROWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto kern = k1_tc_rotate_quant<LOGN, SIGNS, STORE32>;
+  auto kern = k1_tc_rotate_quant<LOGN, SIGNS, STORE32, BITS>;
   int slots = 0;
   cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreads, (int)kSmemBytes, &slots);
   if (err != cudaSuccess) return err;
@@ -561,18 +606,18 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
   return cudaLaunchKernelEx(&cfg, kern, map, tokens, clip, inv_sqrt_n, signs, q, scales, stall_test);
 }
 
-template <int LOGN>
+template <int LOGN, int BITS>
 cudaError_t launch_n(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
                      cudaStream_t stream, int stall_test) {
   const bool a32 = (reinterpret_cast<uintptr_t>(q) & 31u) == 0;  // 32-byte stores need 32-byte alignment
   if constexpr (Shape<LOGN>::SPLIT) {
     if (signs) return cudaErrorInvalidValue;
   } else if (signs) {
-    return a32 ? launch_tc<LOGN, true, true>(x, tokens, clip, signs, q, scales, stream, stall_test)
-               : launch_tc<LOGN, true, false>(x, tokens, clip, signs, q, scales, stream, stall_test);
+    return a32 ? launch_tc<LOGN, true, true, BITS>(x, tokens, clip, signs, q, scales, stream, stall_test)
+               : launch_tc<LOGN, true, false, BITS>(x, tokens, clip, signs, q, scales, stream, stall_test);
   }
-  return a32 ? launch_tc<LOGN, false, true>(x, tokens, clip, nullptr, q, scales, stream, stall_test)
-             : launch_tc<LOGN, false, false>(x, tokens, clip, nullptr, q, scales, stream, stall_test);
+  return a32 ? launch_tc<LOGN, false, true, BITS>(x, tokens, clip, nullptr, q, scales, stream, stall_test)
+             : launch_tc<LOGN, false, false, BITS>(x, tokens, clip, nullptr, q, scales, stream, stall_test);
 }
 
 
@@ -629,7 +674,7 @@ __device__ __forceinline__ float absmax32(const uint32_t *r, float m) {
   return m;
 }
 
-template <int V, bool SIGNS, bool STORE32>
+template <int V, bool SIGNS, bool STORE32, int BITS>
 __global__ void __launch_bounds__(kThreadsS, 1)
     k1_tcs_rotate_quant(const __grid_constant__ CUtensorMap xmap, int64_t tokens, float clip, float inv_sqrt_n,
                         const uint32_t *__restrict__ signs, uint8_t *__restrict__ q, float *__restrict__ scales) {
@@ -759,7 +804,17 @@ __global__ void __launch_bounds__(kThreadsS, 1)
       tc::tc_fence_after();
       const int64_t token = p * TOKG + (V == 1 ? 128 * g : 0) + row;
       const bool live = token < tokens;
-      uint8_t *dst = q + token * (int64_t)(64 * V);
+      constexpr float QMAX = BITS == 4 ? 7.0f : 127.0f, LEVELS = 2.0f * QMAX + 1.0f;
+      uint8_t *dst = q + token * (int64_t)(16 * V * BITS);
+      // 32 code bytes at dst + off: one 32-byte store when aligned, else two 16-byte ones
+      auto put32 = [&](int off, const uint32_t *w) {
+        if constexpr (STORE32) {
+          st_v8_cs(dst + off, w);
+        } else {
+          __stcs(reinterpret_cast<uint4 *>(dst + off), make_uint4(w[0], w[1], w[2], w[3]));
+          __stcs(reinterpret_cast<uint4 *>(dst + off) + 1, make_uint4(w[4], w[5], w[6], w[7]));
+        }
+      };
       float s;
       if constexpr (V == 1) {
         uint32_t r[128];
@@ -774,26 +829,41 @@ __global__ void __launch_bounds__(kThreadsS, 1)
         float mu = 0.0f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) mu = absmax32(r + 32 * c, mu);
-        s = fmaxf(clip * (mu * inv_sqrt_n) / 7.0f, 1e-8f);
-        const float c15 = (inv_sqrt_n / 15.0f) / s;
-        uint32_t words[16];
+        s = fmaxf(clip * (mu * inv_sqrt_n) / QMAX, 1e-8f);
+        const float c15 = (inv_sqrt_n / LEVELS) / s;
+        if constexpr (BITS == 8) {
 #pragma unroll
-        for (int wi = 0; wi < 16; ++wi) {
-          float f[8];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t w8[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(r[8 * wi + k]);
-          words[wi] = codes8(f, c15);
-        }
-        if (live) {
+            for (int h = 0; h < 4; ++h) {
+              float f[8];
 #pragma unroll
-          for (int w8 = 0; w8 < 2; ++w8) {
-            if constexpr (STORE32) {
-              st_v8_cs(dst + 32 * w8, words + 8 * w8);
-            } else {
-              __stcs(reinterpret_cast<uint4 *>(dst + 32 * w8),
-                     make_uint4(words[8 * w8], words[8 * w8 + 1], words[8 * w8 + 2], words[8 * w8 + 3]));
-              __stcs(reinterpret_cast<uint4 *>(dst + 32 * w8) + 1,
-                     make_uint4(words[8 * w8 + 4], words[8 * w8 + 5], words[8 * w8 + 6], words[8 * w8 + 7]));
+              for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(r[32 * c + 8 * h + k]);
+              codes8_int8(f, c15, w8[2 * h], w8[2 * h + 1]);
+            }
+            if (live) put32(32 * c, w8);
+          }
+        } else {
+          uint32_t words[16];
+#pragma unroll
+          for (int wi = 0; wi < 16; ++wi) {
+            float f[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(r[8 * wi + k]);
+            words[wi] = codes8(f, c15);
+          }
+          if (live) {
+#pragma unroll
+            for (int w8 = 0; w8 < 2; ++w8) {
+              if constexpr (STORE32) {
+                st_v8_cs(dst + 32 * w8, words + 8 * w8);
+              } else {
+                __stcs(reinterpret_cast<uint4 *>(dst + 32 * w8),
+                       make_uint4(words[8 * w8], words[8 * w8 + 1], words[8 * w8 + 2], words[8 * w8 + 3]));
+                __stcs(reinterpret_cast<uint4 *>(dst + 32 * w8) + 1,
+                       make_uint4(words[8 * w8 + 4], words[8 * w8 + 5], words[8 * w8 + 6], words[8 * w8 + 7]));
+              }
             }
           }
         }
@@ -812,29 +882,53 @@ __global__ void __launch_bounds__(kThreadsS, 1)
             mu = fmax3(mu, fabsf(y0 + y1), fabsf(y0 - y1));
           }
         }
-        s = fmaxf(clip * (mu * inv_sqrt_n) / 7.0f, 1e-8f);
-        const float c15 = (inv_sqrt_n / 15.0f) / s;
+        s = fmaxf(clip * (mu * inv_sqrt_n) / QMAX, 1e-8f);
+        const float c15 = (inv_sqrt_n / LEVELS) / s;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {  // pass 2: codes of outputs 32c.. of both halves
-          uint32_t a[32], b[32], w0[4], w1[4];
-          tc::tmem_ld32(taddr + 32 * c, a);
-          tc::tmem_ld32(taddr + 128 + 32 * c, b);
-          tc::tmem_wait_ld();
+          uint32_t a[32], b[32];
+          if constexpr (BITS == 8) {
+            uint32_t w0[8], w1[8];
+            tc::tmem_ld32(taddr + 32 * c, a);
+            tc::tmem_ld32(taddr + 128 + 32 * c, b);
+            tc::tmem_wait_ld();
 #pragma unroll
-          for (int wi = 0; wi < 4; ++wi) {
-            float f0[8], f1[8];
+            for (int wi = 0; wi < 4; ++wi) {
+              float f0[8], f1[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const float y0 = __uint_as_float(a[8 * wi + k]), y1 = __uint_as_float(b[8 * wi + k]);
-              f0[k] = y0 + y1;
-              f1[k] = y0 - y1;
+              for (int k = 0; k < 8; ++k) {
+                const float y0 = __uint_as_float(a[8 * wi + k]), y1 = __uint_as_float(b[8 * wi + k]);
+                f0[k] = y0 + y1;
+                f1[k] = y0 - y1;
+              }
+              codes8_int8(f0, c15, w0[2 * wi], w0[2 * wi + 1]);
+              codes8_int8(f1, c15, w1[2 * wi], w1[2 * wi + 1]);
             }
-            w0[wi] = codes8(f0, c15);
-            w1[wi] = codes8(f1, c15);
-          }
-          if (live) {
-            __stcs(reinterpret_cast<uint4 *>(dst + 16 * c), make_uint4(w0[0], w0[1], w0[2], w0[3]));
-            __stcs(reinterpret_cast<uint4 *>(dst + 64 + 16 * c), make_uint4(w1[0], w1[1], w1[2], w1[3]));
+            if (live) {
+              put32(32 * c, w0);
+              put32(128 + 32 * c, w1);
+            }
+          } else {
+            uint32_t w0[4], w1[4];
+            tc::tmem_ld32(taddr + 32 * c, a);
+            tc::tmem_ld32(taddr + 128 + 32 * c, b);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int wi = 0; wi < 4; ++wi) {
+              float f0[8], f1[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const float y0 = __uint_as_float(a[8 * wi + k]), y1 = __uint_as_float(b[8 * wi + k]);
+                f0[k] = y0 + y1;
+                f1[k] = y0 - y1;
+              }
+              w0[wi] = codes8(f0, c15);
+              w1[wi] = codes8(f1, c15);
+            }
+            if (live) {
+              __stcs(reinterpret_cast<uint4 *>(dst + 16 * c), make_uint4(w0[0], w0[1], w0[2], w0[3]));
+              __stcs(reinterpret_cast<uint4 *>(dst + 64 + 16 * c), make_uint4(w1[0], w1[1], w1[2], w1[3]));
+            }
           }
         }
         tc::tc_fence_before();
@@ -857,7 +951,7 @@ __global__ void __launch_bounds__(kThreadsS, 1)
   }
 }
 
-template <int V, bool SIGNS, bool STORE32>
+template <int V, bool SIGNS, bool STORE32, int BITS>
 cudaError_t launch_tcs(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
                        cudaStream_t stream) {
   auto fn = tensor_map_encoder();
@@ -871,7 +965,7 @@ cudaError_t launch_tcs(const void *x, int64_t tokens, float clip, const uint32_t
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto kern = k1_tcs_rotate_quant<V, SIGNS, STORE32>;
+  auto kern = k1_tcs_rotate_quant<V, SIGNS, STORE32, BITS>;
   constexpr uint32_t smem_bytes = SmallLayout<(SIGNS && V == 2) ? 2 : 1>::kSmemBytes;
   int slots = 0;
   cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreadsS, (int)smem_bytes, &slots);
@@ -892,15 +986,17 @@ cudaError_t launch_tcs(const void *x, int64_t tokens, float clip, const uint32_t
   return cudaLaunchKernelEx(&cfg, kern, map, tokens, clip, inv_sqrt_n, signs, q, scales);
 }
 
-template <int V>
+template <int V, int BITS>
 cudaError_t launch_small(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
                          cudaStream_t stream) {
-  const bool a32 = V == 1 && (reinterpret_cast<uintptr_t>(q) & 31u) == 0;  // n = 256 stores 16 B pieces
+  // 32-byte stores need 32-byte alignment; INT4 at n = 256 stores 16-byte pieces
+  constexpr bool W = V == 1 || BITS == 8;
+  const bool a32 = W && (reinterpret_cast<uintptr_t>(q) & 31u) == 0;
   if (signs)
-    return a32 ? launch_tcs<V, true, V == 1>(x, tokens, clip, signs, q, scales, stream)
-               : launch_tcs<V, true, false>(x, tokens, clip, signs, q, scales, stream);
-  return a32 ? launch_tcs<V, false, V == 1>(x, tokens, clip, nullptr, q, scales, stream)
-             : launch_tcs<V, false, false>(x, tokens, clip, nullptr, q, scales, stream);
+    return a32 ? launch_tcs<V, true, W, BITS>(x, tokens, clip, signs, q, scales, stream)
+               : launch_tcs<V, true, false, BITS>(x, tokens, clip, signs, q, scales, stream);
+  return a32 ? launch_tcs<V, false, W, BITS>(x, tokens, clip, nullptr, q, scales, stream)
+             : launch_tcs<V, false, false, BITS>(x, tokens, clip, nullptr, q, scales, stream);
 }
 
 std::atomic<int> g_stall_test{0};
@@ -938,18 +1034,26 @@ bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags, bool h
   return (flags & kTensorCores) || tokens >= 128 * tok_per_group;
 }
 
-cudaError_t launch_rotate_quant_int4_tc(int log_n, const void *x, int64_t tokens, float clip, const uint32_t *signs,
-                                        uint8_t *q, float *scales, cudaStream_t stream) {
-  const int stall = g_stall_test.load(std::memory_order_relaxed);
+template <int BITS>
+cudaError_t launch_tc_bits(int log_n, const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q,
+                           float *scales, cudaStream_t stream, int stall) {
   switch (log_n) {
-    case 7: return launch_small<1>(x, tokens, clip, signs, q, scales, stream);
-    case 8: return launch_small<2>(x, tokens, clip, signs, q, scales, stream);
-    case 12: return launch_n<12>(x, tokens, clip, signs, q, scales, stream, stall);
-    case 13: return launch_n<13>(x, tokens, clip, signs, q, scales, stream, stall);
-    case 14: return launch_n<14>(x, tokens, clip, signs, q, scales, stream, stall);
-    case 15: return launch_n<15>(x, tokens, clip, signs, q, scales, stream, stall);
+    case 7: return launch_small<1, BITS>(x, tokens, clip, signs, q, scales, stream);
+    case 8: return launch_small<2, BITS>(x, tokens, clip, signs, q, scales, stream);
+    case 12: return launch_n<12, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
+    case 13: return launch_n<13, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
+    case 14: return launch_n<14, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
+    case 15: return launch_n<15, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_rotate_quant_tc(int log_n, int bits, const void *x, int64_t tokens, float clip,
+                                   const uint32_t *signs, uint8_t *q, float *scales, cudaStream_t stream) {
+  const int stall = g_stall_test.load(std::memory_order_relaxed);
+  if (bits == 4) return launch_tc_bits<4>(log_n, x, tokens, clip, signs, q, scales, stream, stall);
+  if (bits == 8) return launch_tc_bits<8>(log_n, x, tokens, clip, signs, q, scales, stream, stall);
+  return cudaErrorInvalidValue;
 }
 
 void set_stall_test(int enable) { g_stall_test.store(enable ? 1 : 0, std::memory_order_relaxed); }

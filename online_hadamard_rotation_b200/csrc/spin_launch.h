@@ -21,15 +21,15 @@ cudaError_t resident_slots(const void *kernel, int threads, int dyn_smem, int *s
 // cuTensorMapEncodeTiled from the driver (null if unavailable), looked up once.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
-cudaError_t launch_rotate_quant_int4(const void *x, int64_t tokens, int log_n, float clip,
-                                     const uint32_t *signs, uint32_t flags, uint8_t *q, float *scales,
-                                     cudaStream_t stream);
+// R4 with per-token codes of `bits` = 4 (two per byte) or 8 (one signed byte each).
+cudaError_t launch_rotate_quant(const void *x, int64_t tokens, int log_n, float clip, const uint32_t *signs,
+                                uint32_t flags, int bits, uint8_t *q, float *scales, cudaStream_t stream);
 
-// Tensor-core R4 kernel (n = 4096 to 32768; n = 32768 without a sign diagonal):
-// availability and launcher.
+// Tensor-core R4 kernels (n = 128, 256 and 4096 to 32768; n = 32768 without a
+// sign diagonal): availability and launcher.
 bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags, bool has_signs);
-cudaError_t launch_rotate_quant_int4_tc(int log_n, const void *x, int64_t tokens, float clip, const uint32_t *signs,
-                                        uint8_t *q, float *scales, cudaStream_t stream);
+cudaError_t launch_rotate_quant_tc(int log_n, int bits, const void *x, int64_t tokens, float clip,
+                                   const uint32_t *signs, uint8_t *q, float *scales, cudaStream_t stream);
 
 // Test hook: make the tensor-core R4 kernel withhold one internal signal.
 void set_stall_test(int enable);

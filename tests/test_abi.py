@@ -18,8 +18,9 @@ def L():
 
 def test_header_declares_the_entry_points():
     names = spin.exported_symbols()
-    for fn in ("spin_hadamard_quant_int4", "spin_hadamard_quant_int4_ex", "spin_rope_hadamard_kvquant",
-               "spin_dequant_hadamard_inverse", "spin_status_string", "spin_last_cuda_error", "spin_version"):
+    for fn in ("spin_hadamard_quant_int4", "spin_hadamard_quant_int4_ex", "spin_hadamard_quant_int8",
+               "spin_rope_hadamard_kvquant", "spin_dequant_hadamard_inverse", "spin_status_string",
+               "spin_last_cuda_error", "spin_version"):
         assert fn in names
 
 
@@ -50,6 +51,17 @@ def test_r4_rejects_sizes(L, n):
 @pytest.mark.parametrize("clip", [0.0, -0.5, 1.5, float("nan")])
 def test_r4_rejects_clip(L, clip):
     assert L.spin_hadamard_quant_int4(FAKE, 4, 256, clip, FAKE, FAKE, None) == 1
+
+
+@pytest.mark.parametrize("n", [0, 64, 100, 65536])
+def test_r4_int8_rejects_sizes_and_arguments(L, n):
+    assert L.spin_hadamard_quant_int8(FAKE, 4, n, 1.0, None, 0, FAKE, FAKE, None) == 2
+    assert L.spin_hadamard_quant_int8(FAKE, 4, 256, 1.5, None, 0, FAKE, FAKE, None) == 1
+    assert L.spin_hadamard_quant_int8(FAKE, 4, 256, 1.0, None, 6, FAKE, FAKE, None) == 1  # both kernel bits
+    assert L.spin_hadamard_quant_int8(FAKE, 4, 256, 1.0, None, 8, FAKE, FAKE, None) == 1  # unknown bit
+    assert L.spin_hadamard_quant_int8(None, 0, 256, 1.0, None, 0, None, None, None) == 0  # empty: no-op
+    assert L.spin_hadamard_quant_int8(FAKE, 4, 256, 1.0, None, 0, None, FAKE, None) == 1
+    assert L.spin_hadamard_quant_int8(FAKE, 4, 256, 1.0, None, 0, FAKE + 4, FAKE, None) == 3
 
 
 def test_r4_argument_checks(L):
