@@ -61,12 +61,12 @@ def oracle_r4_rows(oracle, bits, clip, signs, code_bits):
 
 def r4_kernel_name(n: int, tokens: int, has_signs: bool) -> str:
     """The R4 kernel the library's dispatch picks by default: a tensor-core one for
-    n = 128, 256 and 4096 .. 32768 (n = 32768 without a sign diagonal) once the batch
+    n = 128, 256 and 2048 .. 32768 (n = 32768 without a sign diagonal) once the batch
     has at least 128 MMA groups, else the CUDA-core one."""
     log_n = n.bit_length() - 1
     if log_n in (7, 8) and tokens >= 128 * (256 >> (log_n - 7)):
         return "k1_tcs_rotate_quant"
-    if 12 <= log_n <= 15 and not (log_n == 15 and has_signs):
+    if 11 <= log_n <= 15 and not (log_n == 15 and has_signs):
         tokens_per_group = 1 if log_n == 15 else 256 >> (log_n - 7)
         if tokens >= 128 * tokens_per_group:
             return "k1_tc_rotate_quant"

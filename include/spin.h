@@ -113,7 +113,7 @@ spin_status_t spin_hadamard_quant_int4(const void *x_bf16, int64_t tokens, int32
  *             SPIN_NO_ROTATE: quantise x directly (no D, no H), used to
  *               measure the direct-quantisation error;
  *             SPIN_CUDA_CORES_ONLY: at n = 128 and 256 the transform, and at
- *               n = 4096, 8192 and 16384, and at n = 32768 without sign_bits,
+ *               n = 2048 … 16384, and at n = 32768 without sign_bits,
  *               the first H_128 Kronecker factor (two of them at n = 32768),
  *               normally runs on the tensor cores (exact +-1 x bf16 products,
  *               fp32 accumulation; at n = 128 and 256 the diagonal rides in the

@@ -1,5 +1,6 @@
-// k1_tc.cu -- R4 for n = 4096 to 32768 with the first Kronecker factor on the
-// tensor cores.
+// k1_tc.cu -- R4 on the tensor cores: for n = 2048 to 32768 the first Kronecker
+// factor runs on tcgen05 (below); for n = 128 and 256 the whole transform does
+// (tokens as the MMA's M, further down).
 //
 // "Rotations: QuaRot, SpinQuant and incoherence", section "Hadamard matrices":
 // the Sylvester H_n is a Kronecker product of smaller Sylvester matrices, and
@@ -9,8 +10,8 @@
 // Outlier Curse": symmetric INT4, step max|y| / 7.
 //
 // A token row x of n = 128 B bf16 values is the 128 x B matrix X[a][b], with
-// element index e = B a + b (B = 32, 64, 128; n = 32768 is two such blocks, see
-// Shape). Then H_n x = vec(H_128 X H_B):
+// element index e = B a + b (B = 16, 32, 64, 128; n = 32768 is two such blocks,
+// see Shape). Then H_n x = vec(H_128 X H_B):
 //   1. tcgen05.mma computes Y = H_128 X (contraction over a) for 256 / B tokens
 //      at once (M = 128, N = 256, K = 128, bf16 in, fp32 accumulate in TMEM).
 //      H is exactly +-1 and X is exactly bf16, so every product is exact and
@@ -27,7 +28,7 @@
 // SMs and the last groups land wherever an SM is free.
 // Roles (384 threads, one CTA per SM, persistent over groups):
 //   warp 0      TMA producer: 64 KiB per group (boxes of [128 rows][min(B, 64)]
-//               bf16 with 64- or 128-byte swizzle) into a three-stage ring
+//               bf16 with 32-, 64- or 128-byte swizzle) into a three-stage ring
 //   warp 1      TMEM owner and MMA issuer (8 MMAs of K = 16 per group)
 //   warps 2-3   +-1 diagonal: XOR of the bf16 sign bits in shared memory, with
 //               each thread's sign words held in registers
@@ -90,11 +91,11 @@ struct Shape {
   static constexpr int BPT = CBOX * ROWS / 128;     // boxes per token
   static constexpr uint32_t BOXBYTES = 128u * ROWB; // bytes per box
   static constexpr int CPR = ROWB / 16;             // 16-byte chunks per tile row
-  static constexpr uint32_t LAYOUT = ROWB == 128 ? 2u : 4u;  // UMMA swizzle: 128 B or 64 B
+  static constexpr uint32_t LAYOUT = ROWB == 128 ? 2u : ROWB == 64 ? 4u : 6u;  // UMMA swizzle: 128, 64, 32 B
   static constexpr uint32_t TOKBYTES = kGroupBytes / TOK;
   static constexpr int NPOS = (int)(TOKBYTES / 16 / 64);  // sign positions per sign thread
   static constexpr int64_t OUTB = (int64_t(1) << LOGN) / 2;  // code bytes per token
-  static_assert(LOGN >= 12 && LOGN <= 15, "tensor-core R4 covers n = 4096 .. 32768");
+  static_assert(LOGN >= 11 && LOGN <= 15, "this tensor-core R4 kernel covers n = 2048 .. 32768");
 };
 
 constexpr int kRing = 8;  // group ids in flight between the producer and the epilogue
@@ -109,7 +110,7 @@ struct Shared {
   int abort;
   int dec[3];
   long long budget;        // clock cycles a wait may take before the CTA gives up
-  float wmax[2][2][4][4];  // [warpgroup][group parity][warp][token segment]
+  float wmax[2][2][4][8];  // [warpgroup][group parity][warp][token segment]
 };
 static_assert(sizeof(Shared) <= 1024, "barrier area");
 
@@ -394,7 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t pos = ts + 64u * k;  // 16-byte chunk index inside one token's tile
           const uint32_t box = pos / (SH::BOXBYTES / 16), inbox = pos % (SH::BOXBYTES / 16);
           const uint32_t a = inbox / SH::CPR, pc = inbox % SH::CPR;
-          const uint32_t ch = SH::ROWB == 128 ? (pc ^ (a & 7u)) : (pc ^ ((a >> 1) & 3u));
+          const uint32_t ch = SH::ROWB == 128 ? (pc ^ (a & 7u))
+                              : SH::ROWB == 64 ? (pc ^ ((a >> 1) & 3u))
+                                               : (pc ^ ((a >> 2) & 1u));
           const uint32_t e = a * B + box * SH::BOXW + ch * 8u;
           const uint32_t byte = (__ldg(signs + (e >> 5)) >> (e & 31u)) & 0xFFu;
           uint32_t w[4];
@@ -478,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       stage<1>(v);
       stage<2>(v);
       stage<3>(v);
-      stage<4>(v);
+      if constexpr (SH::LOGB > 4) stage<4>(v);
       if constexpr (SH::LOGB > 5) stage<5>(v);
       if constexpr (SH::LOGB > 6) stage<6>(v);
       // per-token max |u|: a tree of three-input maxima per segment, then the warp, then the warpgroup
@@ -514,7 +517,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (token >= tokens) continue;
         const uint32_t orow = SH::SPLIT ? 128u * g + row : row;  // output row of B values
         uint8_t *dst = q + token * (SH::OUTB * (BITS / 4)) + orow * (B * BITS / 8);
-        if constexpr (BITS == 8) {
+        if constexpr (BITS == 8 && B == 16) {  // 16 code bytes per row segment
+          uint32_t w4[4];
+          codes8_int8(v + sg * B, c15, w4[0], w4[1]);
+          codes8_int8(v + sg * B + 8, c15, w4[2], w4[3]);
+          __stcs(reinterpret_cast<uint4 *>(dst), make_uint4(w4[0], w4[1], w4[2], w4[3]));
+        } else if constexpr (BITS == 8) {
           // one code byte per value: 32 bytes (8 words) at a time
 #pragma unroll
           for (int c8 = 0; c8 < B / 32; ++c8) {
@@ -540,7 +548,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0; k < 8; k += 2) round15_x2(t[k], t[k + 1], b[k], b[k + 1]);
             words[wi] = pack8(b);
           }
-          if constexpr (STORE32 && B >= 64) {
+          if constexpr (B == 16) {  // 8 code bytes per row segment
+            __stcs(reinterpret_cast<uint2 *>(dst), make_uint2(words[0], words[1]));
+          } else if constexpr (STORE32 && B >= 64) {
 #pragma unroll
             for (int w8 = 0; w8 < B / 64; ++w8) st_v8_cs(dst + 32 * w8, words + 8 * w8);
           } else {
@@ -582,7 +592,9 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  SH::ROWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  SH::ROWB == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                  : SH::ROWB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                   : CU_TENSOR_MAP_SWIZZLE_32B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   auto kern = k1_tc_rotate_quant<LOGN, SIGNS, STORE32, BITS>;
@@ -1026,7 +1038,7 @@ bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags, bool h
     const int64_t tok_per_group = log_n == 7 ? 256 : 128;
     return (flags & kTensorCores) || tokens >= 128 * tok_per_group;
   }
-  if (log_n < 12 || log_n > 15) return false;
+  if (log_n < 11 || log_n > 15) return false;
   if (log_n == 15 && has_signs) return false;  // its sign masks do not fit the sign warps' registers
   const int64_t rows_per_token = log_n == 15 ? 256 : 128;
   if (tokens * rows_per_token >= (int64_t(1) << 31)) return false;
@@ -1040,6 +1052,7 @@ cudaError_t launch_tc_bits(int log_n, const void *x, int64_t tokens, float clip,
   switch (log_n) {
     case 7: return launch_small<1, BITS>(x, tokens, clip, signs, q, scales, stream);
     case 8: return launch_small<2, BITS>(x, tokens, clip, signs, q, scales, stream);
+    case 11: return launch_n<11, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
     case 12: return launch_n<12, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
     case 13: return launch_n<13, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
     case 14: return launch_n<14, BITS>(x, tokens, clip, signs, q, scales, stream, stall);

@@ -1,6 +1,6 @@
 """R4 with per-token INT8 codes (spin_hadamard_quant_int8) vs the fp64 oracle:
 every supported n, on the CUDA-core kernel and on the tensor-core kernels
-(n = 128, 256 and 4096 .. 32768; n = 32768 without a diagonal), ragged token
+(n = 128, 256 and 2048 .. 32768; n = 32768 without a diagonal), ragged token
 counts, clip 1.0 / 0.9, with and without the +-1 diagonal, direct quantisation,
 special rows, and more MMA groups than resident blocks."""
 import numpy as np
@@ -14,7 +14,7 @@ from tests.gpu_util import to_dev_bf16, to_dev_signs
 pytestmark = pytest.mark.gpu
 
 VARIANTS = {"plain": (1.0, False, False), "clip_signs": (0.9, True, False), "direct": (1.0, False, True)}
-TC_SIZES = (128, 256, 4096, 8192, 16384, 32768)
+TC_SIZES = (128, 256, 2048, 4096, 8192, 16384, 32768)
 
 
 def run(spin, bits, clip, signs, direct=False, path="default"):
