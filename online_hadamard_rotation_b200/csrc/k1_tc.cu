@@ -367,95 +367,95 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
         } else {
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {
-              // A: 16 columns k of H per step. B: rows a = 16 s .. 16 s + 15 of every box
-              // (MN-major: boxes of BOXW columns BOXBYTES apart, 8-row groups 8 ROWB apart).
-              const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-              uint64_t bd = tc::smem_desc(sX + st * kGroupBytes + s * 16 * SH::ROWB, SH::BOXBYTES, 8 * SH::ROWB);
-              bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
-              tc::umma_bf16(tmem + acc * 256, ad, bd, idesc, s > 0 ? 1u : 0u);
-            }
+          for (int s = 0; s < 8; ++s) {
+            // A: 16 columns k of H per step. B: rows a = 16 s .. 16 s + 15 of every box
+            // (MN-major: boxes of BOXW columns BOXBYTES apart, 8-row groups 8 ROWB apart).
+            const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
+            uint64_t bd = tc::smem_desc(sX + st * kGroupBytes + s * 16 * SH::ROWB, SH::BOXBYTES, 8 * SH::ROWB);
+            bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
+            tc::umma_bf16(tmem + acc * 256, ad, bd, idesc, s > 0 ? 1u : 0u);
           }
-          tc::umma_commit(&S.empty[st]);
-          // Stall test hook: withhold the first group's completion signal, so the
-          // epilogue's wait runs out and the CTA takes its abort path.
-          if (!(stall_test && i == 0)) tc::umma_commit(&S.tfull[acc]);
         }
+        tc::umma_commit(&S.empty[st]);
+        // Stall test hook: withhold the first group's completion signal, so the
+        // epilogue's wait runs out and the CTA takes its abort path.
+        if (!(stall_test && i == 0)) tc::umma_commit(&S.tfull[acc]);
       }
-    } else if (warp < 4) {
-      if constexpr (SIGNS) {
-        // Thread ts flips the signs of chunks ts + 64 j of each group's 64 KiB.
-        // Those chunks sit at NPOS distinct positions of a token's tile; their
-        // sign words stay in registers for the whole kernel.
-        constexpr int NPOS = SH::NPOS;
-        const uint32_t ts = threadIdx.x - 64;  // 0..63
-        uint4 mk[NPOS];
+    }
+  } else if (warp < 4) {
+    if constexpr (SIGNS) {
+      // Thread ts flips the signs of chunks ts + 64 j of each group's 64 KiB.
+      // Those chunks sit at NPOS distinct positions of a token's tile; their
+      // sign words stay in registers for the whole kernel.
+      constexpr int NPOS = SH::NPOS;
+      const uint32_t ts = threadIdx.x - 64;  // 0..63
+      uint4 mk[NPOS];
 #pragma unroll
-        for (int k = 0; k < NPOS; ++k) {
-          const uint32_t pos = ts + 64u * k;  // 16-byte chunk index inside one token's tile
-          const uint32_t box = pos / (SH::BOXBYTES / 16), inbox = pos % (SH::BOXBYTES / 16);
-          const uint32_t a = inbox / SH::CPR, pc = inbox % SH::CPR;
-          const uint32_t ch = SH::ROWB == 128 ? (pc ^ (a & 7u))
-                              : SH::ROWB == 64 ? (pc ^ ((a >> 1) & 3u))
-                                               : (pc ^ ((a >> 2) & 1u));
-          const uint32_t e = a * B + box * SH::BOXW + ch * 8u;
-          const uint32_t byte = (__ldg(signs + (e >> 5)) >> (e & 31u)) & 0xFFu;
-          uint32_t w[4];
+      for (int k = 0; k < NPOS; ++k) {
+        const uint32_t pos = ts + 64u * k;  // 16-byte chunk index inside one token's tile
+        const uint32_t box = pos / (SH::BOXBYTES / 16), inbox = pos % (SH::BOXBYTES / 16);
+        const uint32_t a = inbox / SH::CPR, pc = inbox % SH::CPR;
+        const uint32_t ch = SH::ROWB == 128 ? (pc ^ (a & 7u))
+                            : SH::ROWB == 64 ? (pc ^ ((a >> 1) & 3u))
+                                             : (pc ^ ((a >> 2) & 1u));
+        const uint32_t e = a * B + box * SH::BOXW + ch * 8u;
+        const uint32_t byte = (__ldg(signs + (e >> 5)) >> (e & 31u)) & 0xFFu;
+        uint32_t w[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) w[j] = (((byte >> (2 * j)) & 1u) << 15) | (((byte >> (2 * j + 1)) & 1u) << 31);
-          mk[k] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        for (int64_t i = 0;; ++i) {
-          const int st = (int)(i % kStages);
-          if (ts == 0) {
-            int ok = wait_bounded(&S.full[st], (uint32_t)((i / kStages) & 1), S, true) ? 1 : 0;
-            if (ok && S.gid[i % kRing] < 0) {
-              tc::mbar_arrive(&S.sgn[st]);  // pass the end mark on to the MMA
-              ok = 0;
-            }
-            S.dec[2] = ok;
-          }
-          tc::named_sync(3, 64);
-          if (!S.dec[2]) break;
-          uint4 *X = reinterpret_cast<uint4 *>(smem + kOffX + st * kGroupBytes) + ts;
-#pragma unroll
-          for (int j0 = 0; j0 < 64; j0 += 4) {
-            uint4 x[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) x[u] = X[64 * (j0 + u)];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const uint4 m = mk[(j0 + u) % NPOS];
-              X[64 * (j0 + u)] = make_uint4(x[u].x ^ m.x, x[u].y ^ m.y, x[u].z ^ m.z, x[u].w ^ m.w);
-            }
-          }
-          tc::fence_proxy_async_smem();
-          tc::named_sync(3, 64);
-          if (ts == 0) tc::mbar_arrive(&S.sgn[st]);
-        }
+        for (int j = 0; j < 4; ++j) w[j] = (((byte >> (2 * j)) & 1u) << 15) | (((byte >> (2 * j + 1)) & 1u) << 31);
+        mk[k] = make_uint4(w[0], w[1], w[2], w[3]);
       }
-    } else {
-      // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1)
-      const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
-      const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
       for (int64_t i = 0;; ++i) {
-        const int acc = (int)(i & 1);
-        // the step's group from the producer's ring, then its accumulator
-        auto decide = [&](int slot) {
-          int ok = wait_bounded(&S.gfull[i % kRing], (uint32_t)((i / kRing) & 1), S, true) ? 1 : 0;
-          const int64_t gp = ok ? S.gid[i % kRing] : -1;
-          if (gp < 0) ok = 0;
-          if (ok) ok = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
-          S.egid[slot] = gp;
-          S.dec[slot] = ok;
-        };
-        int64_t p;
-        if constexpr (SH::SPLIT) {  // one decision for both warpgroups: they meet at barrier 4 below
-          if (threadIdx.x == 128) decide(0);
-          tc::named_sync(4, 256);
-          if (!S.dec[0]) break;
-          p = S.egid[0];
-        } else {
+        const int st = (int)(i % kStages);
+        if (ts == 0) {
+          int ok = wait_bounded(&S.full[st], (uint32_t)((i / kStages) & 1), S, true) ? 1 : 0;
+          if (ok && S.gid[i % kRing] < 0) {
+            tc::mbar_arrive(&S.sgn[st]);  // pass the end mark on to the MMA
+            ok = 0;
+          }
+          S.dec[2] = ok;
+        }
+        tc::named_sync(3, 64);
+        if (!S.dec[2]) break;
+        uint4 *X = reinterpret_cast<uint4 *>(smem + kOffX + st * kGroupBytes) + ts;
+#pragma unroll
+        for (int j0 = 0; j0 < 64; j0 += 4) {
+          uint4 x[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) x[u] = X[64 * (j0 + u)];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint4 m = mk[(j0 + u) % NPOS];
+            X[64 * (j0 + u)] = make_uint4(x[u].x ^ m.x, x[u].y ^ m.y, x[u].z ^ m.z, x[u].w ^ m.w);
+          }
+        }
+        tc::fence_proxy_async_smem();
+        tc::named_sync(3, 64);
+        if (ts == 0) tc::mbar_arrive(&S.sgn[st]);
+      }
+    }
+  } else {
+    // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1)
+    const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
+    const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
+    for (int64_t i = 0;; ++i) {
+      const int acc = (int)(i & 1);
+      // the step's group from the producer's ring, then its accumulator
+      auto decide = [&](int slot) {
+        int ok = wait_bounded(&S.gfull[i % kRing], (uint32_t)((i / kRing) & 1), S, true) ? 1 : 0;
+        const int64_t gp = ok ? S.gid[i % kRing] : -1;
+        if (gp < 0) ok = 0;
+        if (ok) ok = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
+        S.egid[slot] = gp;
+        S.dec[slot] = ok;
+      };
+      int64_t p;
+      if constexpr (SH::SPLIT) {  // one decision for both warpgroups: they meet at barrier 4 below
+        if (threadIdx.x == 128) decide(0);
+        tc::named_sync(4, 256);
+        if (!S.dec[0]) break;
+        p = S.egid[0];
+      } else {
         if (tg == 0) decide(g);
         tc::named_sync(1 + g, 128);
         if (!S.dec[g]) break;
