@@ -1013,6 +1013,21 @@ cudaError_t launch_small(const void *x, int64_t tokens, float clip, const uint32
 
 std::atomic<int> g_stall_test{0};
 
+template <int BITS>
+cudaError_t launch_tc_bits(int log_n, const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q,
+                           float *scales, cudaStream_t stream, int stall) {
+  switch (log_n) {
+    case 7: return launch_small<1, BITS>(x, tokens, clip, signs, q, scales, stream);
+    case 8: return launch_small<2, BITS>(x, tokens, clip, signs, q, scales, stream);
+    case 11: return launch_n<11, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
+    case 12: return launch_n<12, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
+    case 13: return launch_n<13, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
+    case 14: return launch_n<14, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
+    case 15: return launch_n<15, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 }  // namespace
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -1044,21 +1059,6 @@ bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags, bool h
   if (tokens * rows_per_token >= (int64_t(1) << 31)) return false;
   const int64_t tok_per_group = log_n == 15 ? 1 : int64_t(256) >> (log_n - 7);
   return (flags & kTensorCores) || tokens >= 128 * tok_per_group;
-}
-
-template <int BITS>
-cudaError_t launch_tc_bits(int log_n, const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q,
-                           float *scales, cudaStream_t stream, int stall) {
-  switch (log_n) {
-    case 7: return launch_small<1, BITS>(x, tokens, clip, signs, q, scales, stream);
-    case 8: return launch_small<2, BITS>(x, tokens, clip, signs, q, scales, stream);
-    case 11: return launch_n<11, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
-    case 12: return launch_n<12, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
-    case 13: return launch_n<13, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
-    case 14: return launch_n<14, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
-    case 15: return launch_n<15, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
-    default: return cudaErrorInvalidValue;
-  }
 }
 
 cudaError_t launch_rotate_quant_tc(int log_n, int bits, const void *x, int64_t tokens, float clip,

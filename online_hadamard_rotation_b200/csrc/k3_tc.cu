@@ -44,6 +44,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <type_traits>
 
 #include "spin_launch.h"
 #include "spin_tile.cuh"
@@ -855,12 +856,16 @@ template <int V>
 cudaError_t launch_small(const uint8_t *codes, int64_t rows, const void *scale, const void *zero,
                          const uint32_t *signs, void *out, bool asym, bool f32, cudaStream_t stream) {
   const bool a32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;  // 32-byte stores need 32-byte alignment
-#define SPIN_TCS(S_, F_) \
-  (a32 ? launch_tcs<V, S_, F_, true>(codes, rows, scale, zero, signs, out, asym, stream) \
-       : launch_tcs<V, S_, F_, false>(codes, rows, scale, zero, signs, out, asym, stream))
-  if (signs) return f32 ? SPIN_TCS(true, true) : SPIN_TCS(true, false);
-  return f32 ? SPIN_TCS(false, true) : SPIN_TCS(false, false);
-#undef SPIN_TCS
+  auto go = [&](auto sg, auto fp) {  // sg, fp: std::integral_constant<bool, ...>
+    return a32 ? launch_tcs<V, decltype(sg)::value, decltype(fp)::value, true>(codes, rows, scale, zero, signs, out,
+                                                                             asym, stream)
+               : launch_tcs<V, decltype(sg)::value, decltype(fp)::value, false>(codes, rows, scale, zero, signs, out,
+                                                                              asym, stream);
+  };
+  using T = std::true_type;
+  using F = std::false_type;
+  if (signs) return f32 ? go(T{}, T{}) : go(T{}, F{});
+  return f32 ? go(F{}, T{}) : go(F{}, F{});
 }
 
 }  // namespace
