@@ -219,7 +219,8 @@ def make_workload(name: str, rank: int, tokens: int | None = None):
         k = int(name[len("sweep"):])
         bits = synthetic.sweep(k, tokens=tokens, seed=4 + k + 100 * rank)
         return dict(kind="r4", bits=bits, signs=None, clip=1.0, code_bits=4,
-                    desc={"workload": f"sweep: n=2^{k}, 1 GiB bf16 input, N(0,1) with 0.1% channels x100, clip 1.0",
+                    desc={"workload": f"sweep: n=2^{k}, {'1 GiB' if tokens is None else f'{bits.nbytes >> 20} MiB'} "
+                                      "bf16 input, N(0,1) with 0.1% channels x100, clip 1.0",
                           "tokens": int(bits.shape[0]), "n": 1 << k})
     if name == "r3_kv":
         q, k, v, pos = synthetic.r3_kv(seed=2 + rank)
@@ -282,6 +283,8 @@ def main():
     ap.add_argument("--impl", default="spin", choices=["spin", "reference"])
     ap.add_argument("--workload", default="r4_prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count (R4 workloads; smaller cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -293,7 +296,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        run_reference(args, make_workload(args.workload, 0))
+        run_reference(args, make_workload(args.workload, 0, args.tokens))
         return
 
     import torch
@@ -310,7 +313,7 @@ def main():
     build.build()
     spin.lib()
 
-    wl = make_workload(args.workload, rank)
+    wl = make_workload(args.workload, rank, args.tokens)
     stream = torch.cuda.Stream(dev)
     if wl["kind"] == "r4":
         bits, n = wl["bits"], wl["bits"].shape[1]
