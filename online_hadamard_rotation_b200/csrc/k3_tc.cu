@@ -718,12 +718,8 @@ __global__ void __launch_bounds__(kThreadsS, 1)
       tc::mbar_arrive(&S.afull[as]);
     }
   } else {
-    const uint32_t tg = threadIdx.x - 192;
     const uint32_t row = (warp & 3u) * 32 + lane;
     const uint32_t lane_base = tmem + (((warp & 3u) * 32u) << 16);
-    uint32_t sw[N / 32];  // the diagonal's sign words, the same for every row
-#pragma unroll
-    for (int k = 0; k < N / 32; ++k) sw[k] = SIGNS ? __ldg(signs + k) : 0u;
     // a row's step (fp32; or fp16 step | fp16 zero << 16), loaded one group ahead
     auto load_step = [&](int64_t pp) -> uint32_t {
       const int64_t token = pp * 128 + row;
@@ -739,9 +735,8 @@ __global__ void __launch_bounds__(kThreadsS, 1)
       const uint32_t step_raw = step_next;
       step_next = load_step(p + gridDim.x);
       const int acc = (int)(i & 1);
-      if (tg == 0) S.dec[1] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
-      tc::named_sync(2, 128);
-      if (!S.dec[1]) break;
+      // every epilogue thread sleeps on the accumulator's barrier itself (no meeting point)
+      if (!wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true)) break;
       tc::tc_fence_after();
       const int64_t token = p * 128 + row;
       const bool live = token < rows;
@@ -751,66 +746,79 @@ __global__ void __launch_bounds__(kThreadsS, 1)
       const float m = s * inv_sqrt_n;
       const uint32_t taddr = lane_base + (uint32_t)acc * (128u * V);
       const int64_t off = token * (int64_t)N;
-      // 32 outputs (elements e0 ..) of this row: scale, sign, store
-      auto emit = [&](float (&o)[32], int e0) {
+      // 32 outputs (elements e0 .., fp32 bit patterns in w, updated in place): scale,
+      // sign, store
+      auto emit = [&](uint32_t *w, int e0) {
 #pragma unroll
-        for (int k = 0; k < 32; k += 2) mul2(o[k], o[k + 1], m);
-        if constexpr (SIGNS) {
-          const uint32_t sb = sw[e0 >> 5];
+        for (int k = 0; k < 32; k += 2) {
+          float x0 = __uint_as_float(w[k]), x1 = __uint_as_float(w[k + 1]);
+          mul2(x0, x1, m);
+          w[k] = __float_as_uint(x0);
+          w[k + 1] = __float_as_uint(x1);
+        }
+        if constexpr (SIGNS) {  // the diagonal's sign word of these 32 elements (the same for every row)
+          const uint32_t sb = __ldg(signs + (e0 >> 5));
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __uint_as_float(__float_as_uint(o[k]) ^ (((sb >> k) & 1u) << 31));
+          for (int k = 0; k < 32; ++k) w[k] ^= ((sb >> k) & 1u) << 31;
         }
         if (!live) return;
         if constexpr (F32) {
           float *dst = static_cast<float *>(out) + off + e0;
 #pragma unroll
           for (int k = 0; k < 32; k += 8)
-            store8<STORE32>(dst + k, __float_as_uint(o[k]), __float_as_uint(o[k + 1]), __float_as_uint(o[k + 2]),
-                            __float_as_uint(o[k + 3]), __float_as_uint(o[k + 4]), __float_as_uint(o[k + 5]),
-                            __float_as_uint(o[k + 6]), __float_as_uint(o[k + 7]));
+            store8<STORE32>(dst + k, w[k], w[k + 1], w[k + 2], w[k + 3], w[k + 4], w[k + 5], w[k + 6], w[k + 7]);
         } else {
+          auto f = [&](int k) { return __uint_as_float(w[k]); };
           uint16_t *dst = static_cast<uint16_t *>(out) + off + e0;
 #pragma unroll
           for (int k = 0; k < 32; k += 16)
-            store8<STORE32>(dst + k, pack_bf16x2(o[k], o[k + 1]), pack_bf16x2(o[k + 2], o[k + 3]),
-                            pack_bf16x2(o[k + 4], o[k + 5]), pack_bf16x2(o[k + 6], o[k + 7]),
-                            pack_bf16x2(o[k + 8], o[k + 9]), pack_bf16x2(o[k + 10], o[k + 11]),
-                            pack_bf16x2(o[k + 12], o[k + 13]), pack_bf16x2(o[k + 14], o[k + 15]));
+            store8<STORE32>(dst + k, pack_bf16x2(f(k), f(k + 1)), pack_bf16x2(f(k + 2), f(k + 3)),
+                            pack_bf16x2(f(k + 4), f(k + 5)), pack_bf16x2(f(k + 6), f(k + 7)),
+                            pack_bf16x2(f(k + 8), f(k + 9)), pack_bf16x2(f(k + 10), f(k + 11)),
+                            pack_bf16x2(f(k + 12), f(k + 13)), pack_bf16x2(f(k + 14), f(k + 15)));
         }
       };
+      // TMEM loads are issued 128 columns at a time and waited for once; the
+      // accumulator is released as soon as its last columns are in registers
+      if constexpr (V == 1) {
+        uint32_t r[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tc::tmem_ld32(taddr + 32 * c, r + 32 * c);
+        tc::tmem_wait_ld();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&S.tempty[acc]);
+        r[0] = __float_as_uint(__uint_as_float(r[0]) - corr);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) emit(r + 32 * c, 32 * c);
+      } else {
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        if constexpr (V == 1) {
-          uint32_t r[32];
-          tc::tmem_ld32(taddr + 32 * c, r);
+        for (int h = 0; h < 2; ++h) {  // chunks 2h and 2h + 1 of both halves
+          uint32_t a[64], b[64];
+          tc::tmem_ld32(taddr + 64 * h, a);
+          tc::tmem_ld32(taddr + 64 * h + 32, a + 32);
+          tc::tmem_ld32(taddr + 128 + 64 * h, b);
+          tc::tmem_ld32(taddr + 128 + 64 * h + 32, b + 32);
           tc::tmem_wait_ld();
-          float o[32];
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __uint_as_float(r[k]);
-          if (c == 0) o[0] -= corr;
-          emit(o, 32 * c);
-        } else {
-          uint32_t a[32], b[32];
-          tc::tmem_ld32(taddr + 32 * c, a);
-          tc::tmem_ld32(taddr + 128 + 32 * c, b);
-          tc::tmem_wait_ld();
-          float o0[32], o1[32];
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            float y0 = __uint_as_float(a[k]), y1 = __uint_as_float(b[k]);
-            if (k == 0 && c == 0) {
-              y0 -= corr;
-              y1 -= corr;
-            }
-            o0[k] = y0 + y1;
-            o1[k] = y0 - y1;
+          if (h == 1) {
+            tc::tc_fence_before();
+            tc::mbar_arrive(&S.tempty[acc]);
+          } else {
+            a[0] = __float_as_uint(__uint_as_float(a[0]) - corr);
+            b[0] = __float_as_uint(__uint_as_float(b[0]) - corr);
           }
-          emit(o0, 32 * c);
-          emit(o1, 128 + 32 * c);
+#pragma unroll
+          for (int k = 0; k < 64; ++k) {  // the H_2 halves, in place
+            const float y0 = __uint_as_float(a[k]), y1 = __uint_as_float(b[k]);
+            a[k] = __float_as_uint(y0 + y1);
+            b[k] = __float_as_uint(y0 - y1);
+          }
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            emit(a + 32 * cc, 64 * h + 32 * cc);
+            emit(b + 32 * cc, 128 + 64 * h + 32 * cc);
+          }
         }
       }
-      tc::tc_fence_before();
-      tc::mbar_arrive(&S.tempty[acc]);
     }
   }
 
