@@ -1,5 +1,6 @@
-// k3_tc.cu -- dequantise + inverse rotation for n = 4096 to 32768 with the first
-// Kronecker factor on the tensor cores.
+// k3_tc.cu -- dequantise + inverse rotation on the tensor cores: for n = 4096 to
+// 32768 the first Kronecker factor runs on tcgen05 (below); for n = 128 and 256
+// the whole transform does (rows as the MMA's M, further down).
 //
 // "Rotations: QuaRot, SpinQuant and incoherence", widget "Try it": rotate,
 // quantize, rotate back; section "Hadamard matrices": H_n / sqrt(n) is

@@ -25,7 +25,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 cudaError_t launch_rotate_quant(const void *x, int64_t tokens, int log_n, float clip, const uint32_t *signs,
                                 uint32_t flags, int bits, uint8_t *q, float *scales, cudaStream_t stream);
 
-// Tensor-core R4 kernels (n = 128, 256 and 4096 to 32768; n = 32768 without a
+// Tensor-core R4 kernels (n = 128, 256 and 2048 to 32768; n = 32768 without a
 // sign diagonal): availability and launcher.
 bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags, bool has_signs);
 cudaError_t launch_rotate_quant_tc(int log_n, int bits, const void *x, int64_t tokens, float clip,
@@ -39,7 +39,8 @@ void set_stall_test(int enable);
 cudaError_t read_device_status(unsigned int *status, bool reset);
 cudaError_t read_rope_status(unsigned int *status, bool reset);
 
-// Tensor-core dequantise + inverse kernel (n = 4096 to 32768): availability and launcher.
+// Tensor-core dequantise + inverse kernels (n = 128, 256 and 4096 to 32768): availability
+// and launcher.
 bool tc_dequant_supported(int log_n, int64_t rows, uint32_t flags);
 cudaError_t launch_dequant_inverse_tc(int log_n, const uint8_t *codes, int64_t rows, int mode, const void *scale,
                                       const void *zero, const uint32_t *signs, void *out, int out_dtype,
