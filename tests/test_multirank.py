@@ -63,3 +63,19 @@ def test_reference_arm_only_rank0_prints():
                         "sweep7", "--steps", "1", "--warmup", "3"], capture_output=True, text=True, env=env,
                        timeout=600)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_reference_arm_int8_line():
+    """The reference arm on the INT8 workload (a reduced token count): its line names
+    the INT8 metric, counts 3n + 4 bytes per token and describes the oracle run."""
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "r4_prefill_int8", "--tokens", "16", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and "INT8" in line["metric"]
+    assert line["config"]["tokens"] == 16 and line["config"]["n"] == 16384
+    n = 16384
+    assert np.isclose(line["value"], 16 * (3 * n + 4) / (line["ms_per_step"] / 1e3) / 1e9, rtol=1e-6)
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
