@@ -72,8 +72,9 @@ def lib():
                              vp, vp, vp, _u8p, C.POINTER(C.c_double), C.POINTER(C.c_float)]
     L.orc_r4_row.restype = C.c_int
     L.orc_r4_rows.argtypes = [_u16p, C.c_int64, C.c_int, C.c_double, vp, C.c_uint32, _u8p,
-                              np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")]
+                              np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS"), C.c_int]
     L.orc_r4_rows.restype = C.c_int
+    L.orc_max_threads.restype = C.c_int
     L.orc_rope_half.argtypes = [_dp, C.c_int, C.c_double, C.c_double]
     L.orc_r3_token.argtypes = [_u16p, _u16p, _u16p, C.c_double, C.c_double, C.c_int, C.c_int,
                                C.c_int, C.c_double, vp, _u16p, vp, vp, vp, _u8p, _u8p,
@@ -252,15 +253,21 @@ def r4_row_int8(x_bits, clip, signs=None, no_rotate=False, method=METHOD_FWHT):
     return dict(y=y, pre=pre, codes=codes, scale64=s64.value, scale32=np.float32(s32.value))
 
 
-def r4_rows(x_bits, clip, signs=None, no_rotate=False):
-    """Rows [T, n] through the R4 path with the fast transform."""
+def max_threads() -> int:
+    """Threads the oracle's batch loop uses by default (the host's cores)."""
+    return int(lib().orc_max_threads())
+
+
+def r4_rows(x_bits, clip, signs=None, no_rotate=False, threads=1):
+    """Rows [T, n] through the R4 path with the fast transform, over `threads`
+    OpenMP threads (rows are independent; the results do not depend on it)."""
     x = np.ascontiguousarray(x_bits, dtype=np.uint16)
     T, n = x.shape
     packed = np.empty((T, n // 2), dtype=np.uint8)
     scales = np.empty(T, dtype=np.float32)
     s = _signs(signs)
     rc = lib().orc_r4_rows(x, T, n, float(clip), _ptr(s), NO_ROTATE if no_rotate else 0,
-                           packed, scales)
+                           packed, scales, int(threads))
     if rc:
         raise ValueError(f"orc_r4_rows failed ({rc})")
     return packed, scales

@@ -4,7 +4,8 @@ The oracle is test infrastructure: only the test suite, the smoke check and
 the CPU-baseline leg of the benchmark load it.  It is plain C built with gcc,
 with strict IEEE semantics (no fast-math, no FMA contraction), so that every
 operation it performs is the correctly rounded binary64 operation written in
-the source.
+the source. OpenMP only spreads independent rows of the batch loop over
+threads.
 """
 import os
 import subprocess
@@ -19,7 +20,7 @@ def build(force: bool = False) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off",
-           "-frounding-math", "-Wall", "-Wextra", "-o", LIB + ".tmp", SRC, "-lm"]
+           "-frounding-math", "-fopenmp", "-Wall", "-Wextra", "-o", LIB + ".tmp", SRC, "-lm"]
     subprocess.check_call(cmd)
     os.replace(LIB + ".tmp", LIB)
     return LIB

@@ -45,6 +45,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORC_NO_ROTATE 1u
 #define ORC_METHOD_FWHT 0
@@ -350,15 +353,27 @@ int orc_r4_row_int8(const uint16_t *x, int n, double clip, const uint32_t *signs
   return 0;
 }
 
-/* Many rows with the fast transform (the timed CPU baseline uses this loop). */
+/* Many rows with the fast transform (the timed CPU baseline uses this loop). Rows are
+ * independent, so `threads` > 1 spreads them over OpenMP threads; each row's arithmetic
+ * is the same as with one thread, so the results are identical. */
 int orc_r4_rows(const uint16_t *x, int64_t tokens, int n, double clip, const uint32_t *signs,
-                uint32_t flags, uint8_t *packed, float *scales) {
+                uint32_t flags, uint8_t *packed, float *scales, int threads) {
+  int rc = 0;
+#pragma omp parallel for schedule(dynamic, 16) num_threads(threads > 0 ? threads : 1) reduction(| : rc)
   for (int64_t t = 0; t < tokens; t++) {
-    int rc = orc_r4_row(x + t * n, n, clip, signs, flags, ORC_METHOD_FWHT, NULL, NULL, NULL,
-                        packed + t * (n / 2), NULL, scales + t);
-    if (rc) return rc;
+    rc |= orc_r4_row(x + t * n, n, clip, signs, flags, ORC_METHOD_FWHT, NULL, NULL, NULL,
+                     packed + t * (n / 2), NULL, scales + t);
   }
-  return 0;
+  return rc ? -1 : 0;
+}
+
+/* Threads OpenMP would use by default (the host's cores). */
+int orc_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
 }
 
 /* ------------------------------------------------------------------ */

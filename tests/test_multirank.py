@@ -79,3 +79,14 @@ def test_reference_arm_int8_line():
     n = 16384
     assert np.isclose(line["value"], 16 * (3 * n + 4) / (line["ms_per_step"] / 1e3) / 1e9, rtol=1e-6)
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_cpu_baseline_leg_reports_one_and_all_cores():
+    sys.path.insert(0, ROOT)
+    import bench
+    wl = bench.make_workload("sweep12", 0, tokens=24)
+    cpu = bench.cpu_baseline_leg(wl)
+    assert cpu["kind"] == "oracle" and cpu["cores"] == 1 and cpu["value"] > 0
+    assert cpu["all_cores"]["cores"] >= 1 and cpu["all_cores"]["value"] > 0
+    wl8 = bench.make_workload("r4_prefill_int8", 0, tokens=2)
+    assert bench.cpu_baseline_leg(wl8)["all_cores"]["cores"] == 1  # the INT8 rows run one call at a time

@@ -424,6 +424,14 @@ def test_r4_rows_matches_single_rows(orc):
         assert np.array_equal(r["packed"], packed[t]) and r["scale32"] == scales[t]
 
 
+def test_r4_rows_do_not_depend_on_threads(orc):
+    xb = synthetic.sweep(10, tokens=37, seed=5)
+    sg = synthetic.sign_bits(1024, 2)
+    p1, s1 = orc.r4_rows(xb, 0.9, signs=sg, threads=1)
+    p4, s4 = orc.r4_rows(xb, 0.9, signs=sg, threads=4)
+    assert np.array_equal(p1, p4) and np.array_equal(s1, s4)
+
+
 # --------------------------------------------------------------------------
 # Per-token INT8 (the b = 8 case of "SpinQuant Guide: Learned Rotations for
 # 4-Bit LLMs", section "The Outlier Curse": range [-128, 127], step
