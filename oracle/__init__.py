@@ -57,6 +57,16 @@ def lib():
     L.orc_rotate.restype = C.c_int
     L.orc_quant_sym_int4.argtypes = [_dp, C.c_int, C.c_double, vp, _i8p]
     L.orc_quant_sym_int4.restype = C.c_double
+    L.orc_legendre.argtypes = [C.c_int64, C.c_int64]
+    L.orc_legendre.restype = C.c_int
+    L.orc_paley_type.argtypes = [C.c_int]
+    L.orc_paley_type.restype = C.c_int
+    L.orc_paley_hadamard.argtypes = [C.c_int, _i8p]
+    L.orc_paley_hadamard.restype = C.c_int
+    L.orc_rotate_kron.argtypes = [_dp, C.c_int, C.c_int, vp, _dp]
+    L.orc_rotate_kron.restype = C.c_int
+    L.orc_r4_row_kron.argtypes = [_u16p, C.c_int, C.c_int, C.c_double, vp, vp, vp, _i8p, vp, vp]
+    L.orc_r4_row_kron.restype = C.c_int
     L.orc_quant_sym_int8.argtypes = [_dp, C.c_int, C.c_double, vp, _i8p]
     L.orc_quant_sym_int8.restype = C.c_double
     L.orc_r4_row_int8.argtypes = [_u16p, C.c_int, C.c_double, vp, C.c_uint32, C.c_int, vp, vp, _i8p,
@@ -256,6 +266,52 @@ def r4_row_int8(x_bits, clip, signs=None, no_rotate=False, method=METHOD_FWHT):
 def max_threads() -> int:
     """Threads the oracle's batch loop uses by default (the host's cores)."""
     return int(lib().orc_max_threads())
+
+
+# ---------------------------------------------------------------- n = m * 2^k
+def legendre(a, q) -> int:
+    return int(lib().orc_legendre(int(a), int(q)))
+
+
+def paley_type(m) -> int:
+    """1 or 2 when Paley's construction gives a Hadamard matrix of order m, else 0."""
+    return int(lib().orc_paley_type(int(m)))
+
+
+def paley_hadamard(m) -> np.ndarray:
+    H = np.empty((m, m), dtype=np.int8)
+    rc = lib().orc_paley_hadamard(int(m), H)
+    if rc:
+        raise ValueError(f"no Paley Hadamard matrix of order {m}")
+    return H
+
+
+def rotate_kron(x, m, signs=None) -> np.ndarray:
+    """(H_m (x) H_b) D x / sqrt(n) for a row of n = m b values (b a power of two)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.empty_like(x)
+    s = _signs(signs)
+    rc = lib().orc_rotate_kron(x, int(m), x.size // int(m), _ptr(s), y)
+    if rc:
+        raise ValueError(f"orc_rotate_kron failed ({rc})")
+    return y
+
+
+def r4_row_kron(x_bits, m, clip, signs=None):
+    """One token of n = m b values through the Kronecker rotation and INT4 quantiser."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    n = x.size
+    y = np.empty(n, dtype=np.float64)
+    pre = np.empty(n, dtype=np.float64)
+    codes = np.empty(n, dtype=np.int8)
+    s64 = C.c_double()
+    s32 = C.c_float()
+    s = _signs(signs)
+    rc = lib().orc_r4_row_kron(x, int(m), n // int(m), float(clip), _ptr(s), _ptr(y), _ptr(pre), codes,
+                               C.byref(s64), C.byref(s32))
+    if rc:
+        raise ValueError(f"orc_r4_row_kron failed ({rc})")
+    return dict(y=y, pre=pre, codes=codes, scale64=s64.value, scale32=np.float32(s32.value))
 
 
 def r4_rows(x_bits, clip, signs=None, no_rotate=False, threads=1):

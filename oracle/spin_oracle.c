@@ -38,7 +38,10 @@
  * asymmetric INT4 with an integer zero point whose range is widened to
  * include 0; codes of element 2j in the low nibble of byte j; the diagonal is
  * applied before the transform; the asymmetric quantiser divides by the
- * fp16-rounded scale.
+ * fp16-rounded scale; for n = m 2^k that is not a power of two, the small factor
+ * H_m is Paley's (type I or II, a named published construction: the pages give
+ * none), the product is H_m (x) H_{2^k} with the H_m index as the high part of
+ * the element index, and the diagonal again comes first.
  */
 #include <fenv.h>
 #include <math.h>
@@ -195,6 +198,133 @@ int orc_rotate(const double *x, int n, const uint32_t *signs, int method, double
   for (int i = 0; i < n; i++) y[i] = y[i] / r;
   free(t);
   return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Sizes that are not powers of two: H_m (x) H_b, b a power of two       */
+/* ------------------------------------------------------------------ */
+
+/* [RQ "Hadamard matrices"]: sizes that are not powers of two use a Kronecker
+ * product of a small known Hadamard matrix with a Sylvester one. The pages give
+ * no small matrix, so H_m comes from Paley's construction (R. E. A. C. Paley,
+ * "On orthogonal matrices", 1933) for a prime q:
+ *   type I,  q = 3 (mod 4), m = q + 1:   H = I + S,  S = [[0, 1^T], [-1, Q]];
+ *   type II, q = 1 (mod 4), m = 2(q + 1): H = S (x) [[1, -1], [-1, -1]] + I (x) [[1, 1], [1, -1]],
+ *            S = [[0, 1^T], [1, Q]];
+ * with the Jacobsthal matrix Q[i][j] = chi(j - i), chi the quadratic character
+ * mod q (chi(0) = 0). */
+
+double orc_quant_sym_int4(const double *y, int n, double clip, double *pre, int8_t *codes);
+
+static int is_prime(int64_t q) {
+  if (q < 2) return 0;
+  for (int64_t d = 2; d * d <= q; d++)
+    if (q % d == 0) return 0;
+  return 1;
+}
+
+/* Quadratic character of a mod an odd prime q by Euler's criterion:
+ * a^((q-1)/2) = 1 (residue), q - 1 (non-residue), 0 (a = 0 mod q). */
+int orc_legendre(int64_t a, int64_t q) {
+  int64_t r = ((a % q) + q) % q;
+  if (r == 0) return 0;
+  int64_t e = (q - 1) / 2, acc = 1, b = r;
+  while (e > 0) {
+    if (e & 1) acc = (acc * b) % q;
+    b = (b * b) % q;
+    e >>= 1;
+  }
+  return acc == 1 ? 1 : -1;
+}
+
+/* The Paley type (1 or 2) that gives a Hadamard matrix of order m, or 0. */
+int orc_paley_type(int m) {
+  if (m >= 4 && (m - 1) % 4 == 3 && is_prime(m - 1)) return 1;
+  if (m >= 12 && m % 4 == 0 && (m / 2 - 1) % 4 == 1 && is_prime(m / 2 - 1)) return 2;
+  return 0;
+}
+
+/* H (m x m, row-major, entries +-1) by Paley's construction; -1 if m has none. */
+int orc_paley_hadamard(int m, int8_t *H) {
+  const int type = orc_paley_type(m);
+  if (!type) return -1;
+  const int q = type == 1 ? m - 1 : m / 2 - 1, k = q + 1;
+  int8_t *S = (int8_t *)malloc((size_t)k * (size_t)k);
+  if (!S) return -2;
+  for (int i = 0; i < k; i++)
+    for (int j = 0; j < k; j++) {
+      int v;
+      if (i == 0 && j == 0) v = 0;
+      else if (i == 0) v = 1;
+      else if (j == 0) v = type == 1 ? -1 : 1;
+      else v = orc_legendre((int64_t)(j - 1) - (int64_t)(i - 1), q);
+      S[i * k + j] = (int8_t)v;
+    }
+  if (type == 1) {
+    for (int i = 0; i < k; i++)
+      for (int j = 0; j < k; j++) H[i * m + j] = (int8_t)(S[i * k + j] + (i == j ? 1 : 0));
+  } else {
+    static const int A[2][2] = {{1, -1}, {-1, -1}}, B[2][2] = {{1, 1}, {1, -1}};
+    for (int i = 0; i < k; i++)
+      for (int j = 0; j < k; j++)
+        for (int u = 0; u < 2; u++)
+          for (int v = 0; v < 2; v++)
+            H[(2 * i + u) * m + (2 * j + v)] = (int8_t)(S[i * k + j] * A[u][v] + (i == j ? B[u][v] : 0));
+  }
+  free(S);
+  return 0;
+}
+
+/* y = (H_m (x) H_b) D x / sqrt(m b) for a row of n = m b values, element e = b i + j
+ * (i the H_m index, j the Sylvester one; D first, as for powers of two): H_b on each
+ * of the m blocks of b, then H_m across the blocks, both written out plainly. */
+int orc_rotate_kron(const double *x, int m, int b, const uint32_t *signs, double *y) {
+  if (!is_pow2(b)) return -1;
+  int8_t *H = (int8_t *)malloc((size_t)m * (size_t)m);
+  double *t = (double *)malloc(sizeof(double) * (size_t)m * (size_t)b);
+  if (!H || !t) {
+    free(H); free(t);
+    return -2;
+  }
+  if (orc_paley_hadamard(m, H)) {
+    free(H); free(t);
+    return -1;
+  }
+  const int n = m * b;
+  for (int e = 0; e < n; e++) t[e] = sign_bit(signs, e) ? -x[e] : x[e];
+  for (int i = 0; i < m; i++) orc_fwht(t + (size_t)i * b, b);
+  for (int i = 0; i < m; i++)
+    for (int j = 0; j < b; j++) {
+      double acc = 0.0;
+      for (int k = 0; k < m; k++) acc += H[i * m + k] * t[(size_t)k * b + j];
+      y[(size_t)i * b + j] = acc;
+    }
+  const double r = sqrt((double)n);
+  for (int e = 0; e < n; e++) y[e] = y[e] / r;
+  free(H); free(t);
+  return 0;
+}
+
+/* R4 for n = m b: the Kronecker rotation, then the per-token INT4 quantiser. */
+int orc_r4_row_kron(const uint16_t *x, int m, int b, double clip, const uint32_t *signs, double *y_out,
+                    double *pre, int8_t *codes, double *scale64, float *scale32) {
+  const int n = m * b;
+  double *xd = (double *)malloc(sizeof(double) * (size_t)n);
+  double *y = (double *)malloc(sizeof(double) * (size_t)n);
+  if (!xd || !y) {
+    free(xd); free(y);
+    return -2;
+  }
+  for (int e = 0; e < n; e++) xd[e] = orc_bf16_to_f64(x[e]);
+  int rc = orc_rotate_kron(xd, m, b, signs, y);
+  if (!rc) {
+    double s = orc_quant_sym_int4(y, n, clip, pre, codes);
+    if (y_out) memcpy(y_out, y, sizeof(double) * (size_t)n);
+    if (scale64) *scale64 = s;
+    *scale32 = (float)s;
+  }
+  free(xd); free(y);
+  return rc;
 }
 
 /* ------------------------------------------------------------------ */

@@ -516,3 +516,65 @@ def test_int8_and_int4_share_the_rotation(orc):
     assert np.array_equal(r4["y"], r8["y"])
     assert r8["scale64"] * 127 == pytest.approx(r4["scale64"] * 7, rel=1e-15)
     assert np.max(np.abs(r8["codes"] * r8["scale64"] - r8["y"])) <= r8["scale64"] / 2 * (1 + 1e-12)
+
+
+# --------------------------------------------------------------------------
+# Sizes that are not powers of two ("Rotations: QuaRot, SpinQuant and
+# incoherence", section "Hadamard matrices": a Kronecker product with a small
+# known Hadamard matrix). The small factor comes from Paley's construction.
+# --------------------------------------------------------------------------
+def _primes(limit):
+    return [q for q in range(2, limit) if all(q % d for d in range(2, int(q ** 0.5) + 1))]
+
+
+def test_legendre_symbol_against_squares(orc):
+    for q in [p for p in _primes(60) if p > 2]:
+        squares = {(x * x) % q for x in range(1, q)}
+        for a in range(-q, 2 * q):
+            want = 0 if a % q == 0 else (1 if a % q in squares else -1)
+            assert orc.legendre(a, q) == want
+
+
+def test_paley_orders_and_orthogonality(orc):
+    expect = sorted({q + 1 for q in _primes(100) if q % 4 == 3} | {2 * (q + 1) for q in _primes(50) if q % 4 == 1})
+    got = [m for m in range(1, 101) if orc.paley_type(m)]
+    assert got == [m for m in expect if m <= 100]
+    for m in got:
+        H = orc.paley_hadamard(m).astype(np.int64)
+        assert set(np.unique(H)) == {-1, 1}
+        assert np.array_equal(H @ H.T, m * np.eye(m, dtype=np.int64))
+        assert np.array_equal(H.T @ H, m * np.eye(m, dtype=np.int64))
+
+
+def test_orders_without_paley_are_rejected(orc):
+    for m in (2, 43, 52, 172):
+        assert orc.paley_type(m) == 0
+        with pytest.raises(ValueError):
+            orc.paley_hadamard(m)
+
+
+@pytest.mark.parametrize("m,b", [(12, 4), (20, 8), (28, 64), (36, 2)])
+def test_rotate_kron_matches_numpy_kron(orc, m, b):
+    n = m * b
+    rng = np.random.default_rng(m * b)
+    x = rng.standard_normal(n)
+    signs = synthetic.sign_bits(n, 4)
+    d = np.where(np.unpackbits(signs.view(np.uint8), bitorder="little")[:n].astype(bool), -1.0, 1.0)
+    M = np.kron(orc.paley_hadamard(m).astype(np.float64), scipy.linalg.hadamard(b).astype(np.float64))
+    y = orc.rotate_kron(x, m, signs=signs)
+    assert np.allclose(y, M @ (d * x) / math.sqrt(n), rtol=0, atol=1e-12 * np.linalg.norm(x))
+    assert abs(np.linalg.norm(y) - np.linalg.norm(x)) <= 1e-12 * np.linalg.norm(x)  # orthogonal
+    assert np.allclose(d * (M.T @ y) / math.sqrt(n), x, atol=1e-12 * np.linalg.norm(x))  # transpose undoes it
+
+
+def test_r4_kron_one_hot_at_llama3_width(orc):
+    """n = 14336 = 28 x 512 (the down-projection input of an 8B LLaMA-3 layer): a one-hot
+    row rotates to +-1/sqrt(n) everywhere, so at clip 1 every code is +-7."""
+    m, b = 28, 512
+    n = m * b
+    x = np.zeros(n, np.float32)
+    x[1234] = 5.0
+    r = orc.r4_row_kron(bf16(x), m, 1.0)
+    assert np.allclose(np.abs(r["y"]), 5.0 / math.sqrt(n), rtol=1e-14)
+    assert np.all(np.abs(r["codes"]) == 7)
+    assert r["scale64"] == pytest.approx(5.0 / math.sqrt(n) / 7, rel=1e-14)
