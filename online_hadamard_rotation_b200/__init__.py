@@ -130,13 +130,41 @@ def _stream(stream):
     return stream.cuda_stream
 
 
-def _need(t: torch.Tensor, name: str, dtype, device=None):
+def _need(t: torch.Tensor, name: str, dtype, device=None, shape=None):
+    """Argument checks before a pointer reaches the library: dtype, a contiguous CUDA
+    tensor (a host pointer would reach a kernel), the expected device and shape."""
     if t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if device is not None and t.device != device:
         raise ValueError(f"{name} must be on {device}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _need_signs(signs, n: int, device) -> None:
+    if signs is not None:
+        _need(signs, "signs", torch.int32, device)
+        if signs.numel() < max(1, n // 32):
+            raise ValueError(f"signs: expected {max(1, n // 32)} words for n = {n}, got {signs.numel()}")
+
+
+def _r4_args(x, out, scales, signs, code_dtype, code_cols):
+    _need(x, "x", torch.bfloat16)
+    if x.dim() != 2:
+        raise ValueError(f"x: expected [tokens, n], got shape {tuple(x.shape)}")
+    tokens, n = x.shape
+    if out is None:
+        out = torch.empty((tokens, code_cols(n)), dtype=code_dtype, device=x.device)
+    _need(out, "out", code_dtype, x.device, (tokens, code_cols(n)))
+    if scales is None:
+        scales = torch.empty((tokens,), dtype=torch.float32, device=x.device)
+    _need(scales, "scales", torch.float32, x.device, (tokens,))
+    _need_signs(signs, n, x.device)
+    return tokens, n, out, scales
 
 
 def test_stall_tensor_core_waits(enable: bool) -> None:
@@ -156,14 +184,7 @@ def hadamard_quant_int4(x: torch.Tensor, clip: float = 1.0, signs: torch.Tensor 
                         scales: torch.Tensor | None = None, stream=None, cuda_cores_only: bool = False,
                         tensor_cores: bool = False):
     """R4: x [tokens, n] bf16 (CUDA) -> (codes [tokens, n/2] uint8, scales [tokens] fp32)."""
-    _need(x, "x", torch.bfloat16)
-    tokens, n = x.shape
-    if out is None:
-        out = torch.empty((tokens, n // 2), dtype=torch.uint8, device=x.device)
-    if scales is None:
-        scales = torch.empty((tokens,), dtype=torch.float32, device=x.device)
-    if signs is not None:
-        _need(signs, "signs", torch.int32, x.device)
+    tokens, n, out, scales = _r4_args(x, out, scales, signs, torch.uint8, lambda n: n // 2)
     flags = ((NO_ROTATE if no_rotate else 0) | (CUDA_CORES_ONLY if cuda_cores_only else 0) |
              (TENSOR_CORES if tensor_cores else 0))
     st = spin_hadamard_quant_int4_ex(_ptr(x), tokens, n, float(clip), _ptr(signs), flags,
@@ -177,14 +198,7 @@ def hadamard_quant_int8(x: torch.Tensor, clip: float = 1.0, signs: torch.Tensor 
                         scales: torch.Tensor | None = None, stream=None, cuda_cores_only: bool = False,
                         tensor_cores: bool = False):
     """R4 with INT8 codes: x [tokens, n] bf16 (CUDA) -> (codes [tokens, n] int8, scales [tokens] fp32)."""
-    _need(x, "x", torch.bfloat16)
-    tokens, n = x.shape
-    if out is None:
-        out = torch.empty((tokens, n), dtype=torch.int8, device=x.device)
-    if scales is None:
-        scales = torch.empty((tokens,), dtype=torch.float32, device=x.device)
-    if signs is not None:
-        _need(signs, "signs", torch.int32, x.device)
+    tokens, n, out, scales = _r4_args(x, out, scales, signs, torch.int8, lambda n: n)
     flags = ((NO_ROTATE if no_rotate else 0) | (CUDA_CORES_ONLY if cuda_cores_only else 0) |
              (TENSOR_CORES if tensor_cores else 0))
     st = spin_hadamard_quant_int8(_ptr(x), tokens, n, float(clip), _ptr(signs), flags, _ptr(out), _ptr(scales),
@@ -233,14 +247,24 @@ def rope_hadamard_kvquant(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos
                           q_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """R3 + INT4 KV: q [B,S,hq,d], k/v [B,S,hkv,d] bf16, pos [B,S] int32.
     Writes the cache dict (see alloc_kv_cache) and returns rotated Q (bf16)."""
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        _need(t, name, torch.bfloat16)
-    _need(pos, "pos", torch.int32)
+    _need(q, "q", torch.bfloat16)
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k and v are [batch, seq, heads, head_dim]")
     B, S, hq, d = q.shape
     hkv = k.shape[2]
+    _need(k, "k", torch.bfloat16, q.device, (B, S, hkv, d))
+    _need(v, "v", torch.bfloat16, q.device, (B, S, hkv, d))
+    _need(pos, "pos", torch.int32, q.device, (B, S))
     if q_out is None:
         q_out = torch.empty_like(q)
+    _need(q_out, "q_out", torch.bfloat16, q.device, (B, S, hq, d))
     cache_len = cache["k_cache"].shape[2]
+    for name in ("k_cache", "v_cache"):
+        _need(cache[name], name, torch.uint8, q.device, (B, hkv, cache_len, d // 2))
+    for name in ("k_scale", "k_zero", "v_scale", "v_zero"):
+        _need(cache[name], name, torch.float16, q.device, (B, hkv, cache_len))
+    if cache_offset < 0 or cache_offset + S > cache_len:
+        raise ValueError(f"cache slots {cache_offset} .. {cache_offset + S - 1} outside a cache of {cache_len}")
     st = spin_rope_hadamard_kvquant(
         _ptr(q), _ptr(k), _ptr(v), _ptr(pos), float(theta), d, B, S, hq, hkv, float(clip), _ptr(q_out),
         _ptr(cache["k_cache"]), _ptr(cache["v_cache"]), _ptr(cache["k_scale"]), _ptr(cache["k_zero"]),
@@ -257,9 +281,29 @@ def dequant_hadamard_inverse(codes: torch.Tensor, n: int, scale: torch.Tensor, z
     cuda_cores_only / tensor_cores select the kernel (SPIN_CUDA_CORES_ONLY /
     SPIN_TENSOR_CORES); by default the library picks."""
     _need(codes, "codes", torch.uint8)
+    if n < 2 or codes.dim() < 1 or codes.shape[-1] != n // 2:
+        raise ValueError(f"codes: expected [..., {n // 2}] for n = {n}, got shape {tuple(codes.shape)}")
     rows = codes.numel() // (n // 2)
+    if mode not in (SYM_INT4_F32SCALE, ASYM_INT4_F16SZ):
+        raise ValueError(f"mode {mode}: expected SYM_INT4_F32SCALE or ASYM_INT4_F16SZ")
+    asym = mode == ASYM_INT4_F16SZ
+    _need(scale, "scale", torch.float16 if asym else torch.float32, codes.device)
+    if scale.numel() != rows:
+        raise ValueError(f"scale: expected {rows} values, got {scale.numel()}")
+    if asym:
+        if zero is None:
+            raise ValueError("zero is required for ASYM_INT4_F16SZ")
+        _need(zero, "zero", torch.float16, codes.device)
+        if zero.numel() != rows:
+            raise ValueError(f"zero: expected {rows} values, got {zero.numel()}")
+    _need_signs(signs, n, codes.device)
     if out is None:
+        if out_dtype not in (torch.float32, torch.bfloat16):
+            raise TypeError(f"out_dtype: expected torch.float32 or torch.bfloat16, got {out_dtype}")
         out = torch.empty(tuple(codes.shape[:-1]) + (n,), dtype=out_dtype, device=codes.device)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"out: expected torch.float32 or torch.bfloat16, got {out.dtype}")
+    _need(out, "out", out.dtype, codes.device, tuple(codes.shape[:-1]) + (n,))
     dt = F32 if out.dtype == torch.float32 else BF16
     flags = (NO_ROTATE if no_rotate else 0) | (CUDA_CORES_ONLY if cuda_cores_only else 0) | \
         (TENSOR_CORES if tensor_cores else 0)

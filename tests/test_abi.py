@@ -125,3 +125,22 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(spin, "LIB_PATH", str(tmp_path / "libspin.so"))
     with pytest.raises(ImportError):
         spin.lib()
+
+
+def test_binding_rejects_host_tensors():
+    """A host pointer must never reach a kernel: the binding refuses tensors that are not
+    on a CUDA device before it calls the library."""
+    import torch
+    x = torch.zeros((4, 256), dtype=torch.bfloat16)
+    for fn in (spin.hadamard_quant_int4, spin.hadamard_quant_int8):
+        with pytest.raises(ValueError, match="CUDA"):
+            fn(x, 1.0)
+    with pytest.raises(ValueError, match="CUDA"):
+        spin.dequant_hadamard_inverse(torch.zeros((4, 128), dtype=torch.uint8), 256,
+                                      torch.ones(4, dtype=torch.float32))
+    q = torch.zeros((1, 2, 4, 128), dtype=torch.bfloat16)
+    kv = torch.zeros((1, 2, 1, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        spin.rope_hadamard_kvquant(q, kv, kv, torch.zeros((1, 2), dtype=torch.int32), {}, clip=1.0)
+    with pytest.raises(TypeError):
+        spin.hadamard_quant_int4(torch.zeros((4, 256), dtype=torch.float32), 1.0)
