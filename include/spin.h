@@ -20,11 +20,13 @@
  *  * Calls on the same stream are ordered; calls that run concurrently on
  *    different streams may share inputs but not outputs.
  *
- * Quantised layout (all entry points)
- * -----------------------------------
+ * Quantised layout
+ * ----------------
  *  Two 4-bit codes per byte: element 2j in the low nibble of byte j,
  *  element 2j+1 in the high nibble. Symmetric codes are 4-bit two's
  *  complement in [-8, 7]; asymmetric codes are unsigned in [0, 15].
+ *  spin_hadamard_quant_int8 instead writes one 8-bit two's-complement code
+ *  per element, element j at byte j, in [-128, 127].
  *
  * Sources are cited by page title and section:
  *  "SpinQuant, when rotations are worth learning" -- section "Four rotation
@@ -113,7 +115,7 @@ spin_status_t spin_hadamard_quant_int4(const void *x_bf16, int64_t tokens, int32
  *             SPIN_NO_ROTATE: quantise x directly (no D, no H), used to
  *               measure the direct-quantisation error;
  *             SPIN_CUDA_CORES_ONLY: at n = 128 and 256 the transform, and at
- *               n = 2048 … 16384, and at n = 32768 without sign_bits,
+ *               n = 2048 .. 16384, and at n = 32768 without sign_bits,
  *               the first H_128 Kronecker factor (two of them at n = 32768),
  *               normally runs on the tensor cores (exact +-1 x bf16 products,
  *               fp32 accumulation; at n = 128 and 256 the diagonal rides in the
