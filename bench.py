@@ -63,29 +63,21 @@ def oracle_r4_rows(oracle, bits, clip, signs, code_bits, threads=1) -> int:
     return 1
 
 
-def r4_kernel_name(n: int, tokens: int, has_signs: bool) -> str:
-    """The R4 kernel the library's dispatch picks by default: a tensor-core one for
-    n = 128, 256 and 2048 .. 32768 (n = 32768 without a sign diagonal) once the batch
-    has at least 128 MMA groups, else the CUDA-core one."""
-    log_n = n.bit_length() - 1
-    if log_n in (7, 8) and tokens >= 128 * (256 >> (log_n - 7)):
-        return "k1_tcs_rotate_quant"
-    if 11 <= log_n <= 15 and not (log_n == 15 and has_signs):
-        tokens_per_group = 1 if log_n == 15 else 256 >> (log_n - 7)
-        if tokens >= 128 * tokens_per_group:
-            return "k1_tc_rotate_quant"
-    return "k1_rotate_quant_int4"
+def r4_kernel_name(n: int, tokens: int, has_signs: bool, code_bits: int = 4) -> str:
+    """The R4 kernel the library's dispatch picks by default, asked of the library
+    itself (spin_uses_tensor_cores, a host-only query)."""
+    import online_hadamard_rotation_b200 as spin
+    if spin.uses_tensor_cores(spin.OP_HADAMARD_QUANT, tokens, n, 0, has_signs):
+        return "k1_tcs_rotate_quant" if n <= 256 else "k1_tc_rotate_quant"
+    return f"k1_rotate_quant_int{code_bits}"
 
 
 def k3_kernel_name(n: int, rows: int) -> str:
-    """The dequantise + inverse kernel the library's dispatch picks by default: a
-    tensor-core one for n = 128, 256 and 4096 .. 32768 once the batch has at least
-    128 MMA groups, else the CUDA-core one."""
-    log_n = n.bit_length() - 1
-    if log_n in (7, 8) and rows >= 128 * 128:
-        return "k3_tcs_dequant_inverse"
-    if 12 <= log_n <= 15 and rows >= 128 * (1 if log_n == 15 else 256 >> (log_n - 7)):
-        return "k3_tc_dequant_inverse"
+    """The dequantise + inverse kernel the library's dispatch picks by default (asked
+    of the library, as above)."""
+    import online_hadamard_rotation_b200 as spin
+    if spin.uses_tensor_cores(spin.OP_DEQUANT_INVERSE, rows, n):
+        return "k3_tcs_dequant_inverse" if n <= 256 else "k3_tc_dequant_inverse"
     return "k3_dequant_inverse"
 
 
@@ -523,7 +515,7 @@ def main():
 
     peak, peak_kind = measured_peaks()
     if wl["kind"] == "r4":
-        kname = r4_kernel_name(n, tokens, wl["signs"] is not None)
+        kname = r4_kernel_name(n, tokens, wl["signs"] is not None, wl["code_bits"])
     else:
         kname = "k2_rope_hadamard_kvquant"
     traffic = recorded_traffic(f"{kname}:{args.workload}")

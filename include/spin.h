@@ -258,6 +258,20 @@ spin_status_t spin_device_status(uint32_t *status, int reset);
  */
 void spin_test_stall_tensor_core_waits(int enable);
 
+/* Operations for spin_uses_tensor_cores. */
+#define SPIN_OP_HADAMARD_QUANT 0 /* spin_hadamard_quant_int4[_ex] and spin_hadamard_quant_int8 */
+#define SPIN_OP_DEQUANT_INVERSE 1 /* spin_dequant_hadamard_inverse */
+
+/*
+ * Host-only query (no device access, no launch): 1 if a call of operation `op`
+ * with these arguments would run a tensor-core kernel, 0 if it would run the
+ * CUDA-core kernel, -1 if the arguments are invalid for `op` (n not a supported
+ * power of two, rows < 0, unknown op or flag bits). has_signs != 0 means a
+ * sign_bits mask would be passed. The answer follows the same rules as the
+ * entry points' own dispatch.
+ */
+int spin_uses_tensor_cores(int32_t op, int64_t rows, int32_t n, uint32_t flags, int32_t has_signs);
+
 /* Human-readable name of a status code (static storage). */
 const char *spin_status_string(spin_status_t status);
 

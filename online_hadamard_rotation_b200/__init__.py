@@ -72,6 +72,8 @@ def lib() -> C.CDLL:
     for name in ("spin_hadamard_quant_int4", "spin_hadamard_quant_int4_ex", "spin_hadamard_quant_int8",
                  "spin_rope_hadamard_kvquant", "spin_dequant_hadamard_inverse"):
         getattr(L, name).restype = C.c_int
+    L.spin_uses_tensor_cores.argtypes = [i32, i64, i32, u32, i32]
+    L.spin_uses_tensor_cores.restype = C.c_int
     L.spin_test_stall_tensor_core_waits.argtypes = [C.c_int]
     L.spin_test_stall_tensor_core_waits.restype = None
     L.spin_device_status.argtypes = [C.POINTER(C.c_uint32), C.c_int]
@@ -170,6 +172,19 @@ def _r4_args(x, out, scales, signs, code_dtype, code_cols):
 def test_stall_tensor_core_waits(enable: bool) -> None:
     """Failure-detection test hook (see spin_test_stall_tensor_core_waits)."""
     lib().spin_test_stall_tensor_core_waits(1 if enable else 0)
+
+
+OP_HADAMARD_QUANT = 0
+OP_DEQUANT_INVERSE = 1
+
+
+def uses_tensor_cores(op: int, rows: int, n: int, flags: int = 0, has_signs: bool = False) -> bool:
+    """Whether a call would run a tensor-core kernel (host-only query of the library's
+    dispatch; see spin_uses_tensor_cores)."""
+    r = lib().spin_uses_tensor_cores(int(op), int(rows), int(n), int(flags), 1 if has_signs else 0)
+    if r < 0:
+        raise ValueError(f"invalid arguments for op {op}: rows={rows} n={n} flags={flags}")
+    return bool(r)
 
 
 def device_status(reset: bool = False) -> int:

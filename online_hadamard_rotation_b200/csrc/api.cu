@@ -219,6 +219,18 @@ spin_status_t spin_device_status(uint32_t *status, int reset) {
   return st;
 }
 
+int spin_uses_tensor_cores(int32_t op, int64_t rows, int32_t n, uint32_t flags, int32_t has_signs) {
+  const int log_n = log2_pow2(n);
+  if (log_n < 7 || log_n > 15 || rows < 0) return -1;
+  if ((flags & ~(SPIN_NO_ROTATE | SPIN_CUDA_CORES_ONLY | SPIN_TENSOR_CORES)) != 0 ||
+      (flags & (SPIN_CUDA_CORES_ONLY | SPIN_TENSOR_CORES)) == (SPIN_CUDA_CORES_ONLY | SPIN_TENSOR_CORES))
+    return -1;
+  if (flags & SPIN_CUDA_CORES_ONLY) return 0;
+  if (op == SPIN_OP_HADAMARD_QUANT) return tc_rotate_quant_supported(log_n, rows, flags, has_signs != 0) ? 1 : 0;
+  if (op == SPIN_OP_DEQUANT_INVERSE) return tc_dequant_supported(log_n, rows, flags) ? 1 : 0;
+  return -1;
+}
+
 int spin_version(void) { return 100; }
 
 }  // extern "C"

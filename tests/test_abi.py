@@ -144,3 +144,34 @@ def test_binding_rejects_host_tensors():
         spin.rope_hadamard_kvquant(q, kv, kv, torch.zeros((1, 2), dtype=torch.int32), {}, clip=1.0)
     with pytest.raises(TypeError):
         spin.hadamard_quant_int4(torch.zeros((4, 256), dtype=torch.float32), 1.0)
+
+
+def test_dispatch_query(L):
+    """spin_uses_tensor_cores answers on the host with the entry points' own rules."""
+    R4, INV = 0, 1
+    q = L.spin_uses_tensor_cores
+    q.argtypes = [C.c_int32, C.c_int64, C.c_int32, C.c_uint32, C.c_int32]
+    q.restype = C.c_int
+    assert q(R4, 8192, 16384, 0, 1) == 1              # R4 prefill: tensor cores
+    assert q(R4, 32, 16384, 0, 0) == 0                # decode batch: CUDA cores
+    assert q(R4, 1, 16384, 4, 0) == 1                 # SPIN_TENSOR_CORES at any batch
+    assert q(R4, 8192, 16384, 2, 1) == 0              # SPIN_CUDA_CORES_ONLY
+    assert q(R4, 8192, 16384, 1, 0) == 0              # SPIN_NO_ROTATE
+    assert q(R4, 16384, 32768, 0, 1) == 0             # n = 32768 with a diagonal
+    assert q(R4, 16384, 32768, 0, 0) == 1
+    assert q(R4, 128 * 256, 128, 0, 0) == 1 and q(R4, 128 * 256 - 1, 128, 0, 0) == 0
+    assert q(R4, 10 ** 6, 512, 0, 0) == 0 and q(R4, 10 ** 6, 1024, 4, 0) == 0
+    assert q(R4, 128 * 16, 2048, 0, 0) == 1
+    assert q(INV, 128 * 128, 256, 0, 0) == 1 and q(INV, 128 * 128 - 1, 256, 0, 0) == 0
+    assert q(INV, 10 ** 6, 2048, 0, 0) == 0 and q(INV, 128 * 8, 4096, 0, 0) == 1
+    for bad in ((R4, 4, 100, 0, 0), (R4, -1, 256, 0, 0), (R4, 4, 256, 6, 0), (R4, 4, 256, 8, 0), (7, 4, 256, 0, 0)):
+        assert q(*bad) == -1
+
+
+def test_bench_names_the_dispatched_kernel():
+    import bench
+    assert bench.r4_kernel_name(16384, 8192, True) == "k1_tc_rotate_quant"
+    assert bench.r4_kernel_name(128, 1 << 22, False) == "k1_tcs_rotate_quant"
+    assert bench.r4_kernel_name(1024, 1 << 19, False, 8) == "k1_rotate_quant_int8"
+    assert bench.k3_kernel_name(256, 1 << 21) == "k3_tcs_dequant_inverse"
+    assert bench.k3_kernel_name(2048, 1 << 18) == "k3_dequant_inverse"
