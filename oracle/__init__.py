@@ -74,6 +74,9 @@ def lib():
     L.orc_r4_row_int8.restype = C.c_int
     L.orc_quant_asym_int4.argtypes = [_dp, C.c_int, C.c_double, vp, _u8p,
                                       C.POINTER(C.c_uint16), C.POINTER(C.c_uint16)]
+    L.orc_quant_asym_int4_at.argtypes = [_dp, C.c_int, C.c_double, C.c_uint16, vp, _u8p,
+                                         C.POINTER(C.c_uint16)]
+    L.orc_quant_asym_int4_at.restype = C.c_uint16
     L.orc_asym_unrounded_scale.argtypes = [_dp, C.c_int, C.c_double]
     L.orc_asym_unrounded_scale.restype = C.c_double
     L.orc_pack_nibbles.argtypes = [_i32p, C.c_int, _u8p]
@@ -92,11 +95,14 @@ def lib():
     L.orc_r3_token.restype = C.c_int
     L.orc_r3_batch.argtypes = [_u16p, _u16p, _u16p, _i32p, C.c_double, C.c_int, C.c_int, C.c_int,
                                C.c_int, C.c_int, C.c_double, _u16p, _u8p, _u8p, _u16p, _u16p,
-                               _u16p, _u16p, C.c_int, C.c_int]
+                               _u16p, _u16p, C.c_int, C.c_int, C.c_int]
     L.orc_r3_batch.restype = C.c_int
     L.orc_dequant_inverse_row.argtypes = [_u8p, C.c_int, C.c_int, C.c_double, C.c_double, vp,
                                           C.c_uint32, C.c_int, _dp]
     L.orc_dequant_inverse_row.restype = C.c_int
+    L.orc_dequant_inverse_rows.argtypes = [_u8p, C.c_int64, C.c_int, C.c_int, _dp, vp, vp, C.c_uint32, _dp,
+                                           C.c_int]
+    L.orc_dequant_inverse_rows.restype = C.c_int
     L.orc_rmsnorm.argtypes = [_dp, C.c_int, C.c_double, _dp]
     L.orc_mse.argtypes = [_dp, _dp, C.c_int64]
     L.orc_mse.restype = C.c_double
@@ -205,6 +211,17 @@ def quant_asym_int4(x, clip):
     z16 = C.c_uint16()
     lib().orc_quant_asym_int4(x, x.size, float(clip), _ptr(pre), codes, C.byref(s16), C.byref(z16))
     return codes, int(s16.value), int(z16.value), pre
+
+
+def quant_asym_int4_at(x, clip, s16):
+    """Codes and zero point of an asymmetric group for the given fp16 step pattern.
+    Returns (codes, s16 used, z16, pre)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    pre = np.empty_like(x)
+    codes = np.empty(x.size, dtype=np.uint8)
+    z16 = C.c_uint16()
+    used = lib().orc_quant_asym_int4_at(x, x.size, float(clip), int(s16), _ptr(pre), codes, C.byref(z16))
+    return codes, int(used), int(z16.value), pre
 
 
 def asym_unrounded_scale(x, clip) -> float:
@@ -358,7 +375,9 @@ def r3_token(q_bits, k_bits, v_bits, pos, theta, clip):
     return out
 
 
-def r3_batch(q_bits, k_bits, v_bits, pos, theta, clip, cache_len=None, cache_offset=0):
+def r3_batch(q_bits, k_bits, v_bits, pos, theta, clip, cache_len=None, cache_offset=0, threads=1):
+    """The whole R3 batch into a cache of cache_len slots (token (b, s) at slot
+    cache_offset + s; other slots stay zero); tokens spread over `threads`."""
     q = np.ascontiguousarray(q_bits, dtype=np.uint16)
     k = np.ascontiguousarray(k_bits, dtype=np.uint16)
     v = np.ascontiguousarray(v_bits, dtype=np.uint16)
@@ -374,7 +393,7 @@ def r3_batch(q_bits, k_bits, v_bits, pos, theta, clip, cache_len=None, cache_off
         v_scale=np.zeros((B, hkv, L), dtype=np.uint16), v_zero=np.zeros((B, hkv, L), dtype=np.uint16))
     rc = lib().orc_r3_batch(q, k, v, p, float(theta), d, B, S, hq, hkv, float(clip), out["q_out"],
                             out["k_cache"], out["v_cache"], out["k_scale"], out["k_zero"],
-                            out["v_scale"], out["v_zero"], L, cache_offset)
+                            out["v_scale"], out["v_zero"], L, cache_offset, int(threads))
     if rc:
         raise ValueError(f"orc_r3_batch failed ({rc})")
     return out
@@ -390,6 +409,23 @@ def dequant_inverse_row(packed, n, mode, scale, zero=0.0, signs=None, no_rotate=
                                        NO_ROTATE if no_rotate else 0, method, out)
     if rc:
         raise ValueError(f"orc_dequant_inverse_row failed ({rc})")
+    return out
+
+
+def dequant_inverse_rows(packed, n, mode, scale, zero=None, signs=None, no_rotate=False, threads=1):
+    """Rows [rows, n/2] of codes -> [rows, n] fp64 (fast transform), rows over `threads`."""
+    p = np.ascontiguousarray(packed, dtype=np.uint8).reshape(-1, n // 2)
+    rows = p.shape[0]
+    sc = np.ascontiguousarray(scale, dtype=np.float64).ravel()
+    z = None if zero is None else np.ascontiguousarray(zero, dtype=np.float64).ravel()
+    if sc.size != rows or (z is not None and z.size != rows):
+        raise ValueError("one scale (and zero) per row")
+    out = np.empty((rows, n), dtype=np.float64)
+    s = _signs(signs)
+    rc = lib().orc_dequant_inverse_rows(p, rows, n, int(mode), sc, _ptr(z), _ptr(s),
+                                        NO_ROTATE if no_rotate else 0, out, int(threads))
+    if rc:
+        raise ValueError(f"orc_dequant_inverse_rows failed ({rc})")
     return out
 
 

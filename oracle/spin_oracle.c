@@ -367,24 +367,20 @@ double orc_quant_sym_int8(const double *y, int n, double clip, double *pre, int8
   return s;
 }
 
-/* Asymmetric INT4 over one group (reading of "KV cache stored as 4-bit INT4";
- * the pages give no formula): lo = min(clip*min x, 0), hi = max(clip*max x, 0),
- * s = (hi - lo) / 15 rounded to fp16, z = clamp(rne(-lo/s), 0, 15),
- * q = clamp(rne(x/s) + z, 0, 15). A group whose fp16 scale is 0 gets s = 1,
- * z = 0. `pre` (nullable) receives x/s + z before rounding. */
-void orc_quant_asym_int4(const double *x, int n, double clip, double *pre, uint8_t *codes,
-                         uint16_t *s16, uint16_t *z16) {
-  double mn = x[0], mx = x[0];
-  for (int j = 1; j < n; j++) {
-    mn = fmin(mn, x[j]);
-    mx = fmax(mx, x[j]);
-  }
-  double lo = fmin(clip * mn, 0.0), hi = fmax(clip * mx, 0.0);
-  uint16_t sh = orc_f64_to_f16((hi - lo) / 15.0);
-  double s = orc_f16_to_f64(sh);
+/* Codes and zero point of one asymmetric INT4 group for a given fp16 step s16
+ * (the steps of the asymmetric rule that follow the step's rounding):
+ * lo = min(clip*min x, 0), z = clamp(rne(-lo/s), 0, 15), q = clamp(rne(x/s) + z, 0, 15);
+ * a step of 0 becomes s = 1, z = 0. `pre` (nullable) receives x/s + z before rounding.
+ * Returns the fp16 pattern of the step actually used (s16, or 1.0 for a zero step). */
+uint16_t orc_quant_asym_int4_at(const double *x, int n, double clip, uint16_t s16, double *pre,
+                                uint8_t *codes, uint16_t *z16) {
+  double mn = x[0];
+  for (int j = 1; j < n; j++) mn = fmin(mn, x[j]);
+  double lo = fmin(clip * mn, 0.0);
+  double s = orc_f16_to_f64(s16);
   double z;
   if (s == 0.0) {
-    sh = 0x3C00; /* 1.0 */
+    s16 = 0x3C00; /* 1.0 */
     s = 1.0;
     z = 0.0;
   } else {
@@ -395,8 +391,20 @@ void orc_quant_asym_int4(const double *x, int n, double clip, double *pre, uint8
     if (pre) pre[j] = p;
     codes[j] = (uint8_t)clampd(nearbyint(x[j] / s) + z, 0.0, 15.0);
   }
-  *s16 = sh;
   *z16 = orc_f64_to_f16(z);
+  return s16;
+}
+
+double orc_asym_unrounded_scale(const double *x, int n, double clip);
+
+/* Asymmetric INT4 over one group (reading of "KV cache stored as 4-bit INT4";
+ * the pages give no formula): lo = min(clip*min x, 0), hi = max(clip*max x, 0),
+ * s = (hi - lo) / 15 rounded to fp16, then z and the codes as in
+ * orc_quant_asym_int4_at. `pre` (nullable) receives x/s + z before rounding. */
+void orc_quant_asym_int4(const double *x, int n, double clip, double *pre, uint8_t *codes,
+                         uint16_t *s16, uint16_t *z16) {
+  uint16_t sh = orc_f64_to_f16(orc_asym_unrounded_scale(x, n, clip));
+  *s16 = orc_quant_asym_int4_at(x, n, clip, sh, pre, codes, z16);
 }
 
 /* The asymmetric step before its rounding to fp16, (hi - lo) / 15 (used to
@@ -574,21 +582,28 @@ int orc_r3_token(const uint16_t *q, const uint16_t *k, const uint16_t *v, double
 
 /* Whole R3 batch: q [B,S,hq,d], k/v [B,S,hkv,d], pos [B,S]; cache slot of
  * token (b, s) is cache_offset + s; caches are [B, hkv, cache_len, d/2] and
- * scale/zero arrays [B, hkv, cache_len] fp16. q_out [B,S,hq,d] bf16. */
+ * scale/zero arrays [B, hkv, cache_len] fp16. q_out [B,S,hq,d] bf16. Slots
+ * outside [cache_offset, cache_offset + S) are not written. Tokens are
+ * independent and write disjoint slots, so `threads` > 1 spreads them over
+ * OpenMP threads with identical results. */
 int orc_r3_batch(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *pos,
                  double theta, int d, int B, int S, int hq, int hkv, double clip, uint16_t *q_out,
                  uint8_t *k_cache, uint8_t *v_cache, uint16_t *k_scale, uint16_t *k_zero,
-                 uint16_t *v_scale, uint16_t *v_zero, int cache_len, int cache_offset) {
-  uint8_t *kp = (uint8_t *)malloc((size_t)hkv * d / 2), *vp = (uint8_t *)malloc((size_t)hkv * d / 2);
-  uint16_t *ks = (uint16_t *)malloc(2 * (size_t)hkv), *kz = (uint16_t *)malloc(2 * (size_t)hkv);
-  uint16_t *vs = (uint16_t *)malloc(2 * (size_t)hkv), *vz = (uint16_t *)malloc(2 * (size_t)hkv);
+                 uint16_t *v_scale, uint16_t *v_zero, int cache_len, int cache_offset, int threads) {
+  if (cache_offset < 0 || cache_offset + S > cache_len) return -1;
   int rc = 0;
-  for (int b = 0; b < B && rc == 0; b++)
-    for (int s = 0; s < S && rc == 0; s++) {
-      size_t tok = (size_t)b * S + s;
-      rc = orc_r3_token(q + tok * hq * d, k + tok * hkv * d, v + tok * hkv * d, (double)pos[tok],
-                        theta, d, hq, hkv, clip, NULL, q_out + tok * hq * d, NULL, NULL, NULL, kp,
-                        vp, ks, kz, vs, vz);
+#pragma omp parallel for schedule(dynamic, 8) num_threads(threads > 0 ? threads : 1) reduction(| : rc)
+  for (int64_t tok = 0; tok < (int64_t)B * S; tok++) {
+    int b = (int)(tok / S), s = (int)(tok % S);
+    uint8_t *kp = (uint8_t *)malloc((size_t)hkv * d / 2), *vp = (uint8_t *)malloc((size_t)hkv * d / 2);
+    uint16_t *ks = (uint16_t *)malloc(2 * (size_t)hkv), *kz = (uint16_t *)malloc(2 * (size_t)hkv);
+    uint16_t *vs = (uint16_t *)malloc(2 * (size_t)hkv), *vz = (uint16_t *)malloc(2 * (size_t)hkv);
+    int r = (kp && vp && ks && kz && vs && vz) ? 0 : -2;
+    if (r == 0)
+      r = orc_r3_token(q + (size_t)tok * hq * d, k + (size_t)tok * hkv * d, v + (size_t)tok * hkv * d,
+                       (double)pos[tok], theta, d, hq, hkv, clip, NULL, q_out + (size_t)tok * hq * d, NULL,
+                       NULL, NULL, kp, vp, ks, kz, vs, vz);
+    if (r == 0) {
       int slot = cache_offset + s;
       for (int h = 0; h < hkv; h++) {
         size_t row = ((size_t)b * hkv + h) * cache_len + slot;
@@ -600,8 +615,10 @@ int orc_r3_batch(const uint16_t *q, const uint16_t *k, const uint16_t *v, const 
         v_zero[row] = vz[h];
       }
     }
-  free(kp); free(vp); free(ks); free(kz); free(vs); free(vz);
-  return rc;
+    free(kp); free(vp); free(ks); free(kz); free(vs); free(vz);
+    rc |= r;
+  }
+  return rc ? -1 : 0;
 }
 
 /* ------------------------------------------------------------------ */
@@ -641,6 +658,21 @@ int orc_dequant_inverse_row(const uint8_t *packed, int n, int mode, double scale
   }
   free(c); free(v);
   return 0;
+}
+
+/* Many rows through orc_dequant_inverse_row with the fast transform: codes
+ * [rows, n/2], scale [rows] (fp64 values), zero [rows] (mode 1; NULL for mode 0),
+ * out [rows, n] fp64. Rows are independent; `threads` > 1 spreads them over
+ * OpenMP threads with identical results. */
+int orc_dequant_inverse_rows(const uint8_t *packed, int64_t rows, int n, int mode, const double *scale,
+                             const double *zero, const uint32_t *signs, uint32_t flags, double *out,
+                             int threads) {
+  int rc = 0;
+#pragma omp parallel for schedule(dynamic, 16) num_threads(threads > 0 ? threads : 1) reduction(| : rc)
+  for (int64_t r = 0; r < rows; r++)
+    rc |= orc_dequant_inverse_row(packed + r * (n / 2), n, mode, scale[r], zero ? zero[r] : 0.0, signs, flags,
+                                  ORC_METHOD_FWHT, out + r * n);
+  return rc ? -1 : 0;
 }
 
 /* ------------------------------------------------------------------ */

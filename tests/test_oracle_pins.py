@@ -285,6 +285,83 @@ def test_asymmetric_dequant_error_bound(orc):
         assert np.max(np.abs(deq - x)) <= 0.5 * s * 1.02 + abs(z - (-min(x.min(), 0) / s)) * s
 
 
+def test_asymmetric_at_given_step(orc):
+    """The codes-at-a-step half of the asymmetric rule, against numpy's own
+    rounding (rint: half to even) and fp16 conversion: with the rule's step it
+    reproduces the full quantiser; with either fp16 neighbour of the step it gives
+    numpy's codes for that step; a zero step becomes 1 with zero point 0."""
+    rng = np.random.default_rng(31)
+    for clip in (0.95, 1.0):
+        for _ in range(20):
+            x = rng.standard_normal(128) * rng.uniform(0.1, 30) + rng.uniform(-5, 5)
+            codes, s16, z16, pre = orc.quant_asym_int4(x, clip)
+            c2, used, z2, pre2 = orc.quant_asym_int4_at(x, clip, s16)
+            assert used == s16 and z2 == z16 and np.array_equal(codes, c2) and np.array_equal(pre, pre2)
+            lo = min(clip * x.min(), 0.0)
+            for cand in (s16 - 1, s16 + 1):
+                s = float(np.array([cand], dtype=np.uint16).view(np.float16)[0])
+                z = float(np.clip(np.rint(-lo / s), 0, 15)) + 0.0  # a zero point of -0 is stored as +0
+                want = np.clip(np.rint(x / s) + z, 0, 15).astype(np.uint8)
+                c3, used3, z3, pre3 = orc.quant_asym_int4_at(x, clip, cand)
+                assert used3 == cand and np.array_equal(c3, want)
+                assert z3 == int(np.array([z], dtype=np.float16).view(np.uint16)[0])
+                assert np.allclose(pre3, x / s + z, rtol=0, atol=1e-12 * np.abs(x / s).max())
+    c0, used0, z0, _ = orc.quant_asym_int4_at(np.zeros(128), 1.0, 0)
+    assert used0 == 0x3C00 and z0 == 0 and np.all(c0 == 0)
+
+
+def test_r3_batch_scatter_layout(orc):
+    """The batch entry writes token (b, s) to slot cache_offset + s of the
+    [B, hkv, cache_len, d/2] caches and [B, hkv, cache_len] scale/zero arrays
+    (placement computed here with numpy indexing), leaves other slots at zero,
+    and does not depend on the thread count."""
+    B, S, hq, hkv, d = 2, 5, 4, 2, 128
+    q, k, v, _ = synthetic.r3_kv(B, S, hq, hkv, d, seed=41)
+    pos = (np.arange(S)[None, :] * 3 + 7 * np.arange(B)[:, None]).astype(np.int32)
+    off, L = 2, S + 4
+    out = orc.r3_batch(q, k, v, pos, 1e4, 0.95, cache_len=L, cache_offset=off)
+    out4 = orc.r3_batch(q, k, v, pos, 1e4, 0.95, cache_len=L, cache_offset=off, threads=4)
+    for name in out:
+        assert np.array_equal(out[name], out4[name]), name
+    for b in range(B):
+        for s in range(S):
+            r = orc.r3_token(q[b, s], k[b, s], v[b, s], pos[b, s], 1e4, 0.95)
+            assert np.array_equal(out["q_out"][b, s], r["q_bf16"])
+            for h in range(hkv):
+                assert np.array_equal(out["k_cache"][b, h, off + s], r["k_packed"][h])
+                assert np.array_equal(out["v_cache"][b, h, off + s], r["v_packed"][h])
+                assert out["k_scale"][b, h, off + s] == r["k_s"][h] and out["k_zero"][b, h, off + s] == r["k_z"][h]
+                assert out["v_scale"][b, h, off + s] == r["v_s"][h] and out["v_zero"][b, h, off + s] == r["v_z"][h]
+    untouched = np.r_[0:off, off + S:L]
+    for name in ("k_cache", "v_cache", "k_scale", "k_zero", "v_scale", "v_zero"):
+        assert np.all(out[name][:, :, untouched] == 0), name
+    with pytest.raises(ValueError):
+        orc.r3_batch(q, k, v, pos, 1e4, 0.95, cache_len=S, cache_offset=1)
+
+
+def test_dequant_inverse_rows_matches_matrix_product(orc):
+    """Batched inverse = D H_n (code scale) / sqrt(n) per row with scipy's H_n
+    (symmetric codes) and (code - zero) scale without rotation (asymmetric);
+    independent of the thread count."""
+    rng = np.random.default_rng(33)
+    n, rows = 256, 9
+    H = scipy.linalg.hadamard(n) / math.sqrt(n)
+    sg = synthetic.sign_bits(n, 8)
+    d = synthetic.sign_vector(sg, n)
+    codes = rng.integers(-8, 8, size=(rows, n))
+    packed = np.stack([orc.pack_nibbles(c) for c in codes])
+    scale = rng.uniform(0.01, 2.0, rows)
+    out = orc.dequant_inverse_rows(packed, n, 0, scale, signs=sg)
+    ref = (codes * scale[:, None]) @ H.T * d[None, :]
+    assert np.max(np.abs(out - ref)) < 1e-12
+    assert np.array_equal(out, orc.dequant_inverse_rows(packed, n, 0, scale, signs=sg, threads=4))
+    ucodes = rng.integers(0, 16, size=(rows, n))
+    upacked = np.stack([orc.pack_nibbles(c) for c in ucodes])
+    zero = rng.integers(0, 16, rows).astype(np.float64)
+    out = orc.dequant_inverse_rows(upacked, n, 1, scale, zero, no_rotate=True)
+    assert np.array_equal(out, (ucodes - zero[:, None]) * scale[:, None])
+
+
 # --------------------------------------------------------------------------
 # Storage converters: hand-listed bit patterns and library conversions.
 # --------------------------------------------------------------------------
