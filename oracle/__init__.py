@@ -103,6 +103,9 @@ def lib():
     L.orc_dequant_inverse_rows.argtypes = [_u8p, C.c_int64, C.c_int, C.c_int, _dp, vp, vp, C.c_uint32, _dp,
                                            C.c_int]
     L.orc_dequant_inverse_rows.restype = C.c_int
+    L.orc_decode_attention_batch.argtypes = [_u16p, _u8p, _u8p, _u16p, _u16p, _u16p, _u16p, _i32p, C.c_int,
+                                             C.c_int, C.c_int, C.c_int, C.c_int, C.c_double, _dp, C.c_int]
+    L.orc_decode_attention_batch.restype = C.c_int
     L.orc_rmsnorm.argtypes = [_dp, C.c_int, C.c_double, _dp]
     L.orc_mse.argtypes = [_dp, _dp, C.c_int64]
     L.orc_mse.restype = C.c_double
@@ -426,6 +429,28 @@ def dequant_inverse_rows(packed, n, mode, scale, zero=None, signs=None, no_rotat
                                         NO_ROTATE if no_rotate else 0, out, int(threads))
     if rc:
         raise ValueError(f"orc_dequant_inverse_rows failed ({rc})")
+    return out
+
+
+# ---------------------------------------------------------------- decode attention
+def decode_attention(q_bits, cache, lens, softmax_scale=None, threads=1):
+    """One decode step per batch row over the INT4 KV cache: q [B, hq, d] bf16
+    patterns; cache dict of numpy arrays (k_cache, v_cache [B, hkv, L, d/2] uint8;
+    k_scale, k_zero, v_scale, v_zero [B, hkv, L] fp16 patterns); lens [B] slots
+    attended. Returns out [B, hq, d] fp64."""
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    B, hq, d = q.shape
+    kc = np.ascontiguousarray(cache["k_cache"], dtype=np.uint8)
+    hkv, L = kc.shape[1], kc.shape[2]
+    arr = {k: np.ascontiguousarray(cache[k]).view(np.uint16) for k in ("k_scale", "k_zero", "v_scale", "v_zero")}
+    ln = np.ascontiguousarray(np.broadcast_to(np.asarray(lens, dtype=np.int32), (B,)))
+    out = np.empty((B, hq, d), dtype=np.float64)
+    sc = 1.0 / np.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    rc = lib().orc_decode_attention_batch(q, kc, np.ascontiguousarray(cache["v_cache"], dtype=np.uint8),
+                                          arr["k_scale"], arr["k_zero"], arr["v_scale"], arr["v_zero"], ln, B, hq,
+                                          hkv, d, L, sc, out, int(threads))
+    if rc:
+        raise ValueError(f"orc_decode_attention_batch failed ({rc})")
     return out
 
 

@@ -676,6 +676,85 @@ int orc_dequant_inverse_rows(const uint8_t *packed, int64_t rows, int n, int mod
 }
 
 /* ------------------------------------------------------------------ */
+/* Decode attention over the 4-bit KV cache ["SpinQuant Guide", the KV4 */
+/* serving diagram: rotated keys stored in the cache as INT4, then a     */
+/* "Fused INT4 Dot Product" with the rotated queries; "SpinQuant: rotate */
+/* before you round", "Deployment implications": a rotation only pays   */
+/* once the runtime has KV4 kernels]                                    */
+/* ------------------------------------------------------------------ */
+
+/* One decode step of one batch row. q: [hq][d] bf16 bit patterns (queries after
+ * RoPE and R3, as the R3 kernel writes them). Cache of one batch row: k_codes,
+ * v_codes [hkv][cache_len][d/2] (unsigned nibbles, element 2j low), k_s, k_z,
+ * v_s, v_z [hkv][cache_len] fp16 patterns; slots 0 .. len-1 are attended.
+ * Query head h reads kv head h / (hq / hkv). In fp64, plainly:
+ *   khat_j = (code - z) s,  score_j = (q . khat_j) * softmax_scale,
+ *   p = exp(score - max score) / sum,  out_h = sum_j p_j vhat_j.
+ * Since R3 rotates q and k by the same orthogonal H/sqrt(d), q . k is the
+ * unrotated product; V is not rotated, so out is in the value basis.
+ * out: [hq][d] fp64. Returns 0, or -1 for bad sizes. */
+int orc_decode_attention(const uint16_t *q, const uint8_t *k_codes, const uint8_t *v_codes,
+                         const uint16_t *k_s, const uint16_t *k_z, const uint16_t *v_s, const uint16_t *v_z,
+                         int hq, int hkv, int d, int cache_len, int len, double softmax_scale, double *out) {
+  if (hq <= 0 || hkv <= 0 || hq % hkv != 0 || d < 2 || (d & 1) || len <= 0 || len > cache_len) return -1;
+  double *sc = (double *)malloc(sizeof(double) * (size_t)len);
+  double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+  int32_t *c = (int32_t *)malloc(sizeof(int32_t) * (size_t)d);
+  if (!sc || !qd || !c) {
+    free(sc); free(qd); free(c);
+    return -2;
+  }
+  const int group = hq / hkv;
+  for (int h = 0; h < hq; h++) {
+    const int g = h / group;
+    for (int i = 0; i < d; i++) qd[i] = orc_bf16_to_f64(q[(size_t)h * d + i]);
+    double mx = -INFINITY;
+    for (int j = 0; j < len; j++) {
+      const size_t row = (size_t)g * cache_len + j;
+      orc_unpack_nibbles(k_codes + row * (d / 2), d, 0, c);
+      const double s = orc_f16_to_f64(k_s[row]), z = orc_f16_to_f64(k_z[row]);
+      double dot = 0.0;
+      for (int i = 0; i < d; i++) dot += qd[i] * (((double)c[i] - z) * s);
+      sc[j] = dot * softmax_scale;
+      if (sc[j] > mx) mx = sc[j];
+    }
+    double den = 0.0;
+    for (int j = 0; j < len; j++) {
+      sc[j] = exp(sc[j] - mx);
+      den += sc[j];
+    }
+    for (int i = 0; i < d; i++) out[(size_t)h * d + i] = 0.0;
+    for (int j = 0; j < len; j++) {
+      const size_t row = (size_t)g * cache_len + j;
+      orc_unpack_nibbles(v_codes + row * (d / 2), d, 0, c);
+      const double s = orc_f16_to_f64(v_s[row]), z = orc_f16_to_f64(v_z[row]);
+      const double p = sc[j] / den;
+      for (int i = 0; i < d; i++) out[(size_t)h * d + i] += p * (((double)c[i] - z) * s);
+    }
+  }
+  free(sc); free(qd); free(c);
+  return 0;
+}
+
+/* Batch of decode steps: q [B][hq][d]; caches [B][hkv][cache_len][d/2] and
+ * [B][hkv][cache_len]; lens [B] (slots attended per batch row); out [B][hq][d].
+ * Rows are independent; `threads` > 1 spreads them over OpenMP threads. */
+int orc_decode_attention_batch(const uint16_t *q, const uint8_t *k_codes, const uint8_t *v_codes,
+                               const uint16_t *k_s, const uint16_t *k_z, const uint16_t *v_s,
+                               const uint16_t *v_z, const int32_t *lens, int B, int hq, int hkv, int d,
+                               int cache_len, double softmax_scale, double *out, int threads) {
+  int rc = 0;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(threads > 0 ? threads : 1) reduction(| : rc)
+  for (int b = 0; b < B; b++) {
+    const size_t cb = (size_t)b * hkv * cache_len;
+    rc |= orc_decode_attention(q + (size_t)b * hq * d, k_codes + cb * (d / 2), v_codes + cb * (d / 2),
+                               k_s + cb, k_z + cb, v_s + cb, v_z + cb, hq, hkv, d, cache_len, lens[b],
+                               softmax_scale, out + (size_t)b * hq * d);
+  }
+  return rc ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* Self-test helpers: RMSNorm [SW "The math, slowly"; RQ "Computational */
 /* invariance"]                                                         */
 /* ------------------------------------------------------------------ */

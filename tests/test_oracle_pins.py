@@ -13,6 +13,7 @@ import os
 import numpy as np
 import pytest
 import scipy.linalg
+import scipy.special
 import torch
 
 import synthetic
@@ -655,3 +656,82 @@ def test_r4_kron_one_hot_at_llama3_width(orc):
     assert np.allclose(np.abs(r["y"]), 5.0 / math.sqrt(n), rtol=1e-14)
     assert np.all(np.abs(r["codes"]) == 7)
     assert r["scale64"] == pytest.approx(5.0 / math.sqrt(n) / 7, rel=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Decode attention over the INT4 KV cache -- "SpinQuant Guide: Learned
+# Rotations for 4-Bit LLMs", the KV4 serving diagram (rotated keys stored as
+# 4-bit INT4, then a fused INT4 dot product with the rotated queries);
+# attention itself is the textbook softmax(q k^T / sqrt(d)) v.
+# --------------------------------------------------------------------------
+def _random_cache(rng, B, hkv, L, d):
+    f16 = lambda a: np.asarray(a, dtype=np.float16).view(np.uint16)
+    return dict(k_cache=rng.integers(0, 256, (B, hkv, L, d // 2), dtype=np.uint8),
+                v_cache=rng.integers(0, 256, (B, hkv, L, d // 2), dtype=np.uint8),
+                k_scale=f16(rng.uniform(0.01, 0.3, (B, hkv, L))), k_zero=f16(rng.integers(0, 16, (B, hkv, L))),
+                v_scale=f16(rng.uniform(0.01, 0.3, (B, hkv, L))), v_zero=f16(rng.integers(0, 16, (B, hkv, L))))
+
+
+def _dequant_numpy(codes, scale, zero):
+    c = np.empty(codes.shape[:-1] + (2 * codes.shape[-1],), dtype=np.float64)
+    c[..., 0::2] = codes & 0xF
+    c[..., 1::2] = codes >> 4
+    s = scale.view(np.float16).astype(np.float64)[..., None]
+    z = zero.view(np.float16).astype(np.float64)[..., None]
+    return (c - z) * s
+
+
+def test_decode_attention_matches_numpy_softmax(orc):
+    """Against numpy dequantisation and scipy's softmax on the same cache, with
+    grouped query heads (head h reads kv head h // (hq / hkv)) and per-row lengths."""
+    import scipy.special
+    rng = np.random.default_rng(51)
+    B, hq, hkv, d, L = 3, 8, 2, 128, 37
+    cache = _random_cache(rng, B, hkv, L, d)
+    q = bf16(rng.standard_normal((B, hq, d)).astype(np.float32) * 2)
+    lens = np.array([37, 1, 20], dtype=np.int32)
+    out = orc.decode_attention(q, cache, lens)
+    K = _dequant_numpy(cache["k_cache"], cache["k_scale"], cache["k_zero"])
+    V = _dequant_numpy(cache["v_cache"], cache["v_scale"], cache["v_zero"])
+    qf = synthetic.bf16_bits_to_f32(q).astype(np.float64)
+    for b in range(B):
+        for h in range(hq):
+            g = h // (hq // hkv)
+            p = scipy.special.softmax(K[b, g, :lens[b]] @ qf[b, h] / math.sqrt(d))
+            assert np.max(np.abs(out[b, h] - p @ V[b, g, :lens[b]])) < 1e-12
+    assert np.array_equal(out, orc.decode_attention(q, cache, lens, threads=3))
+
+
+def test_decode_attention_special_cases(orc):
+    """One attended slot returns its value row exactly; a zero query weighs every
+    slot equally (the mean of the value rows); slots past the length are ignored."""
+    rng = np.random.default_rng(52)
+    B, hq, hkv, d, L = 1, 4, 4, 128, 16
+    cache = _random_cache(rng, B, hkv, L, d)
+    V = _dequant_numpy(cache["v_cache"], cache["v_scale"], cache["v_zero"])
+    q = bf16(rng.standard_normal((B, hq, d)).astype(np.float32))
+    one = orc.decode_attention(q, cache, [1])
+    assert np.array_equal(one[0], V[0, :, 0])
+    zero_q = np.zeros((B, hq, d), dtype=np.uint16)
+    mean = orc.decode_attention(zero_q, cache, [L])
+    assert np.max(np.abs(mean[0] - V[0].mean(axis=1))) < 1e-12
+    short = orc.decode_attention(q, cache, [9])
+    cache2 = {k: v.copy() for k, v in cache.items()}
+    cache2["k_cache"][:, :, 9:] ^= 0x5A
+    cache2["v_cache"][:, :, 9:] ^= 0xA5
+    assert np.array_equal(short, orc.decode_attention(q, cache2, [9]))
+
+
+def test_decode_attention_scores_survive_r3(orc):
+    """R3 rotates q and k by the same orthogonal H/sqrt(d): the attention over a
+    cache of H-rotated keys with H-rotated queries equals the attention over the
+    unrotated keys and queries (values unrotated), to fp64 rounding."""
+    rng = np.random.default_rng(53)
+    d, L = 128, 24
+    H = scipy.linalg.hadamard(d) / math.sqrt(d)
+    k = rng.standard_normal((L, d))
+    v = rng.standard_normal((L, d))
+    q = rng.standard_normal(d)
+    ref = scipy.special.softmax(k @ q / math.sqrt(d)) @ v
+    rot = scipy.special.softmax((k @ H.T) @ (H @ q) / math.sqrt(d)) @ v
+    assert np.max(np.abs(ref - rot)) < 1e-12
