@@ -25,6 +25,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -43,8 +44,11 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 def metric_for(wl) -> str:
-    """The headline metric, or its INT8 counterpart for the INT8 workload."""
-    return METRIC.replace("INT4", "INT8") if wl.get("code_bits", 4) == 8 else METRIC
+    """The headline metric, or its counterpart for the INT8 and Kronecker-size workloads."""
+    m = METRIC.replace("INT4", "INT8") if wl.get("code_bits", 4) == 8 else METRIC
+    if wl.get("kron_m"):
+        m = m.replace("at n=16384", f"at n={wl['bits'].shape[1]} (H_{wl['kron_m']} Paley x Sylvester)")
+    return m
 
 
 def algorithmic_bytes_r4(tokens: int, n: int, code_bits: int = 4) -> int:
@@ -52,9 +56,13 @@ def algorithmic_bytes_r4(tokens: int, n: int, code_bits: int = 4) -> int:
     return tokens * (2 * n + n * code_bits // 8 + 4)
 
 
-def oracle_r4_rows(oracle, bits, clip, signs, code_bits, threads=1) -> int:
-    """The oracle over rows: its C loop for INT4 (rows spread over `threads`), one call
-    per row for INT8 (one thread). Returns the threads used."""
+def oracle_r4_rows(oracle, bits, clip, signs, code_bits, threads=1, kron_m=None) -> int:
+    """The oracle over rows: its C loop for INT4 (rows spread over `threads`; the
+    Kronecker loop for n = m 2^k), one call per row for INT8 (one thread). Returns
+    the threads used."""
+    if kron_m:
+        oracle.r4_rows_kron(bits, kron_m, clip, signs, threads=threads)
+        return threads
     if code_bits == 4:
         oracle.r4_rows(bits, clip, signs, threads=threads)
         return threads
@@ -205,6 +213,14 @@ def make_workload(name: str, rank: int, tokens: int | None = None):
                                       "seeded +-1 diagonal, H_16384 = H_128 (x) H_128, clip 0.9"
                                       + (", per-token INT8 codes" if code_bits == 8 else ""),
                           "tokens": int(bits.shape[0]), "n": int(bits.shape[1])})
+    if name.startswith("kron"):
+        n = int(name[len("kron"):] or 14336)
+        m = {14336: 28, 6144: 12, 10240: 20, 12288: 12}[n]
+        bits, signs, _ = synthetic.r4_prefill(tokens=tokens or 8192, n=n, seed=1 + rank)
+        return dict(kind="r4", bits=bits, signs=signs, clip=0.9, code_bits=4, kron_m=m,
+                    desc={"workload": f"R4 prefill at n={n} = {m} x {n // m} (H_{m} Paley (x) H_{n // m}): "
+                                      f"{bits.shape[0]} tokens, SwiGLU-like bf16, 0.1% channels x100, seeded +-1 "
+                                      "diagonal, clip 0.9", "tokens": int(bits.shape[0]), "n": n, "m": m})
     if name.startswith("decode"):
         n = int(name[len("decode"):] or 16384)
         bits = synthetic.decode(tokens or 32, n, seed=3 + rank)
@@ -250,10 +266,10 @@ def run_reference(args, wl):
     rows = bits[:sample]
     threads = oracle.max_threads()  # the host's cores
     for _ in range(args.warmup):
-        oracle_r4_rows(oracle, rows[:1], wl["clip"], wl["signs"], wl["code_bits"], threads)
+        oracle_r4_rows(oracle, rows[:1], wl["clip"], wl["signs"], wl["code_bits"], threads, wl.get("kron_m"))
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        cores = oracle_r4_rows(oracle, rows, wl["clip"], wl["signs"], wl["code_bits"], threads)
+        cores = oracle_r4_rows(oracle, rows, wl["clip"], wl["signs"], wl["code_bits"], threads, wl.get("kron_m"))
     dt = time.perf_counter() - t0
     tok_s = args.steps * sample / dt
     gbs = algorithmic_bytes_r4(sample, n, wl["code_bits"]) * args.steps / dt / 1e9
@@ -269,31 +285,177 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline_leg(wl) -> dict:
+def cpu_baseline_leg(wl):
     """The fp64 oracle on this host over the workload's rows (all of them from
     n = 4096 up, else at most 65536): one pass on one thread, and one pass with the
-    rows spread over the host's cores."""
+    rows spread over the host's cores. Returns the baseline record and, for the
+    spot check of the GPU's last timed step, (oracle module, packed codes, steps,
+    rows) of the all-cores pass (INT4 workloads)."""
     import oracle
     oracle.lib()
     bits = wl["bits"]
     sample = bits.shape[0] if bits.shape[1] >= 4096 else min(bits.shape[0], 65536)
     cpu_bytes = algorithmic_bytes_r4(sample, bits.shape[1], wl["code_bits"])
     t0 = time.perf_counter()
-    oracle_r4_rows(oracle, bits[:sample], wl["clip"], wl["signs"], wl["code_bits"])
+    oracle_r4_rows(oracle, bits[:sample], wl["clip"], wl["signs"], wl["code_bits"], kron_m=wl.get("kron_m"))
     dt = time.perf_counter() - t0
     cpu = {"value": cpu_bytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle", "tokens_per_s": sample / dt,
            "sample": f"{sample} of {bits.shape[0]} tokens, one pass, fp64 fast transform, 1 thread"}
+    ref = None
     t0 = time.perf_counter()
-    used = oracle_r4_rows(oracle, bits[:sample], wl["clip"], wl["signs"], wl["code_bits"], oracle.max_threads())
+    if wl.get("kron_m"):
+        used = oracle.max_threads()
+        packed, scales = oracle.r4_rows_kron(bits[:sample], wl["kron_m"], wl["clip"], wl["signs"], threads=used)
+        ref = (oracle, packed, scales.astype(np.float64), sample)
+    elif wl["code_bits"] == 4:
+        used = oracle.max_threads()
+        packed, scales = oracle.r4_rows(bits[:sample], wl["clip"], wl["signs"], threads=used)
+        ref = (oracle, packed, scales.astype(np.float64), sample)
+    else:
+        used = oracle_r4_rows(oracle, bits[:sample], wl["clip"], wl["signs"], wl["code_bits"], oracle.max_threads())
     dt = time.perf_counter() - t0
     cpu["all_cores"] = {"value": cpu_bytes / dt / 1e9, "unit": "GB/s", "cores": used, "tokens_per_s": sample / dt,
                         "sample": "the same rows, spread over the host's cores"}
-    return cpu
+    return cpu, ref
 
 
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+def timed_windows(step, steps, stream, dev, world, min_seconds, first=0):
+    """Device time of windows of exactly `steps` calls of step(i), each window
+    bracketed by a barrier (N > 1) and a device synchronisation, timed with CUDA
+    events on `stream` and reduced to the maximum over ranks. Windows repeat until
+    about `min_seconds` of device time is sampled (the count is fixed after the first
+    window from its max-over-ranks time, so every rank runs the same number).
+    Returns the list of window times in ms."""
+    import torch
+    import torch.distributed as dist
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    windows, target, i = [], None, first
+    while target is None or len(windows) < target:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(steps):
+            step(i)
+            i += 1
+        ev1.record(stream)
+        ev1.synchronize()
+        torch.cuda.synchronize()
+        ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
+        windows.append(ms)
+        if target is None:
+            target = windows_needed(ms, min_seconds)
+    return windows
+
+
+def windows_needed(first_ms: float, min_seconds: float) -> int:
+    """Windows to time so that about `min_seconds` of device time is sampled,
+    from the first window's (max-over-ranks) time; between 1 and 400."""
+    return max(1, min(400, math.ceil(min_seconds * 1e3 / max(first_ms, 1e-3))))
+
+
+def require_clean_status(spin, what):
+    """The library's device status word must be zero after a timed loop: a kernel
+    that gave up on a bounded wait stops early and would time as a faster run."""
+    import torch
+    torch.cuda.synchronize()
+    st = spin.device_status(reset=True)
+    if st:
+        raise SystemExit(f"{what}: the device status word is {st:#x} (a kernel stopped early); no number reported")
+
+
+def window_stats(windows, steps):
+    med = statistics.median(windows)
+    return med / steps, {"count": len(windows), "steps_each": steps, "ms_min": min(windows), "ms_median": med,
+                         "ms_max": max(windows), "device_seconds": sum(windows) / 1e3}
+
+
+def spot_check(oracle, wl, packed_ref, scales_ref, q_dev, s_dev, rows):
+    """The GPU's codes and steps of `rows` (last timed step) against the oracle's
+    batch output for the same rows: steps within 1e-5 relative; rows whose bytes
+    differ are re-run through the single-row oracle, and every differing code must
+    be one step away with the oracle's pre-round value within 1e-3 of a .5 tie."""
+    q = q_dev[:rows].cpu().numpy()
+    s = s_dev[:rows].cpu().numpy()
+    rel = np.abs(s.astype(np.float64) - scales_ref) / np.abs(scales_ref)
+    ok = bool(np.all(rel <= 1e-5))
+    diff_rows = np.nonzero((q != packed_ref).any(axis=1))[0]
+    bad_codes = 0
+    n = wl["bits"].shape[1]
+    for t in diff_rows[:4096]:
+        if wl.get("kron_m"):
+            r = oracle.r4_row_kron(wl["bits"][t], wl["kron_m"], wl["clip"], signs=wl["signs"])
+        else:
+            r = oracle.r4_row(wl["bits"][t], wl["clip"], signs=wl["signs"])
+        g = q[t].astype(np.int32)
+        c = np.empty(n, np.int32)
+        c[0::2], c[1::2] = g & 0xF, g >> 4
+        c = np.where(c >= 8, c - 16, c)
+        d = c != r["codes"]
+        pre = r["pre"][d]
+        frac = np.abs(pre - np.floor(pre) - 0.5)
+        bad_codes += int(np.sum(~((frac <= 1e-3) & (np.abs(c[d] - r["codes"][d]) == 1))))
+    ok = ok and bad_codes == 0 and len(diff_rows) <= 4096
+    return {"rows": int(rows), "rows_bit_identical": int(rows - len(diff_rows)),
+            "rows_with_tie_band_codes": int(len(diff_rows)), "codes_outside_tie_band": bad_codes,
+            "max_step_rel_err": float(rel.max()), "ok": ok}
+
+
+def extra_workloads(spin, dev, world, rank, stream, args, peak):
+    """Compact measurements of the other throughput workloads, carried in the
+    default line: the 1 GiB sweeps at n = 4096 .. 32768 (the n >= 4096 target) and
+    R3 + KV. Same timing method as the headline, about 0.25 s of device time each."""
+    import torch
+    out = {"sweep": [], "r3_kv": None}
+    for k in (12, 13, 14, 15):
+        wl = make_workload(f"sweep{k}", rank)
+        n, tokens = 1 << k, wl["bits"].shape[0]
+        x = torch.from_numpy(wl["bits"].view(np.int16)).view(torch.bfloat16).to(dev)
+        del wl
+        q = torch.empty((tokens, n // 2), dtype=torch.uint8, device=dev)
+        s = torch.empty((tokens,), dtype=torch.float32, device=dev)
+
+        def step(i):
+            spin.hadamard_quant_int4(x, 1.0, None, out=q, scales=s, stream=stream)
+
+        for i in range(args.warmup):
+            step(i)
+        windows = timed_windows(step, args.steps, stream, dev, world, 0.25)
+        require_clean_status(spin, f"sweep n={n}")
+        ms, _ = window_stats(windows, args.steps)
+        gbs = algorithmic_bytes_r4(tokens, n) / (ms / 1e3) / 1e9
+        out["sweep"].append({"n": n, "tokens": tokens, "kernel": r4_kernel_name(n, tokens, False),
+                             "ms_per_step": ms, "achieved_gbs": gbs * world, "frac": gbs / peak,
+                             "windows": len(windows)})
+        del x, q, s
+    wl = make_workload("r3_kv", rank)
+    qh, kh, vh, pos = wl["q"], wl["k"], wl["v"], wl["pos"]
+    B, S, hq, d = qh.shape
+    hkv = kh.shape[2]
+    t = {name: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+         for name, a in (("q", qh), ("k", kh), ("v", vh))}
+    pos_d = torch.from_numpy(pos).to(dev)
+    qo = torch.empty((B, S, hq, d), dtype=torch.bfloat16, device=dev)
+    cache = spin.alloc_kv_cache(B, hkv, S, d, device=dev)
+
+    def r3_step(i):
+        spin.rope_hadamard_kvquant(t["q"], t["k"], t["v"], pos_d, cache, clip=wl["clip"], q_out=qo, stream=stream)
+
+    for i in range(args.warmup):
+        r3_step(i)
+    windows = timed_windows(r3_step, args.steps, stream, dev, world, 0.25)
+    require_clean_status(spin, "R3 + KV")
+    ms, _ = window_stats(windows, args.steps)
+    gbs = r3_bytes(B * S, hq, hkv, d) / (ms / 1e3) / 1e9
+    out["r3_kv"] = {"kernel": "k2_rope_hadamard_kvquant", "tokens": B * S, "ms_per_step": ms,
+                    "achieved_gbs": gbs * world, "frac": gbs / peak, "tokens_per_s": world * B * S / (ms / 1e3),
+                    "windows": len(windows)}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -302,6 +464,10 @@ def main():
     ap.add_argument("--impl", default="spin", choices=["spin", "reference"])
     ap.add_argument("--workload", default="r4_prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="leave out the sweep and R3 + KV sub-measurements of the default line")
+    ap.add_argument("--min-seconds", type=float, default=0.5,
+                    help="repeat the timed window of --steps steps until this much device time is sampled")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's token count (R4 workloads; smaller cases for profiling)")
     args = ap.parse_args()
@@ -331,6 +497,7 @@ def main():
     from online_hadamard_rotation_b200 import build
     build.build()
     spin.lib()
+    spin.device_status(reset=True)
 
     wl = make_workload(args.workload, rank, args.tokens)
     stream = torch.cuda.Stream(dev)
@@ -341,6 +508,9 @@ def main():
         code_bits = wl["code_bits"]
         qshape, qtype = ((tokens, n // 2), torch.uint8) if code_bits == 4 else ((tokens, n), torch.int8)
         quant = spin.hadamard_quant_int4 if code_bits == 4 else spin.hadamard_quant_int8
+        if "kron_m" in wl:
+            def quant(x, clip, signs, out, scales, stream, cuda_cores_only=False):  # noqa: F811
+                return spin.hadamard_quant_kron(x, wl["kron_m"], clip, signs, out=out, scales=scales, stream=stream)
         sets = []
         for _ in range(2):
             sets.append(dict(x=host.to(dev), q=torch.empty(qshape, dtype=qtype, device=dev),
@@ -375,68 +545,54 @@ def main():
     for i in range(args.warmup):
         step(i)
     stream.synchronize()
+    require_clean_status(spin, "warm-up")
 
-    # ---- device-timed region: inputs resident in HBM
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
+    # ---- device-timed region: inputs resident in HBM; windows of exactly --steps steps
     with ClockSampler(local_rank) as clocks:
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        ev1.record(stream)
-        ev1.synchronize()
-    torch.cuda.synchronize()
-    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
+        windows = timed_windows(step, args.steps, stream, dev, world, args.min_seconds)
+    require_clean_status(spin, "timed region")
+    ms_per_step, window_info = window_stats(windows, args.steps)
+    last = sets[(args.steps * len(windows) - 1) & 1]  # buffers of the last timed step, kept for the spot check
+    last = {"q": last["q"].clone(), "s": last["s"].clone()} if wl["kind"] == "r4" else None
     if world > 1:
         dist.barrier()
-    ms_per_step = ms / args.steps
-    gbs, tok_s = aggregate(world, step_bytes, tokens, args.steps, ms)
+    gbs, tok_s = aggregate(world, step_bytes, tokens, args.steps, ms_per_step * args.steps)
 
-    # ---- end to end through the public API from pinned host memory
+    # ---- end to end through the public API from pinned host memory: the batch in
+    # eight slices whose copy in, kernel and copy out overlap on three streams
     e2e = None
     if wl["kind"] == "r4":
-        q_host = torch.empty(qshape, dtype=qtype).pin_memory()
-        s_host = torch.empty((tokens,), dtype=torch.float32).pin_memory()
-        b = sets[0]
         e2e_steps = max(3, args.steps // 5)
-
-        def e2e_step():
-            with torch.cuda.stream(stream):
-                b["x"].copy_(host, non_blocking=True)
-                quant(b["x"], wl["clip"], signs, out=b["q"], scales=b["s"], stream=stream)
-                q_host.copy_(b["q"], non_blocking=True)
-                s_host.copy_(b["s"], non_blocking=True)
-
+        bufs = None
         for _ in range(2):
-            e2e_step()
-        stream.synchronize()
+            _, _, bufs = spin.hadamard_quant_host(host, wl["clip"], signs, code_bits, dev, stream, bufs,
+                                                  m=wl.get("kron_m"))
         if world > 1:
             dist.barrier()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev0.record(stream)
         for _ in range(e2e_steps):
-            e2e_step()
+            q_host, s_host, bufs = spin.hadamard_quant_host(host, wl["clip"], signs, code_bits, dev, stream, bufs,
+                                                            m=wl.get("kron_m"))
         ev1.record(stream)
         ev1.synchronize()
+        require_clean_status(spin, "end-to-end leg")
         ems = max_over_ranks(ev0.elapsed_time(ev1), dev)
         e_gbs, e_tok = aggregate(world, step_bytes, tokens, e2e_steps, ems)
         e2e = {"value": e_gbs, "unit": "GB/s", "tokens_per_s": e_tok,
                "h2d_bytes_per_step": int(host.numel() * 2), "d2h_bytes_per_step": int(q_host.numel() + 4 * tokens),
-               "steps": e2e_steps}
+               "steps": e2e_steps, "pipeline": "8 token slices, copy in / kernel / copy out on three streams"}
+        del bufs
 
     # ---- the same steps on the all-CUDA-core kernel, for comparison (not the headline)
     cores = None
-    if wl["kind"] == "r4" and r4_kernel_name(n, tokens, wl["signs"] is not None) == "k1_tc_rotate_quant":
+    if wl["kind"] == "r4" and "kron_m" not in wl and \
+            r4_kernel_name(n, tokens, wl["signs"] is not None) == "k1_tc_rotate_quant":
         for i in range(args.warmup):
             step(i, True)
-        stream.synchronize()
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(i, True)
-        ev1.record(stream)
-        ev1.synchronize()
-        cms = ev0.elapsed_time(ev1) / args.steps
+        cwin = timed_windows(lambda i: step(i, True), args.steps, stream, dev, world, 0.1)
+        require_clean_status(spin, "CUDA-core comparison leg")
+        cms, _ = window_stats(cwin, args.steps)
         cores = {"kernel": f"k1_rotate_quant_int{code_bits} (all butterflies on CUDA cores)", "ms_per_step": cms,
                  "achieved_gbs": step_bytes / (cms / 1e3) / 1e9}
 
@@ -455,13 +611,9 @@ def main():
 
         for _ in range(args.warmup):
             inverse(b["q"], b["s"])
-        stream.synchronize()
-        ev0.record(stream)
-        for _ in range(args.steps):
-            inverse(b["q"], b["s"])
-        ev1.record(stream)
-        ev1.synchronize()
-        rms = max_over_ranks(ev0.elapsed_time(ev1), dev) / args.steps
+        rwin = timed_windows(lambda i: inverse(b["q"], b["s"]), args.steps, stream, dev, world, 0.25)
+        require_clean_status(spin, "round trip")
+        rms, _ = window_stats(rwin, args.steps)
         rt_bytes = tokens * (n // 2 + 4 + 2 * n)
         x32 = b["x"].float()
         mse = {}
@@ -488,6 +640,7 @@ def main():
         for _ in range(10):
             step(0)
         stream.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev0.record(stream)
         for _ in range(calls):
             step(0)
@@ -510,11 +663,14 @@ def main():
         ev1.synchronize()
         graph_us = ev0.elapsed_time(ev1) / calls * 1e3
         del graph
+        require_clean_status(spin, "decode latency")
         latency = {"us_per_call_plain": plain_us, "us_per_call_graph": graph_us, "calls": calls,
                    "note": "inputs are L2-resident at this size (1.3 MB or less)"}
 
     peak, peak_kind = measured_peaks()
-    if wl["kind"] == "r4":
+    if wl["kind"] == "r4" and "kron_m" in wl:
+        kname = "k1_tc_rotate_quant"
+    elif wl["kind"] == "r4":
         kname = r4_kernel_name(n, tokens, wl["signs"] is not None, wl["code_bits"])
     else:
         kname = "k2_rope_hadamard_kvquant"
@@ -525,9 +681,17 @@ def main():
                 "algorithmic_bytes_per_launch": step_bytes,
                 "peak_source": f"{peak_kind} hbm_gbs (STREAM-style copy)"}
 
+    extras = None
+    if args.workload == "r4_prefill" and not args.no_extras and args.tokens is None:
+        extras = extra_workloads(spin, dev, world, rank, stream, args, peak)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and wl["kind"] == "r4":
-        cpu = cpu_baseline_leg(wl)
+        cpu, ref_out = cpu_baseline_leg(wl)
+        cpu["spot_check"] = (spot_check(ref_out[0], wl, ref_out[1], ref_out[2], last["q"], last["s"], ref_out[3])
+                             if ref_out is not None else None)
+        if cpu["spot_check"] is not None and not cpu["spot_check"]["ok"]:
+            raise SystemExit(f"the last timed step disagrees with the oracle: {cpu['spot_check']}")
 
     if rank == 0:
         line = {"metric": metric_for(wl), "value": gbs, "unit": "GB/s", "tokens_per_s": tok_s,
@@ -535,9 +699,9 @@ def main():
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": config_for(wl, world, args.workload),
-                "gpu_launches": args.steps, "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu,
-                "cuda_core_kernel": cores, "decode_latency": latency, "round_trip": round_trip,
-                "clocks": clocks.summary()}
+                "gpu_launches": args.steps, "timed_windows": window_info, "e2e": e2e, "roofline": roofline,
+                "cpu_baseline": cpu, "cuda_core_kernel": cores, "decode_latency": latency,
+                "round_trip": round_trip, "other_workloads": extras, "clocks": clocks.summary()}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -6,7 +6,9 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  * Pointers are device pointers the caller owns (allocated by any means).
- *    The library allocates, frees and synchronises nothing; it never blocks.
+ *    The library allocates, frees and synchronises nothing, and no entry
+ *    point blocks, with one exception: spin_device_status() reads the
+ *    device status word synchronously (see there).
  *  * Each call validates its arguments on the host, then enqueues its kernels
  *    on `stream` (a cudaStream_t; NULL is the legacy default stream) and
  *    returns. A non-SPIN_OK status means nothing was enqueued, except
@@ -157,6 +159,39 @@ spin_status_t spin_hadamard_quant_int8(const void *x_bf16, int64_t tokens, int32
                                        float *scales_f32, spin_stream_t stream);
 
 /*
+ * R4 for a row length that is not a power of two, n = m b with b = 2^k
+ * ("Rotations: QuaRot, SpinQuant and incoherence", section "Hadamard matrices":
+ * other sizes use a Kronecker product of a Sylvester matrix with a small known
+ * Hadamard matrix). The pages name no small matrix; H_m here is Paley's
+ * construction from the quadratic character chi mod a prime q, with the core
+ * matrix C of order q + 1: C[0][0] = 0, C[0][j] = 1, C[i][j] = chi(j - i) for
+ * i, j > 0, and C[i][0] = -1 (type I) or +1 (type II).
+ *   type I  (q = m - 1 prime, q = 3 mod 4):        H_m = C + I
+ *   type II (q = m/2 - 1 prime, q = 1 mod 4, and m - 1 not a type I prime):
+ *           H_m = C (x) [[1, -1], [-1, -1]] + I (x) [[1, 1], [1, -1]]
+ * For each of `tokens` rows x (element e = b i + j: i < m indexes H_m, j < b the
+ * Sylvester H_b; the diagonal D comes first, as for powers of two):
+ *   y = (H_m (x) H_b) D x / sqrt(n), then the per-token rule of
+ *   spin_hadamard_quant_int4 (bits = 4) or spin_hadamard_quant_int8 (bits = 8).
+ *
+ *  x_bf16     [tokens, n] bf16, 16-byte aligned
+ *  m          order of H_m: one with a Paley form (12, 20, 24, 28, 44, 48, ...)
+ *  n          m b with b a power of two >= 128 and n / 128 a multiple of 16, at most
+ *             128 (n = 6144, 10240, 12288 or 14336 for m = 12, 20, 12 or 28, ...);
+ *             tokens * n / 128 < 2^31
+ *  sign_bits  nullable, [ceil(n/32)] words, bit e set => d_e = -1, 4-byte aligned
+ *  flags      0 or SPIN_TENSOR_CORES (one kernel, on the tensor cores, for every batch)
+ *  bits       4: q is [tokens, n/2] packed INT4 bytes; 8: q is [tokens, n] int8 codes
+ *  q          16-byte aligned, written; scales_f32 [tokens] fp32, 4-byte aligned, written
+ * Errors: SPIN_ERR_UNSUPPORTED_SIZE ((m, n) outside the above), SPIN_ERR_INVALID_ARG
+ * (null pointer with tokens > 0, tokens < 0, clip outside (0, 1], bits not 4 or 8,
+ * other flag bits), SPIN_ERR_MISALIGNED, SPIN_ERR_DEVICE, SPIN_ERR_CUDA.
+ */
+spin_status_t spin_hadamard_quant_kron(const void *x_bf16, int64_t tokens, int32_t m, int32_t n, float clip,
+                                       const uint32_t *sign_bits, uint32_t flags, int32_t bits, void *q,
+                                       float *scales_f32, spin_stream_t stream);
+
+/*
  * R3 + INT4 KV cache ("SpinQuant, when rotations are worth learning", "Four
  * rotation sites": R3 is a fixed Hadamard on queries and keys after RoPE,
  * there only to make the KV cache quantisable; "SpinQuant Guide", "RoPE
@@ -242,7 +277,9 @@ spin_status_t spin_dequant_hadamard_inverse(const uint8_t *codes, int64_t rows, 
  * library gave up on an internal wait (a pipeline barrier that did not
  * complete within about two seconds); that kernel then stopped early and its
  * outputs are incomplete. Copies the word to *status and, if reset != 0,
- * clears it. Synchronous: it waits for work on the legacy default stream.
+ * clears it. Synchronous, the one entry point that blocks: it waits for work
+ * on the legacy default stream (and so for every launch of this library that
+ * the caller has enqueued on a blocking stream) before it reads the word.
  * Errors: SPIN_ERR_INVALID_ARG (status NULL), SPIN_ERR_CUDA.
  */
 spin_status_t spin_device_status(uint32_t *status, int reset);
@@ -266,9 +303,10 @@ void spin_test_stall_tensor_core_waits(int enable);
  * Host-only query (no device access, no launch): 1 if a call of operation `op`
  * with these arguments would run a tensor-core kernel, 0 if it would run the
  * CUDA-core kernel, -1 if the arguments are invalid for `op` (n not a supported
- * power of two, rows < 0, unknown op or flag bits). has_signs != 0 means a
- * sign_bits mask would be passed. The answer follows the same rules as the
- * entry points' own dispatch.
+ * power of two, rows < 0 or above the entry point's limit -- 2^47 - 1 tokens for
+ * SPIN_OP_HADAMARD_QUANT, 2^46 - 1 rows for SPIN_OP_DEQUANT_INVERSE --, unknown op
+ * or flag bits). has_signs != 0 means a sign_bits mask would be passed. The
+ * answer follows the same rules as the entry points' own dispatch.
  */
 int spin_uses_tensor_cores(int32_t op, int64_t rows, int32_t n, uint32_t flags, int32_t has_signs);
 

@@ -19,6 +19,7 @@ import torch
 
 __all__ = [
     "lib", "SpinError", "hadamard_quant_int4", "hadamard_quant_int8", "hadamard_quant_int4_host",
+    "hadamard_quant_host", "hadamard_quant_kron",
     "rope_hadamard_kvquant",
     "dequant_hadamard_inverse", "alloc_kv_cache", "NO_ROTATE", "SYM_INT4_F32SCALE", "ASYM_INT4_F16SZ",
     "BF16", "F32", "HEADER", "LIB_PATH", "exported_symbols", "CUDA_CORES_ONLY", "TENSOR_CORES", "device_status",
@@ -69,8 +70,9 @@ def lib() -> C.CDLL:
                                              vp, vp, vp, vp, i32, i32, vp]
     L.spin_hadamard_quant_int8.argtypes = [vp, i64, i32, f32, vp, u32, vp, vp, vp]
     L.spin_dequant_hadamard_inverse.argtypes = [vp, i64, i32, i32, vp, vp, vp, u32, vp, i32, vp]
+    L.spin_hadamard_quant_kron.argtypes = [vp, i64, i32, i32, f32, vp, u32, i32, vp, vp, vp]
     for name in ("spin_hadamard_quant_int4", "spin_hadamard_quant_int4_ex", "spin_hadamard_quant_int8",
-                 "spin_rope_hadamard_kvquant", "spin_dequant_hadamard_inverse"):
+                 "spin_rope_hadamard_kvquant", "spin_dequant_hadamard_inverse", "spin_hadamard_quant_kron"):
         getattr(L, name).restype = C.c_int
     L.spin_uses_tensor_cores.argtypes = [i32, i64, i32, u32, i32]
     L.spin_uses_tensor_cores.restype = C.c_int
@@ -111,6 +113,10 @@ def spin_hadamard_quant_int4_ex(x_bf16, tokens, n, clip, sign_bits, flags, q_pac
 
 def spin_hadamard_quant_int8(x_bf16, tokens, n, clip, sign_bits, flags, q_i8, scales_f32, stream) -> int:
     return lib().spin_hadamard_quant_int8(x_bf16, tokens, n, clip, sign_bits, flags, q_i8, scales_f32, stream)
+
+
+def spin_hadamard_quant_kron(x_bf16, tokens, m, n, clip, sign_bits, flags, bits, q, scales_f32, stream) -> int:
+    return lib().spin_hadamard_quant_kron(x_bf16, tokens, m, n, clip, sign_bits, flags, bits, q, scales_f32, stream)
 
 
 def spin_rope_hadamard_kvquant(*args) -> int:
@@ -222,28 +228,90 @@ def hadamard_quant_int8(x: torch.Tensor, clip: float = 1.0, signs: torch.Tensor 
     return out, scales
 
 
-def hadamard_quant_int4_host(x_host: torch.Tensor, clip: float = 1.0, signs: torch.Tensor | None = None,
-                             device=None, stream=None, buffers=None):
-    """End-to-end R4 from host memory: copy x (pinned, bf16) to the device, run
-    the kernel, copy codes and scales back into pinned host tensors. Returns
-    (codes_host, scales_host); synchronises the stream before returning."""
+_host_streams = {}
+
+
+def _pipeline_streams(device):
+    """Three streams per device (copy in, compute, copy out), created once."""
+    key = torch.device(device).index
+    if key not in _host_streams:
+        _host_streams[key] = tuple(torch.cuda.Stream(device) for _ in range(3))
+    return _host_streams[key]
+
+
+def hadamard_quant_kron(x: torch.Tensor, m: int, clip: float = 1.0, signs: torch.Tensor | None = None,
+                        bits: int = 4, out: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                        stream=None):
+    """R4 for n = m 2^k (H_m of Paley (x) Sylvester H_{2^k}): x [tokens, n] bf16 (CUDA) ->
+    (codes [tokens, n/2] uint8 for bits = 4, or [tokens, n] int8 for bits = 8; scales [tokens] fp32)."""
+    if bits not in (4, 8):
+        raise ValueError("bits must be 4 or 8")
+    ctype, cols = (torch.uint8, lambda n: n // 2) if bits == 4 else (torch.int8, lambda n: n)
+    tokens, n, out, scales = _r4_args(x, out, scales, signs, ctype, cols)
+    st = spin_hadamard_quant_kron(_ptr(x), tokens, int(m), n, float(clip), _ptr(signs), 0, bits, _ptr(out),
+                                  _ptr(scales), _stream(stream))
+    _check("spin_hadamard_quant_kron", st)
+    return out, scales
+
+
+def hadamard_quant_host(x_host: torch.Tensor, clip: float = 1.0, signs: torch.Tensor | None = None, bits: int = 4,
+                        device=None, stream=None, buffers=None, chunks: int = 8, m: int | None = None):
+    """End-to-end R4 from host memory: copy x (pinned, bf16 [tokens, n]) to the
+    device, run the kernel, copy codes and steps back into pinned host tensors.
+    The batch is cut into `chunks` slices of whole tokens that flow through three
+    streams, so the copy in of one slice, the kernel of the previous one and the
+    copy out of the one before overlap. Work is ordered after what is already
+    enqueued on `stream` (default: the current stream), which is made to wait for
+    all of it; the call synchronises `stream` before it returns (codes_host,
+    steps_host). `buffers` (from a previous call's return of the same shape) may
+    be passed to reuse the device and pinned buffers. With `m`, the row length is
+    n = m 2^k and the kernel is hadamard_quant_kron's."""
     device = torch.device(device or "cuda")
+    if bits not in (4, 8):
+        raise ValueError("bits must be 4 or 8")
+    if x_host.dim() != 2 or x_host.dtype != torch.bfloat16 or x_host.is_cuda:
+        raise ValueError("x_host: expected a host [tokens, n] bfloat16 tensor")
     tokens, n = x_host.shape
+    cols, ctype = (n // 2, torch.uint8) if bits == 4 else (n, torch.int8)
     if buffers is None:
         buffers = dict(
             x=torch.empty((tokens, n), dtype=torch.bfloat16, device=device),
-            q=torch.empty((tokens, n // 2), dtype=torch.uint8, device=device),
+            q=torch.empty((tokens, cols), dtype=ctype, device=device),
             s=torch.empty((tokens,), dtype=torch.float32, device=device),
-            q_host=torch.empty((tokens, n // 2), dtype=torch.uint8, pin_memory=True),
+            q_host=torch.empty((tokens, cols), dtype=ctype, pin_memory=True),
             s_host=torch.empty((tokens,), dtype=torch.float32, pin_memory=True))
-    s = stream or torch.cuda.current_stream(device)
-    with torch.cuda.stream(s):
-        buffers["x"].copy_(x_host, non_blocking=True)
-        hadamard_quant_int4(buffers["x"], clip, signs, out=buffers["q"], scales=buffers["s"], stream=s)
-        buffers["q_host"].copy_(buffers["q"], non_blocking=True)
-        buffers["s_host"].copy_(buffers["s"], non_blocking=True)
-    s.synchronize()
-    return buffers["q_host"], buffers["s_host"]
+    if m is not None:
+        def quant(x, clip, signs, out, scales, stream):
+            return hadamard_quant_kron(x, m, clip, signs, bits, out, scales, stream)
+    else:
+        quant = hadamard_quant_int4 if bits == 4 else hadamard_quant_int8
+    s0 = stream or torch.cuda.current_stream(device)
+    h2d, comp, d2h = _pipeline_streams(device)
+    start = torch.cuda.Event()
+    start.record(s0)
+    for st in (h2d, comp, d2h):
+        st.wait_event(start)
+    step = max(1, -(-tokens // max(1, chunks)))
+    for t0 in range(0, tokens, step):
+        t1 = min(tokens, t0 + step)
+        with torch.cuda.stream(h2d):
+            buffers["x"][t0:t1].copy_(x_host[t0:t1], non_blocking=True)
+        comp.wait_stream(h2d)
+        quant(buffers["x"][t0:t1], clip, signs, out=buffers["q"][t0:t1], scales=buffers["s"][t0:t1], stream=comp)
+        d2h.wait_stream(comp)
+        with torch.cuda.stream(d2h):
+            buffers["q_host"][t0:t1].copy_(buffers["q"][t0:t1], non_blocking=True)
+            buffers["s_host"][t0:t1].copy_(buffers["s"][t0:t1], non_blocking=True)
+    s0.wait_stream(d2h)
+    s0.synchronize()
+    return buffers["q_host"], buffers["s_host"], buffers
+
+
+def hadamard_quant_int4_host(x_host: torch.Tensor, clip: float = 1.0, signs: torch.Tensor | None = None,
+                             device=None, stream=None, buffers=None, chunks: int = 8):
+    """hadamard_quant_host with INT4 codes; returns (codes_host, steps_host)."""
+    q, s, _ = hadamard_quant_host(x_host, clip, signs, 4, device, stream, buffers, chunks)
+    return q, s
 
 
 def alloc_kv_cache(batch: int, n_kv_heads: int, cache_len: int, head_dim: int = 128, device="cuda"):

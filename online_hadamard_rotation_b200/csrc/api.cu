@@ -143,6 +143,23 @@ spin_status_t spin_hadamard_quant_int4(const void *x_bf16, int64_t tokens, int32
   return spin_hadamard_quant_int4_ex(x_bf16, tokens, n, clip, nullptr, 0u, q_packed_u8, scales_f32, stream);
 }
 
+spin_status_t spin_hadamard_quant_kron(const void *x_bf16, int64_t tokens, int32_t m, int32_t n, float clip,
+                                       const uint32_t *sign_bits, uint32_t flags, int32_t bits, void *q,
+                                       float *scales_f32, spin_stream_t stream) {
+  if (!kron_supported(m, n)) return SPIN_ERR_UNSUPPORTED_SIZE;
+  if (tokens < 0 || !valid_clip(clip) || (flags & ~SPIN_TENSOR_CORES) != 0 || (bits != 4 && bits != 8))
+    return SPIN_ERR_INVALID_ARG;
+  if (tokens == 0) return SPIN_OK;
+  if (!x_bf16 || !q || !scales_f32) return SPIN_ERR_INVALID_ARG;
+  if (tokens >= ((int64_t(1) << 31) / (n / 128))) return SPIN_ERR_UNSUPPORTED_SIZE;  // 32-bit TMA row coordinates
+  if (!aligned(x_bf16, 16) || !aligned(q, 16) || !aligned(scales_f32, 4) || (sign_bits && !aligned(sign_bits, 4)))
+    return SPIN_ERR_MISALIGNED;
+  spin_status_t st = check_device();
+  if (st != SPIN_OK) return st;
+  return cuda_status(launch_rotate_quant_kron(m, n, bits, x_bf16, tokens, clip, sign_bits, static_cast<uint8_t *>(q),
+                                              scales_f32, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 spin_status_t spin_rope_hadamard_kvquant(const void *q, const void *k, const void *v, const int32_t *pos,
                                          float theta, int32_t head_dim, int32_t batch, int32_t seq,
                                          int32_t n_q_heads, int32_t n_kv_heads, float clip, void *q_out,
@@ -225,10 +242,17 @@ int spin_uses_tensor_cores(int32_t op, int64_t rows, int32_t n, uint32_t flags, 
   if ((flags & ~(SPIN_NO_ROTATE | SPIN_CUDA_CORES_ONLY | SPIN_TENSOR_CORES)) != 0 ||
       (flags & (SPIN_CUDA_CORES_ONLY | SPIN_TENSOR_CORES)) == (SPIN_CUDA_CORES_ONLY | SPIN_TENSOR_CORES))
     return -1;
+  // the entry points' own upper bounds on the row count
+  if (op == SPIN_OP_HADAMARD_QUANT) {
+    if (rows > (INT64_MAX >> 16)) return -1;
+  } else if (op == SPIN_OP_DEQUANT_INVERSE) {
+    if (rows > (INT64_MAX >> 17)) return -1;
+  } else {
+    return -1;
+  }
   if (flags & SPIN_CUDA_CORES_ONLY) return 0;
   if (op == SPIN_OP_HADAMARD_QUANT) return tc_rotate_quant_supported(log_n, rows, flags, has_signs != 0) ? 1 : 0;
-  if (op == SPIN_OP_DEQUANT_INVERSE) return tc_dequant_supported(log_n, rows, flags) ? 1 : 0;
-  return -1;
+  return tc_dequant_supported(log_n, rows, flags) ? 1 : 0;
 }
 
 int spin_version(void) { return 100; }

@@ -26,14 +26,18 @@
 // resident CTA, after its own group, takes over groups of CTAs that have not started
 // yet (cluster launch control `try_cancel`), so the work spreads dynamically over the
 // SMs and the last groups land wherever an SM is free.
-// Roles (384 threads, one CTA per SM, persistent over groups):
-//   warp 0      TMA producer: 64 KiB per group (boxes of [128 rows][min(B, 64)]
-//               bf16 with 32-, 64- or 128-byte swizzle) into a three-stage ring
-//   warp 1      TMEM owner and MMA issuer (8 MMAs of K = 16 per group)
-//   warps 2-3   +-1 diagonal: XOR of the bf16 sign bits in shared memory, with
-//               each thread's sign words held in registers
+// Roles (512 threads in four warpgroups, one CTA per SM, persistent over groups):
+//   warps 0-3   +-1 diagonal: XOR of the bf16 sign bits in shared memory, with
+//               each thread's sign words held in registers; one warp on each of
+//               the SM's four schedulers, so the pass loads them evenly
 //   warps 4-7   epilogue for TMEM columns 0-127 of each group
 //   warps 8-11  epilogue for columns 128-255
+//   warp 12     TMA producer: 64 KiB per group (boxes of [128 rows][min(B, 64)]
+//               bf16 with 32-, 64- or 128-byte swizzle) into a three-stage ring
+//   warp 13     TMEM owner and MMA issuer (8 MMAs of K = 16 per group)
+//   warps 14-15 idle
+// setmaxnreg moves registers from the sign and control warpgroups to the epilogue
+// warpgroups, whose threads hold 128 fp32 values each.
 // TMEM holds two 256-column accumulators, so the MMA of group i + 1 overlaps
 // the epilogue of group i. Each epilogue thread stores its code bytes straight
 // to global memory. The launch allows programmatic dependent launch: the
@@ -61,7 +65,14 @@ __device__ unsigned int g_device_status = 0u;
 
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
+constexpr int kProducerWarp = 12, kMmaWarp = 13;
+// Registers per thread: 128 at launch (65536 / 512); after the split, the sign
+// warpgroup keeps 96, the epilogue warpgroups get 176 and the control warpgroup
+// (producer, MMA issuer, two idle warps) keeps 56. The split adds up to at most the
+// launch's total, so no increase waits for registers that are not there.
+constexpr int kLaunchRegs = 128, kRegsSign = 96, kRegsEpi = 176, kRegsCtl = 56;
+static_assert(kRegsSign * 128 + kRegsEpi * 256 + kRegsCtl * 128 <= kLaunchRegs * kThreads, "register split");
 constexpr int kStages = 3;
 constexpr uint32_t kGroupBytes = 65536;            // one MMA group: 128 rows x 256 columns of bf16
 constexpr uint32_t kOffH = 0;                      // A operand: H_128, K-major, 2 x 16 KiB
@@ -77,40 +88,97 @@ constexpr long long kStallTestCycles = 2000000LL;      // about a millisecond, f
 // MMA accumulates H_128 X_0 + H_128 X_1 into TMEM columns 0-127 and H_128 X_0 -
 // H_128 X_1 (negated A) into columns 128-255, so epilogue warpgroup g holds output
 // rows 128 g + a' and the token's max spans both warpgroups.
-template <int LOGN>
+//
+// KR > 0 (KRON) is a row of n = m 2^k = 128 KR values that is not a power of two
+// ("Rotations: QuaRot, SpinQuant and incoherence", "Hadamard matrices": sizes that
+// are not powers of two use a Kronecker product with a small known Hadamard matrix):
+// element e = b i + j (i < m the index of Paley's H_m, j < b = 2^k the Sylvester
+// index) is row r = (b / 128) i + (j >> 7), column j & 127 of a KR x 128 tile, and
+// H_m (x) H_b = (H_m (x) H_{b/128}) (x) H_128. The MMA's A operand is the KR x KR
+// matrix H_m (x) H_{b/128} (zero-padded to 128 x 128) instead of H_128; everything
+// after it is the n = 16384 shape with KR rows per token.
+template <int LOGN, int KR = 0>
 struct Shape {
-  static constexpr bool SPLIT = LOGN == 15;
-  static constexpr int B = SPLIT ? 128 : 1 << (LOGN - 7);  // columns per row (last factor size)
-  static constexpr int LOGB = SPLIT ? 7 : LOGN - 7;
-  static constexpr int ROWS = SPLIT ? 256 : 128;    // rows per token
-  static constexpr int TOK = SPLIT ? 1 : 256 / B;   // tokens per MMA group
-  static constexpr int SEG = SPLIT ? 1 : 128 / B;   // token segments per epilogue thread
-  static constexpr int BOXW = B < 64 ? B : 64;      // TMA box width (columns)
-  static constexpr int ROWB = BOXW * 2;             // bytes per smem tile row (64 or 128)
-  static constexpr int CBOX = B / BOXW;             // column boxes per 128-row block
-  static constexpr int BPT = CBOX * ROWS / 128;     // boxes per token
-  static constexpr uint32_t BOXBYTES = 128u * ROWB; // bytes per box
-  static constexpr int CPR = ROWB / 16;             // 16-byte chunks per tile row
+  static constexpr bool KRON = KR > 0;
+  static constexpr bool SPLIT = !KRON && LOGN == 15;
+  static constexpr int B = (SPLIT || KRON) ? 128 : 1 << (LOGN - 7);  // columns per row (last factor size)
+  static constexpr int LOGB = (SPLIT || KRON) ? 7 : LOGN - 7;
+  static constexpr int BOXH = KRON ? KR : 128;     // rows per TMA box and per MMA contraction
+  static constexpr int ROWS = SPLIT ? 256 : BOXH;  // rows per token
+  static constexpr int TOK = SPLIT ? 1 : 256 / B;  // tokens per MMA group
+  static constexpr int SEG = SPLIT ? 1 : 128 / B;  // token segments per epilogue thread
+  static constexpr int BOXW = B < 64 ? B : 64;     // TMA box width (columns)
+  static constexpr int ROWB = BOXW * 2;            // bytes per smem tile row (64 or 128)
+  static constexpr int CBOX = B / BOXW;            // column boxes per row block
+  static constexpr int BPT = CBOX * ROWS / BOXH;   // boxes per token
+  static constexpr uint32_t BOXBYTES = (uint32_t)BOXH * ROWB;  // bytes per box
+  static constexpr int CPR = ROWB / 16;            // 16-byte chunks per tile row
   static constexpr uint32_t LAYOUT = ROWB == 128 ? 2u : ROWB == 64 ? 4u : 6u;  // UMMA swizzle: 128, 64, 32 B
-  static constexpr uint32_t TOKBYTES = kGroupBytes / TOK;
-  static constexpr int NPOS = (int)(TOKBYTES / 16 / 64);  // sign positions per sign thread
-  static constexpr int64_t OUTB = (int64_t(1) << LOGN) / 2;  // code bytes per token
-  static_assert(LOGN >= 11 && LOGN <= 15, "this tensor-core R4 kernel covers n = 2048 .. 32768");
+  static constexpr uint32_t TOKBYTES = BPT * BOXBYTES;
+  static constexpr int NPOS = (int)(TOKBYTES / 16 / 128);  // sign positions per sign thread
+  static constexpr int SIGN_ITERS = (int)(TOK * TOKBYTES / 16 / 128);  // chunks per sign thread per group
+  static constexpr int KSTEPS = BOXH / 16;         // MMA steps of K = 16 per row block
+  static constexpr int64_t OUTB = (int64_t)ROWS * B / 2;  // code bytes per token (INT4)
+  static_assert(KRON ? (KR % 16 == 0 && KR >= 16 && KR <= 128) : (LOGN >= 11 && LOGN <= 15),
+                "this tensor-core R4 kernel covers n = 2048 .. 32768 and n = 128 KR, KR = 16 .. 128");
+  static_assert(TOK * TOKBYTES <= kGroupBytes && SIGN_ITERS % 4 == 0, "stage layout");
 };
 
-constexpr int kRing = 8;  // group ids in flight between the producer and the epilogue
+// Paley's Hadamard matrix of order m, as a kernel argument: type I (q = m - 1, prime,
+// q = 3 mod 4) or type II (q = m/2 - 1, prime, q = 1 mod 4); qr bit a is set when a
+// (0 < a < q) is a square mod q. bq = b / 128 = KR / m.
+struct KronParams {
+  int m, type, q, bq;
+  uint32_t qr[4];
+};
+
+// Quadratic character of a mod q from the residue mask: 0, +1 or -1.
+__device__ __forceinline__ int chi(int a, const KronParams &kp) {
+  a %= kp.q;
+  if (a < 0) a += kp.q;
+  if (a == 0) return 0;
+  return ((kp.qr[a >> 5] >> (a & 31)) & 1u) ? 1 : -1;
+}
+
+// Entry (i, j) of Paley's H_m. With the core matrix C of order q + 1 -- C[0][0] = 0,
+// C[0][j] = 1, C[i][0] = -1 (type I) or +1 (type II), C[i][j] = chi(j - i) otherwise --
+// type I is C + I and type II replaces each entry c of C by c [[1, -1], [-1, -1]]
+// plus [[1, 1], [1, -1]] on the diagonal.
+__device__ __forceinline__ int paley_entry(int i, int j, const KronParams &kp) {
+  auto core = [&](int a, int b) {
+    if (a == 0 && b == 0) return 0;
+    if (a == 0) return 1;
+    if (b == 0) return kp.type == 1 ? -1 : 1;
+    return chi(b - a, kp);
+  };
+  if (kp.type == 1) return core(i, j) + (i == j ? 1 : 0);
+  const int u = i & 1, v = j & 1, c = core(i >> 1, j >> 1);
+  const int am = (u == 0 && v == 0) ? 1 : -1;   // [[1, -1], [-1, -1]]
+  const int bm = (u == 1 && v == 1) ? -1 : 1;   // [[1, 1], [1, -1]]
+  return c * am + ((i >> 1) == (j >> 1) ? bm : 0);
+}
+
+// Group ids in flight from the producer to the sign warps, the MMA issuer and the
+// epilogue. The producer writes step i + kRing only after waiting for the stage of
+// that step to come free, i.e. after the MMA of step i + kRing - kStages (= i + 2)
+// completed; that MMA waited for its accumulator to be released by the step that
+// used it before, i (two accumulators), and the warpgroup(s) of step i release it
+// only after reading the id of step i. So with kRing = kStages + 2 no id is
+// overwritten before every consumer has read it, both when each warpgroup takes
+// every other step and when both take every step.
+constexpr int kRing = kStages + 2;
 
 struct Shared {
   uint4 clc_resp;          // response of the pending work-stealing request
   uint64_t full[kStages], sgn[kStages], empty[kStages], tfull[2], tempty[2], drain, clc;
-  uint64_t gfull[kRing];   // group id i & 7 written
-  int64_t gid[kRing];      // group of the CTA's i-th step (i & 7), -1 once there is none
+  uint64_t gfull[kRing];   // group id of step i written (slot i % kRing)
+  int64_t gid[kRing];      // group of the CTA's i-th step (slot i % kRing), -1 once there is none
   int64_t egid[2];         // epilogue warpgroup g's current group
   uint32_t tmem_base;
   int abort;
   int dec[3];
   long long budget;        // clock cycles a wait may take before the CTA gives up
-  float wmax[2][2][4][8];  // [warpgroup][group parity][warp][token segment]
+  float wmax[2][2][4][8];  // [warpgroup][parity of the half processed][warp][token segment]
 };
 static_assert(sizeof(Shared) <= 1024, "barrier area");
 
@@ -221,25 +289,25 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&b)[8]) {
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t ch) { return r * 128u + ((ch ^ (r & 7u)) << 4); }
 
 // Issue the TMA copies of group p (tokens p * TOK ...) into `dst`.
-template <int LOGN>
+template <int LOGN, int KR>
 __device__ __forceinline__ void load_group(uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int64_t p,
                                            int64_t tokens) {
-  using SH = Shape<LOGN>;
+  using SH = Shape<LOGN, KR>;
   const int64_t t0 = p * SH::TOK;
   const int nvalid = (int)((tokens - t0) < SH::TOK ? (tokens - t0) : SH::TOK);
   tc::mbar_arrive_expect_tx(bar, (uint32_t)nvalid * SH::TOKBYTES);
   for (int t = 0; t < nvalid; ++t)
     for (int j = 0; j < SH::BPT; ++j)
       tc::tma_load_2d(dst + (t * SH::BPT + j) * SH::BOXBYTES, map, bar, (j % SH::CBOX) * SH::BOXW,
-                      (int)((t0 + t) * SH::ROWS + (j / SH::CBOX) * 128));
+                      (int)((t0 + t) * SH::ROWS + (j / SH::CBOX) * SH::BOXH));
 }
 
-template <int LOGN, bool SIGNS, bool STORE32, int BITS>
+template <int LOGN, int KR, bool SIGNS, bool STORE32, int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
     k1_tc_rotate_quant(const __grid_constant__ CUtensorMap xmap, int64_t tokens, float clip, float inv_sqrt_n,
                        const uint32_t *__restrict__ signs, uint8_t *__restrict__ q, float *__restrict__ scales,
-                       int stall_test) {
-  using SH = Shape<LOGN>;
+                       int stall_test, const __grid_constant__ KronParams kp) {
+  using SH = Shape<LOGN, KR>;
   constexpr int B = SH::B, SEG = SH::SEG;
   static_assert(!(SIGNS && SH::SPLIT), "the sign masks of n = 32768 do not fit in registers");
   extern __shared__ uint8_t smem_raw[];
@@ -255,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // finished (programmatic dependent launch lets this prologue overlap their tail).
   tc::grid_dep_wait();
   int64_t first_issued = 0;  // groups the producer issues before the setup barrier
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == kProducerWarp * 32) {
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&S.full[s], 1);
       tc::mbar_init(&S.sgn[s], 1);
@@ -263,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       tc::mbar_init(&S.tfull[a], 1);
-      tc::mbar_init(&S.tempty[a], 256);
+      tc::mbar_init(&S.tempty[a], SH::SPLIT ? 256 : 128);  // the warpgroup(s) that read the accumulator
     }
     tc::mbar_init(&S.drain, 1);
     tc::mbar_init(&S.clc, 1);
@@ -276,26 +344,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     // latency overlaps the rest of the setup; ask for the next group at once.
     S.gid[0] = blockIdx.x;
     tc::mbar_arrive(&S.gfull[0]);
-    load_group<LOGN>(smem + kOffX, &xmap, &S.full[0], blockIdx.x, tokens);
+    load_group<LOGN, KR>(smem + kOffX, &xmap, &S.full[0], blockIdx.x, tokens);
     first_issued = 1;
     clc_request(&S.clc_resp, &S.clc);
   }
   tc::grid_dep_launch();
-  // H_128 as the A operand: K-major, two K blocks of [128 rows m][64 k], 128-byte swizzle.
+  // H_128 (KRON: H_m (x) H_{b/128}, zero outside its KR x KR corner) as the A operand:
+  // K-major, two K blocks of [128 rows m][64 k], 128-byte swizzle.
+  auto a_entry = [&](uint32_t m, uint32_t k) -> uint32_t {  // bf16 pattern of A[m][k]
+    if constexpr (SH::KRON) {
+      if (m >= (uint32_t)KR || k >= (uint32_t)KR) return 0u;
+      const int h = paley_entry((int)m / kp.bq, (int)k / kp.bq, kp) *
+                    ((__popc((m % kp.bq) & (k % kp.bq)) & 1) ? -1 : 1);
+      return h > 0 ? 0x3F80u : 0xBF80u;
+    } else {
+      return (__popc(m & k) & 1) ? 0xBF80u : 0x3F80u;
+    }
+  };
   for (uint32_t c = threadIdx.x; c < 2048; c += kThreads) {
     const uint32_t kb = c >> 10, m = (c >> 3) & 127u, ch = c & 7u;
     uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint32_t k0 = kb * 64 + ch * 8 + 2 * j;
-      const uint32_t lo = (__popc(m & k0) & 1) ? 0xBF80u : 0x3F80u;
-      const uint32_t hi = (__popc(m & (k0 + 1)) & 1) ? 0xBF80u : 0x3F80u;
-      w[j] = lo | (hi << 16);
+      w[j] = a_entry(m, k0) | (a_entry(m, k0 + 1) << 16);
     }
     *reinterpret_cast<uint4 *>(smem + kOffH + kb * 16384 + sw128(m, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   tc::fence_proxy_async_smem();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc::tmem_alloc(&S.tmem_base, 512);
     tc::tmem_relinquish();
   }
@@ -305,7 +382,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = S.tmem_base;
 
   // ------------------------------------------------------------ roles
-  if (warp == 0) {
+  // Each role block starts with its warpgroup's register change (every warp of a
+  // warpgroup, idle ones included, executes it; a block dominated by its own
+  // setmaxnreg is compiled to that register count).
+  if (warp == kProducerWarp) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl) : "memory");
     if (lane == 0) {
       int64_t last[kStages] = {-1, -1, -1};
       for (int64_t i = 0; i < first_issued; ++i) last[i] = i;
@@ -329,9 +410,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p < 0) {
           tc::mbar_arrive(&S.full[st]);  // no copies: the sign warps and the MMA read the end mark
           last[st] = -1;  // its previous copy was consumed before the slot came free
+          // The warpgroup that would take step i + 1 waits for that step's id: mark it
+          // as the end too (its ring slot is free once step i + 1's stage is).
+          const int st1 = (int)((i + 1) % kStages);
+          if (wait_bounded(&S.empty[st1], (uint32_t)(((i + 1) / kStages) & 1) ^ 1u, S, true)) {
+            last[st1] = -1;
+            S.gid[(i + 1) % kRing] = -1;
+            tc::mbar_arrive(&S.gfull[(i + 1) % kRing]);
+          }
           break;
         }
-        load_group<LOGN>(smem + kOffX + st * kGroupBytes, &xmap, &S.full[st], p, tokens);
+        load_group<LOGN, KR>(smem + kOffX + st * kGroupBytes, &xmap, &S.full[st], p, tokens);
         last[st] = i;
       }
       // every issued copy (and work request) has landed before the CTA can leave
@@ -339,7 +428,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (last[s] >= 0) wait_bounded(&S.full[s], (uint32_t)((last[s] / kStages) & 1), S, false);
       if (pending) wait_bounded(&S.clc, clc_phase, S, false);
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl) : "memory");
     if (lane == 0) {
       constexpr uint32_t idesc = tc::idesc_bf16(128, SH::SPLIT ? 128 : 256, true);
       constexpr uint32_t idesc_neg = idesc | (1u << 13);  // negate A
@@ -367,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
         } else {
 #pragma unroll
-          for (int s = 0; s < 8; ++s) {
+          for (int s = 0; s < SH::KSTEPS; ++s) {
             // A: 16 columns k of H per step. B: rows a = 16 s .. 16 s + 15 of every box
             // (MN-major: boxes of BOXW columns BOXBYTES apart, 8-row groups 8 ROWB apart).
             const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
@@ -383,16 +473,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSign) : "memory");
     if constexpr (SIGNS) {
-      // Thread ts flips the signs of chunks ts + 64 j of each group's 64 KiB.
+      // Thread ts flips the signs of chunks ts + 128 j of each group's 64 KiB.
       // Those chunks sit at NPOS distinct positions of a token's tile; their
       // sign words stay in registers for the whole kernel.
       constexpr int NPOS = SH::NPOS;
-      const uint32_t ts = threadIdx.x - 64;  // 0..63
+      const uint32_t ts = threadIdx.x;  // 0..127
       uint4 mk[NPOS];
 #pragma unroll
       for (int k = 0; k < NPOS; ++k) {
-        const uint32_t pos = ts + 64u * k;  // 16-byte chunk index inside one token's tile
+        const uint32_t pos = ts + 128u * k;  // 16-byte chunk index inside one token's tile
         const uint32_t box = pos / (SH::BOXBYTES / 16), inbox = pos % (SH::BOXBYTES / 16);
         const uint32_t a = inbox / SH::CPR, pc = inbox % SH::CPR;
         const uint32_t ch = SH::ROWB == 128 ? (pc ^ (a & 7u))
@@ -415,30 +506,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           S.dec[2] = ok;
         }
-        tc::named_sync(3, 64);
+        tc::named_sync(3, 128);
         if (!S.dec[2]) break;
         uint4 *X = reinterpret_cast<uint4 *>(smem + kOffX + st * kGroupBytes) + ts;
 #pragma unroll
-        for (int j0 = 0; j0 < 64; j0 += 4) {
+        for (int j0 = 0; j0 < SH::SIGN_ITERS; j0 += 4) {
           uint4 x[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) x[u] = X[64 * (j0 + u)];
+          for (int u = 0; u < 4; ++u) x[u] = X[128 * (j0 + u)];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const uint4 m = mk[(j0 + u) % NPOS];
-            X[64 * (j0 + u)] = make_uint4(x[u].x ^ m.x, x[u].y ^ m.y, x[u].z ^ m.z, x[u].w ^ m.w);
+            X[128 * (j0 + u)] = make_uint4(x[u].x ^ m.x, x[u].y ^ m.y, x[u].z ^ m.z, x[u].w ^ m.w);
           }
         }
         tc::fence_proxy_async_smem();
-        tc::named_sync(3, 64);
+        tc::named_sync(3, 128);
         if (ts == 0) tc::mbar_arrive(&S.sgn[st]);
       }
     }
-  } else {
-    // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1)
+  } else if (warp < 12) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi) : "memory");
+    // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1). Below n = 32768,
+    // warpgroup g takes whole groups, those of steps g, g + 2, ... (accumulator g),
+    // and works through the group's two 128-column halves one after the other, so
+    // the two warpgroups run out of phase (one in its butterflies while the other
+    // waits for TMEM or a barrier). At n = 32768 both take every step, half g each.
     const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
     const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
-    for (int64_t i = 0;; ++i) {
+    constexpr int kStep = SH::SPLIT ? 1 : 2, kHalves = SH::SPLIT ? 1 : 2;
+    uint32_t par = 0;  // max buffer in use: alternates with every half processed
+    for (int64_t i = SH::SPLIT ? 0 : g;; i += kStep) {
       const int acc = (int)(i & 1);
       // the step's group from the producer's ring, then its accumulator
       auto decide = [&](int slot) {
@@ -462,113 +560,122 @@ __global__ void __launch_bounds__(kThreads, 1)
         p = S.egid[g];
       }
       tc::tc_fence_after();
-      float v[kRegs];
-      {
-        uint32_t r[kRegs];
-        const uint32_t taddr = tmem + ((wq * 32u) << 16) + (uint32_t)acc * 256u + g * 128u;
-        tc::tmem_ld32(taddr, r);
-        tc::tmem_ld32(taddr + 32, r + 32);
-        tc::tmem_ld32(taddr + 64, r + 64);
-        tc::tmem_ld32(taddr + 96, r + 96);
-        tc::tmem_wait_ld();
+#pragma unroll 1
+      for (int hh = 0; hh < kHalves; ++hh, par ^= 1u) {
+        const uint32_t half = SH::SPLIT ? g : (uint32_t)hh;  // accumulator columns 128 half ..
+        float v[kRegs];
+        {
+          uint32_t r[kRegs];
+          const uint32_t taddr = tmem + ((wq * 32u) << 16) + (uint32_t)acc * 256u + half * 128u;
+          tc::tmem_ld32(taddr, r);
+          tc::tmem_ld32(taddr + 32, r + 32);
+          tc::tmem_ld32(taddr + 64, r + 64);
+          tc::tmem_ld32(taddr + 96, r + 96);
+          tc::tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < kRegs; ++k) v[k] = __uint_as_float(r[k]);
-      }
-      tc::tc_fence_before();
-      tc::mbar_arrive(&S.tempty[acc]);
-      // second Kronecker factor: H_B over b inside each token segment, in registers
-      stage<0>(v);
-      stage<1>(v);
-      stage<2>(v);
-      stage<3>(v);
-      if constexpr (SH::LOGB > 4) stage<4>(v);
-      if constexpr (SH::LOGB > 5) stage<5>(v);
-      if constexpr (SH::LOGB > 6) stage<6>(v);
-      // per-token max |u|: a tree of three-input maxima per segment, then the warp, then the warpgroup
-#pragma unroll
-      for (int sg = 0; sg < SEG; ++sg) {
-        float mx[B / 8];
-#pragma unroll
-        for (int k = 0; k < B / 8; ++k) {
-          const float *w = v + sg * B + 8 * k;
-          mx[k] = fmax3(fmax3(fabsf(w[0]), fabsf(w[1]), fabsf(w[2])), fmax3(fabsf(w[3]), fabsf(w[4]), fabsf(w[5])),
-                        fmaxf(fabsf(w[6]), fabsf(w[7])));
+          for (int k = 0; k < kRegs; ++k) v[k] = __uint_as_float(r[k]);
         }
+        if (hh == kHalves - 1) {  // the accumulator is in registers: the MMA may reuse it
+          tc::tc_fence_before();
+          tc::mbar_arrive(&S.tempty[acc]);
+        }
+        // second Kronecker factor: H_B over b inside each token segment, in registers
+        stage<0>(v);
+        stage<1>(v);
+        stage<2>(v);
+        stage<3>(v);
+        if constexpr (SH::LOGB > 4) stage<4>(v);
+        if constexpr (SH::LOGB > 5) stage<5>(v);
+        if constexpr (SH::LOGB > 6) stage<6>(v);
+        // per-token max |u|: a tree of three-input maxima per segment, then the warp, then the warpgroup
 #pragma unroll
-        for (int h = B / 16; h >= 1; h >>= 1)
+        for (int sg = 0; sg < SEG; ++sg) {
+          float mx[B / 8];
 #pragma unroll
-          for (int k = 0; k < h; ++k) mx[k] = fmaxf(mx[k], mx[k + h]);
-        const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mx[0]));
-        if (lane == 0) S.wmax[g][i & 1][wq][sg] = __uint_as_float(wm);
-      }
-      if constexpr (SH::SPLIT) tc::named_sync(4, 256);
-      else tc::named_sync(1 + g, 128);
-      constexpr float k815 = 8.0f / 15.0f;
+          for (int k = 0; k < B / 8; ++k) {
+            const float *w = v + sg * B + 8 * k;
+            mx[k] = fmax3(fmax3(fabsf(w[0]), fabsf(w[1]), fabsf(w[2])), fmax3(fabsf(w[3]), fabsf(w[4]), fabsf(w[5])),
+                          fmaxf(fabsf(w[6]), fabsf(w[7])));
+          }
 #pragma unroll
-      for (int sg = 0; sg < SEG; ++sg) {
-        float mu = fmaxf(fmaxf(S.wmax[g][i & 1][0][sg], S.wmax[g][i & 1][1][sg]),
-                         fmaxf(S.wmax[g][i & 1][2][sg], S.wmax[g][i & 1][3][sg]));
-        if constexpr (SH::SPLIT)
-          mu = fmaxf(mu, fmaxf(fmaxf(S.wmax[g ^ 1][i & 1][0][0], S.wmax[g ^ 1][i & 1][1][0]),
-                               fmaxf(S.wmax[g ^ 1][i & 1][2][0], S.wmax[g ^ 1][i & 1][3][0])));
-        const float s = fmaxf(clip * (mu * inv_sqrt_n) / (BITS == 4 ? 7.0f : 127.0f), 1e-8f);
-        const float c15 = (inv_sqrt_n / (BITS == 4 ? 15.0f : 255.0f)) / s;
-        const int64_t token = SH::SPLIT ? p : p * SH::TOK + g * SEG + sg;
-        if (token >= tokens) continue;
-        const uint32_t orow = SH::SPLIT ? 128u * g + row : row;  // output row of B values
-        uint8_t *dst = q + token * (SH::OUTB * (BITS / 4)) + orow * (B * BITS / 8);
-        if constexpr (BITS == 8 && B == 16) {  // 16 code bytes per row segment
-          uint32_t w4[4];
-          codes8_int8(v + sg * B, c15, w4[0], w4[1]);
-          codes8_int8(v + sg * B + 8, c15, w4[2], w4[3]);
-          __stcs(reinterpret_cast<uint4 *>(dst), make_uint4(w4[0], w4[1], w4[2], w4[3]));
-        } else if constexpr (BITS == 8) {
-          // one code byte per value: 32 bytes (8 words) at a time
+          for (int h = B / 16; h >= 1; h >>= 1)
 #pragma unroll
-          for (int c8 = 0; c8 < B / 32; ++c8) {
-            uint32_t w8[8];
+            for (int k = 0; k < h; ++k) mx[k] = fmaxf(mx[k], mx[k + h]);
+          const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mx[0]));
+          if (lane == 0) S.wmax[g][par][wq][sg] = __uint_as_float(wm);
+        }
+        if constexpr (SH::SPLIT) tc::named_sync(4, 256);
+        else tc::named_sync(1 + g, 128);
+        constexpr float k815 = 8.0f / 15.0f;
 #pragma unroll
-            for (int h = 0; h < 4; ++h) codes8_int8(v + sg * B + 32 * c8 + 8 * h, c15, w8[2 * h], w8[2 * h + 1]);
-            if constexpr (STORE32) {
-              st_v8_cs(dst + 32 * c8, w8);
+        for (int sg = 0; sg < SEG; ++sg) {
+          float mu = fmaxf(fmaxf(S.wmax[g][par][0][sg], S.wmax[g][par][1][sg]),
+                           fmaxf(S.wmax[g][par][2][sg], S.wmax[g][par][3][sg]));
+          if constexpr (SH::SPLIT)
+            mu = fmaxf(mu, fmaxf(fmaxf(S.wmax[g ^ 1][par][0][0], S.wmax[g ^ 1][par][1][0]),
+                                 fmaxf(S.wmax[g ^ 1][par][2][0], S.wmax[g ^ 1][par][3][0])));
+          const float s = fmaxf(clip * (mu * inv_sqrt_n) / (BITS == 4 ? 7.0f : 127.0f), 1e-8f);
+          const float c15 = (inv_sqrt_n / (BITS == 4 ? 15.0f : 255.0f)) / s;
+          const int64_t token = SH::SPLIT ? p : p * SH::TOK + half * SEG + sg;
+          if (token >= tokens) continue;
+          if (SH::KRON && row >= (uint32_t)KR) continue;  // TMEM lanes past the tile's rows hold zeros
+          const uint32_t orow = SH::SPLIT ? 128u * g + row : row;  // output row of B values
+          uint8_t *dst = q + token * (SH::OUTB * (BITS / 4)) + orow * (B * BITS / 8);
+          if constexpr (BITS == 8 && B == 16) {  // 16 code bytes per row segment
+            uint32_t w4[4];
+            codes8_int8(v + sg * B, c15, w4[0], w4[1]);
+            codes8_int8(v + sg * B + 8, c15, w4[2], w4[3]);
+            __stcs(reinterpret_cast<uint4 *>(dst), make_uint4(w4[0], w4[1], w4[2], w4[3]));
+          } else if constexpr (BITS == 8) {
+            // one code byte per value: 32 bytes (8 words) at a time
+#pragma unroll
+            for (int c8 = 0; c8 < B / 32; ++c8) {
+              uint32_t w8[8];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) codes8_int8(v + sg * B + 32 * c8 + 8 * h, c15, w8[2 * h], w8[2 * h + 1]);
+              if constexpr (STORE32) {
+                st_v8_cs(dst + 32 * c8, w8);
+              } else {
+                __stcs(reinterpret_cast<uint4 *>(dst + 32 * c8), make_uint4(w8[0], w8[1], w8[2], w8[3]));
+                __stcs(reinterpret_cast<uint4 *>(dst + 32 * c8) + 1, make_uint4(w8[4], w8[5], w8[6], w8[7]));
+              }
+            }
+          } else {
+            uint32_t words[B / 8];
+#pragma unroll
+            for (int wi = 0; wi < B / 8; ++wi) {
+              uint32_t b[8];
+              float t[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) t[k] = fma_sat(v[sg * B + 8 * wi + k], c15, k815);
+#pragma unroll
+              for (int k = 0; k < 8; k += 2) round15_x2(t[k], t[k + 1], b[k], b[k + 1]);
+              words[wi] = pack8(b);
+            }
+            if constexpr (B == 16) {  // 8 code bytes per row segment
+              __stcs(reinterpret_cast<uint2 *>(dst), make_uint2(words[0], words[1]));
+            } else if constexpr (STORE32 && B >= 64) {
+#pragma unroll
+              for (int w8 = 0; w8 < B / 64; ++w8) st_v8_cs(dst + 32 * w8, words + 8 * w8);
             } else {
-              __stcs(reinterpret_cast<uint4 *>(dst + 32 * c8), make_uint4(w8[0], w8[1], w8[2], w8[3]));
-              __stcs(reinterpret_cast<uint4 *>(dst + 32 * c8) + 1, make_uint4(w8[4], w8[5], w8[6], w8[7]));
+#pragma unroll
+              for (int w4 = 0; w4 < B / 32; ++w4)
+                __stcs(reinterpret_cast<uint4 *>(dst) + w4,
+                       make_uint4(words[4 * w4], words[4 * w4 + 1], words[4 * w4 + 2], words[4 * w4 + 3]));
             }
           }
-        } else {
-          uint32_t words[B / 8];
-#pragma unroll
-          for (int wi = 0; wi < B / 8; ++wi) {
-            uint32_t b[8];
-            float t[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) t[k] = fma_sat(v[sg * B + 8 * wi + k], c15, k815);
-#pragma unroll
-            for (int k = 0; k < 8; k += 2) round15_x2(t[k], t[k + 1], b[k], b[k + 1]);
-            words[wi] = pack8(b);
-          }
-          if constexpr (B == 16) {  // 8 code bytes per row segment
-            __stcs(reinterpret_cast<uint2 *>(dst), make_uint2(words[0], words[1]));
-          } else if constexpr (STORE32 && B >= 64) {
-#pragma unroll
-            for (int w8 = 0; w8 < B / 64; ++w8) st_v8_cs(dst + 32 * w8, words + 8 * w8);
-          } else {
-#pragma unroll
-            for (int w4 = 0; w4 < B / 32; ++w4)
-              __stcs(reinterpret_cast<uint4 *>(dst) + w4,
-                     make_uint4(words[4 * w4], words[4 * w4 + 1], words[4 * w4 + 2], words[4 * w4 + 3]));
-          }
+          if (tg == 0 && (!SH::SPLIT || g == 0)) scales[token] = s;
         }
-        if (tg == 0 && (!SH::SPLIT || g == 0)) scales[token] = s;
       }
     }
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl) : "memory");  // idle warps 14-15
   }
 
   // ------------------------------------------------------------ teardown
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     if (lane == 0) {
       tc::umma_commit(&S.drain);  // arrives once every MMA this thread issued is complete
       wait_bounded(&S.drain, 0, S, false);
@@ -579,16 +686,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int LOGN, bool SIGNS, bool STORE32, int BITS>
+template <int LOGN, int KR, bool SIGNS, bool STORE32, int BITS>
 cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
-                      cudaStream_t stream, int stall_test) {
-  using SH = Shape<LOGN>;
+                      cudaStream_t stream, int stall_test, const KronParams &kp) {
+  using SH = Shape<LOGN, KR>;
   auto fn = tensor_map_encoder();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap map;
   const cuuint64_t dims[2] = {(cuuint64_t)SH::B, (cuuint64_t)tokens * SH::ROWS};
   const cuuint64_t strides[1] = {(cuuint64_t)SH::B * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)SH::BOXW, 128};
+  const cuuint32_t box[2] = {(cuuint32_t)SH::BOXW, (cuuint32_t)SH::BOXH};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -597,14 +704,21 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
                                    : CU_TENSOR_MAP_SWIZZLE_32B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto kern = k1_tc_rotate_quant<LOGN, SIGNS, STORE32, BITS>;
+  auto kern = k1_tc_rotate_quant<LOGN, KR, SIGNS, STORE32, BITS>;
+  static cudaError_t checked = [&] {  // the register split assumes this count at launch
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(kern));
+    if (e != cudaSuccess) return e;
+    return fa.numRegs == kLaunchRegs ? cudaSuccess : cudaErrorInvalidConfiguration;
+  }();
+  if (checked != cudaSuccess) return checked;
   int slots = 0;
   cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreads, (int)kSmemBytes, &slots);
   if (err != cudaSuccess) return err;
   // One CTA per group: the resident ones take the groups of CTAs that have not started
   // yet (cluster launch control), so the groups spread over the SMs as they free up.
   const int64_t grid = (tokens + SH::TOK - 1) / SH::TOK;
-  const float inv_sqrt_n = (float)(1.0 / std::sqrt((double)(1 << LOGN)));
+  const float inv_sqrt_n = (float)(1.0 / std::sqrt((double)SH::ROWS * SH::B));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(kThreads);
@@ -615,23 +729,32 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, map, tokens, clip, inv_sqrt_n, signs, q, scales, stall_test);
+  return cudaLaunchKernelEx(&cfg, kern, map, tokens, clip, inv_sqrt_n, signs, q, scales, stall_test, kp);
 }
 
 template <int LOGN, int BITS>
 cudaError_t launch_n(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q, float *scales,
                      cudaStream_t stream, int stall_test) {
   const bool a32 = (reinterpret_cast<uintptr_t>(q) & 31u) == 0;  // 32-byte stores need 32-byte alignment
+  const KronParams none = {};
   if constexpr (Shape<LOGN>::SPLIT) {
     if (signs) return cudaErrorInvalidValue;
   } else if (signs) {
-    return a32 ? launch_tc<LOGN, true, true, BITS>(x, tokens, clip, signs, q, scales, stream, stall_test)
-               : launch_tc<LOGN, true, false, BITS>(x, tokens, clip, signs, q, scales, stream, stall_test);
+    return a32 ? launch_tc<LOGN, 0, true, true, BITS>(x, tokens, clip, signs, q, scales, stream, stall_test, none)
+               : launch_tc<LOGN, 0, true, false, BITS>(x, tokens, clip, signs, q, scales, stream, stall_test, none);
   }
-  return a32 ? launch_tc<LOGN, false, true, BITS>(x, tokens, clip, nullptr, q, scales, stream, stall_test)
-             : launch_tc<LOGN, false, false, BITS>(x, tokens, clip, nullptr, q, scales, stream, stall_test);
+  return a32 ? launch_tc<LOGN, 0, false, true, BITS>(x, tokens, clip, nullptr, q, scales, stream, stall_test, none)
+             : launch_tc<LOGN, 0, false, false, BITS>(x, tokens, clip, nullptr, q, scales, stream, stall_test, none);
 }
 
+// n = 128 KR: 16-byte code stores (the output need only be 16-byte aligned), with or
+// without the diagonal.
+template <int KR, int BITS>
+cudaError_t launch_kron_rows(const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q,
+                             float *scales, cudaStream_t stream, int stall_test, const KronParams &kp) {
+  return signs ? launch_tc<14, KR, true, false, BITS>(x, tokens, clip, signs, q, scales, stream, stall_test, kp)
+               : launch_tc<14, KR, false, false, BITS>(x, tokens, clip, nullptr, q, scales, stream, stall_test, kp);
+}
 
 // ============================================================================ n = 128, 256
 // Tokens as the MMA's M. A token row of n = 128 V (V = 1, 2) is V chunks x_v of 128
@@ -1028,7 +1151,65 @@ cudaError_t launch_tc_bits(int log_n, const void *x, int64_t tokens, float clip,
   }
 }
 
+template <int BITS>
+cudaError_t launch_kron_bits(int rows, const void *x, int64_t tokens, float clip, const uint32_t *signs, uint8_t *q,
+                             float *scales, cudaStream_t stream, int stall, const KronParams &kp) {
+  switch (rows) {
+    case 16: return launch_kron_rows<16, BITS>(x, tokens, clip, signs, q, scales, stream, stall, kp);
+    case 32: return launch_kron_rows<32, BITS>(x, tokens, clip, signs, q, scales, stream, stall, kp);
+    case 48: return launch_kron_rows<48, BITS>(x, tokens, clip, signs, q, scales, stream, stall, kp);
+    case 64: return launch_kron_rows<64, BITS>(x, tokens, clip, signs, q, scales, stream, stall, kp);
+    case 80: return launch_kron_rows<80, BITS>(x, tokens, clip, signs, q, scales, stream, stall, kp);
+    case 96: return launch_kron_rows<96, BITS>(x, tokens, clip, signs, q, scales, stream, stall, kp);
+    case 112: return launch_kron_rows<112, BITS>(x, tokens, clip, signs, q, scales, stream, stall, kp);
+    case 128: return launch_kron_rows<128, BITS>(x, tokens, clip, signs, q, scales, stream, stall, kp);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+bool is_prime(int v) {
+  if (v < 2) return false;
+  for (int d = 2; d * d <= v; ++d)
+    if (v % d == 0) return false;
+  return true;
+}
+
 }  // namespace
+
+// Paley's construction applies to m when q = m - 1 is a prime = 3 mod 4 (type I) or
+// q = m/2 - 1 is a prime = 1 mod 4 (type II); type I is taken when both do.
+int paley_type(int m) {
+  if (m >= 4 && (m - 1) % 4 == 3 && is_prime(m - 1)) return 1;
+  if (m >= 12 && m % 4 == 0 && (m / 2 - 1) % 4 == 1 && is_prime(m / 2 - 1)) return 2;
+  return 0;
+}
+
+bool kron_supported(int m, int64_t n) {
+  if (!paley_type(m) || n <= 0 || n % m != 0) return false;
+  const int64_t b = n / m;
+  if (b < 128 || (b & (b - 1)) != 0) return false;
+  const int64_t rows = n / 128;
+  return rows >= 16 && rows <= 128 && rows % 16 == 0;
+}
+
+cudaError_t launch_rotate_quant_kron(int m, int n, int bits, const void *x, int64_t tokens, float clip,
+                                     const uint32_t *signs, uint8_t *q, float *scales, cudaStream_t stream) {
+  if (!kron_supported(m, n)) return cudaErrorInvalidValue;
+  KronParams kp = {};
+  kp.m = m;
+  kp.type = paley_type(m);
+  kp.q = kp.type == 1 ? m - 1 : m / 2 - 1;
+  kp.bq = (n / m) / 128;
+  for (int a = 1; a < kp.q; ++a) {  // the nonzero squares mod q
+    const int sq = (a * a) % kp.q;
+    kp.qr[sq >> 5] |= 1u << (sq & 31);
+  }
+  const int rows = n / 128;
+  const int stall = g_stall_test.load(std::memory_order_relaxed);
+  if (bits == 4) return launch_kron_bits<4>(rows, x, tokens, clip, signs, q, scales, stream, stall, kp);
+  if (bits == 8) return launch_kron_bits<8>(rows, x, tokens, clip, signs, q, scales, stream, stall, kp);
+  return cudaErrorInvalidValue;
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static std::once_flag once;

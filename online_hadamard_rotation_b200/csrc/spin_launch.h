@@ -28,6 +28,13 @@ cudaError_t launch_rotate_quant(const void *x, int64_t tokens, int log_n, float 
 // Tensor-core R4 kernels (n = 128, 256 and 2048 to 32768; n = 32768 without a
 // sign diagonal): availability and launcher.
 bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags, bool has_signs);
+// n = m 2^k that is not a power of two: Paley's type for m (1, 2, or 0 for none), whether
+// the tensor-core kernel covers (m, n) (2^k >= 128, n / 128 a multiple of 16 up to 128),
+// and its launch (k1_tc.cu).
+int paley_type(int m);
+bool kron_supported(int m, int64_t n);
+cudaError_t launch_rotate_quant_kron(int m, int n, int bits, const void *x, int64_t tokens, float clip,
+                                     const uint32_t *signs, uint8_t *q, float *scales, cudaStream_t stream);
 cudaError_t launch_rotate_quant_tc(int log_n, int bits, const void *x, int64_t tokens, float clip,
                                    const uint32_t *signs, uint8_t *q, float *scales, cudaStream_t stream);
 

@@ -67,6 +67,9 @@ def lib():
     L.orc_rotate_kron.restype = C.c_int
     L.orc_r4_row_kron.argtypes = [_u16p, C.c_int, C.c_int, C.c_double, vp, vp, vp, _i8p, vp, vp]
     L.orc_r4_row_kron.restype = C.c_int
+    L.orc_r4_rows_kron.argtypes = [_u16p, C.c_int64, C.c_int, C.c_int, C.c_double, vp, _u8p,
+                                   np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS"), C.c_int]
+    L.orc_r4_rows_kron.restype = C.c_int
     L.orc_quant_sym_int8.argtypes = [_dp, C.c_int, C.c_double, vp, _i8p]
     L.orc_quant_sym_int8.restype = C.c_double
     L.orc_r4_row_int8.argtypes = [_u16p, C.c_int, C.c_double, vp, C.c_uint32, C.c_int, vp, vp, _i8p,
@@ -77,6 +80,8 @@ def lib():
     L.orc_quant_asym_int4_at.argtypes = [_dp, C.c_int, C.c_double, C.c_uint16, vp, _u8p,
                                          C.POINTER(C.c_uint16)]
     L.orc_quant_asym_int4_at.restype = C.c_uint16
+    L.orc_asym_codes_at.argtypes = [_dp, C.c_int, C.c_double, C.c_uint16, C.c_double, vp, _u8p]
+    L.orc_asym_codes_at.restype = C.c_double
     L.orc_asym_unrounded_scale.argtypes = [_dp, C.c_int, C.c_double]
     L.orc_asym_unrounded_scale.restype = C.c_double
     L.orc_pack_nibbles.argtypes = [_i32p, C.c_int, _u8p]
@@ -227,6 +232,16 @@ def quant_asym_int4_at(x, clip, s16):
     return codes, int(used), int(z16.value), pre
 
 
+def asym_codes_at(x, clip, s16, z):
+    """Codes for the given fp16 step pattern and integer zero point; also the zero
+    point before rounding (-lo/s). Returns (codes, zero_pre, pre)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    pre = np.empty_like(x)
+    codes = np.empty(x.size, dtype=np.uint8)
+    zpre = lib().orc_asym_codes_at(x, x.size, float(clip), int(s16), float(z), _ptr(pre), codes)
+    return codes, float(zpre), pre
+
+
 def asym_unrounded_scale(x, clip) -> float:
     x = np.ascontiguousarray(x, dtype=np.float64)
     return lib().orc_asym_unrounded_scale(x, x.size, float(clip))
@@ -332,6 +347,20 @@ def r4_row_kron(x_bits, m, clip, signs=None):
     if rc:
         raise ValueError(f"orc_r4_row_kron failed ({rc})")
     return dict(y=y, pre=pre, codes=codes, scale64=s64.value, scale32=np.float32(s32.value))
+
+
+def r4_rows_kron(x_bits, m, clip, signs=None, threads=1):
+    """Rows [T, n = m b] through the Kronecker rotation and INT4 quantiser over
+    `threads` OpenMP threads: (packed codes [T, n/2], fp32 steps [T])."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    T, n = x.shape
+    packed = np.empty((T, n // 2), dtype=np.uint8)
+    scales = np.empty(T, dtype=np.float32)
+    rc = lib().orc_r4_rows_kron(x, T, int(m), n // int(m), float(clip), _ptr(_signs(signs)), packed, scales,
+                                int(threads))
+    if rc:
+        raise ValueError(f"orc_r4_rows_kron failed ({rc})")
+    return packed, scales
 
 
 def r4_rows(x_bits, clip, signs=None, no_rotate=False, threads=1):

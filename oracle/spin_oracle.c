@@ -327,6 +327,29 @@ int orc_r4_row_kron(const uint16_t *x, int m, int b, double clip, const uint32_t
   return rc;
 }
 
+void orc_pack_nibbles(const int32_t *codes, int n, uint8_t *packed);
+
+/* Many rows of n = m b through orc_r4_row_kron (INT4 codes packed two per byte,
+ * element 2j in the low nibble, and fp32 steps); rows spread over `threads`. */
+int orc_r4_rows_kron(const uint16_t *x, int64_t tokens, int m, int b, double clip, const uint32_t *signs,
+                     uint8_t *packed, float *scales, int threads) {
+  const int n = m * b;
+  int rc = 0;
+#pragma omp parallel for schedule(dynamic, 8) num_threads(threads > 0 ? threads : 1) reduction(| : rc)
+  for (int64_t t = 0; t < tokens; t++) {
+    int8_t *codes = (int8_t *)malloc((size_t)n);
+    int32_t *c32 = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+    int r = (codes && c32) ? orc_r4_row_kron(x + t * n, m, b, clip, signs, NULL, NULL, codes, NULL, scales + t) : -2;
+    if (r == 0) {
+      for (int j = 0; j < n; j++) c32[j] = codes[j];
+      orc_pack_nibbles(c32, n, packed + t * (n / 2));
+    }
+    free(codes); free(c32);
+    rc |= r;
+  }
+  return rc ? -1 : 0;
+}
+
 /* ------------------------------------------------------------------ */
 /* Quantisers                                                          */
 /* ------------------------------------------------------------------ */
@@ -396,6 +419,25 @@ uint16_t orc_quant_asym_int4_at(const double *x, int n, double clip, uint16_t s1
 }
 
 double orc_asym_unrounded_scale(const double *x, int n, double clip);
+
+/* The asymmetric zero point before its rounding, -lo/s with lo = min(clip*min x, 0)
+ * and s the given fp16 step (a zero step counts as 1), and the codes for that
+ * step and a given integer zero point z: q = clamp(rne(x/s) + z, 0, 15); `pre`
+ * (nullable) receives x/s + z. Used to check a zero point whose rounding sits on
+ * a .5 tie against the oracle's own result for the other rounding. */
+double orc_asym_codes_at(const double *x, int n, double clip, uint16_t s16, double z, double *pre,
+                         uint8_t *codes) {
+  double mn = x[0];
+  for (int j = 1; j < n; j++) mn = fmin(mn, x[j]);
+  double lo = fmin(clip * mn, 0.0);
+  double s = orc_f16_to_f64(s16);
+  if (s == 0.0) s = 1.0;
+  for (int j = 0; j < n; j++) {
+    if (pre) pre[j] = x[j] / s + z;
+    codes[j] = (uint8_t)clampd(nearbyint(x[j] / s) + z, 0.0, 15.0);
+  }
+  return -lo / s;
+}
 
 /* Asymmetric INT4 over one group (reading of "KV cache stored as 4-bit INT4";
  * the pages give no formula): lo = min(clip*min x, 0), hi = max(clip*max x, 0),

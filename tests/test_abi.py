@@ -164,8 +164,14 @@ def test_dispatch_query(L):
     assert q(R4, 128 * 16, 2048, 0, 0) == 1
     assert q(INV, 128 * 128, 256, 0, 0) == 1 and q(INV, 128 * 128 - 1, 256, 0, 0) == 0
     assert q(INV, 10 ** 6, 2048, 0, 0) == 0 and q(INV, 128 * 8, 4096, 0, 0) == 1
-    for bad in ((R4, 4, 100, 0, 0), (R4, -1, 256, 0, 0), (R4, 4, 256, 6, 0), (R4, 4, 256, 8, 0), (7, 4, 256, 0, 0)):
+    for bad in ((R4, 4, 100, 0, 0), (R4, -1, 256, 0, 0), (R4, 4, 256, 6, 0), (R4, 4, 256, 8, 0), (7, 4, 256, 0, 0),
+                (7, 4, 256, 2, 0)):
         assert q(*bad) == -1
+    # the entry points' row limits apply (no signed overflow in the size checks)
+    assert q(R4, (1 << 47) - 1, 32768, 2, 0) == 0 and q(R4, 1 << 47, 32768, 0, 0) == -1
+    assert q(R4, 1 << 56, 32768, 4, 0) == -1 and q(R4, 1 << 62, 128, 4, 0) == -1
+    assert q(INV, (1 << 46) - 1, 32768, 2, 0) == 0 and q(INV, 1 << 46, 32768, 0, 0) == -1
+    assert q(INV, 1 << 56, 32768, 4, 0) == -1
 
 
 def test_bench_names_the_dispatched_kernel():
@@ -175,3 +181,23 @@ def test_bench_names_the_dispatched_kernel():
     assert bench.r4_kernel_name(1024, 1 << 19, False, 8) == "k1_rotate_quant_int8"
     assert bench.k3_kernel_name(256, 1 << 21) == "k3_tcs_dequant_inverse"
     assert bench.k3_kernel_name(2048, 1 << 18) == "k3_dequant_inverse"
+
+
+def test_kron_size_rules(L):
+    """spin_hadamard_quant_kron accepts n = m 2^k with a Paley order m, 2^k >= 128 and
+    n / 128 a multiple of 16 up to 128; with tokens = 0 the call returns before any
+    device access, so the size rules are checked here without a GPU."""
+    f = L.spin_hadamard_quant_kron
+    f.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_int32, C.c_float, C.c_void_p, C.c_uint32, C.c_int32,
+                  C.c_void_p, C.c_void_p, C.c_void_p]
+    f.restype = C.c_int
+    OK, BAD, SIZE = 0, 1, 2
+    for m, n in ((28, 14336), (12, 6144), (12, 12288), (20, 10240), (24, 6144), (48, 6144), (4, 2048), (8, 4096)):
+        assert f(None, 0, m, n, 1.0, None, 0, 4, None, None, None) == OK, (m, n)
+    for m, n in ((16, 4096), (28, 7168), (36, 18432), (12, 3072), (20, 2560), (40, 10240), (28, 14336 * 2),
+                 (28, 14000), (0, 2048), (-12, 6144), (12, 0)):
+        assert f(None, 0, m, n, 1.0, None, 0, 4, None, None, None) == SIZE, (m, n)
+    assert f(None, 0, 28, 14336, 1.0, None, 0, 5, None, None, None) == BAD      # bits
+    assert f(None, 0, 28, 14336, 1.0, None, 1, 4, None, None, None) == BAD      # SPIN_NO_ROTATE is not a flag here
+    assert f(None, 0, 28, 14336, 1.5, None, 0, 4, None, None, None) == BAD      # clip
+    assert f(None, 4, 28, 14336, 1.0, None, 0, 4, None, None, None) == BAD      # null pointers

@@ -85,8 +85,10 @@ def test_cpu_baseline_leg_reports_one_and_all_cores():
     sys.path.insert(0, ROOT)
     import bench
     wl = bench.make_workload("sweep12", 0, tokens=24)
-    cpu = bench.cpu_baseline_leg(wl)
+    cpu, ref = bench.cpu_baseline_leg(wl)
     assert cpu["kind"] == "oracle" and cpu["cores"] == 1 and cpu["value"] > 0
     assert cpu["all_cores"]["cores"] >= 1 and cpu["all_cores"]["value"] > 0
+    assert ref[1].shape == (24, 2048) and ref[2].shape == (24,) and ref[3] == 24  # kept for the spot check
     wl8 = bench.make_workload("r4_prefill_int8", 0, tokens=2)
-    assert bench.cpu_baseline_leg(wl8)["all_cores"]["cores"] == 1  # the INT8 rows run one call at a time
+    cpu8, ref8 = bench.cpu_baseline_leg(wl8)
+    assert cpu8["all_cores"]["cores"] == 1 and ref8 is None  # the INT8 rows run one call at a time

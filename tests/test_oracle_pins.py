@@ -309,6 +309,13 @@ def test_asymmetric_at_given_step(orc):
                 assert np.allclose(pre3, x / s + z, rtol=0, atol=1e-12 * np.abs(x / s).max())
     c0, used0, z0, _ = orc.quant_asym_int4_at(np.zeros(128), 1.0, 0)
     assert used0 == 0x3C00 and z0 == 0 and np.all(c0 == 0)
+    # codes for a given step and zero point, and the zero point before rounding
+    x = rng.standard_normal(128) * 3 - 1
+    for clip, s16, z in ((1.0, 0x3800, 7.0), (0.95, 0x3A00, 3.0)):
+        s = float(np.array([s16], dtype=np.uint16).view(np.float16)[0])
+        codes, zpre, pre = orc.asym_codes_at(x, clip, s16, z)
+        assert np.array_equal(codes, np.clip(np.rint(x / s) + z, 0, 15).astype(np.uint8))
+        assert zpre == -min(clip * x.min(), 0.0) / s and np.allclose(pre, x / s + z, rtol=0, atol=1e-12)
 
 
 def test_r3_batch_scatter_layout(orc):
@@ -735,3 +742,14 @@ def test_decode_attention_scores_survive_r3(orc):
     ref = scipy.special.softmax(k @ q / math.sqrt(d)) @ v
     rot = scipy.special.softmax((k @ H.T) @ (H @ q) / math.sqrt(d)) @ v
     assert np.max(np.abs(ref - rot)) < 1e-12
+
+
+def test_r4_rows_kron_matches_single_rows(orc):
+    """The threaded Kronecker batch packs each row's codes (element 2j in the low
+    nibble) and fp32 step as the single-row function computes them."""
+    bits = synthetic.r4_prefill(tokens=5, n=6144, seed=8)[0]
+    sg = synthetic.sign_bits(6144, 3)
+    packed, scales = orc.r4_rows_kron(bits, 12, 0.9, sg, threads=3)
+    for t in range(5):
+        r = orc.r4_row_kron(bits[t], 12, 0.9, signs=sg)
+        assert np.array_equal(packed[t], orc.pack_nibbles(r["codes"])) and scales[t] == r["scale32"]
