@@ -44,7 +44,10 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 def metric_for(wl) -> str:
-    """The headline metric, or its counterpart for the INT8 and Kronecker-size workloads."""
+    """The headline metric, or its counterpart for the INT8, Kronecker-size and
+    decode-attention workloads."""
+    if wl.get("kind") == "attn":
+        return "decode attention over the INT4 KV cache: HBM GB/s (% of B200 peak) and us per step"
     m = METRIC.replace("INT4", "INT8") if wl.get("code_bits", 4) == 8 else METRIC
     if wl.get("kron_m"):
         m = m.replace("at n=16384", f"at n={wl['bits'].shape[1]} (H_{wl['kron_m']} Paley x Sylvester)")
@@ -213,6 +216,13 @@ def make_workload(name: str, rank: int, tokens: int | None = None):
                                       "seeded +-1 diagonal, H_16384 = H_128 (x) H_128, clip 0.9"
                                       + (", per-token INT8 codes" if code_bits == 8 else ""),
                           "tokens": int(bits.shape[0]), "n": int(bits.shape[1])})
+    if name.startswith("decode_attn"):
+        batch = int(name[len("decode_attn_b"):]) if name.startswith("decode_attn_b") else 4
+        q, k, v, pos = synthetic.r3_kv(batch=batch, seed=2 + rank)
+        return dict(kind="attn", q=q, k=k, v=v, pos=pos, clip=0.95,
+                    desc={"workload": f"decode attention over the INT4 KV cache: batch {batch} x 4096 cached slots "
+                                      "(the R3+KV workload's cache, written by the R3 kernel), 32 q / 8 kv heads, "
+                                      "head_dim 128, one query token per row", "tokens": batch})
     if name.startswith("kron"):
         n = int(name[len("kron"):] or 14336)
         m = {14336: 28, 6144: 12, 10240: 20, 12288: 12}[n]
@@ -256,11 +266,50 @@ def r3_bytes(tokens, hq=32, hkv=8, d=128):
 # ---------------------------------------------------------------------------
 # reference arm: the fp64 CPU oracle on the host cores
 # ---------------------------------------------------------------------------
+def attn_bytes(B, S, hq, hkv, d=128):
+    """Bytes one decode-attention step must move: both caches' codes, fp16 scales and
+    zeros, the bf16 queries and the fp32 output."""
+    return B * hkv * S * (2 * d // 2 + 4 * 2) + B * hq * d * (2 + 4)
+
+
+def run_reference_attn(args, wl):
+    """The oracle's decode attention over the oracle's own cache of the workload, all
+    batch rows spread over the host's cores."""
+    import oracle
+    oracle.lib()
+    q, k, v, pos = wl["q"], wl["k"], wl["v"], wl["pos"]
+    B, S, hq, d = q.shape
+    hkv = k.shape[2]
+    threads = oracle.max_threads()
+    ref = oracle.r3_batch(q, k, v, pos, 1e4, wl["clip"], cache_len=S, threads=threads)
+    qs = ref["q_out"][:, S - 1]
+    lens = [S] * B
+    for _ in range(args.warmup):
+        oracle.decode_attention(qs[:1], {n: a[:1] for n, a in ref.items() if n != "q_out"}, lens[:1])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.decode_attention(qs, ref, lens, threads=threads)
+    dt = time.perf_counter() - t0
+    gbs = attn_bytes(B, S, hq, hkv, d) * args.steps / dt / 1e9
+    line = {"impl": "reference", "metric": metric_for(wl), "value": gbs, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_for(wl, args.gpus, args.workload),
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": f"the whole batch ({B} rows x {S} slots) per step, fp64, rows over "
+                                       f"{threads} host thread(s)"},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args, wl):
     import oracle
     oracle.lib()
+    if wl["kind"] == "attn":
+        return run_reference_attn(args, wl)
     if wl["kind"] != "r4":
-        raise SystemExit("the reference arm times the R4 workloads")
+        raise SystemExit("the reference arm times the R4 and decode-attention workloads")
     bits, n = wl["bits"], wl["bits"].shape[1]
     sample = min(bits.shape[0], max(8, (1 << 22) // n))  # about 0.1-0.2 s of oracle work per step
     rows = bits[:sample]
@@ -521,6 +570,31 @@ def main():
         def step(i, cores_only=False):
             b = sets[i & 1]
             quant(b["x"], wl["clip"], signs, out=b["q"], scales=b["s"], stream=stream, cuda_cores_only=cores_only)
+    elif wl["kind"] == "attn":
+        # the cache as the R3 kernel writes it from the workload's Q, K, V; one query per row
+        q, k, v, pos = wl["q"], wl["k"], wl["v"], wl["pos"]
+        B, S, hq, d = q.shape
+        hkv = k.shape[2]
+        tokens = B
+        sets = []
+        for _ in range(2):
+            cache = spin.alloc_kv_cache(B, hkv, S, d, device=dev)
+            qo = spin.rope_hadamard_kvquant(*(torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+                                              for a in (q, k, v)), torch.from_numpy(pos).to(dev), cache,
+                                            clip=wl["clip"])
+            sets.append(dict(q=qo[:, S - 1].contiguous(), cache=cache,
+                             lens=torch.full((B,), S, dtype=torch.int32, device=dev),
+                             out=torch.empty((B, hq, d), dtype=torch.float32, device=dev),
+                             ws=torch.empty((spin.decode_attention_workspace_bytes(B, hq, S),), dtype=torch.uint8,
+                                            device=dev)))
+            del qo
+        torch.cuda.synchronize()
+        step_bytes = attn_bytes(B, S, hq, hkv, d)
+
+        def step(i, cores_only=False):
+            b = sets[i & 1]
+            spin.decode_attention_int4kv(b["q"], b["cache"], b["lens"], out=b["out"], workspace=b["ws"],
+                                         stream=stream)
     else:
         q, k, v, pos = wl["q"], wl["k"], wl["v"], wl["pos"]
         B, S, hq, d = q.shape
@@ -554,6 +628,8 @@ def main():
     ms_per_step, window_info = window_stats(windows, args.steps)
     last = sets[(args.steps * len(windows) - 1) & 1]  # buffers of the last timed step, kept for the spot check
     last = {"q": last["q"].clone(), "s": last["s"].clone()} if wl["kind"] == "r4" else None
+    if wl["kind"] == "attn":  # per-call latency: the cache of the R3 + KV workload is L2-resident
+        latency = {"us_per_call": ms_per_step * 1e3, "launches_per_call": 2}
     if world > 1:
         dist.barrier()
     gbs, tok_s = aggregate(world, step_bytes, tokens, args.steps, ms_per_step * args.steps)
@@ -633,8 +709,9 @@ def main():
                       "mse_ratio": mse[False] / mse[True] if mse[True] > 0 else None}
 
     # ---- decode: per-call latency, plain launches and CUDA-graph replay
-    latency = None
-    if args.workload.startswith("decode"):
+    if wl["kind"] != "attn":
+        latency = None
+    if args.workload.startswith("decode") and wl["kind"] == "r4":
         calls = 1000
         b = sets[0]
         for _ in range(10):
@@ -668,7 +745,9 @@ def main():
                    "note": "inputs are L2-resident at this size (1.3 MB or less)"}
 
     peak, peak_kind = measured_peaks()
-    if wl["kind"] == "r4" and "kron_m" in wl:
+    if wl["kind"] == "attn":
+        kname = "k4_attn_partial"
+    elif wl["kind"] == "r4" and "kron_m" in wl:
         kname = "k1_tc_rotate_quant"
     elif wl["kind"] == "r4":
         kname = r4_kernel_name(n, tokens, wl["signs"] is not None, wl["code_bits"])
@@ -699,7 +778,7 @@ def main():
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": config_for(wl, world, args.workload),
-                "gpu_launches": args.steps, "timed_windows": window_info, "e2e": e2e, "roofline": roofline,
+                "gpu_launches": args.steps * (2 if wl["kind"] == "attn" else 1), "timed_windows": window_info, "e2e": e2e, "roofline": roofline,
                 "cpu_baseline": cpu, "cuda_core_kernel": cores, "decode_latency": latency,
                 "round_trip": round_trip, "other_workloads": extras, "clocks": clocks.summary()}
         print(json.dumps(line), flush=True)

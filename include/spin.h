@@ -48,6 +48,7 @@
 #ifndef SPIN_H_
 #define SPIN_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -271,6 +272,51 @@ spin_status_t spin_dequant_hadamard_inverse(const uint8_t *codes, int64_t rows, 
                                             int32_t mode, const void *scale, const void *zero,
                                             const uint32_t *sign_bits, uint32_t flags, void *out,
                                             int32_t out_dtype, spin_stream_t stream);
+
+/*
+ * Decode attention over the INT4 KV cache that spin_rope_hadamard_kvquant writes
+ * ("SpinQuant Guide: Learned Rotations for 4-Bit LLMs", the KV4 serving diagram:
+ * rotated keys stored in the cache as INT4 meet the rotated queries in a fused INT4
+ * dot product; "SpinQuant: rotate before you round", section "Deployment
+ * implications": the rotation pays only with KV4 kernels). One step: for batch row
+ * b, query head h and its kv head g = h / (n_q_heads / n_kv_heads), over the cache
+ * slots j < lens[b] of row (b, g):
+ *   khat_j = (code_j - zero_j) * scale_j      (K and V alike, fp16 scale and zero)
+ *   score_j = (q_h . khat_j) * softmax_scale
+ *   out_h = sum_j softmax(score)_j * vhat_j
+ * R3 rotated q and k by the same orthogonal matrix, so the scores need no inverse
+ * rotation; V was not rotated, so out is in the value basis. Arithmetic is fp32.
+ *
+ *  q          [batch, n_q_heads, head_dim] bf16 (the rotated queries, as q_out of
+ *             spin_rope_hadamard_kvquant), 16-byte aligned
+ *  k_cache, v_cache  [batch, n_kv_heads, cache_len, head_dim/2] bytes, 16-byte aligned
+ *  k_scale, k_zero, v_scale, v_zero  [batch, n_kv_heads, cache_len] fp16, 2-byte aligned
+ *  lens       [batch] int32 in device memory: slots attended in each row; a value
+ *             outside [0, cache_len] is clamped to it, and a row with 0 slots gives 0
+ *  head_dim   128; n_q_heads / n_kv_heads in {1, 2, 4, 8}; batch, n_q_heads and
+ *             n_kv_heads at most 65535 (else SPIN_ERR_UNSUPPORTED_SIZE)
+ *  softmax_scale  > 0 and finite, usually 1 / sqrt(head_dim)
+ *  out        [batch, n_q_heads, head_dim] bf16 or fp32 (out_dtype), 16-byte aligned
+ *  workspace  caller-owned device scratch of at least
+ *             spin_decode_attention_workspace_bytes(batch, n_q_heads, cache_len) bytes,
+ *             16-byte aligned; its contents on entry do not matter and are
+ *             overwritten (the per-chunk partials); calls that may run at the same
+ *             time need separate workspaces
+ * Two kernels on `stream`: per 256-slot chunk partials, then their merge.
+ * Errors: SPIN_ERR_INVALID_ARG (null pointer with batch > 0, cache_len < 1, sizes
+ * < 0, softmax_scale, out_dtype, workspace too small), SPIN_ERR_UNSUPPORTED_SIZE,
+ * SPIN_ERR_MISALIGNED, SPIN_ERR_DEVICE, SPIN_ERR_CUDA.
+ */
+spin_status_t spin_decode_attention_int4kv(const void *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                                           const void *k_scale, const void *k_zero, const void *v_scale,
+                                           const void *v_zero, const int32_t *lens, int32_t batch,
+                                           int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                           int32_t cache_len, float softmax_scale, void *out, int32_t out_dtype,
+                                           void *workspace, size_t workspace_bytes, spin_stream_t stream);
+
+/* Workspace bytes spin_decode_attention_int4kv needs (batch x n_q_heads x
+ * ceil(cache_len / 256) partials of head_dim + 2 fp32 values); 0 for sizes <= 0. */
+size_t spin_decode_attention_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t cache_len);
 
 /*
  * Device status word of the current device: nonzero once a kernel of this

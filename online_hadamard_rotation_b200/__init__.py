@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "lib", "SpinError", "hadamard_quant_int4", "hadamard_quant_int8", "hadamard_quant_int4_host",
-    "hadamard_quant_host", "hadamard_quant_kron",
+    "hadamard_quant_host", "hadamard_quant_kron", "decode_attention_int4kv", "decode_attention_workspace_bytes",
     "rope_hadamard_kvquant",
     "dequant_hadamard_inverse", "alloc_kv_cache", "NO_ROTATE", "SYM_INT4_F32SCALE", "ASYM_INT4_F16SZ",
     "BF16", "F32", "HEADER", "LIB_PATH", "exported_symbols", "CUDA_CORES_ONLY", "TENSOR_CORES", "device_status",
@@ -71,8 +71,13 @@ def lib() -> C.CDLL:
     L.spin_hadamard_quant_int8.argtypes = [vp, i64, i32, f32, vp, u32, vp, vp, vp]
     L.spin_dequant_hadamard_inverse.argtypes = [vp, i64, i32, i32, vp, vp, vp, u32, vp, i32, vp]
     L.spin_hadamard_quant_kron.argtypes = [vp, i64, i32, i32, f32, vp, u32, i32, vp, vp, vp]
+    L.spin_decode_attention_int4kv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32,
+                                               vp, C.c_size_t, vp]
+    L.spin_decode_attention_workspace_bytes.argtypes = [i32, i32, i32]
+    L.spin_decode_attention_workspace_bytes.restype = C.c_size_t
     for name in ("spin_hadamard_quant_int4", "spin_hadamard_quant_int4_ex", "spin_hadamard_quant_int8",
-                 "spin_rope_hadamard_kvquant", "spin_dequant_hadamard_inverse", "spin_hadamard_quant_kron"):
+                 "spin_rope_hadamard_kvquant", "spin_dequant_hadamard_inverse", "spin_hadamard_quant_kron",
+                 "spin_decode_attention_int4kv"):
         getattr(L, name).restype = C.c_int
     L.spin_uses_tensor_cores.argtypes = [i32, i64, i32, u32, i32]
     L.spin_uses_tensor_cores.restype = C.c_int
@@ -117,6 +122,10 @@ def spin_hadamard_quant_int8(x_bf16, tokens, n, clip, sign_bits, flags, q_i8, sc
 
 def spin_hadamard_quant_kron(x_bf16, tokens, m, n, clip, sign_bits, flags, bits, q, scales_f32, stream) -> int:
     return lib().spin_hadamard_quant_kron(x_bf16, tokens, m, n, clip, sign_bits, flags, bits, q, scales_f32, stream)
+
+
+def spin_decode_attention_int4kv(*args) -> int:
+    return lib().spin_decode_attention_int4kv(*args)
 
 
 def spin_rope_hadamard_kvquant(*args) -> int:
@@ -354,6 +363,49 @@ def rope_hadamard_kvquant(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos
         _ptr(cache["v_scale"]), _ptr(cache["v_zero"]), cache_len, cache_offset, _stream(stream))
     _check("spin_rope_hadamard_kvquant", st)
     return q_out
+
+
+def decode_attention_workspace_bytes(batch: int, n_q_heads: int, cache_len: int) -> int:
+    """Scratch bytes decode_attention_int4kv needs (see spin_decode_attention_workspace_bytes)."""
+    return int(lib().spin_decode_attention_workspace_bytes(int(batch), int(n_q_heads), int(cache_len)))
+
+
+def decode_attention_int4kv(q: torch.Tensor, cache: dict, lens: torch.Tensor, softmax_scale: float | None = None,
+                            out_dtype=torch.float32, out: torch.Tensor | None = None,
+                            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One decode step over the INT4 KV cache: q [B, hq, d] bf16 (rotated queries),
+    cache as alloc_kv_cache returns it ([B, hkv, L, d/2] codes, [B, hkv, L] fp16 scale
+    and zero), lens [B] int32 slots attended. Returns out [B, hq, d] (fp32 or bf16).
+    `workspace` (uint8, at least decode_attention_workspace_bytes) is allocated
+    through torch when not given."""
+    _need(q, "q", torch.bfloat16)
+    if q.dim() != 3:
+        raise ValueError(f"q: expected [batch, n_q_heads, head_dim], got shape {tuple(q.shape)}")
+    B, hq, d = q.shape
+    hkv, L = cache["k_cache"].shape[1], cache["k_cache"].shape[2]
+    for name in ("k_cache", "v_cache"):
+        _need(cache[name], name, torch.uint8, q.device, (B, hkv, L, d // 2))
+    for name in ("k_scale", "k_zero", "v_scale", "v_zero"):
+        _need(cache[name], name, torch.float16, q.device, (B, hkv, L))
+    _need(lens, "lens", torch.int32, q.device, (B,))
+    if out is None:
+        if out_dtype not in (torch.float32, torch.bfloat16):
+            raise TypeError(f"out_dtype: expected torch.float32 or torch.bfloat16, got {out_dtype}")
+        out = torch.empty((B, hq, d), dtype=out_dtype, device=q.device)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"out: expected torch.float32 or torch.bfloat16, got {out.dtype}")
+    _need(out, "out", out.dtype, q.device, (B, hq, d))
+    need = decode_attention_workspace_bytes(B, hq, L)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", torch.uint8, q.device)
+    scale = float(softmax_scale) if softmax_scale is not None else 1.0 / float(d) ** 0.5
+    st = spin_decode_attention_int4kv(
+        _ptr(q), _ptr(cache["k_cache"]), _ptr(cache["v_cache"]), _ptr(cache["k_scale"]), _ptr(cache["k_zero"]),
+        _ptr(cache["v_scale"]), _ptr(cache["v_zero"]), _ptr(lens), B, hq, hkv, d, L, scale, _ptr(out),
+        F32 if out.dtype == torch.float32 else BF16, _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("spin_decode_attention_int4kv", st)
+    return out
 
 
 def dequant_hadamard_inverse(codes: torch.Tensor, n: int, scale: torch.Tensor, zero: torch.Tensor | None = None,

@@ -187,6 +187,39 @@ spin_status_t spin_rope_hadamard_kvquant(const void *q, const void *k, const voi
                                                   reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t spin_decode_attention_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t cache_len) {
+  if (batch <= 0 || n_q_heads <= 0 || cache_len <= 0) return 0;
+  return decode_attention_workspace_bytes(batch, n_q_heads, cache_len);
+}
+
+spin_status_t spin_decode_attention_int4kv(const void *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                                           const void *k_scale, const void *k_zero, const void *v_scale,
+                                           const void *v_zero, const int32_t *lens, int32_t batch,
+                                           int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                           int32_t cache_len, float softmax_scale, void *out, int32_t out_dtype,
+                                           void *workspace, size_t workspace_bytes, spin_stream_t stream) {
+  if (batch < 0 || n_q_heads <= 0 || n_kv_heads <= 0 || cache_len < 1 || n_q_heads % n_kv_heads != 0 ||
+      !(softmax_scale > 0.0f) || !std::isfinite(softmax_scale) || (out_dtype != SPIN_BF16 && out_dtype != SPIN_F32))
+    return SPIN_ERR_INVALID_ARG;
+  if (head_dim != 128 || !decode_attention_group_supported(n_q_heads / n_kv_heads) || batch > 65535 ||
+      n_q_heads > 65535 || n_kv_heads > 65535)
+    return SPIN_ERR_UNSUPPORTED_SIZE;
+  if (batch == 0) return SPIN_OK;
+  if (!q || !k_cache || !v_cache || !k_scale || !k_zero || !v_scale || !v_zero || !lens || !out || !workspace)
+    return SPIN_ERR_INVALID_ARG;
+  if (workspace_bytes < decode_attention_workspace_bytes(batch, n_q_heads, cache_len)) return SPIN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(workspace, 16) || !aligned(lens, 4) || !aligned(k_scale, 2) || !aligned(k_zero, 2) ||
+      !aligned(v_scale, 2) || !aligned(v_zero, 2))
+    return SPIN_ERR_MISALIGNED;
+  spin_status_t st = check_device();
+  if (st != SPIN_OK) return st;
+  return cuda_status(launch_decode_attention(q, k_cache, v_cache, k_scale, k_zero, v_scale, v_zero, lens, batch,
+                                             n_q_heads, n_kv_heads, cache_len, softmax_scale, out,
+                                             out_dtype == SPIN_F32, static_cast<float *>(workspace),
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
 spin_status_t spin_dequant_hadamard_inverse(const uint8_t *codes, int64_t rows, int32_t n, int32_t mode,
                                             const void *scale, const void *zero, const uint32_t *sign_bits,
                                             uint32_t flags, void *out, int32_t out_dtype,

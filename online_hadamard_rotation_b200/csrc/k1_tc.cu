@@ -26,18 +26,14 @@
 // resident CTA, after its own group, takes over groups of CTAs that have not started
 // yet (cluster launch control `try_cancel`), so the work spreads dynamically over the
 // SMs and the last groups land wherever an SM is free.
-// Roles (512 threads in four warpgroups, one CTA per SM, persistent over groups):
-//   warps 0-3   +-1 diagonal: XOR of the bf16 sign bits in shared memory, with
-//               each thread's sign words held in registers; one warp on each of
-//               the SM's four schedulers, so the pass loads them evenly
+// Roles (384 threads, one CTA per SM, persistent over groups):
+//   warp 0      TMA producer: 64 KiB per group (boxes of [128 rows][min(B, 64)]
+//               bf16 with 32-, 64- or 128-byte swizzle) into a three-stage ring
+//   warp 1      TMEM owner and MMA issuer (8 MMAs of K = 16 per group)
+//   warps 2-3   +-1 diagonal: XOR of the bf16 sign bits in shared memory, with
+//               each thread's sign words held in registers
 //   warps 4-7   epilogue for TMEM columns 0-127 of each group
 //   warps 8-11  epilogue for columns 128-255
-//   warp 12     TMA producer: 64 KiB per group (boxes of [128 rows][min(B, 64)]
-//               bf16 with 32-, 64- or 128-byte swizzle) into a three-stage ring
-//   warp 13     TMEM owner and MMA issuer (8 MMAs of K = 16 per group)
-//   warps 14-15 idle
-// setmaxnreg moves registers from the sign and control warpgroups to the epilogue
-// warpgroups, whose threads hold 128 fp32 values each.
 // TMEM holds two 256-column accumulators, so the MMA of group i + 1 overlaps
 // the epilogue of group i. Each epilogue thread stores its code bytes straight
 // to global memory. The launch allows programmatic dependent launch: the
@@ -65,14 +61,7 @@ __device__ unsigned int g_device_status = 0u;
 
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kProducerWarp = 12, kMmaWarp = 13;
-// Registers per thread: 128 at launch (65536 / 512); after the split, the sign
-// warpgroup keeps 96, the epilogue warpgroups get 176 and the control warpgroup
-// (producer, MMA issuer, two idle warps) keeps 56. The split adds up to at most the
-// launch's total, so no increase waits for registers that are not there.
-constexpr int kLaunchRegs = 128, kRegsSign = 96, kRegsEpi = 176, kRegsCtl = 56;
-static_assert(kRegsSign * 128 + kRegsEpi * 256 + kRegsCtl * 128 <= kLaunchRegs * kThreads, "register split");
+constexpr int kThreads = 384;
 constexpr int kStages = 3;
 constexpr uint32_t kGroupBytes = 65536;            // one MMA group: 128 rows x 256 columns of bf16
 constexpr uint32_t kOffH = 0;                      // A operand: H_128, K-major, 2 x 16 KiB
@@ -115,8 +104,8 @@ struct Shape {
   static constexpr int CPR = ROWB / 16;            // 16-byte chunks per tile row
   static constexpr uint32_t LAYOUT = ROWB == 128 ? 2u : ROWB == 64 ? 4u : 6u;  // UMMA swizzle: 128, 64, 32 B
   static constexpr uint32_t TOKBYTES = BPT * BOXBYTES;
-  static constexpr int NPOS = (int)(TOKBYTES / 16 / 128);  // sign positions per sign thread
-  static constexpr int SIGN_ITERS = (int)(TOK * TOKBYTES / 16 / 128);  // chunks per sign thread per group
+  static constexpr int NPOS = (int)(TOKBYTES / 16 / 64);  // sign positions per sign thread
+  static constexpr int SIGN_ITERS = (int)(TOK * TOKBYTES / 16 / 64);  // chunks per sign thread per group
   static constexpr int KSTEPS = BOXH / 16;         // MMA steps of K = 16 per row block
   static constexpr int64_t OUTB = (int64_t)ROWS * B / 2;  // code bytes per token (INT4)
   static_assert(KRON ? (KR % 16 == 0 && KR >= 16 && KR <= 128) : (LOGN >= 11 && LOGN <= 15),
@@ -158,27 +147,19 @@ __device__ __forceinline__ int paley_entry(int i, int j, const KronParams &kp) {
   return c * am + ((i >> 1) == (j >> 1) ? bm : 0);
 }
 
-// Group ids in flight from the producer to the sign warps, the MMA issuer and the
-// epilogue. The producer writes step i + kRing only after waiting for the stage of
-// that step to come free, i.e. after the MMA of step i + kRing - kStages (= i + 2)
-// completed; that MMA waited for its accumulator to be released by the step that
-// used it before, i (two accumulators), and the warpgroup(s) of step i release it
-// only after reading the id of step i. So with kRing = kStages + 2 no id is
-// overwritten before every consumer has read it, both when each warpgroup takes
-// every other step and when both take every step.
-constexpr int kRing = kStages + 2;
+constexpr int kRing = 8;  // group ids in flight between the producer and the epilogue
 
 struct Shared {
   uint4 clc_resp;          // response of the pending work-stealing request
   uint64_t full[kStages], sgn[kStages], empty[kStages], tfull[2], tempty[2], drain, clc;
-  uint64_t gfull[kRing];   // group id of step i written (slot i % kRing)
-  int64_t gid[kRing];      // group of the CTA's i-th step (slot i % kRing), -1 once there is none
+  uint64_t gfull[kRing];   // group id i & 7 written
+  int64_t gid[kRing];      // group of the CTA's i-th step (i & 7), -1 once there is none
   int64_t egid[2];         // epilogue warpgroup g's current group
   uint32_t tmem_base;
   int abort;
   int dec[3];
   long long budget;        // clock cycles a wait may take before the CTA gives up
-  float wmax[2][2][4][8];  // [warpgroup][parity of the half processed][warp][token segment]
+  float wmax[2][2][4][8];  // [warpgroup][group parity][warp][token segment]
 };
 static_assert(sizeof(Shared) <= 1024, "barrier area");
 
@@ -223,48 +204,64 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, SS 
   }
 }
 
-__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+
+// Codes on the subnormal grid. For 0 <= t < 2^23 the bit pattern of t * 2^-149 (a
+// multiply by the smallest subnormal, rounded to nearest even) is rne(t), because the
+// grid's spacing is 2^-149; for t < 0 the sign bit is set, so the pattern read as a
+// signed integer is negative. cvt.pack.sat then clamps two such integers to the code
+// range and packs them: biased codes u = code + 2^(b-1) need no clamp of their own.
+// (r0, r1) = rne(v0 cq + bias), rne(v1 cq + bias) as such patterns: one packed FMA and
+// one packed multiply (c2 = {cq, cq}, b2 = {bias, bias}).
+__device__ __forceinline__ void biased_codes_x2(float v0, float v1, uint64_t c2, uint64_t b2, uint32_t &r0,
+                                                uint32_t &r1) {
+  uint64_t A, T, R;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(v0), "f"(v1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(T) : "l"(A), "l"(c2), "l"(b2));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(R) : "l"(T), "l"(0x0000000100000001ull));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(R));
+}
+
+// 1 / x from the hardware reciprocal (within an ulp or so, for the normal x used here).
+__device__ __forceinline__ float rcp_approx(float x) {
   float r;
-  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
 }
 
-// (r0, r1) = bit patterns of fma(a0, 15, 1.5 * 2^23), fma(a1, 15, 1.5 * 2^23): one packed
-// f32x2 FMA rounds two scaled codes to integers (ties to even) in their low mantissa bits.
-__device__ __forceinline__ void round15_x2(float a0, float a1, uint32_t &r0, uint32_t &r1) {
-  uint64_t A, R;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(R) : "l"(A), "l"(0x4170000041700000ull), "l"(0x4B4000004B400000ull));
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(R));
+__device__ __forceinline__ uint64_t pair(float x) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(x));
+  return r;
 }
 
-// INT8 variant: (r0, r1) = bit patterns of fma(a, 255, 1.5 * 2^23), rounding 255 a to
-// an integer (ties to even) in the low mantissa bits.
-__device__ __forceinline__ void round255_x2(float a0, float a1, uint32_t &r0, uint32_t &r1) {
-  uint64_t A, R;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(R) : "l"(A), "l"(0x437F0000437F0000ull), "l"(0x4B4000004B400000ull));
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(R));
-}
-
-// four biased INT8 codes (0..255 in the low byte of each word) -> one word, code k in
-// byte k, converted to two's complement
-__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
-  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410) ^ 0x80808080u;
-}
-
-// 8 consecutive values -> two words of INT8 codes (c255 = 1 / (255 step) in the
-// values' scale)
-__device__ __forceinline__ void codes8_int8(const float *v, float c255, uint32_t &w0, uint32_t &w1) {
-  constexpr float k128 = 128.0f / 255.0f;
-  uint32_t b[8];
-  float t[8];
+// 8 consecutive values -> one word of INT4 codes, value k in nibble k (two's
+// complement): u = clamp(rne(v cq) + 8, 0, 15), code = u - 8 (cq = 1 / step, in the
+// values' scale).
+__device__ __forceinline__ uint32_t codes8(const float *v, uint64_t c2) {
+  constexpr uint64_t kBias = 0x4100000041000000ull;  // {8, 8}
+  uint32_t r[8], d = 0u;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) t[k] = fma_sat(v[k], c255, k128);
+  for (int k = 0; k < 8; k += 2) biased_codes_x2(v[k], v[k + 1], c2, kBias, r[k], r[k + 1]);
 #pragma unroll
-  for (int k = 0; k < 8; k += 2) round255_x2(t[k], t[k + 1], b[k], b[k + 1]);
-  w0 = pack4(b[0], b[1], b[2], b[3]);
-  w1 = pack4(b[4], b[5], b[6], b[7]);
+  for (int k = 6; k >= 0; k -= 2)  // d = (d << 8) | sat(r[k + 1]) << 4 | sat(r[k])
+    asm("cvt.pack.sat.u4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(r[k + 1]), "r"(r[k]), "r"(d));
+  return d ^ 0x88888888u;
+}
+
+// 8 consecutive values -> two words of INT8 codes, value k in byte k (two's
+// complement): u = clamp(rne(v cq) + 128, 0, 255), code = u - 128.
+__device__ __forceinline__ void codes8_int8(const float *v, uint64_t c2, uint32_t &w0, uint32_t &w1) {
+  constexpr uint64_t kBias = 0x4300000043000000ull;  // {128, 128}
+  uint32_t r[8];
+#pragma unroll
+  for (int k = 0; k < 8; k += 2) biased_codes_x2(v[k], v[k + 1], c2, kBias, r[k], r[k + 1]);
+  uint32_t d0 = 0u, d1 = 0u;
+  asm("cvt.pack.sat.u8.s32.b32 %0, %1, %2, %3;" : "=r"(d0) : "r"(r[3]), "r"(r[2]), "r"(d0));
+  asm("cvt.pack.sat.u8.s32.b32 %0, %1, %2, %3;" : "=r"(d0) : "r"(r[1]), "r"(r[0]), "r"(d0));
+  asm("cvt.pack.sat.u8.s32.b32 %0, %1, %2, %3;" : "=r"(d1) : "r"(r[7]), "r"(r[6]), "r"(d1));
+  asm("cvt.pack.sat.u8.s32.b32 %0, %1, %2, %3;" : "=r"(d1) : "r"(r[5]), "r"(r[4]), "r"(d1));
+  w0 = d0 ^ 0x80808080u;
+  w1 = d1 ^ 0x80808080u;
 }
 
 __device__ __forceinline__ void st_v8_cs(void *p, const uint32_t *w) {
@@ -279,11 +276,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-__device__ __forceinline__ uint32_t pack8(const uint32_t (&b)[8]) {
-  const uint32_t e = __byte_perm(__byte_perm(b[0], b[2], 0x0040), __byte_perm(b[4], b[6], 0x0040), 0x5410);
-  const uint32_t o = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
-  return (e | (o << 4)) ^ 0x88888888u;
-}
 
 // byte offset of 16-byte chunk `ch` (0..7) of row `r` in a 128-byte-swizzled [rows][128 B] tile
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t ch) { return r * 128u + ((ch ^ (r & 7u)) << 4); }
@@ -309,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        int stall_test, const __grid_constant__ KronParams kp) {
   using SH = Shape<LOGN, KR>;
   constexpr int B = SH::B, SEG = SH::SEG;
+  const float step_per_unit = clip * inv_sqrt_n / (BITS == 4 ? 7.0f : 127.0f);
   static_assert(!(SIGNS && SH::SPLIT), "the sign masks of n = 32768 do not fit in registers");
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array itself so that accesses
@@ -323,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // finished (programmatic dependent launch lets this prologue overlap their tail).
   tc::grid_dep_wait();
   int64_t first_issued = 0;  // groups the producer issues before the setup barrier
-  if (threadIdx.x == kProducerWarp * 32) {
+  if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&S.full[s], 1);
       tc::mbar_init(&S.sgn[s], 1);
@@ -331,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       tc::mbar_init(&S.tfull[a], 1);
-      tc::mbar_init(&S.tempty[a], SH::SPLIT ? 256 : 128);  // the warpgroup(s) that read the accumulator
+      tc::mbar_init(&S.tempty[a], 256);
     }
     tc::mbar_init(&S.drain, 1);
     tc::mbar_init(&S.clc, 1);
@@ -369,10 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t k0 = kb * 64 + ch * 8 + 2 * j;
       w[j] = a_entry(m, k0) | (a_entry(m, k0 + 1) << 16);
     }
+
     *reinterpret_cast<uint4 *>(smem + kOffH + kb * 16384 + sw128(m, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   tc::fence_proxy_async_smem();
-  if (warp == kMmaWarp) {
+  if (warp == 1) {
     tc::tmem_alloc(&S.tmem_base, 512);
     tc::tmem_relinquish();
   }
@@ -382,11 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = S.tmem_base;
 
   // ------------------------------------------------------------ roles
-  // Each role block starts with its warpgroup's register change (every warp of a
-  // warpgroup, idle ones included, executes it; a block dominated by its own
-  // setmaxnreg is compiled to that register count).
-  if (warp == kProducerWarp) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl) : "memory");
+  if (warp == 0) {
     if (lane == 0) {
       int64_t last[kStages] = {-1, -1, -1};
       for (int64_t i = 0; i < first_issued; ++i) last[i] = i;
@@ -410,14 +400,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p < 0) {
           tc::mbar_arrive(&S.full[st]);  // no copies: the sign warps and the MMA read the end mark
           last[st] = -1;  // its previous copy was consumed before the slot came free
-          // The warpgroup that would take step i + 1 waits for that step's id: mark it
-          // as the end too (its ring slot is free once step i + 1's stage is).
-          const int st1 = (int)((i + 1) % kStages);
-          if (wait_bounded(&S.empty[st1], (uint32_t)(((i + 1) / kStages) & 1) ^ 1u, S, true)) {
-            last[st1] = -1;
-            S.gid[(i + 1) % kRing] = -1;
-            tc::mbar_arrive(&S.gfull[(i + 1) % kRing]);
-          }
           break;
         }
         load_group<LOGN, KR>(smem + kOffX + st * kGroupBytes, &xmap, &S.full[st], p, tokens);
@@ -428,8 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (last[s] >= 0) wait_bounded(&S.full[s], (uint32_t)((last[s] / kStages) & 1), S, false);
       if (pending) wait_bounded(&S.clc, clc_phase, S, false);
     }
-  } else if (warp == kMmaWarp) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl) : "memory");
+  } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = tc::idesc_bf16(128, SH::SPLIT ? 128 : 256, true);
       constexpr uint32_t idesc_neg = idesc | (1u << 13);  // negate A
@@ -473,17 +454,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSign) : "memory");
     if constexpr (SIGNS) {
-      // Thread ts flips the signs of chunks ts + 128 j of each group's 64 KiB.
+      // Thread ts flips the signs of chunks ts + 64 j of each group's 64 KiB.
       // Those chunks sit at NPOS distinct positions of a token's tile; their
       // sign words stay in registers for the whole kernel.
       constexpr int NPOS = SH::NPOS;
-      const uint32_t ts = threadIdx.x;  // 0..127
+      const uint32_t ts = threadIdx.x - 64;  // 0..63
       uint4 mk[NPOS];
 #pragma unroll
       for (int k = 0; k < NPOS; ++k) {
-        const uint32_t pos = ts + 128u * k;  // 16-byte chunk index inside one token's tile
+        const uint32_t pos = ts + 64u * k;  // 16-byte chunk index inside one token's tile
         const uint32_t box = pos / (SH::BOXBYTES / 16), inbox = pos % (SH::BOXBYTES / 16);
         const uint32_t a = inbox / SH::CPR, pc = inbox % SH::CPR;
         const uint32_t ch = SH::ROWB == 128 ? (pc ^ (a & 7u))
@@ -506,37 +486,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           S.dec[2] = ok;
         }
-        tc::named_sync(3, 128);
+        tc::named_sync(3, 64);
         if (!S.dec[2]) break;
         uint4 *X = reinterpret_cast<uint4 *>(smem + kOffX + st * kGroupBytes) + ts;
 #pragma unroll
         for (int j0 = 0; j0 < SH::SIGN_ITERS; j0 += 4) {
           uint4 x[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) x[u] = X[128 * (j0 + u)];
+          for (int u = 0; u < 4; ++u) x[u] = X[64 * (j0 + u)];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const uint4 m = mk[(j0 + u) % NPOS];
-            X[128 * (j0 + u)] = make_uint4(x[u].x ^ m.x, x[u].y ^ m.y, x[u].z ^ m.z, x[u].w ^ m.w);
+            X[64 * (j0 + u)] = make_uint4(x[u].x ^ m.x, x[u].y ^ m.y, x[u].z ^ m.z, x[u].w ^ m.w);
           }
         }
         tc::fence_proxy_async_smem();
-        tc::named_sync(3, 128);
+        tc::named_sync(3, 64);
         if (ts == 0) tc::mbar_arrive(&S.sgn[st]);
       }
     }
-  } else if (warp < 12) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi) : "memory");
-    // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1). Below n = 32768,
-    // warpgroup g takes whole groups, those of steps g, g + 2, ... (accumulator g),
-    // and works through the group's two 128-column halves one after the other, so
-    // the two warpgroups run out of phase (one in its butterflies while the other
-    // waits for TMEM or a barrier). At n = 32768 both take every step, half g each.
+  } else {
+    // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1)
     const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
     const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
-    constexpr int kStep = SH::SPLIT ? 1 : 2, kHalves = SH::SPLIT ? 1 : 2;
-    uint32_t par = 0;  // max buffer in use: alternates with every half processed
-    for (int64_t i = SH::SPLIT ? 0 : g;; i += kStep) {
+    for (int64_t i = 0;; ++i) {
       const int acc = (int)(i & 1);
       // the step's group from the producer's ring, then its accumulator
       auto decide = [&](int slot) {
@@ -560,122 +533,108 @@ __global__ void __launch_bounds__(kThreads, 1)
         p = S.egid[g];
       }
       tc::tc_fence_after();
-#pragma unroll 1
-      for (int hh = 0; hh < kHalves; ++hh, par ^= 1u) {
-        const uint32_t half = SH::SPLIT ? g : (uint32_t)hh;  // accumulator columns 128 half ..
-        float v[kRegs];
-        {
-          uint32_t r[kRegs];
-          const uint32_t taddr = tmem + ((wq * 32u) << 16) + (uint32_t)acc * 256u + half * 128u;
-          tc::tmem_ld32(taddr, r);
-          tc::tmem_ld32(taddr + 32, r + 32);
-          tc::tmem_ld32(taddr + 64, r + 64);
-          tc::tmem_ld32(taddr + 96, r + 96);
-          tc::tmem_wait_ld();
+      float v[kRegs];
+      {
+        uint32_t r[kRegs];
+        const uint32_t taddr = tmem + ((wq * 32u) << 16) + (uint32_t)acc * 256u + g * 128u;
+        tc::tmem_ld32(taddr, r);
+        tc::tmem_ld32(taddr + 32, r + 32);
+        tc::tmem_ld32(taddr + 64, r + 64);
+        tc::tmem_ld32(taddr + 96, r + 96);
+        tc::tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < kRegs; ++k) v[k] = __uint_as_float(r[k]);
+        for (int k = 0; k < kRegs; ++k) v[k] = __uint_as_float(r[k]);
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&S.tempty[acc]);
+      // second Kronecker factor: H_B over b inside each token segment, in registers
+      stage<0>(v);
+      stage<1>(v);
+      stage<2>(v);
+      stage<3>(v);
+      if constexpr (SH::LOGB > 4) stage<4>(v);
+      if constexpr (SH::LOGB > 5) stage<5>(v);
+      if constexpr (SH::LOGB > 6) stage<6>(v);
+      // per-token max |u|: a tree of three-input maxima per segment, then the warp, then the warpgroup
+#pragma unroll
+      for (int sg = 0; sg < SEG; ++sg) {
+        float mx[B / 8];
+#pragma unroll
+        for (int k = 0; k < B / 8; ++k) {
+          const float *w = v + sg * B + 8 * k;
+          mx[k] = fmax3(fmax3(fabsf(w[0]), fabsf(w[1]), fabsf(w[2])), fmax3(fabsf(w[3]), fabsf(w[4]), fabsf(w[5])),
+                        fmaxf(fabsf(w[6]), fabsf(w[7])));
         }
-        if (hh == kHalves - 1) {  // the accumulator is in registers: the MMA may reuse it
-          tc::tc_fence_before();
-          tc::mbar_arrive(&S.tempty[acc]);
-        }
-        // second Kronecker factor: H_B over b inside each token segment, in registers
-        stage<0>(v);
-        stage<1>(v);
-        stage<2>(v);
-        stage<3>(v);
-        if constexpr (SH::LOGB > 4) stage<4>(v);
-        if constexpr (SH::LOGB > 5) stage<5>(v);
-        if constexpr (SH::LOGB > 6) stage<6>(v);
-        // per-token max |u|: a tree of three-input maxima per segment, then the warp, then the warpgroup
 #pragma unroll
-        for (int sg = 0; sg < SEG; ++sg) {
-          float mx[B / 8];
+        for (int h = B / 16; h >= 1; h >>= 1)
 #pragma unroll
-          for (int k = 0; k < B / 8; ++k) {
-            const float *w = v + sg * B + 8 * k;
-            mx[k] = fmax3(fmax3(fabsf(w[0]), fabsf(w[1]), fabsf(w[2])), fmax3(fabsf(w[3]), fabsf(w[4]), fabsf(w[5])),
-                          fmaxf(fabsf(w[6]), fabsf(w[7])));
-          }
+          for (int k = 0; k < h; ++k) mx[k] = fmaxf(mx[k], mx[k + h]);
+        const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mx[0]));
+        if (lane == 0) S.wmax[g][i & 1][wq][sg] = __uint_as_float(wm);
+      }
+      if constexpr (SH::SPLIT) tc::named_sync(4, 256);
+      else tc::named_sync(1 + g, 128);
 #pragma unroll
-          for (int h = B / 16; h >= 1; h >>= 1)
+      for (int sg = 0; sg < SEG; ++sg) {
+        float mu = fmaxf(fmaxf(S.wmax[g][i & 1][0][sg], S.wmax[g][i & 1][1][sg]),
+                         fmaxf(S.wmax[g][i & 1][2][sg], S.wmax[g][i & 1][3][sg]));
+        if constexpr (SH::SPLIT)
+          mu = fmaxf(mu, fmaxf(fmaxf(S.wmax[g ^ 1][i & 1][0][0], S.wmax[g ^ 1][i & 1][1][0]),
+                               fmaxf(S.wmax[g ^ 1][i & 1][2][0], S.wmax[g ^ 1][i & 1][3][0])));
+        // step = max(clip m / qmax, 1e-8) (m in the transform's units times 1/sqrt(n)), and
+        // 1 / step for the codes; a few ulp from the correctly rounded forms, far inside
+        // the step tolerance, and the codes' pre-round values move by ~1e-7 of a step
+        const float s = fmaxf(mu * step_per_unit, 1e-8f);
+        const uint64_t cq = pair(inv_sqrt_n * rcp_approx(s));
+        const int64_t token = SH::SPLIT ? p : p * SH::TOK + g * SEG + sg;
+        if (token >= tokens) continue;
+        if (SH::KRON && row >= (uint32_t)KR) continue;  // TMEM lanes past the tile's rows hold zeros
+        const uint32_t orow = SH::SPLIT ? 128u * g + row : row;  // output row of B values
+        uint8_t *dst = q + token * (SH::OUTB * (BITS / 4)) + orow * (B * BITS / 8);
+        if constexpr (BITS == 8 && B == 16) {  // 16 code bytes per row segment
+          uint32_t w4[4];
+          codes8_int8(v + sg * B, cq, w4[0], w4[1]);
+          codes8_int8(v + sg * B + 8, cq, w4[2], w4[3]);
+          __stcs(reinterpret_cast<uint4 *>(dst), make_uint4(w4[0], w4[1], w4[2], w4[3]));
+        } else if constexpr (BITS == 8) {
+          // one code byte per value: 32 bytes (8 words) at a time
 #pragma unroll
-            for (int k = 0; k < h; ++k) mx[k] = fmaxf(mx[k], mx[k + h]);
-          const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mx[0]));
-          if (lane == 0) S.wmax[g][par][wq][sg] = __uint_as_float(wm);
-        }
-        if constexpr (SH::SPLIT) tc::named_sync(4, 256);
-        else tc::named_sync(1 + g, 128);
-        constexpr float k815 = 8.0f / 15.0f;
+          for (int c8 = 0; c8 < B / 32; ++c8) {
+            uint32_t w8[8];
 #pragma unroll
-        for (int sg = 0; sg < SEG; ++sg) {
-          float mu = fmaxf(fmaxf(S.wmax[g][par][0][sg], S.wmax[g][par][1][sg]),
-                           fmaxf(S.wmax[g][par][2][sg], S.wmax[g][par][3][sg]));
-          if constexpr (SH::SPLIT)
-            mu = fmaxf(mu, fmaxf(fmaxf(S.wmax[g ^ 1][par][0][0], S.wmax[g ^ 1][par][1][0]),
-                                 fmaxf(S.wmax[g ^ 1][par][2][0], S.wmax[g ^ 1][par][3][0])));
-          const float s = fmaxf(clip * (mu * inv_sqrt_n) / (BITS == 4 ? 7.0f : 127.0f), 1e-8f);
-          const float c15 = (inv_sqrt_n / (BITS == 4 ? 15.0f : 255.0f)) / s;
-          const int64_t token = SH::SPLIT ? p : p * SH::TOK + half * SEG + sg;
-          if (token >= tokens) continue;
-          if (SH::KRON && row >= (uint32_t)KR) continue;  // TMEM lanes past the tile's rows hold zeros
-          const uint32_t orow = SH::SPLIT ? 128u * g + row : row;  // output row of B values
-          uint8_t *dst = q + token * (SH::OUTB * (BITS / 4)) + orow * (B * BITS / 8);
-          if constexpr (BITS == 8 && B == 16) {  // 16 code bytes per row segment
-            uint32_t w4[4];
-            codes8_int8(v + sg * B, c15, w4[0], w4[1]);
-            codes8_int8(v + sg * B + 8, c15, w4[2], w4[3]);
-            __stcs(reinterpret_cast<uint4 *>(dst), make_uint4(w4[0], w4[1], w4[2], w4[3]));
-          } else if constexpr (BITS == 8) {
-            // one code byte per value: 32 bytes (8 words) at a time
-#pragma unroll
-            for (int c8 = 0; c8 < B / 32; ++c8) {
-              uint32_t w8[8];
-#pragma unroll
-              for (int h = 0; h < 4; ++h) codes8_int8(v + sg * B + 32 * c8 + 8 * h, c15, w8[2 * h], w8[2 * h + 1]);
-              if constexpr (STORE32) {
-                st_v8_cs(dst + 32 * c8, w8);
-              } else {
-                __stcs(reinterpret_cast<uint4 *>(dst + 32 * c8), make_uint4(w8[0], w8[1], w8[2], w8[3]));
-                __stcs(reinterpret_cast<uint4 *>(dst + 32 * c8) + 1, make_uint4(w8[4], w8[5], w8[6], w8[7]));
-              }
-            }
-          } else {
-            uint32_t words[B / 8];
-#pragma unroll
-            for (int wi = 0; wi < B / 8; ++wi) {
-              uint32_t b[8];
-              float t[8];
-#pragma unroll
-              for (int k = 0; k < 8; ++k) t[k] = fma_sat(v[sg * B + 8 * wi + k], c15, k815);
-#pragma unroll
-              for (int k = 0; k < 8; k += 2) round15_x2(t[k], t[k + 1], b[k], b[k + 1]);
-              words[wi] = pack8(b);
-            }
-            if constexpr (B == 16) {  // 8 code bytes per row segment
-              __stcs(reinterpret_cast<uint2 *>(dst), make_uint2(words[0], words[1]));
-            } else if constexpr (STORE32 && B >= 64) {
-#pragma unroll
-              for (int w8 = 0; w8 < B / 64; ++w8) st_v8_cs(dst + 32 * w8, words + 8 * w8);
+            for (int h = 0; h < 4; ++h) codes8_int8(v + sg * B + 32 * c8 + 8 * h, cq, w8[2 * h], w8[2 * h + 1]);
+            if constexpr (STORE32) {
+              st_v8_cs(dst + 32 * c8, w8);
             } else {
-#pragma unroll
-              for (int w4 = 0; w4 < B / 32; ++w4)
-                __stcs(reinterpret_cast<uint4 *>(dst) + w4,
-                       make_uint4(words[4 * w4], words[4 * w4 + 1], words[4 * w4 + 2], words[4 * w4 + 3]));
+              __stcs(reinterpret_cast<uint4 *>(dst + 32 * c8), make_uint4(w8[0], w8[1], w8[2], w8[3]));
+              __stcs(reinterpret_cast<uint4 *>(dst + 32 * c8) + 1, make_uint4(w8[4], w8[5], w8[6], w8[7]));
             }
           }
-          if (tg == 0 && (!SH::SPLIT || g == 0)) scales[token] = s;
+        } else {
+          uint32_t words[B / 8];
+#pragma unroll
+          for (int wi = 0; wi < B / 8; ++wi) words[wi] = codes8(v + sg * B + 8 * wi, cq);
+          if constexpr (B == 16) {  // 8 code bytes per row segment
+            __stcs(reinterpret_cast<uint2 *>(dst), make_uint2(words[0], words[1]));
+          } else if constexpr (STORE32 && B >= 64) {
+#pragma unroll
+            for (int w8 = 0; w8 < B / 64; ++w8) st_v8_cs(dst + 32 * w8, words + 8 * w8);
+          } else {
+#pragma unroll
+            for (int w4 = 0; w4 < B / 32; ++w4)
+              __stcs(reinterpret_cast<uint4 *>(dst) + w4,
+                     make_uint4(words[4 * w4], words[4 * w4 + 1], words[4 * w4 + 2], words[4 * w4 + 3]));
+          }
         }
+        if (tg == 0 && (!SH::SPLIT || g == 0)) scales[token] = s;
       }
     }
-  } else {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl) : "memory");  // idle warps 14-15
   }
 
   // ------------------------------------------------------------ teardown
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == 1) {
     if (lane == 0) {
       tc::umma_commit(&S.drain);  // arrives once every MMA this thread issued is complete
       wait_bounded(&S.drain, 0, S, false);
@@ -705,13 +664,6 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   auto kern = k1_tc_rotate_quant<LOGN, KR, SIGNS, STORE32, BITS>;
-  static cudaError_t checked = [&] {  // the register split assumes this count at launch
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(kern));
-    if (e != cudaSuccess) return e;
-    return fa.numRegs == kLaunchRegs ? cudaSuccess : cudaErrorInvalidConfiguration;
-  }();
-  if (checked != cudaSuccess) return checked;
   int slots = 0;
   cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreads, (int)kSmemBytes, &slots);
   if (err != cudaSuccess) return err;
@@ -789,19 +741,6 @@ struct SharedS {
   int dec[2];
   long long budget;
 };
-
-// 8 consecutive outputs t[0..7] (already multiplied into the code domain) to one
-// word of 8 nibbles
-__device__ __forceinline__ uint32_t codes8(const float *v, float c15) {
-  constexpr float k815 = 8.0f / 15.0f;
-  uint32_t b[8];
-  float t[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) t[k] = fma_sat(v[k], c15, k815);
-#pragma unroll
-  for (int k = 0; k < 8; k += 2) round15_x2(t[k], t[k + 1], b[k], b[k + 1]);
-  return pack8(b);
-}
 
 __device__ __forceinline__ float absmax32(const uint32_t *r, float m) {
 #pragma unroll
@@ -939,7 +878,8 @@ __global__ void __launch_bounds__(kThreadsS, 1)
       tc::tc_fence_after();
       const int64_t token = p * TOKG + (V == 1 ? 128 * g : 0) + row;
       const bool live = token < tokens;
-      constexpr float QMAX = BITS == 4 ? 7.0f : 127.0f, LEVELS = 2.0f * QMAX + 1.0f;
+      constexpr float QMAX = BITS == 4 ? 7.0f : 127.0f;
+      const float step_per_unit = clip * inv_sqrt_n / QMAX;
       uint8_t *dst = q + token * (int64_t)(16 * V * BITS);
       // 32 code bytes at dst + off: one 32-byte store when aligned, else two 16-byte ones
       auto put32 = [&](int off, const uint32_t *w) {
@@ -964,8 +904,8 @@ __global__ void __launch_bounds__(kThreadsS, 1)
         float mu = 0.0f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) mu = absmax32(r + 32 * c, mu);
-        s = fmaxf(clip * (mu * inv_sqrt_n) / QMAX, 1e-8f);
-        const float c15 = (inv_sqrt_n / LEVELS) / s;
+        s = fmaxf(mu * step_per_unit, 1e-8f);  // as in the large-n kernel
+        const uint64_t cq = pair(inv_sqrt_n * rcp_approx(s));
         if constexpr (BITS == 8) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -975,7 +915,7 @@ __global__ void __launch_bounds__(kThreadsS, 1)
               float f[8];
 #pragma unroll
               for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(r[32 * c + 8 * h + k]);
-              codes8_int8(f, c15, w8[2 * h], w8[2 * h + 1]);
+              codes8_int8(f, cq, w8[2 * h], w8[2 * h + 1]);
             }
             if (live) put32(32 * c, w8);
           }
@@ -986,7 +926,7 @@ __global__ void __launch_bounds__(kThreadsS, 1)
             float f[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(r[8 * wi + k]);
-            words[wi] = codes8(f, c15);
+            words[wi] = codes8(f, cq);
           }
           if (live) {
 #pragma unroll
@@ -1017,8 +957,8 @@ __global__ void __launch_bounds__(kThreadsS, 1)
             mu = fmax3(mu, fabsf(y0 + y1), fabsf(y0 - y1));
           }
         }
-        s = fmaxf(clip * (mu * inv_sqrt_n) / QMAX, 1e-8f);
-        const float c15 = (inv_sqrt_n / LEVELS) / s;
+        s = fmaxf(mu * step_per_unit, 1e-8f);  // as in the large-n kernel
+        const uint64_t cq = pair(inv_sqrt_n * rcp_approx(s));
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {  // pass 2: codes of outputs 32c.. of both halves
           uint32_t a[32], b[32];
@@ -1036,8 +976,8 @@ __global__ void __launch_bounds__(kThreadsS, 1)
                 f0[k] = y0 + y1;
                 f1[k] = y0 - y1;
               }
-              codes8_int8(f0, c15, w0[2 * wi], w0[2 * wi + 1]);
-              codes8_int8(f1, c15, w1[2 * wi], w1[2 * wi + 1]);
+              codes8_int8(f0, cq, w0[2 * wi], w0[2 * wi + 1]);
+              codes8_int8(f1, cq, w1[2 * wi], w1[2 * wi + 1]);
             }
             if (live) {
               put32(32 * c, w0);
@@ -1057,8 +997,8 @@ __global__ void __launch_bounds__(kThreadsS, 1)
                 f0[k] = y0 + y1;
                 f1[k] = y0 - y1;
               }
-              w0[wi] = codes8(f0, c15);
-              w1[wi] = codes8(f1, c15);
+              w0[wi] = codes8(f0, cq);
+              w1[wi] = codes8(f1, cq);
             }
             if (live) {
               __stcs(reinterpret_cast<uint4 *>(dst + 16 * c), make_uint4(w0[0], w0[1], w0[2], w0[3]));

@@ -35,6 +35,15 @@ int paley_type(int m);
 bool kron_supported(int m, int64_t n);
 cudaError_t launch_rotate_quant_kron(int m, int n, int bits, const void *x, int64_t tokens, float clip,
                                      const uint32_t *signs, uint8_t *q, float *scales, cudaStream_t stream);
+// Decode attention over the INT4 KV cache (k4_decode_attn.cu): workspace bytes for
+// the split partials, supported query heads per kv head, and the two launches.
+size_t decode_attention_workspace_bytes(int batch, int n_q_heads, int cache_len);
+bool decode_attention_group_supported(int group);
+cudaError_t launch_decode_attention(const void *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                                    const void *k_scale, const void *k_zero, const void *v_scale,
+                                    const void *v_zero, const int32_t *lens, int batch, int n_q_heads,
+                                    int n_kv_heads, int cache_len, float softmax_scale, void *out, bool out_f32,
+                                    float *workspace, cudaStream_t stream);
 cudaError_t launch_rotate_quant_tc(int log_n, int bits, const void *x, int64_t tokens, float clip,
                                    const uint32_t *signs, uint8_t *q, float *scales, cudaStream_t stream);
 

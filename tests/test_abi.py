@@ -201,3 +201,26 @@ def test_kron_size_rules(L):
     assert f(None, 0, 28, 14336, 1.0, None, 1, 4, None, None, None) == BAD      # SPIN_NO_ROTATE is not a flag here
     assert f(None, 0, 28, 14336, 1.5, None, 0, 4, None, None, None) == BAD      # clip
     assert f(None, 4, 28, 14336, 1.0, None, 0, 4, None, None, None) == BAD      # null pointers
+
+
+def test_decode_attention_host_rules(L):
+    """Workspace size and argument rules of the decode-attention entry point; batch = 0
+    and every rejected argument return before any device access."""
+    ws = L.spin_decode_attention_workspace_bytes
+    ws.argtypes = [C.c_int32] * 3
+    ws.restype = C.c_size_t
+    assert ws(4, 32, 4096) == 4 * 32 * 16 * 130 * 4  # 16 chunks of 256 slots, 128 + 2 floats each
+    assert ws(1, 8, 257) == 8 * 2 * 130 * 4 and ws(0, 8, 10) == 0 and ws(1, 8, 0) == 0
+    f = L.spin_decode_attention_int4kv
+    f.argtypes = [C.c_void_p] * 8 + [C.c_int32] * 5 + [C.c_float, C.c_void_p, C.c_int32, C.c_void_p, C.c_size_t,
+                                                      C.c_void_p]
+    f.restype = C.c_int
+    z = [None] * 8
+    assert f(*z, 0, 32, 8, 128, 4096, 0.088, None, 1, None, 0, None) == 0      # batch 0: no-op
+    assert f(*z, 0, 32, 8, 64, 4096, 0.088, None, 1, None, 0, None) == 2       # head_dim
+    assert f(*z, 0, 24, 8, 128, 4096, 0.088, None, 1, None, 0, None) == 2      # 3 query heads per kv head
+    assert f(*z, 0, 30, 8, 128, 4096, 0.088, None, 1, None, 0, None) == 1      # not a multiple
+    assert f(*z, 0, 32, 8, 128, 0, 0.088, None, 1, None, 0, None) == 1         # empty cache
+    assert f(*z, 0, 32, 8, 128, 4096, -1.0, None, 1, None, 0, None) == 1       # softmax scale
+    assert f(*z, 0, 32, 8, 128, 4096, 0.088, None, 7, None, 0, None) == 1      # out dtype
+    assert f(*z, 2, 32, 8, 128, 4096, 0.088, None, 1, None, 0, None) == 1      # null pointers
