@@ -69,11 +69,6 @@ constexpr double k2PiHi = 6.283185307179586;         // 2 pi rounded to double
 constexpr double k2PiLo = 2.4492935982947064e-16;    // 2 pi - k2PiHi
 constexpr long long kTimeoutCycles = 4000000000LL;   // about two seconds
 
-__device__ __forceinline__ float fma_sat(float a, float b, float c) {
-  float r;
-  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -85,16 +80,34 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return r;
 }
 
-// (r0, r1) = bit patterns of fma(a, 15, 1.5 * 2^23) for a pair: one packed FMA rounds two
-// scaled codes to integers (ties to even) in their low mantissa bits.
-__device__ __forceinline__ void round15_x2(float a0, float a1, uint32_t &r0, uint32_t &r1) {
-  uint64_t A, R;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(R) : "l"(A), "l"(0x4170000041700000ull), "l"(0x4B4000004B400000ull));
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(R));
+// Eight consecutive values -> one word of unsigned INT4 codes, value k in nibble k:
+// u = clamp(rne(v c + z), 0, 15) (c = 1 / step, z the integer zero point). One packed
+// FMA forms v c + z, a packed multiply by 2^-149 (the smallest subnormal) rounds it to
+// nearest even onto the subnormal grid, so the bit pattern is the integer (negative
+// values keep the sign bit), and cvt.pack.sat clamps two of them to [0, 15] and packs
+// them (second operand in the low nibble).
+__device__ __forceinline__ uint32_t codes8_asym(const float *v, uint64_t c2, uint64_t z2) {
+  uint32_t r[8], d = 0u;
+#pragma unroll
+  for (int k = 0; k < 8; k += 2) {
+    uint64_t A, T, R;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(v[k]), "f"(v[k + 1]));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(T) : "l"(A), "l"(c2), "l"(z2));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(R) : "l"(T), "l"(0x0000000100000001ull));
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(r[k]), "=r"(r[k + 1]) : "l"(R));
+  }
+#pragma unroll
+  for (int k = 6; k >= 0; k -= 2)  // d = (d << 8) | sat(r[k + 1]) << 4 | sat(r[k])
+    asm("cvt.pack.sat.u4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(r[k + 1]), "r"(r[k]), "r"(d));
+  return d;
 }
 
-// (a0, a1) <- (a0, a1) * (s, s) + (w0, w1)
+__device__ __forceinline__ uint64_t pair(float x) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(x));
+  return r;
+}
+
 __device__ __forceinline__ void fma_pair(float &a0, float &a1, float s, float w0, float w1) {
   uint64_t A, S, Wv, R;
   asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
@@ -279,22 +292,12 @@ __device__ __forceinline__ void quant_asym_store(const float (&x)[64], float cli
   } else {
     z = fminf(fmaxf(rintf(-lo / s), 0.f), 15.f);
   }
-  const float c15 = (1.0f / s) / 15.0f, z15 = z / 15.0f;
+  const uint64_t c2 = pair(1.0f / s), z2 = pair(z);
   uint32_t words[2][4];
 #pragma unroll
   for (int wi = 0; wi < 4; ++wi) {  // registers 8 wi .. 8 wi + 7 and 32 + 8 wi .. 32 + 8 wi + 7
-    uint32_t c[2][8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int j = 8 * wi + i;
-      round15_x2(fma_sat(x[j], c15, z15), fma_sat(x[j + 32], c15, z15), c[0][i], c[1][i]);
-    }
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const uint32_t e = __byte_perm(__byte_perm(c[q][0], c[q][2], 0x0040), __byte_perm(c[q][4], c[q][6], 0x0040), 0x5410);
-      const uint32_t o = __byte_perm(__byte_perm(c[q][1], c[q][3], 0x0040), __byte_perm(c[q][5], c[q][7], 0x0040), 0x5410);
-      words[q][wi] = e | (o << 4);
-    }
+    words[0][wi] = codes8_asym(x + 8 * wi, c2, z2);
+    words[1][wi] = codes8_asym(x + 32 + 8 * wi, c2, z2);
   }
   // registers 32 q .. 32 q + 31 -> code bytes 32 q + 16 h .. + 15
   __stcs(reinterpret_cast<uint4 *>(codes_row + 16 * h), make_uint4(words[0][0], words[0][1], words[0][2], words[0][3]));
