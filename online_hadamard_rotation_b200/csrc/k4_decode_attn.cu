@@ -108,6 +108,27 @@ __global__ void __launch_bounds__(kThreads)
     return;
   }
   const int64_t row0 = ((int64_t)b * hkv + g) * cache_len + start;  // first cache row of the chunk
+  const int dg = t & 15, sg = t >> 4;  // value phase: dims 8 dg .. 8 dg + 7 of slots sg, sg + 16, ...
+
+  // every global load of the block is issued here, before any barrier, so their
+  // latencies overlap: thread t's key row (slot t), and its 16 words of value codes
+  uint4 krow[4] = {};
+  float ksc = 0.0f, kzr = 0.0f, vsc = 0.0f, vzr = 0.0f;
+  if (t < cnt) {
+    const uint4 *kr = reinterpret_cast<const uint4 *>(kc + (row0 + t) * (kD / 2));
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) krow[c4] = __ldg(kr + c4);
+    ksc = __half2float(ks[row0 + t]);
+    kzr = __half2float(kz[row0 + t]);
+    vsc = __half2float(vs[row0 + t]);
+    vzr = __half2float(vz[row0 + t]);
+  }
+  uint32_t vw[kChunk / 16];
+#pragma unroll
+  for (int u = 0; u < kChunk / 16; ++u) {
+    const int j = sg + 16 * u;
+    vw[u] = j < cnt ? __ldg(reinterpret_cast<const uint32_t *>(vc + (row0 + j) * (kD / 2)) + dg) : 0u;
+  }
 
   // queries of the G heads as fp32, and their sums
   for (int i = t; i < G * kD; i += kThreads)
@@ -124,15 +145,12 @@ __global__ void __launch_bounds__(kThreads)
   // scores: thread t takes slot start + t
   float sc[G];
   if (t < cnt) {
-    const int64_t row = row0 + t;
-    const uint4 *kr = reinterpret_cast<const uint4 *>(kc + row * (kD / 2));
     float2 acc[G];
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) acc[hh] = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4) {
-      const uint4 wv = __ldg(kr + c4);
-      const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+      const uint32_t words[4] = {krow[c4].x, krow[c4].y, krow[c4].z, krow[c4].w};
 #pragma unroll
       for (int wi = 0; wi < 4; ++wi) {
         float2 f[4];
@@ -149,9 +167,8 @@ __global__ void __launch_bounds__(kThreads)
         }
       }
     }
-    const float s = __half2float(ks[row]), z = __half2float(kz[row]);
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) sc[hh] = s * ((acc[hh].x + acc[hh].y) - z * S.qsum[hh]) * softmax_scale;
+    for (int hh = 0; hh < G; ++hh) sc[hh] = ksc * ((acc[hh].x + acc[hh].y) - kzr * S.qsum[hh]) * softmax_scale;
   } else {
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) sc[hh] = -INFINITY;
@@ -173,11 +190,6 @@ __global__ void __launch_bounds__(kThreads)
   // p_j = exp(score_j - m), l = sum p_j; w_j = p_j s'_j and sum_j w_j z'_j
   float p[G], wz[G];
   {
-    float vsc = 0.0f, vzr = 0.0f;
-    if (t < cnt) {
-      vsc = __half2float(vs[row0 + t]);
-      vzr = __half2float(vz[row0 + t]);
-    }
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
       p[hh] = t < cnt ? __expf(sc[hh] - S.m[hh]) : 0.0f;
@@ -212,18 +224,20 @@ __global__ void __launch_bounds__(kThreads)
     S.z[t] = v;
   }
 
-  // value sums: thread t takes dims 8 (t & 15) .. + 7 of every 16th slot from t >> 4
+  // value sums: thread t takes dims 8 dg .. 8 dg + 7 of every 16th slot from sg (the
+  // code words loaded at the start)
   {
-    const int dg = t & 15, sg = t >> 4;
     float2 acc[G][4];
 #pragma unroll
     for (int hh = 0; hh < G; ++hh)
 #pragma unroll
       for (int k = 0; k < 4; ++k) acc[hh][k] = make_float2(0.0f, 0.0f);
-    for (int j = sg; j < cnt; j += 16) {
-      const uint32_t wv = __ldg(reinterpret_cast<const uint32_t *>(vc + (row0 + j) * (kD / 2)) + dg);
+#pragma unroll
+    for (int u = 0; u < kChunk / 16; ++u) {
+      const int j = sg + 16 * u;
+      if (j >= cnt) break;
       float2 f[4];
-      nibbles8(wv, f);
+      nibbles8(vw[u], f);
       float wj[G];
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) wj[hh] = S.w[j][hh];
@@ -274,13 +288,31 @@ __global__ void __launch_bounds__(kD)
   len = len < 0 ? 0 : (len > cache_len ? cache_len : len);
   const int used = (len + kChunk - 1) / kChunk;  // chunks that hold slots of this row
   const float *pp = ws + ((int64_t)b * hq + h) * nsplit * kPart;
-  float M = -INFINITY;
-  for (int c = 0; c < used; ++c) M = fmaxf(M, pp[c * kPart]);
-  float num = 0.0f, den = 0.0f;
-  for (int c = 0; c < used; ++c) {
-    const float e = __expf(pp[c * kPart] - M);
-    den += e * pp[c * kPart + 1];
-    num += e * pp[c * kPart + 2 + i];
+  // chunks in batches of 8 whose loads are all issued before any is used; a running
+  // maximum rescales the sums when it grows
+  float M = -INFINITY, num = 0.0f, den = 0.0f;
+  for (int c0 = 0; c0 < used; c0 += 8) {
+    float m[8], l[8], a[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const bool in = c0 + u < used;
+      m[u] = in ? pp[(c0 + u) * kPart] : -INFINITY;
+      l[u] = in ? pp[(c0 + u) * kPart + 1] : 0.0f;
+      a[u] = in ? pp[(c0 + u) * kPart + 2 + i] : 0.0f;
+    }
+    float Mn = M;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) Mn = fmaxf(Mn, m[u]);
+    const float r = M == -INFINITY ? 0.0f : __expf(M - Mn);
+    num *= r;
+    den *= r;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float e = m[u] == -INFINITY ? 0.0f : __expf(m[u] - Mn);
+      den += e * l[u];
+      num += e * a[u];
+    }
+    M = Mn;
   }
   const float r = used > 0 ? num / den : 0.0f;
   const int64_t o = ((int64_t)b * hq + h) * kD + i;
