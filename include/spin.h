@@ -118,12 +118,12 @@ spin_status_t spin_hadamard_quant_int4(const void *x_bf16, int64_t tokens, int32
  *             SPIN_NO_ROTATE: quantise x directly (no D, no H), used to
  *               measure the direct-quantisation error;
  *             SPIN_CUDA_CORES_ONLY: at n = 128 and 256 the transform, and at
- *               n = 2048 .. 16384, and at n = 32768 without sign_bits,
- *               the first H_128 Kronecker factor (two of them at n = 32768),
- *               normally runs on the tensor cores (exact +-1 x bf16 products,
- *               fp32 accumulation; at n = 128 and 256 the diagonal rides in the
- *               +-1 operand); this bit selects the kernel that runs every
- *               butterfly on the CUDA cores instead.
+ *               n = 512 .. 16384, and at n = 32768 without sign_bits,
+ *               the first Kronecker factor (H_128; two of them at n = 32768;
+ *               H_64 at n = 512) normally runs on the tensor cores (exact
+ *               +-1 x bf16 products, fp32 accumulation; at n = 128 and 256 the
+ *               diagonal rides in the +-1 operand); this bit selects the kernel
+ *               that runs every butterfly on the CUDA cores instead.
  *               Both give the same codes up to the rounding-tie band and the
  *               same steps to fp32 accumulation order. By default the
  *               tensor-core kernel runs only when the batch has at least 128 MMA
@@ -255,16 +255,16 @@ spin_status_t spin_rope_hadamard_kvquant(const void *q, const void *k, const voi
  *  sign_bits  nullable, as in spin_hadamard_quant_int4_ex
  *  flags      bitwise OR of SPIN_NO_ROTATE and at most one of
  *             SPIN_CUDA_CORES_ONLY: at n = 128 and 256 the transform, and at
- *               n = 4096 .. 32768 its first H_128 Kronecker factor, normally
- *               run on the tensor cores (the codes minus the zero point are
- *               exact fp16 integers and so is every sum, so both kernels give
- *               the same bits); this bit selects the kernel that runs every
- *               butterfly on the CUDA cores instead. By default the tensor-core
- *               kernel runs only from 128 MMA groups up (128 rows per group at
- *               n = 128 and 256, 128 x max(1, 256 / (n/128)) rows from 4096);
- *             SPIN_TENSOR_CORES: use the tensor-core kernel wherever n allows
- *               (n = 128, 256 or n >= 4096, not with SPIN_NO_ROTATE), whatever
- *               the row count.
+ *               n = 512 .. 32768 its first Kronecker factor (H_128; H_64 at
+ *               n = 512), normally run on the tensor cores (the codes minus the
+ *               zero point are exact fp16 integers and so is every sum, so both
+ *               kernels give the same bits); this bit selects the kernel that
+ *               runs every butterfly on the CUDA cores instead. By default the
+ *               tensor-core kernel runs only from 128 MMA groups up (128 rows per
+ *               group at n = 128 and 256, 64 at n = 512, 128 x max(1, 256 /
+ *               (n/128)) rows from 1024);
+ *             SPIN_TENSOR_CORES: use the tensor-core kernel at any row count
+ *               (not with SPIN_NO_ROTATE).
  *             Other bits: SPIN_ERR_INVALID_ARG.
  *  out        [rows, n] bf16 or fp32 (out_dtype), 16-byte aligned
  */

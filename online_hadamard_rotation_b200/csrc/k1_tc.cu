@@ -10,7 +10,8 @@
 // Outlier Curse": symmetric INT4, step max|y| / 7.
 //
 // A token row x of n = 128 B bf16 values is the 128 x B matrix X[a][b], with
-// element index e = B a + b (B = 16, 32, 64, 128; n = 32768 is two such blocks,
+// element index e = B a + b (B = 8, 16, 32, 64, 128; n = 32768 is two such blocks,
+// n = 512 two 64-row tokens per 128-row block,
 // see Shape). Then H_n x = vec(H_128 X H_B):
 //   1. tcgen05.mma computes Y = H_128 X (contraction over a) for 256 / B tokens
 //      at once (M = 128, N = 256, K = 128, bf16 in, fp32 accumulate in TMEM).
@@ -67,7 +68,7 @@ constexpr uint32_t kGroupBytes = 65536;            // one MMA group: 128 rows x 
 constexpr uint32_t kOffH = 0;                      // A operand: H_128, K-major, 2 x 16 KiB
 constexpr uint32_t kOffX = 32768;                  // ring of kStages x 64 KiB
 constexpr uint32_t kOffBar = kOffX + kStages * kGroupBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 1024 + 1024;  // barrier area + alignment slack
+constexpr uint32_t kSmemBytes = kOffBar + 2048 + 1024;  // barrier area + alignment slack (227 KiB in all)
 constexpr long long kTimeoutCycles = 4000000000LL;     // about two seconds
 constexpr long long kStallTestCycles = 2000000LL;      // about a millisecond, for the stall test hook
 
@@ -90,27 +91,39 @@ template <int LOGN, int KR = 0>
 struct Shape {
   static constexpr bool KRON = KR > 0;
   static constexpr bool SPLIT = !KRON && LOGN == 15;
-  static constexpr int B = (SPLIT || KRON) ? 128 : 1 << (LOGN - 7);  // columns per row (last factor size)
-  static constexpr int LOGB = (SPLIT || KRON) ? 7 : LOGN - 7;
+  // n = 512 (PAIR): a token is 64 rows of B = 8 columns (H_512 = H_64 (x) H_8) and each
+  // 128-row TMA box holds two consecutive tokens, rows 0-63 and 64-127. The MMA's A
+  // operand is H_64 (+) H_64 (block diagonal), so the two tokens stay apart; TMEM lanes
+  // 0-63 hold the first token's rows, 64-127 the second's, and a token's max spans two
+  // of an epilogue warpgroup's warps.
+  static constexpr bool PAIR = !KRON && LOGN == 9;
+  static constexpr int B = (SPLIT || KRON) ? 128 : PAIR ? 8 : 1 << (LOGN - 7);  // columns per row
+  static constexpr int LOGB = (SPLIT || KRON) ? 7 : PAIR ? 3 : LOGN - 7;
   static constexpr int BOXH = KRON ? KR : 128;     // rows per TMA box and per MMA contraction
-  static constexpr int ROWS = SPLIT ? 256 : BOXH;  // rows per token
-  static constexpr int TOK = SPLIT ? 1 : 256 / B;  // tokens per MMA group
-  static constexpr int SEG = SPLIT ? 1 : 128 / B;  // token segments per epilogue thread
+  static constexpr int ROWS = SPLIT ? 256 : PAIR ? 64 : BOXH;  // rows per token
+  static constexpr int TPB = PAIR ? 2 : 1;         // tokens per 128-row box
+  static constexpr int TOK = SPLIT ? 1 : TPB * 256 / B;  // tokens per MMA group
+  static constexpr int SEG = SPLIT ? 1 : 128 / B;  // column segments per epilogue thread
   static constexpr int BOXW = B < 64 ? B : 64;     // TMA box width (columns)
-  static constexpr int ROWB = BOXW * 2;            // bytes per smem tile row (64 or 128)
+  static constexpr int ROWB = BOXW * 2;            // bytes per smem tile row (16, 32, 64 or 128)
   static constexpr int CBOX = B / BOXW;            // column boxes per row block
-  static constexpr int BPT = CBOX * ROWS / BOXH;   // boxes per token
+  static constexpr int BPT = PAIR ? 1 : CBOX * ROWS / BOXH;  // boxes per token (PAIR: per token pair)
   static constexpr uint32_t BOXBYTES = (uint32_t)BOXH * ROWB;  // bytes per box
   static constexpr int CPR = ROWB / 16;            // 16-byte chunks per tile row
-  static constexpr uint32_t LAYOUT = ROWB == 128 ? 2u : ROWB == 64 ? 4u : 6u;  // UMMA swizzle: 128, 64, 32 B
-  static constexpr uint32_t TOKBYTES = BPT * BOXBYTES;
+  static constexpr uint32_t LAYOUT = ROWB == 128 ? 2u : ROWB == 64 ? 4u : ROWB == 32 ? 6u : 0u;  // UMMA swizzle: 128, 64, 32 B, none
+  // MN-major B operand strides: swizzled tiles step by box along N and by 8 rows along
+  // K; the no-swizzle layout (16-byte rows, one 8 x 16 B core matrix per 8 rows) swaps
+  // the roles of the two offsets, its leading offset stepping along K.
+  static constexpr uint32_t LBO = LAYOUT == 0 ? 8u * ROWB : BOXBYTES;
+  static constexpr uint32_t SBO = LAYOUT == 0 ? BOXBYTES : 8u * ROWB;
+  static constexpr uint32_t TOKBYTES = (uint32_t)ROWS * B * 2;  // input bytes of one token
   static constexpr int NPOS = (int)(TOKBYTES / 16 / 64);  // sign positions per sign thread
   static constexpr int SIGN_ITERS = (int)(TOK * TOKBYTES / 16 / 64);  // chunks per sign thread per group
   static constexpr int KSTEPS = BOXH / 16;         // MMA steps of K = 16 per row block
   static constexpr int64_t OUTB = (int64_t)ROWS * B / 2;  // code bytes per token (INT4)
-  static_assert(KRON ? (KR % 16 == 0 && KR >= 16 && KR <= 128) : (LOGN >= 11 && LOGN <= 15),
-                "this tensor-core R4 kernel covers n = 2048 .. 32768 and n = 128 KR, KR = 16 .. 128");
-  static_assert(TOK * TOKBYTES <= kGroupBytes && SIGN_ITERS % 4 == 0, "stage layout");
+  static_assert(KRON ? (KR % 16 == 0 && KR >= 16 && KR <= 128) : (LOGN >= 9 && LOGN <= 15),
+                "this tensor-core R4 kernel covers n = 512 .. 32768 and n = 128 KR, KR = 16 .. 128");
+  static_assert(TOK * TOKBYTES <= kGroupBytes && SIGN_ITERS % 4 == 0 && NPOS >= 1, "stage layout");
 };
 
 // Paley's Hadamard matrix of order m, as a kernel argument: type I (q = m - 1, prime,
@@ -159,9 +172,9 @@ struct Shared {
   int abort;
   int dec[3];
   long long budget;        // clock cycles a wait may take before the CTA gives up
-  float wmax[2][2][4][8];  // [warpgroup][group parity][warp][token segment]
+  float wmax[2][2][4][16];  // [warpgroup][group parity][warp][token segment]
 };
-static_assert(sizeof(Shared) <= 1024, "barrier area");
+static_assert(sizeof(Shared) <= 2048, "barrier area");
 
 // Work stealing by cluster launch control: ask the hardware to cancel a CTA of this
 // grid that has not started yet; its 16-byte response lands in `resp` and completes
@@ -287,6 +300,13 @@ __device__ __forceinline__ void load_group(uint8_t *dst, const CUtensorMap *map,
   using SH = Shape<LOGN, KR>;
   const int64_t t0 = p * SH::TOK;
   const int nvalid = (int)((tokens - t0) < SH::TOK ? (tokens - t0) : SH::TOK);
+  if constexpr (SH::PAIR) {  // whole boxes of two tokens; rows past the last token read as zero
+    const int nbox = (nvalid + 1) / 2;
+    tc::mbar_arrive_expect_tx(bar, (uint32_t)nbox * SH::BOXBYTES);
+    for (int i = 0; i < nbox; ++i)
+      tc::tma_load_2d(dst + i * SH::BOXBYTES, map, bar, 0, (int)((t0 + 2 * i) * SH::ROWS));
+    return;
+  }
   tc::mbar_arrive_expect_tx(bar, (uint32_t)nvalid * SH::TOKBYTES);
   for (int t = 0; t < nvalid; ++t)
     for (int j = 0; j < SH::BPT; ++j)
@@ -350,6 +370,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int h = paley_entry((int)m / kp.bq, (int)k / kp.bq, kp) *
                     ((__popc((m % kp.bq) & (k % kp.bq)) & 1) ? -1 : 1);
       return h > 0 ? 0x3F80u : 0xBF80u;
+    } else if constexpr (SH::PAIR) {  // H_64 (+) H_64
+      if ((m >> 6) != (k >> 6)) return 0u;
+      return (__popc(m & k & 63u) & 1) ? 0xBF80u : 0x3F80u;
     } else {
       return (__popc(m & k) & 1) ? 0xBF80u : 0x3F80u;
     }
@@ -431,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int s = 0; s < 8; ++s) {
                 const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
                 uint64_t bd = tc::smem_desc(sX + st * kGroupBytes + v * SH::CBOX * SH::BOXBYTES + s * 16 * SH::ROWB,
-                                            SH::BOXBYTES, 8 * SH::ROWB);
+                                            SH::LBO, SH::SBO);
                 bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
                 tc::umma_bf16(tmem + acc * 256 + u * 128, ad, bd, (u & v) ? idesc_neg : idesc,
                               (v > 0 || s > 0) ? 1u : 0u);
@@ -442,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // A: 16 columns k of H per step. B: rows a = 16 s .. 16 s + 15 of every box
             // (MN-major: boxes of BOXW columns BOXBYTES apart, 8-row groups 8 ROWB apart).
             const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-            uint64_t bd = tc::smem_desc(sX + st * kGroupBytes + s * 16 * SH::ROWB, SH::BOXBYTES, 8 * SH::ROWB);
+            uint64_t bd = tc::smem_desc(sX + st * kGroupBytes + s * 16 * SH::ROWB, SH::LBO, SH::SBO);
             bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
             tc::umma_bf16(tmem + acc * 256, ad, bd, idesc, s > 0 ? 1u : 0u);
           }
@@ -468,7 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a = inbox / SH::CPR, pc = inbox % SH::CPR;
         const uint32_t ch = SH::ROWB == 128 ? (pc ^ (a & 7u))
                             : SH::ROWB == 64 ? (pc ^ ((a >> 1) & 3u))
-                                             : (pc ^ ((a >> 2) & 1u));
+                            : SH::ROWB == 32 ? (pc ^ ((a >> 2) & 1u))
+                                             : pc;  // 16-byte rows: no swizzle
         const uint32_t e = a * B + box * SH::BOXW + ch * 8u;
         const uint32_t byte = (__ldg(signs + (e >> 5)) >> (e & 31u)) & 0xFFu;
         uint32_t w[4];
@@ -551,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       stage<0>(v);
       stage<1>(v);
       stage<2>(v);
-      stage<3>(v);
+      if constexpr (SH::LOGB > 3) stage<3>(v);
       if constexpr (SH::LOGB > 4) stage<4>(v);
       if constexpr (SH::LOGB > 5) stage<5>(v);
       if constexpr (SH::LOGB > 6) stage<6>(v);
@@ -576,8 +600,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       else tc::named_sync(1 + g, 128);
 #pragma unroll
       for (int sg = 0; sg < SEG; ++sg) {
-        float mu = fmaxf(fmaxf(S.wmax[g][i & 1][0][sg], S.wmax[g][i & 1][1][sg]),
-                         fmaxf(S.wmax[g][i & 1][2][sg], S.wmax[g][i & 1][3][sg]));
+        float mu;
+        if constexpr (SH::PAIR)  // the token of this thread's row: warps 0-1 or 2-3
+          mu = fmaxf(S.wmax[g][i & 1][wq & 2u][sg], S.wmax[g][i & 1][(wq & 2u) + 1][sg]);
+        else
+          mu = fmaxf(fmaxf(S.wmax[g][i & 1][0][sg], S.wmax[g][i & 1][1][sg]),
+                     fmaxf(S.wmax[g][i & 1][2][sg], S.wmax[g][i & 1][3][sg]));
         if constexpr (SH::SPLIT)
           mu = fmaxf(mu, fmaxf(fmaxf(S.wmax[g ^ 1][i & 1][0][0], S.wmax[g ^ 1][i & 1][1][0]),
                                fmaxf(S.wmax[g ^ 1][i & 1][2][0], S.wmax[g ^ 1][i & 1][3][0])));
@@ -586,12 +614,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the step tolerance, and the codes' pre-round values move by ~1e-7 of a step
         const float s = fmaxf(mu * step_per_unit, 1e-8f);
         const uint64_t cq = pair(inv_sqrt_n * rcp_approx(s));
-        const int64_t token = SH::SPLIT ? p : p * SH::TOK + g * SEG + sg;
+        const int64_t token = SH::SPLIT ? p
+                              : SH::PAIR ? p * SH::TOK + 2 * (g * SEG + sg) + (row >> 6)
+                                         : p * SH::TOK + g * SEG + sg;
         if (token >= tokens) continue;
         if (SH::KRON && row >= (uint32_t)KR) continue;  // TMEM lanes past the tile's rows hold zeros
-        const uint32_t orow = SH::SPLIT ? 128u * g + row : row;  // output row of B values
+        const uint32_t orow = SH::SPLIT ? 128u * g + row : SH::PAIR ? (row & 63u) : row;  // output row of B values
         uint8_t *dst = q + token * (SH::OUTB * (BITS / 4)) + orow * (B * BITS / 8);
-        if constexpr (BITS == 8 && B == 16) {  // 16 code bytes per row segment
+        if constexpr (BITS == 8 && B == 8) {  // 8 code bytes per row segment
+          uint32_t w2[2];
+          codes8_int8(v + sg * B, cq, w2[0], w2[1]);
+          __stcs(reinterpret_cast<uint2 *>(dst), make_uint2(w2[0], w2[1]));
+        } else if constexpr (BITS == 4 && B == 8) {  // 4 code bytes per row segment
+          __stcs(reinterpret_cast<unsigned int *>(dst), codes8(v + sg * B, cq));
+        } else if constexpr (BITS == 8 && B == 16) {  // 16 code bytes per row segment
           uint32_t w4[4];
           codes8_int8(v + sg * B, cq, w4[0], w4[1]);
           codes8_int8(v + sg * B + 8, cq, w4[2], w4[3]);
@@ -626,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      make_uint4(words[4 * w4], words[4 * w4 + 1], words[4 * w4 + 2], words[4 * w4 + 3]));
           }
         }
-        if (tg == 0 && (!SH::SPLIT || g == 0)) scales[token] = s;
+        if ((SH::PAIR ? (tg & 63u) : tg) == 0 && (!SH::SPLIT || g == 0)) scales[token] = s;
       }
     }
   }
@@ -660,7 +696,8 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
                   SH::ROWB == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
                   : SH::ROWB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                   : CU_TENSOR_MAP_SWIZZLE_32B,
+                  : SH::ROWB == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                   : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   auto kern = k1_tc_rotate_quant<LOGN, KR, SIGNS, STORE32, BITS>;
@@ -1082,6 +1119,8 @@ cudaError_t launch_tc_bits(int log_n, const void *x, int64_t tokens, float clip,
   switch (log_n) {
     case 7: return launch_small<1, BITS>(x, tokens, clip, signs, q, scales, stream);
     case 8: return launch_small<2, BITS>(x, tokens, clip, signs, q, scales, stream);
+    case 9: return launch_n<9, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
+    case 10: return launch_n<10, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
     case 11: return launch_n<11, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
     case 12: return launch_n<12, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
     case 13: return launch_n<13, BITS>(x, tokens, clip, signs, q, scales, stream, stall);
@@ -1174,10 +1213,11 @@ bool tc_rotate_quant_supported(int log_n, int64_t tokens, uint32_t flags, bool h
     const int64_t tok_per_group = log_n == 7 ? 256 : 128;
     return (flags & kTensorCores) || tokens >= 128 * tok_per_group;
   }
-  if (log_n < 11 || log_n > 15) return false;
+  if (log_n < 9 || log_n > 15) return false;
   if (log_n == 15 && has_signs) return false;  // its sign masks do not fit the sign warps' registers
-  const int64_t rows_per_token = log_n == 15 ? 256 : 128;
+  const int64_t rows_per_token = log_n == 15 ? 256 : log_n == 9 ? 64 : 128;
   if (tokens * rows_per_token >= (int64_t(1) << 31)) return false;
+  // tokens per MMA group: one at n = 32768, 256 / (n / 128) below, 64 at n = 512 (two per box)
   const int64_t tok_per_group = log_n == 15 ? 1 : int64_t(256) >> (log_n - 7);
   return (flags & kTensorCores) || tokens >= 128 * tok_per_group;
 }

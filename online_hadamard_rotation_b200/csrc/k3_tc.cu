@@ -1,5 +1,6 @@
-// k3_tc.cu -- dequantise + inverse rotation on the tensor cores: for n = 4096 to
-// 32768 the first Kronecker factor runs on tcgen05 (below); for n = 128 and 256
+// k3_tc.cu -- dequantise + inverse rotation on the tensor cores: for n = 512 to
+// 32768 the first Kronecker factor runs on tcgen05 (below; at n = 512 two 64-row
+// token rows share a tile and the factor is H_64 (+) H_64); for n = 128 and 256
 // the whole transform does (rows as the MMA's M, further down).
 //
 // "Rotations: QuaRot, SpinQuant and incoherence", widget "Try it": rotate,
@@ -76,19 +77,28 @@ static_assert(kRegsLow * 128 + kRegsHigh * 256 == kLaunchRegs * kThreads, "regis
 template <int LOGN>
 struct Shape {
   static constexpr bool SPLIT = LOGN == 15;
-  static constexpr int B = SPLIT ? 128 : 1 << (LOGN - 7);  // columns per row
-  static constexpr int LOGB = SPLIT ? 7 : LOGN - 7;
-  static constexpr int ROWS = SPLIT ? 256 : 128;    // matrix rows per token row
-  static constexpr int TOK = SPLIT ? 1 : 256 / B;   // token rows per group
-  static constexpr int SEG = SPLIT ? 1 : 128 / B;   // token rows per epilogue thread
+  // n = 512 (PAIR): a row is 64 x 8 and each 128-row operand tile holds two consecutive
+  // rows (matrix rows 0-63 and 64-127); the A operand is H_64 (+) H_64.
+  static constexpr bool PAIR = LOGN == 9;
+  static constexpr int B = SPLIT ? 128 : PAIR ? 8 : 1 << (LOGN - 7);  // columns per row
+  static constexpr int LOGB = SPLIT ? 7 : PAIR ? 3 : LOGN - 7;
+  static constexpr int ROWS = SPLIT ? 256 : PAIR ? 64 : 128;  // matrix rows per token row
+  static constexpr int TPT = PAIR ? 2 : 1;          // token rows per 128-row tile
+  static constexpr int TOK = SPLIT ? 1 : TPT * 256 / B;  // token rows per group
+  static constexpr int SEG = SPLIT ? 1 : 128 / B;   // column segments per epilogue thread
   static constexpr int BOXW = B < 64 ? B : 64;      // operand tile width (columns)
   static constexpr int ROWB = BOXW * 2;             // bytes per operand tile row
   static constexpr int CBOX = B / BOXW;             // column tiles per 128-row block
-  static constexpr int BPT = CBOX * ROWS / 128;     // tiles per token row
+  static constexpr int BPT = PAIR ? 1 : CBOX * ROWS / 128;  // tiles per token row (PAIR: per pair)
   static constexpr uint32_t BOXBYTES = 128u * ROWB; // bytes per tile
-  static constexpr uint32_t LAYOUT = ROWB == 128 ? 2u : 4u;  // UMMA swizzle: 128 B or 64 B
+  static constexpr uint32_t LAYOUT = ROWB == 128 ? 2u : ROWB == 64 ? 4u : ROWB == 32 ? 6u : 0u;  // UMMA swizzle
+  // MN-major B operand strides: swizzled tiles step by box along N and by 8 rows along
+  // K; the no-swizzle layout (16-byte rows, one 8 x 16 B core matrix per 8 rows) swaps
+  // the roles of the two offsets, its leading offset stepping along K.
+  static constexpr uint32_t LBO = LAYOUT == 0 ? 8u * ROWB : BOXBYTES;
+  static constexpr uint32_t SBO = LAYOUT == 0 ? BOXBYTES : 8u * ROWB;
   static constexpr int WPT = (1 << LOGN) / 8;       // code words (8 nibbles) per token row
-  static_assert(LOGN >= 12 && LOGN <= 15, "tensor-core dequantise covers n = 4096 .. 32768");
+  static_assert(LOGN >= 9 && LOGN <= 15, "tensor-core dequantise covers n = 512 .. 32768");
 };
 
 struct Shared {
@@ -225,9 +235,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint32_t k0 = kb * 64 + ch * 8 + 2 * j;
-      const uint32_t lo = (__popc(m & k0) & 1) ? 0xBC00u : 0x3C00u;
-      const uint32_t hi = (__popc(m & (k0 + 1)) & 1) ? 0xBC00u : 0x3C00u;
-      w[j] = lo | (hi << 16);
+      auto entry = [&](uint32_t k) -> uint32_t {  // fp16 +-1 of H_128, or of H_64 (+) H_64
+        if (SH::PAIR && (m >> 6) != (k >> 6)) return 0u;
+        return (__popc(m & k & (SH::PAIR ? 63u : 127u)) & 1) ? 0xBC00u : 0x3C00u;
+      };
+      w[j] = entry(k0) | (entry(k0 + 1) << 16);
     }
     *reinterpret_cast<uint4 *>(smem + kOffH + kb * 16384 + m * 128u + ((ch ^ (m & 7u)) << 4)) =
         make_uint4(w[0], w[1], w[2], w[3]);
@@ -271,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int s = 0; s < 8; ++s) {
                 const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
                 uint64_t bd = tc::smem_desc(sO + os * kOpBytes + v * SH::CBOX * SH::BOXBYTES + s * 16 * SH::ROWB,
-                                            SH::BOXBYTES, 8 * SH::ROWB);
+                                            SH::LBO, SH::SBO);
                 bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
                 tc::umma_bf16(tmem + acc * 256 + u * 128, ad, bd, (u & v) ? idesc_neg : idesc,
                               (v > 0 || s > 0) ? 1u : 0u);
@@ -280,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int s = 0; s < 8; ++s) {
             const uint64_t ad = tc::smem_desc(sH + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-            uint64_t bd = tc::smem_desc(sO + os * kOpBytes + s * 16 * SH::ROWB, SH::BOXBYTES, 8 * SH::ROWB);
+            uint64_t bd = tc::smem_desc(sO + os * kOpBytes + s * 16 * SH::ROWB, SH::LBO, SH::SBO);
             bd = (bd & ~(7ull << 61)) | ((uint64_t)SH::LAYOUT << 61);
             tc::umma_bf16(tmem + acc * 256, ad, bd, idesc, s > 0 ? 1u : 0u);
           }
@@ -316,6 +328,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint4 *cw = reinterpret_cast<const uint4 *>(smem + kOffC + cs * kCodeBytes);
       uint8_t *op = smem + kOffO + os * kOpBytes;
       const uint32_t flip = asym ? 0u : 0x88888888u;
+      if constexpr (SH::B <= 16) {
+        // 16- and 32-byte tile rows: one code word (8 elements) -> one 16-byte chunk.
+        // Chunk c is chunk (c & (B/8 - 1)) of tile row (c / (B/8)) & 127 of tile
+        // c / (128 B/8); consecutive lanes fill consecutive 16-byte slots of a tile (a
+        // 128-byte store phase touches eight different bank groups), and read
+        // consecutive code words: element e of token row t is word t WPT + e / 8, and
+        // a tile's words are contiguous (PAIR: a tile is two token rows of 64 words).
+        constexpr uint32_t CPRW = SH::B / 8;  // chunks per tile row
+        const uint32_t *cwords = reinterpret_cast<const uint32_t *>(cw);
+#pragma unroll 4
+        for (uint32_t c = cid; c < 4096u; c += kConv) {
+          const uint32_t tile = c / (128u * CPRW), inrow = c % (128u * CPRW);
+          const uint32_t a = inrow / CPRW, cr = inrow % CPRW;
+          const uint32_t w = cwords[c] ^ flip;  // the tile's words are contiguous: word c
+          const uint32_t sx = SH::ROWB == 32 ? ((a >> 2) & 1u) : 0u;  // 32-byte swizzle
+          *reinterpret_cast<uint4 *>(op + tile * SH::BOXBYTES + a * SH::ROWB + ((cr ^ sx) << 4)) = expand8(w);
+        }
+      } else {
 #pragma unroll 2
       for (uint32_t q = cid; q < 1024u; q += kConv) {
         constexpr uint32_t HB = SH::BOXW / 32, LHB = HB == 2 ? 1 : 0;  // quads per tile row
@@ -330,6 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ws[4] = {w.x ^ flip, w.y ^ flip, w.z ^ flip, w.w ^ flip};
 #pragma unroll
         for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4 *>(rowp + (((c0 + u) ^ sx) << 4)) = expand8(ws[u]);
+      }
       }
       tc::fence_proxy_async_smem();
       tc::named_sync(3, kConv);
@@ -350,17 +381,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1)
     const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
     const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
-    const uint32_t orow = SH::SPLIT ? 128u * g + row : row;  // output matrix row
-    uint32_t sw[B / 32];  // this row's sign words (the same for every token row)
+    const uint32_t orow = SH::SPLIT ? 128u * g + row : SH::PAIR ? (row & 63u) : row;  // output matrix row
+    // this row's sign bits (the same for every token row): B / 32 words, or for B < 32
+    // the word holding them, shifted so that bit k is element orow B + k
+    constexpr int NSW = B >= 32 ? B / 32 : 1;
+    uint32_t sw[NSW];
 #pragma unroll
-    for (int k = 0; k < B / 32; ++k) sw[k] = SIGNS ? __ldg(signs + (orow * B) / 32 + k) : 0u;
+    for (int k = 0; k < NSW; ++k)
+      sw[k] = SIGNS ? (__ldg(signs + (orow * B) / 32 + k) >> (B >= 32 ? 0u : (orow * B) & 31u)) : 0u;
     // The row steps (and zero points) of a group are loaded one group ahead, so their
     // DRAM latency hides behind the previous group's work: raw bits, converted when used
     // (fp32 step, or fp16 step in the low and fp16 zero in the high half).
-    auto load_steps = [&](int64_t pp, uint32_t (&dst)[SEG]) {
+      auto load_steps = [&](int64_t pp, uint32_t (&dst)[SEG]) {
 #pragma unroll
       for (int sg = 0; sg < SEG; ++sg) {
-        const int64_t token = SH::SPLIT ? pp : pp * SH::TOK + g * SEG + sg;
+        const int64_t token = SH::SPLIT ? pp
+                              : SH::PAIR ? pp * SH::TOK + 2 * (g * SEG + sg) + (row >> 6)
+                                         : pp * SH::TOK + g * SEG + sg;
         dst[sg] = 0u;
         if (pp < ngroups && token < rows)
           dst[sg] = asym ? (uint32_t)__ldg(static_cast<const unsigned short *>(scale) + token) |
@@ -400,11 +437,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the row's zero point). H_128 of a constant is nonzero only in matrix row 0
       // (128 times it; twice that in the top half at n = 32768, nothing in the bottom
       // half), so the thread holding row 0 takes it out before H_B; all exact integers.
-      if (row == 0 && (!SH::SPLIT || g == 0)) {
+      // (PAIR: H_64 (+) H_64 puts 64 times it in rows 0 and 64, one per token row.)
+      if ((SH::PAIR ? (row & 63u) : row) == 0 && (!SH::SPLIT || g == 0)) {
 #pragma unroll
         for (int sg = 0; sg < SEG; ++sg) {
           const float K = asym ? __half2float(__ushort_as_half((unsigned short)(step_raw[sg] >> 16))) : 8.0f;
-          const float corr = (SH::SPLIT ? 256.0f : 128.0f) * (1024.0f + K);
+          const float corr = (SH::SPLIT ? 256.0f : SH::PAIR ? 64.0f : 128.0f) * (1024.0f + K);
 #pragma unroll
           for (int k = 0; k < B; ++k) v[sg * B + k] -= corr;
         }
@@ -413,22 +451,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       stage<0>(v);
       stage<1>(v);
       stage<2>(v);
-      stage<3>(v);
-      stage<4>(v);
+      if constexpr (SH::LOGB > 3) stage<3>(v);
+      if constexpr (SH::LOGB > 4) stage<4>(v);
       if constexpr (SH::LOGB > 5) stage<5>(v);
       if constexpr (SH::LOGB > 6) stage<6>(v);
 #pragma unroll
       for (int sg = 0; sg < SEG; ++sg) {
-        const int64_t token = SH::SPLIT ? p : p * SH::TOK + g * SEG + sg;
+        const int64_t token = SH::SPLIT ? p
+                              : SH::PAIR ? p * SH::TOK + 2 * (g * SEG + sg) + (row >> 6)
+                                         : p * SH::TOK + g * SEG + sg;
         if (token >= rows) continue;
         const float s = asym ? __half2float(__ushort_as_half((unsigned short)step_raw[sg]))
                              : __uint_as_float(step_raw[sg]);
         const float m = s * inv_sqrt_n;
         const float *w = v + sg * B;
         const int64_t off = token * (int64_t)(B * SH::ROWS) + (int64_t)orow * B;  // first element of the row
-        // one 8 (fp32) or 16 (bf16) element piece at a time, in element order: scale,
-        // diagonal sign, store
-        constexpr int P = F32 ? 8 : 16;
+        // one 8 (fp32) or 16 (bf16; 8 when B = 8) element piece at a time, in element
+        // order: scale, diagonal sign, store
+        constexpr int P = (F32 || B == 8) ? 8 : 16;
 #pragma unroll
         for (int k = 0; k < B; k += P) {
           float o[P];
@@ -439,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mul2(o[u], o[u + 1], m);
           }
           if constexpr (SIGNS) {
-            const uint32_t sb = sw[k >> 5] >> (k & 31);
+            const uint32_t sb = B >= 32 ? sw[k >> 5] >> (k & 31) : sw[0] >> k;
 #pragma unroll
             for (int u = 0; u < P; ++u) o[u] = __uint_as_float(__float_as_uint(o[u]) ^ (((sb >> u) & 1u) << 31));
           }
@@ -447,6 +487,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             store8<STORE32>(static_cast<float *>(out) + off + k, __float_as_uint(o[0]), __float_as_uint(o[1]),
                             __float_as_uint(o[2]), __float_as_uint(o[3]), __float_as_uint(o[4]),
                             __float_as_uint(o[5]), __float_as_uint(o[6]), __float_as_uint(o[7]));
+          } else if constexpr (P == 8) {  // 8 bf16: one 16-byte store
+            __stcs(reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + off + k),
+                   make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                              pack_bf16x2(o[6], o[7])));
           } else {
             store8<STORE32>(static_cast<uint16_t *>(out) + off + k, pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
                             pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]), pack_bf16x2(o[8], o[9]),
@@ -881,8 +925,10 @@ cudaError_t launch_small(const uint8_t *codes, int64_t rows, const void *scale, 
 
 bool tc_dequant_supported(int log_n, int64_t rows, uint32_t flags) {
   if ((flags & kNoRotate) || rows <= 0) return false;
-  if (!(log_n == 7 || log_n == 8 || (log_n >= 12 && log_n <= 15))) return false;
+  if (log_n < 7 || log_n > 15) return false;
   if (rows * (int64_t(1) << log_n) >= (int64_t(1) << 40)) return false;
+  // rows per MMA group: 128 at n = 128 and 256, 64 at n = 512 (two per tile), 256 / (n / 128)
+  // from n = 1024, one at n = 32768
   const int64_t rows_per_group = log_n <= 8 ? 128 : log_n == 15 ? 1 : int64_t(256) >> (log_n - 7);
   return (flags & kTensorCores) || rows >= 128 * rows_per_group;
 }
@@ -894,6 +940,9 @@ cudaError_t launch_dequant_inverse_tc(int log_n, const uint8_t *codes, int64_t r
   switch (log_n) {
     case 7: return launch_small<1>(codes, rows, scale, zero, signs, out, asym, f32, stream);
     case 8: return launch_small<2>(codes, rows, scale, zero, signs, out, asym, f32, stream);
+    case 9: return launch_n<9>(codes, rows, scale, zero, signs, out, asym, f32, stream);
+    case 10: return launch_n<10>(codes, rows, scale, zero, signs, out, asym, f32, stream);
+    case 11: return launch_n<11>(codes, rows, scale, zero, signs, out, asym, f32, stream);
     case 12: return launch_n<12>(codes, rows, scale, zero, signs, out, asym, f32, stream);
     case 13: return launch_n<13>(codes, rows, scale, zero, signs, out, asym, f32, stream);
     case 14: return launch_n<14>(codes, rows, scale, zero, signs, out, asym, f32, stream);

@@ -160,10 +160,12 @@ def test_dispatch_query(L):
     assert q(R4, 16384, 32768, 0, 1) == 0             # n = 32768 with a diagonal
     assert q(R4, 16384, 32768, 0, 0) == 1
     assert q(R4, 128 * 256, 128, 0, 0) == 1 and q(R4, 128 * 256 - 1, 128, 0, 0) == 0
-    assert q(R4, 10 ** 6, 512, 0, 0) == 0 and q(R4, 10 ** 6, 1024, 4, 0) == 0
+    assert q(R4, 10 ** 6, 512, 0, 0) == 1 and q(R4, 10 ** 6, 1024, 4, 0) == 1   # tensor cores from n = 512
+    assert q(R4, 128 * 64 - 1, 512, 0, 0) == 0 and q(R4, 128 * 32, 1024, 0, 0) == 1
     assert q(R4, 128 * 16, 2048, 0, 0) == 1
     assert q(INV, 128 * 128, 256, 0, 0) == 1 and q(INV, 128 * 128 - 1, 256, 0, 0) == 0
-    assert q(INV, 10 ** 6, 2048, 0, 0) == 0 and q(INV, 128 * 8, 4096, 0, 0) == 1
+    assert q(INV, 10 ** 6, 2048, 0, 0) == 1 and q(INV, 128 * 8, 4096, 0, 0) == 1
+    assert q(INV, 128 * 64, 512, 0, 0) == 1 and q(INV, 128 * 64 - 1, 512, 0, 0) == 0
     for bad in ((R4, 4, 100, 0, 0), (R4, -1, 256, 0, 0), (R4, 4, 256, 6, 0), (R4, 4, 256, 8, 0), (7, 4, 256, 0, 0),
                 (7, 4, 256, 2, 0)):
         assert q(*bad) == -1
@@ -178,9 +180,11 @@ def test_bench_names_the_dispatched_kernel():
     import bench
     assert bench.r4_kernel_name(16384, 8192, True) == "k1_tc_rotate_quant"
     assert bench.r4_kernel_name(128, 1 << 22, False) == "k1_tcs_rotate_quant"
-    assert bench.r4_kernel_name(1024, 1 << 19, False, 8) == "k1_rotate_quant_int8"
+    assert bench.r4_kernel_name(1024, 1 << 19, False, 8) == "k1_tc_rotate_quant"
+    assert bench.r4_kernel_name(1024, 32, False, 8) == "k1_rotate_quant_int8"  # a decode-size batch
     assert bench.k3_kernel_name(256, 1 << 21) == "k3_tcs_dequant_inverse"
-    assert bench.k3_kernel_name(2048, 1 << 18) == "k3_dequant_inverse"
+    assert bench.k3_kernel_name(2048, 1 << 18) == "k3_tc_dequant_inverse"
+    assert bench.k3_kernel_name(2048, 100) == "k3_dequant_inverse"
 
 
 def test_kron_size_rules(L):

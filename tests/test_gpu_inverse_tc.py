@@ -5,7 +5,8 @@ constant H_128 (H_2 of n = 256 in the epilogue), at n = 4096 .. 32768 the first
 H_128 factor runs on tcgen05 and the second in registers. Both kernels transform
 exact integers and scale once at the end, so their outputs must agree bit for
 bit. Row counts leave partial MMA groups (128 rows per group at n = 128 and 256;
-8, 4, 2 and 1 from 4096)."""
+64 at n = 512, whose odd row counts split a two-row tile; 32, 16, 8, 4, 2 and 1 from
+1024)."""
 import numpy as np
 import pytest
 import torch
@@ -16,7 +17,7 @@ from tests.gpu_util import to_dev_signs
 
 pytestmark = pytest.mark.gpu
 
-SIZES = [128, 256, 4096, 8192, 16384, 32768]
+SIZES = [128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768]
 
 
 def inverse(spin, packed, n, scale, zero, mode, signs, out_dtype, cores_only=False):
@@ -106,7 +107,7 @@ def test_tc_leaves_tail_untouched(spin_gpu, orc, n):
     parity.check_f32_rows(out[:rows].cpu().numpy().astype(np.float64), ref, f"tc inverse n={n} into a slice")
 
 
-@pytest.mark.parametrize("n", [128, 256])
+@pytest.mark.parametrize("n", [128, 256, 512, 1024, 2048])
 @pytest.mark.parametrize("mode", [0, 1])
 def test_tc_small_n_many_groups(spin_gpu, orc, n, mode):
     """More 128-row groups than resident blocks (every block loops, every ring

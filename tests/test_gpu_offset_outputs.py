@@ -2,7 +2,7 @@
 view into a larger buffer. The tensor-core kernels store 32 bytes at a time
 when the output pointer allows it and switch to 16-byte stores otherwise; these
 tests run that second form of every tensor-core kernel (R4 INT4 and INT8 at
-n = 128, 256 and 2048 .. 32768, with and without the diagonal, and both
+n = 128 .. 32768, with and without the diagonal, and both
 tensor-core inverses, bf16 and fp32 out) against the oracle, with canary bytes
 on both sides of the output."""
 import numpy as np
@@ -18,8 +18,9 @@ pytestmark = pytest.mark.gpu
 CANARY = 0xA5
 PAD = 64  # bytes of canary after the view
 # tokens: several MMA groups plus a ragged tail (tokens per group: 256 at n = 128,
-# 128 at n = 256, 256 / (n / 128) from 2048, 1 at 32768)
-TOKENS = {128: 3 * 256 + 77, 256: 3 * 128 + 37, 2048: 5 * 16 + 7, 4096: 5 * 8 + 3, 8192: 9 * 4 + 1,
+# 128 at n = 256, 64 at n = 512 (an odd tail splits a two-token box), 256 / (n / 128)
+# from 1024, 1 at 32768)
+TOKENS = {128: 3 * 256 + 77, 256: 3 * 128 + 37, 512: 3 * 64 + 33, 1024: 3 * 32 + 5, 2048: 5 * 16 + 7, 4096: 5 * 8 + 3, 8192: 9 * 4 + 1,
           16384: 11 * 2 + 1, 32768: 7}
 
 
@@ -70,7 +71,8 @@ def test_r4_tensor_core_output_at_16_byte_offset(spin_gpu, orc, n, with_signs, b
             parity.check_codes(q_np[t].astype(np.int32), r["codes"], r["pre"], f"{what}: codes row {t}")
 
 
-@pytest.mark.parametrize("n,rows", [(128, 300), (256, 150), (4096, 19), (8192, 9), (16384, 5), (32768, 3)])
+@pytest.mark.parametrize("n,rows", [(128, 300), (256, 150), (512, 131), (1024, 67), (2048, 35), (4096, 19), (8192, 9),
+                                    (16384, 5), (32768, 3)])
 @pytest.mark.parametrize("with_signs", [False, True])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_inverse_tensor_core_output_at_16_byte_offset(spin_gpu, orc, n, rows, with_signs, out_dtype):

@@ -14,7 +14,7 @@ from tests.gpu_util import to_dev_bf16, to_dev_signs
 pytestmark = pytest.mark.gpu
 
 VARIANTS = {"plain": (1.0, False, False), "clip_signs": (0.9, True, False), "direct": (1.0, False, True)}
-TC_SIZES = (128, 256, 2048, 4096, 8192, 16384, 32768)
+TC_SIZES = (128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768)
 
 
 def run(spin, bits, clip, signs, direct=False, path="default"):
@@ -80,7 +80,7 @@ def test_int8_many_groups(spin_gpu, orc, n, tokens):
     assert spin_gpu.device_status() == 0
 
 
-@pytest.mark.parametrize("n", [128, 1024, 16384])
+@pytest.mark.parametrize("n", [128, 512, 1024, 16384])
 def test_int8_leaves_tail_untouched(spin_gpu, n):
     bits = synthetic.r4_prefill(tokens=5, n=n, seed=3)[0]
     out = torch.full((8, n), 0x5A, dtype=torch.int8, device="cuda")

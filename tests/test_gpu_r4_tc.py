@@ -2,11 +2,12 @@
 selected with SPIN_CUDA_CORES_ONLY:
   n = 128, 256: tokens as the MMA's M (128 tokens per MMA, the diagonal folded
     into the constant operand, H_2 of n = 256 in the epilogue);
-  n = 2048 .. 16384: first H_128 Kronecker factor on tcgen05, second on CUDA
-    cores; n = 32768: H_2 and H_128 on tcgen05, without a sign diagonal.
-Token counts leave partial MMA groups (256 / 128 tokens per group at n = 128 /
-256; 16, 8, 4 and 2 at the large sizes). At n = 32768 with sign_bits the CUDA-core
-kernel runs."""
+  n = 1024 .. 16384: first H_128 Kronecker factor on tcgen05, second on CUDA
+    cores; n = 512: two 64-row tokens per 128-row tile with H_64 (+) H_64 on
+    tcgen05; n = 32768: H_2 and H_128 on tcgen05, without a sign diagonal.
+Token counts leave partial MMA groups (256 / 128 / 64 tokens per group at n = 128 /
+256 / 512; 32, 16, 8, 4 and 2 at n = 1024 .. 16384) and, at n = 512, odd tails that
+split a two-token tile. At n = 32768 with sign_bits the CUDA-core kernel runs."""
 import numpy as np
 import pytest
 import torch
@@ -17,7 +18,7 @@ from tests.gpu_util import to_dev_bf16, to_dev_signs
 
 pytestmark = pytest.mark.gpu
 
-SIZES = [128, 256, 2048, 4096, 8192, 16384, 32768]
+SIZES = [128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768]
 
 
 def run(spin, bits, clip, signs, cores_only=False):
