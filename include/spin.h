@@ -64,7 +64,8 @@ typedef enum spin_status_t {
   SPIN_ERR_UNSUPPORTED_SIZE = 2, /* n or head_dim not a supported power of two */
   SPIN_ERR_MISALIGNED = 3,       /* a pointer is not 16-byte aligned */
   SPIN_ERR_CUDA = 4,             /* a CUDA call or launch failed: see spin_last_cuda_error() */
-  SPIN_ERR_DEVICE = 5            /* the current device is not compute capability 10.0 */
+  SPIN_ERR_DEVICE = 5,           /* the current device is not compute capability 10.0 */
+  SPIN_ERR_SCRATCH_LIMIT = 6     /* the call needs more scratch than the library's built-in array */
 } spin_status_t;
 
 /* flags */
@@ -317,6 +318,41 @@ spin_status_t spin_decode_attention_int4kv(const void *q, const uint8_t *k_cache
 /* Workspace bytes spin_decode_attention_int4kv needs (batch x n_q_heads x
  * ceil(cache_len / 256) partials of head_dim + 2 fp32 values); 0 for sizes <= 0. */
 size_t spin_decode_attention_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t cache_len);
+
+/* Bytes of the scratch array built into the library for
+ * spin_decode_attention_int4kv_noalloc (held by every GPU that loads the library). */
+#define SPIN_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * spin_decode_attention_int4kv for callers that cannot allocate device memory
+ * (no counterpart on the pages). Some callers have no way to provide the workspace:
+ * a plugin inside an inference engine that owns all device memory and gives the plugin
+ * no scratch, or a latency-critical serving loop that must not call cudaMalloc
+ * because it can synchronise the device. This entry point takes the same arguments
+ * except the workspace and allocates nothing: the per-chunk partials go to a scratch
+ * array compiled into the library, SPIN_NOALLOC_SCRATCH_BYTES (4 MiB) on every GPU
+ * that loads the library, kept until the process exits.
+ *  * Limit: batch x n_q_heads x ceil(cache_len / 256) x 520 bytes (the value of
+ *    spin_decode_attention_workspace_bytes) must not exceed SPIN_NOALLOC_SCRATCH_BYTES,
+ *    e.g. 4 rows x 32 heads of a 4096-slot cache use 1.06 MB; larger calls return
+ *    SPIN_ERR_SCRATCH_LIMIT and enqueue nothing.
+ *  * The first call on a device looks up the array's device address on the host
+ *    (cudaGetSymbolAddress, with that device current) and keeps it; make that first
+ *    call on each device before any stream capture.
+ *  * Every call on a device shares the one array, and nothing in it needs to start at
+ *    zero (each call writes every partial it reads). Calls whose kernels can overlap
+ *    on the GPU -- on different streams or from different host threads without an
+ *    ordering between them -- race on the array and give wrong results; order them
+ *    (one stream, or events).
+ * Errors: those of spin_decode_attention_int4kv (other than a small workspace),
+ * SPIN_ERR_SCRATCH_LIMIT, and SPIN_ERR_CUDA if the address lookup fails.
+ */
+spin_status_t spin_decode_attention_int4kv_noalloc(const void *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                                                   const void *k_scale, const void *k_zero, const void *v_scale,
+                                                   const void *v_zero, const int32_t *lens, int32_t batch,
+                                                   int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                                   int32_t cache_len, float softmax_scale, void *out,
+                                                   int32_t out_dtype, spin_stream_t stream);
 
 /*
  * Device status word of the current device: nonzero once a kernel of this

@@ -54,6 +54,8 @@ spin_status_t check_device() {
 bool valid_clip(float clip) { return clip > 0.0f && clip <= 1.0f; }  // false for NaN
 }  // namespace
 
+int report_cuda_error(cudaError_t e) { return static_cast<int>(cuda_status(e)); }
+
 cudaError_t resident_slots(const void *kernel, int threads, int dyn_smem, int *slots) {
   static std::mutex mu;
   static std::map<std::tuple<const void *, int, int, int>, int> cache;
@@ -253,6 +255,7 @@ const char *spin_status_string(spin_status_t status) {
     case SPIN_ERR_MISALIGNED: return "SPIN_ERR_MISALIGNED";
     case SPIN_ERR_CUDA: return "SPIN_ERR_CUDA";
     case SPIN_ERR_DEVICE: return "SPIN_ERR_DEVICE";
+    case SPIN_ERR_SCRATCH_LIMIT: return "SPIN_ERR_SCRATCH_LIMIT";
   }
   return "SPIN_ERR_UNKNOWN";
 }

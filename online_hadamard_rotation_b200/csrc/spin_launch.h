@@ -13,6 +13,10 @@ constexpr uint32_t kNoRotate = 1u;        // same value as SPIN_NO_ROTATE
 constexpr uint32_t kCudaCoresOnly = 2u;   // same value as SPIN_CUDA_CORES_ONLY
 constexpr uint32_t kTensorCores = 4u;     // same value as SPIN_TENSOR_CORES
 
+// SPIN_OK for cudaSuccess; otherwise records `e` for spin_last_cuda_error() and
+// returns SPIN_ERR_CUDA (as every entry point reports a failed CUDA call).
+int report_cuda_error(cudaError_t e);
+
 // Number of blocks of `kernel` that are resident on the current device at once
 // (SM count x blocks per SM), with the dynamic shared-memory opt-in applied.
 // Cached per kernel and device after the first call.
