@@ -24,8 +24,10 @@
 //      integer below 2^24.
 //   3. Each epilogue thread owns one TMEM lane (row a') over 128 columns, runs the
 //      log2(B) butterfly stages of H_B in registers (still exact), multiplies by
-//      s / sqrt(n), flips the signs of D (its row's sign words stay in registers)
-//      and stores bf16 or fp32 straight to the output row.
+//      s / sqrt(n) and flips the signs of D (its row's sign words stay in
+//      registers). Output rows of 64 bytes or more go through a swizzled staging
+//      tile per warp and a TMA tensor store of the warp's 32 rows (whole lines);
+//      narrower rows are stored from registers.
 // n = 32768 is H_2 (x) H_128 (x) H_128: a row is 256 x 128, the MMA accumulates
 // H_128 C'_0 + H_128 C'_1 and H_128 C'_0 - H_128 C'_1 (negate-A bit) into the two
 // 128-column halves, and epilogue warpgroup g writes output rows 128 g + a'.
@@ -33,7 +35,8 @@
 // Roles (384 threads, one CTA per SM, persistent over groups):
 //   warps 0, 2, 3  converters: codes -> fp16 operand (two-stage ring of 64 KiB);
 //                  thread 0 also issues each group's 16 KiB bulk copy of codes
-//                  into a three-stage ring
+//                  into a three-stage ring (two stages where the output staging
+//                  tiles take the third's space)
 //   warp 1         TMEM owner and MMA issuer
 //   warps 4-11     epilogue, two warpgroups over TMEM columns 0-127 and 128-255
 // (setmaxnreg moves registers from warps 0-3 to the epilogue warpgroups).
@@ -46,6 +49,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstring>
 #include <type_traits>
 
 #include "spin_launch.h"
@@ -60,15 +64,25 @@ __device__ unsigned int g_dequant_status = 0u;
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kCStages = 3;                        // codes ring
 constexpr int kOStages = 2;                        // fp16 operand ring
 constexpr uint32_t kCodeBytes = 16384;             // codes of one group (32768 nibbles)
 constexpr uint32_t kOpBytes = 65536;               // fp16 operand of one group
 constexpr uint32_t kOffH = 0;                      // A operand: H_128 in fp16, K-major, 2 x 16 KiB
 constexpr uint32_t kOffO = 32768;                  // operand ring
-constexpr uint32_t kOffC = kOffO + kOStages * kOpBytes;
-constexpr uint32_t kOffBar = kOffC + kCStages * kCodeBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
+constexpr uint32_t kStageBytes = 4096;             // output staging per epilogue warp (TMA-store shapes)
+
+// Shared-memory layout. Shapes whose output rows are written by TMA tensor stores
+// (`ts`) give up one codes stage (two groups of lead time still cover the DRAM
+// latency) for a 4 KiB staging tile per epilogue warp.
+template <bool TS>
+struct Layout {
+  static constexpr int CS = TS ? 2 : 3;              // codes ring stages
+  static constexpr uint32_t kOffC = kOffO + kOStages * kOpBytes;
+  static constexpr uint32_t kOffS = kOffC + CS * kCodeBytes;  // 8 staging tiles (TS)
+  static constexpr uint32_t kOffBar = kOffS + (TS ? 8u * kStageBytes : 0u);
+  static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
 constexpr long long kTimeoutCycles = 4000000000LL;     // about two seconds
 constexpr int kLaunchRegs = 168;                       // registers per thread at launch (65536 / 384, rounded)
 constexpr int kRegsLow = 104, kRegsHigh = 200;         // after the split: warps 0-3, warps 4-11
@@ -98,11 +112,17 @@ struct Shape {
   static constexpr uint32_t LBO = LAYOUT == 0 ? 8u * ROWB : BOXBYTES;
   static constexpr uint32_t SBO = LAYOUT == 0 ? BOXBYTES : 8u * ROWB;
   static constexpr int WPT = (1 << LOGN) / 8;       // code words (8 nibbles) per token row
+  // Output rows of at least 64 bytes (bf16 from n = 4096, fp32 from n = 2048) go out
+  // through TMA tensor stores from a swizzled staging tile: a warp's 32 rows of a row
+  // segment are one contiguous range, written as whole lines. Narrower rows are
+  // stored from registers (their warp stores are contiguous already).
+  template <bool F32>
+  static constexpr bool ts() { return !PAIR && B * (F32 ? 4 : 2) >= 64; }
   static_assert(LOGN >= 9 && LOGN <= 15, "tensor-core dequantise covers n = 512 .. 32768");
 };
 
 struct Shared {
-  uint64_t cfull[kCStages], ofull[kOStages], oempty[kOStages], tfull[2], tempty[2], drain;
+  uint64_t cfull[3], ofull[kOStages], oempty[kOStages], tfull[2], tempty[2], drain;
   uint32_t tmem_base;
   int abort;
   int dec[3];
@@ -155,6 +175,15 @@ __device__ __forceinline__ void store8(void *p, uint32_t w0, uint32_t w1, uint32
   }
 }
 
+// TMA tensor store of a staged box (3-D map: element, piece, row) to global memory,
+// tracked by the issuing thread's bulk group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(tc::smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
 // (a0, a1) <- (a0, a1) * (m, m), one packed multiply
 __device__ __forceinline__ void mul2(float &a0, float &a1, float m) {
   uint64_t A, M, R;
@@ -182,11 +211,15 @@ __host__ __device__ constexpr int pos8(int e) { return (e >> 1) | ((e & 1) << 2)
 
 template <int LOGN, bool SIGNS, bool F32, bool STORE32>
 __global__ void __launch_bounds__(kThreads, 1)
-    k3_tc_dequant_inverse(const uint8_t *__restrict__ codes, int64_t rows, float inv_sqrt_n,
+    k3_tc_dequant_inverse(const __grid_constant__ CUtensorMap omap, const uint8_t *__restrict__ codes, int64_t rows, float inv_sqrt_n,
                           const void *__restrict__ scale, const __half *__restrict__ zero,
                           const uint32_t *__restrict__ signs, void *__restrict__ out, int asym) {
   using SH = Shape<LOGN>;
   constexpr int B = SH::B, SEG = SH::SEG;
+  constexpr bool TS = SH::template ts<F32>();
+  using LY = Layout<TS>;
+  constexpr int kCStages = LY::CS;
+  constexpr uint32_t kOffC = LY::kOffC, kOffBar = LY::kOffBar;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array itself so that accesses
   // through it stay shared-memory accesses
@@ -312,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // in it has been converted.
     constexpr uint32_t kConv = 96;
     const uint32_t cid = warp == 0 ? lane : threadIdx.x - 32;
-    int64_t last[kCStages] = {-1, -1, -1};  // converter 0: last group index issued per stage
+    int64_t last[3] = {-1, -1, -1};  // converter 0: last group index issued per stage
     for (int64_t i = 0; i < first_issued; ++i) last[i] = i;
     for (int64_t i = 0;; ++i) {
       const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
@@ -379,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (last[s2] >= 0) wait_bounded(&S.cfull[s2], (uint32_t)((last[s2] / kCStages) & 1), S, false);
   } else {
     // epilogue warpgroup g: warps 4..7 (g = 0) and 8..11 (g = 1)
-    const uint32_t g = (warp - 4) >> 2, wq = warp & 3u, tg = threadIdx.x - 128 - 128 * g;
+    const uint32_t g = (warp - 4) >> 2, wq = warp & 3u;
     const uint32_t row = wq * 32 + lane;  // a' = TMEM lane
     const uint32_t orow = SH::SPLIT ? 128u * g + row : SH::PAIR ? (row & 63u) : row;  // output matrix row
     // this row's sign bits (the same for every token row): B / 32 words, or for B < 32
@@ -415,9 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int sg = 0; sg < SEG; ++sg) step_raw[sg] = step_next[sg];
       load_steps(p + gridDim.x, step_next);
       const int acc = (int)(i & 1);
-      if (tg == 0) S.dec[g] = wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true) ? 1 : 0;
-      tc::named_sync(1 + g, 128);
-      if (!S.dec[g]) break;
+      // every thread sleeps on the accumulator's barrier itself (no block-level barrier
+      // between the epilogue warps)
+      if (!wait_bounded(&S.tfull[acc], (uint32_t)((i >> 1) & 1), S, true)) break;
       tc::tc_fence_after();
       float v[kRegs];
       {
@@ -455,6 +488,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (SH::LOGB > 4) stage<4>(v);
       if constexpr (SH::LOGB > 5) stage<5>(v);
       if constexpr (SH::LOGB > 6) stage<6>(v);
+      if constexpr (TS) {
+        // A warp's 32 rows of a row segment are one contiguous range of the output. Each
+        // piece (128 or 64 bytes of every row) is written into the warp's staging tile
+        // with the TMA swizzle (row `lane` at lane x OROWB, 16-byte chunk c at position
+        // c ^ (row bits), so the eight lanes of a store phase hit eight bank groups),
+        // then one lane issues the tensor store that writes it out as whole lines.
+        constexpr int OE = F32 ? 4 : 2;                  // output bytes per element
+        constexpr int OROWB = B * OE >= 128 ? 128 : 64;  // staged bytes per row (the swizzle span)
+        constexpr int PE = OROWB / OE;                   // elements per piece
+        constexpr int NP = B / PE;                       // pieces per row segment
+        constexpr int CH = OROWB / 16;                   // 16-byte chunks per staged row
+        uint8_t *stg = smem + LY::kOffS + (warp - 4) * kStageBytes;
+        const uint32_t srow = tc::smem_u32(stg) + lane * (uint32_t)OROWB;
+        const uint32_t swz = OROWB == 128 ? (lane & 7u) : ((lane >> 1) & 3u);
+        const int orow0 = (SH::SPLIT ? 128 * (int)g : 0) + 32 * (int)wq;
+#pragma unroll
+        for (int sg = 0; sg < SEG; ++sg) {
+          const int64_t token = SH::SPLIT ? p : p * SH::TOK + g * SEG + sg;
+          if (token >= rows) continue;  // the same for the whole warpgroup
+          const float s = asym ? __half2float(__ushort_as_half((unsigned short)step_raw[sg]))
+                               : __uint_as_float(step_raw[sg]);
+          const float m = s * inv_sqrt_n;
+          const float *w = v + sg * B;
+#pragma unroll
+          for (int pc = 0; pc < NP; ++pc) {
+            uint32_t wv[CH * 4];
+#pragma unroll
+            for (int u = 0; u < PE; u += 2) {
+              const int k = pc * PE + u;  // element of the row segment (even)
+              float o0 = w[(k & ~7) + pos8(k & 7)], o1 = w[(k & ~7) + pos8((k + 1) & 7)];
+              mul2(o0, o1, m);
+              if constexpr (SIGNS) {
+                const uint32_t sb = B >= 32 ? sw[k >> 5] >> (k & 31) : sw[0] >> k;
+                o0 = __uint_as_float(__float_as_uint(o0) ^ ((sb & 1u) << 31));
+                o1 = __uint_as_float(__float_as_uint(o1) ^ (((sb >> 1) & 1u) << 31));
+              }
+              if constexpr (F32) {
+                wv[u] = __float_as_uint(o0);
+                wv[u + 1] = __float_as_uint(o1);
+              } else {
+                wv[u >> 1] = pack_bf16x2(o0, o1);
+              }
+            }
+            if (lane == 0) tc::bulk_wait_read0();  // the tile's previous piece has been read out
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < CH; ++c)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(srow + ((c ^ swz) << 4)),
+                           "r"(wv[4 * c]), "r"(wv[4 * c + 1]), "r"(wv[4 * c + 2]), "r"(wv[4 * c + 3])
+                           : "memory");
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&omap, stg, 0, pc, (int)(token * SH::ROWS) + orow0);
+              tc::bulk_commit();
+            }
+          }
+        }
+        continue;
+      }
 #pragma unroll
       for (int sg = 0; sg < SEG; ++sg) {
         const int64_t token = SH::SPLIT ? p
@@ -499,6 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if constexpr (TS)
+      if (lane == 0) tc::bulk_wait0();  // every tensor store has completed before the CTA leaves
   }
 
   // ------------------------------------------------------------ teardown
@@ -527,6 +622,28 @@ cudaError_t launch_tc(const uint8_t *codes, int64_t rows, const void *scale, con
     return fa.numRegs == kLaunchRegs ? cudaSuccess : cudaErrorInvalidConfiguration;
   }();
   if (checked != cudaSuccess) return checked;
+  constexpr bool TS = SH::template ts<F32>();
+  constexpr uint32_t kSmemBytes = Layout<TS>::kSmemBytes;
+  // Output map for the tensor stores: (element within a 128- or 64-byte piece, piece
+  // within a matrix row, matrix row = token row x rows-per-token + a'), boxes of one
+  // piece x 32 rows, swizzled like the staging tile.
+  CUtensorMap omap;
+  std::memset(&omap, 0, sizeof(omap));
+  if constexpr (TS) {
+    constexpr int OE = F32 ? 4 : 2, OROWB = SH::B * OE >= 128 ? 128 : 64, PE = OROWB / OE;
+    if (rows * SH::ROWS >= (int64_t(1) << 31)) return cudaErrorInvalidValue;  // row coordinates are 32-bit
+    auto fn = tensor_map_encoder();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)PE, (cuuint64_t)(SH::B / PE), (cuuint64_t)(rows * SH::ROWS)};
+    const cuuint64_t strides[2] = {(cuuint64_t)OROWB, (cuuint64_t)SH::B * OE};
+    const cuuint32_t box[3] = {(cuuint32_t)PE, 1, 32};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(&omap, F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    OROWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
   int slots = 0;
   cudaError_t err = resident_slots(reinterpret_cast<const void *>(kern), kThreads, (int)kSmemBytes, &slots);
   if (err != cudaSuccess) return err;
@@ -543,8 +660,8 @@ cudaError_t launch_tc(const uint8_t *codes, int64_t rows, const void *scale, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, codes, rows, inv_sqrt_n, scale, static_cast<const __half *>(zero), signs,
-                            out, asym ? 1 : 0);
+  return cudaLaunchKernelEx(&cfg, kern, omap, codes, rows, inv_sqrt_n, scale, static_cast<const __half *>(zero),
+                            signs, out, asym ? 1 : 0);
 }
 
 template <int LOGN, bool SIGNS>
