@@ -546,48 +546,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        continue;
-      }
+      } else {
 #pragma unroll
-      for (int sg = 0; sg < SEG; ++sg) {
-        const int64_t token = SH::SPLIT ? p
-                              : SH::PAIR ? p * SH::TOK + 2 * (g * SEG + sg) + (row >> 6)
-                                         : p * SH::TOK + g * SEG + sg;
-        if (token >= rows) continue;
-        const float s = asym ? __half2float(__ushort_as_half((unsigned short)step_raw[sg]))
-                             : __uint_as_float(step_raw[sg]);
-        const float m = s * inv_sqrt_n;
-        const float *w = v + sg * B;
-        const int64_t off = token * (int64_t)(B * SH::ROWS) + (int64_t)orow * B;  // first element of the row
-        // one 8 (fp32) or 16 (bf16; 8 when B = 8) element piece at a time, in element
-        // order: scale, diagonal sign, store
-        constexpr int P = (F32 || B == 8) ? 8 : 16;
+        for (int sg = 0; sg < SEG; ++sg) {
+          const int64_t token = SH::SPLIT ? p
+                                : SH::PAIR ? p * SH::TOK + 2 * (g * SEG + sg) + (row >> 6)
+                                           : p * SH::TOK + g * SEG + sg;
+          if (token >= rows) continue;
+          const float s = asym ? __half2float(__ushort_as_half((unsigned short)step_raw[sg]))
+                               : __uint_as_float(step_raw[sg]);
+          const float m = s * inv_sqrt_n;
+          const float *w = v + sg * B;
+          const int64_t off = token * (int64_t)(B * SH::ROWS) + (int64_t)orow * B;  // first element of the row
+          // one 8 (fp32) or 16 (bf16; 8 when B = 8) element piece at a time, in element
+          // order: scale, diagonal sign, store
+          constexpr int P = (F32 || B == 8) ? 8 : 16;
 #pragma unroll
-        for (int k = 0; k < B; k += P) {
-          float o[P];
+          for (int k = 0; k < B; k += P) {
+            float o[P];
 #pragma unroll
-          for (int u = 0; u < P; u += 2) {
-            o[u] = w[k + (u & ~7) + pos8(u & 7)];
-            o[u + 1] = w[k + (u & ~7) + pos8((u + 1) & 7)];
-            mul2(o[u], o[u + 1], m);
-          }
-          if constexpr (SIGNS) {
-            const uint32_t sb = B >= 32 ? sw[k >> 5] >> (k & 31) : sw[0] >> k;
+            for (int u = 0; u < P; u += 2) {
+              o[u] = w[k + (u & ~7) + pos8(u & 7)];
+              o[u + 1] = w[k + (u & ~7) + pos8((u + 1) & 7)];
+              mul2(o[u], o[u + 1], m);
+            }
+            if constexpr (SIGNS) {
+              const uint32_t sb = B >= 32 ? sw[k >> 5] >> (k & 31) : sw[0] >> k;
 #pragma unroll
-            for (int u = 0; u < P; ++u) o[u] = __uint_as_float(__float_as_uint(o[u]) ^ (((sb >> u) & 1u) << 31));
-          }
-          if constexpr (F32) {
-            store8<STORE32>(static_cast<float *>(out) + off + k, __float_as_uint(o[0]), __float_as_uint(o[1]),
-                            __float_as_uint(o[2]), __float_as_uint(o[3]), __float_as_uint(o[4]),
-                            __float_as_uint(o[5]), __float_as_uint(o[6]), __float_as_uint(o[7]));
-          } else if constexpr (P == 8) {  // 8 bf16: one 16-byte store
-            __stcs(reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + off + k),
-                   make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                              pack_bf16x2(o[6], o[7])));
-          } else {
-            store8<STORE32>(static_cast<uint16_t *>(out) + off + k, pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
-                            pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]), pack_bf16x2(o[8], o[9]),
-                            pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]), pack_bf16x2(o[14], o[15]));
+              for (int u = 0; u < P; ++u) o[u] = __uint_as_float(__float_as_uint(o[u]) ^ (((sb >> u) & 1u) << 31));
+            }
+            if constexpr (F32) {
+              store8<STORE32>(static_cast<float *>(out) + off + k, __float_as_uint(o[0]), __float_as_uint(o[1]),
+                              __float_as_uint(o[2]), __float_as_uint(o[3]), __float_as_uint(o[4]),
+                              __float_as_uint(o[5]), __float_as_uint(o[6]), __float_as_uint(o[7]));
+            } else if constexpr (P == 8) {  // 8 bf16: one 16-byte store
+              __stcs(reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + off + k),
+                     make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                                pack_bf16x2(o[6], o[7])));
+            } else {
+              store8<STORE32>(static_cast<uint16_t *>(out) + off + k, pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                              pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]), pack_bf16x2(o[8], o[9]),
+                              pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]), pack_bf16x2(o[14], o[15]));
+            }
           }
         }
       }
