@@ -293,13 +293,35 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // byte offset of 16-byte chunk `ch` (0..7) of row `r` in a 128-byte-swizzled [rows][128 B] tile
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t ch) { return r * 128u + ((ch ^ (r & 7u)) << 4); }
 
-// Issue the TMA copies of group p (tokens p * TOK ...) into `dst`.
+// One bulk copy global -> shared that completes `bar`'s transaction count (16-byte
+// aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   tc::smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+               : "memory");
+}
+
+// Issue the copies of group p (tokens p * TOK ...) into `dst`. Tiles of 16-byte rows
+// without swizzle (n = 512 and 1024) hold a group's bytes in their global order, so a
+// full group arrives by one bulk copy of its contiguous 64 KiB (the TMA boxes of 16-byte
+// rows cost the copy engine one request per row, 4096 per group). A partial group takes
+// the boxes, whose rows past the last token read as zero: at n = 512 the block-diagonal
+// A operand multiplies the other token's rows by zero, which must not meet stale data.
 template <int LOGN, int KR>
-__device__ __forceinline__ void load_group(uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int64_t p,
-                                           int64_t tokens) {
+__device__ __forceinline__ void load_group(uint8_t *dst, const CUtensorMap *map, const uint16_t *x, uint64_t *bar,
+                                           int64_t p, int64_t tokens) {
   using SH = Shape<LOGN, KR>;
   const int64_t t0 = p * SH::TOK;
   const int nvalid = (int)((tokens - t0) < SH::TOK ? (tokens - t0) : SH::TOK);
+  if constexpr (SH::LAYOUT == 0) {
+    static_assert(SH::TOK * SH::TOKBYTES == kGroupBytes, "a full group is one contiguous range");
+    if (nvalid == SH::TOK) {
+      tc::mbar_arrive_expect_tx(bar, kGroupBytes);
+      bulk_load(dst, x + t0 * (int64_t)(SH::ROWS * SH::B), kGroupBytes, bar);
+      return;
+    }
+  }
   if constexpr (SH::PAIR) {  // whole boxes of two tokens; rows past the last token read as zero
     const int nbox = (nvalid + 1) / 2;
     tc::mbar_arrive_expect_tx(bar, (uint32_t)nbox * SH::BOXBYTES);
@@ -316,7 +338,8 @@ __device__ __forceinline__ void load_group(uint8_t *dst, const CUtensorMap *map,
 
 template <int LOGN, int KR, bool SIGNS, bool STORE32, int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
-    k1_tc_rotate_quant(const __grid_constant__ CUtensorMap xmap, int64_t tokens, float clip, float inv_sqrt_n,
+    k1_tc_rotate_quant(const __grid_constant__ CUtensorMap xmap, const uint16_t *__restrict__ x, int64_t tokens,
+                       float clip, float inv_sqrt_n,
                        const uint32_t *__restrict__ signs, uint8_t *__restrict__ q, float *__restrict__ scales,
                        int stall_test, const __grid_constant__ KronParams kp) {
   using SH = Shape<LOGN, KR>;
@@ -357,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // latency overlaps the rest of the setup; ask for the next group at once.
     S.gid[0] = blockIdx.x;
     tc::mbar_arrive(&S.gfull[0]);
-    load_group<LOGN, KR>(smem + kOffX, &xmap, &S.full[0], blockIdx.x, tokens);
+    load_group<LOGN, KR>(smem + kOffX, &xmap, x, &S.full[0], blockIdx.x, tokens);
     first_issued = 1;
     clc_request(&S.clc_resp, &S.clc);
   }
@@ -425,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           last[st] = -1;  // its previous copy was consumed before the slot came free
           break;
         }
-        load_group<LOGN, KR>(smem + kOffX + st * kGroupBytes, &xmap, &S.full[st], p, tokens);
+        load_group<LOGN, KR>(smem + kOffX + st * kGroupBytes, &xmap, x, &S.full[st], p, tokens);
         last[st] = i;
       }
       // every issued copy (and work request) has landed before the CTA can leave
@@ -718,7 +741,8 @@ cudaError_t launch_tc(const void *x, int64_t tokens, float clip, const uint32_t 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, map, tokens, clip, inv_sqrt_n, signs, q, scales, stall_test, kp);
+  return cudaLaunchKernelEx(&cfg, kern, map, static_cast<const uint16_t *>(x), tokens, clip, inv_sqrt_n, signs, q,
+                            scales, stall_test, kp);
 }
 
 template <int LOGN, int BITS>
