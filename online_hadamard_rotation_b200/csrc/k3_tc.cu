@@ -422,31 +422,44 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int k = 0; k < NSW; ++k)
       sw[k] = SIGNS ? (__ldg(signs + (orow * B) / 32 + k) >> (B >= 32 ? 0u : (orow * B) & 31u)) : 0u;
+    // The thread's token row in segment sg of group pp is first_token(pp) + sg TSTEP
+    // (PAIR: the warp's half of the tile picks the odd or even token rows).
+    constexpr int TSTEP = SH::PAIR ? 2 : 1;
+    auto first_token = [&](int64_t pp) -> int64_t {
+      return SH::SPLIT ? pp : SH::PAIR ? pp * SH::TOK + 2 * g * SEG + (wq >> 1) : pp * SH::TOK + g * SEG;
+    };
     // The row steps (and zero points) of a group are loaded one group ahead, so their
-    // DRAM latency hides behind the previous group's work: raw bits, converted when used
-    // (fp32 step, or fp16 step in the low and fp16 zero in the high half).
-      auto load_steps = [&](int64_t pp, uint32_t (&dst)[SEG]) {
+    // DRAM latency hides behind the previous group's work: raw bits (fp32 step, or fp16
+    // step in the low and fp16 zero in the high half). With 8 or more segments per thread
+    // (n <= 2048) lane sg loads segment sg's and each thread takes them by shuffle when
+    // the group starts; otherwise every thread loads its few segments' itself.
+    constexpr bool LANES = SEG >= 8;
+    constexpr int NST = LANES ? 1 : SEG;  // raw steps a thread prefetches
+    auto load_steps = [&](int64_t pp, uint32_t (&dst)[NST]) {
 #pragma unroll
-      for (int sg = 0; sg < SEG; ++sg) {
-        const int64_t token = SH::SPLIT ? pp
-                              : SH::PAIR ? pp * SH::TOK + 2 * (g * SEG + sg) + (row >> 6)
-                                         : pp * SH::TOK + g * SEG + sg;
-        dst[sg] = 0u;
-        if (pp < ngroups && token < rows)
-          dst[sg] = asym ? (uint32_t)__ldg(static_cast<const unsigned short *>(scale) + token) |
-                               ((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(zero) + token) << 16)
-                         : __float_as_uint(__ldg(static_cast<const float *>(scale) + token));
+      for (int j = 0; j < NST; ++j) {
+        const int sg = LANES ? (int)lane : j;
+        const int64_t token = first_token(pp) + (int64_t)sg * TSTEP;
+        dst[j] = 0u;
+        if (sg < SEG && pp < ngroups && token < rows)
+          dst[j] = asym ? (uint32_t)__ldg(static_cast<const unsigned short *>(scale) + token) |
+                              ((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(zero) + token) << 16)
+                        : __float_as_uint(__ldg(static_cast<const float *>(scale) + token));
       }
     };
-    uint32_t step_next[SEG];
+    uint32_t step_next[NST];
     load_steps(blockIdx.x, step_next);
     for (int64_t i = 0;; ++i) {
       const int64_t p = blockIdx.x + i * (int64_t)gridDim.x;
       if (p >= ngroups) break;
       uint32_t step_raw[SEG];
 #pragma unroll
-      for (int sg = 0; sg < SEG; ++sg) step_raw[sg] = step_next[sg];
+      for (int sg = 0; sg < SEG; ++sg)
+        step_raw[sg] = LANES ? __shfl_sync(0xffffffffu, step_next[0], sg) : step_next[LANES ? 0 : sg];
       load_steps(p + gridDim.x, step_next);
+      const int64_t tok0 = first_token(p);
+      // segments 0 .. nseg - 1 hold token rows below `rows` (the same for the warp)
+      const int nseg = rows - tok0 >= (int64_t)SEG * TSTEP ? SEG : (int)((rows - tok0 + TSTEP - 1) / TSTEP);
       const int acc = (int)(i & 1);
       // every thread sleeps on the accumulator's barrier itself (no block-level barrier
       // between the epilogue warps)
@@ -505,8 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int orow0 = (SH::SPLIT ? 128 * (int)g : 0) + 32 * (int)wq;
 #pragma unroll
         for (int sg = 0; sg < SEG; ++sg) {
-          const int64_t token = SH::SPLIT ? p : p * SH::TOK + g * SEG + sg;
-          if (token >= rows) continue;  // the same for the whole warpgroup
+          if (sg >= nseg) break;  // the same for the whole warpgroup
+          const int64_t token = tok0 + sg;
           const float s = asym ? __half2float(__ushort_as_half((unsigned short)step_raw[sg]))
                                : __uint_as_float(step_raw[sg]);
           const float m = s * inv_sqrt_n;
@@ -547,17 +560,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
+        // first element of this thread's row in segment 0; segment sg starts sg TSTEP
+        // token rows further (a constant offset the compiler folds into the stores)
+        const int64_t off0 = tok0 * (int64_t)(B * SH::ROWS) + (int64_t)orow * B;
 #pragma unroll
         for (int sg = 0; sg < SEG; ++sg) {
-          const int64_t token = SH::SPLIT ? p
-                                : SH::PAIR ? p * SH::TOK + 2 * (g * SEG + sg) + (row >> 6)
-                                           : p * SH::TOK + g * SEG + sg;
-          if (token >= rows) continue;
+          if (sg >= nseg) break;
           const float s = asym ? __half2float(__ushort_as_half((unsigned short)step_raw[sg]))
                                : __uint_as_float(step_raw[sg]);
           const float m = s * inv_sqrt_n;
           const float *w = v + sg * B;
-          const int64_t off = token * (int64_t)(B * SH::ROWS) + (int64_t)orow * B;  // first element of the row
+          const int64_t off = off0 + (int64_t)sg * TSTEP * (B * SH::ROWS);
           // one 8 (fp32) or 16 (bf16; 8 when B = 8) element piece at a time, in element
           // order: scale, diagonal sign, store
           constexpr int P = (F32 || B == 8) ? 8 : 16;
