@@ -128,22 +128,22 @@ struct Shape {
 
 // Paley's Hadamard matrix of order m, as a kernel argument: type I (q = m - 1, prime,
 // q = 3 mod 4) or type II (q = m/2 - 1, prime, q = 1 mod 4); qr bit a is set when a
-// (0 < a < q) is a square mod q. bq = b / 128 = KR / m.
+// (0 < a < q) is a square mod q. bq = b / 128 = KR / m, a power of two 2^lbq.
 struct KronParams {
-  int m, type, q, bq;
+  int m, type, q, bq, lbq;
   uint32_t qr[4];
 };
 
-// Quadratic character of a mod q from the residue mask: 0, +1 or -1.
+// Quadratic character of a mod q from the residue mask, for -q < a < q: 0, +1 or -1.
 __device__ __forceinline__ int chi(int a, const KronParams &kp) {
-  a %= kp.q;
   if (a < 0) a += kp.q;
   if (a == 0) return 0;
   return ((kp.qr[a >> 5] >> (a & 31)) & 1u) ? 1 : -1;
 }
 
 // Entry (i, j) of Paley's H_m. With the core matrix C of order q + 1 -- C[0][0] = 0,
-// C[0][j] = 1, C[i][0] = -1 (type I) or +1 (type II), C[i][j] = chi(j - i) otherwise --
+// C[0][j] = 1, C[i][0] = -1 (type I) or +1 (type II), C[i][j] = chi(j - i) otherwise
+// (1 <= i, j <= q, so -q < j - i < q) --
 // type I is C + I and type II replaces each entry c of C by c [[1, -1], [-1, -1]]
 // plus [[1, 1], [1, -1]] on the diagonal.
 __device__ __forceinline__ int paley_entry(int i, int j, const KronParams &kp) {
@@ -390,8 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto a_entry = [&](uint32_t m, uint32_t k) -> uint32_t {  // bf16 pattern of A[m][k]
     if constexpr (SH::KRON) {
       if (m >= (uint32_t)KR || k >= (uint32_t)KR) return 0u;
-      const int h = paley_entry((int)m / kp.bq, (int)k / kp.bq, kp) *
-                    ((__popc((m % kp.bq) & (k % kp.bq)) & 1) ? -1 : 1);
+      const uint32_t mask = (uint32_t)kp.bq - 1u;
+      const int h = paley_entry((int)(m >> kp.lbq), (int)(k >> kp.lbq), kp) * ((__popc(m & k & mask) & 1) ? -1 : 1);
       return h > 0 ? 0x3F80u : 0xBF80u;
     } else if constexpr (SH::PAIR) {  // H_64 (+) H_64
       if ((m >> 6) != (k >> 6)) return 0u;
@@ -1202,7 +1202,8 @@ cudaError_t launch_rotate_quant_kron(int m, int n, int bits, const void *x, int6
   kp.m = m;
   kp.type = paley_type(m);
   kp.q = kp.type == 1 ? m - 1 : m / 2 - 1;
-  kp.bq = (n / m) / 128;
+  kp.bq = (n / m) / 128;  // a power of two: n / m = 2^k with 2^k >= 128
+  while ((1 << kp.lbq) < kp.bq) ++kp.lbq;
   for (int a = 1; a < kp.q; ++a) {  // the nonzero squares mod q
     const int sq = (a * a) % kp.q;
     kp.qr[sq >> 5] |= 1u << (sq & 31);
