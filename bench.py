@@ -44,13 +44,19 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 def metric_for(wl) -> str:
-    """The headline metric, or its counterpart for the INT8, Kronecker-size and
-    decode-attention workloads."""
+    """The headline metric, or its counterpart for the INT8, other-n, Kronecker-size,
+    R3 + KV and decode-attention workloads."""
     if wl.get("kind") == "attn":
         return "decode attention over the INT4 KV cache: HBM GB/s (% of B200 peak) and us per step"
+    if wl.get("kind") == "r3":
+        return ("fused RoPE + Hadamard (R3) on Q/K + asymmetric INT4 KV-cache quant: HBM GB/s (% of B200 peak) "
+                "and tokens/s at head_dim=128")
     m = METRIC.replace("INT4", "INT8") if wl.get("code_bits", 4) == 8 else METRIC
+    n = int(wl["bits"].shape[1]) if "bits" in wl else 16384
     if wl.get("kron_m"):
-        m = m.replace("at n=16384", f"at n={wl['bits'].shape[1]} (H_{wl['kron_m']} Paley x Sylvester)")
+        m = m.replace("at n=16384", f"at n={n} (H_{wl['kron_m']} Paley x Sylvester)")
+    elif n != 16384:
+        m = m.replace("at n=16384", f"at n={n}")
     return m
 
 
