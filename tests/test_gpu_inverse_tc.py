@@ -1,8 +1,10 @@
 """The tensor-core dequantise + inverse kernels vs the fp64 oracle, and vs the
 all-CUDA-core kernel selected with SPIN_CUDA_CORES_ONLY. Codes are expanded to
 exact fp16 integers; at n = 128 and 256 the rows are the MMA's M against a
-constant H_128 (H_2 of n = 256 in the epilogue), at n = 4096 .. 32768 the first
-H_128 factor runs on tcgen05 and the second in registers. Both kernels transform
+constant H_128 (H_2 of n = 256 in the epilogue), at n = 512 .. 32768 the first
+Kronecker factor (H_64 (+) H_64 at n = 512) runs on tcgen05 and the second in
+registers, and rows of 64 bytes or more (bf16 from n = 4096, fp32 from 2048) leave
+through TMA tensor stores from swizzled staging tiles. Both kernels transform
 exact integers and scale once at the end, so their outputs must agree bit for
 bit. Row counts leave partial MMA groups (128 rows per group at n = 128 and 256;
 64 at n = 512, whose odd row counts split a two-row tile; 32, 16, 8, 4, 2 and 1 from
