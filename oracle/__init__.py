@@ -27,6 +27,7 @@ _u16p = np.ctypeslib.ndpointer(dtype=np.uint16, flags="C_CONTIGUOUS")
 _u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
 _i8p = np.ctypeslib.ndpointer(dtype=np.int8, flags="C_CONTIGUOUS")
 _i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+_f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
 
 
 def lib():
@@ -92,6 +93,8 @@ def lib():
     L.orc_r4_rows.argtypes = [_u16p, C.c_int64, C.c_int, C.c_double, vp, C.c_uint32, _u8p,
                               np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS"), C.c_int]
     L.orc_r4_rows.restype = C.c_int
+    L.orc_w4a4_gemm.argtypes = [_u8p, _f32p, C.c_int64, _u8p, _f32p, C.c_int, C.c_int, _dp, C.c_int]
+    L.orc_w4a4_gemm.restype = C.c_int
     L.orc_max_threads.restype = C.c_int
     L.orc_rope_half.argtypes = [_dp, C.c_int, C.c_double, C.c_double]
     L.orc_r3_token.argtypes = [_u16p, _u16p, _u16p, C.c_double, C.c_double, C.c_int, C.c_int,
@@ -376,6 +379,35 @@ def r4_rows(x_bits, clip, signs=None, no_rotate=False, threads=1):
     if rc:
         raise ValueError(f"orc_r4_rows failed ({rc})")
     return packed, scales
+
+
+# ---------------------------------------------------------------- W4A4 GEMM
+def bake_weights(w_bits, signs=None, clip=1.0, threads=1):
+    """Offline weight baking: each output row w_o of W [n_out, k] (bf16 bits) becomes a
+    row of W R^T = (R w_o)^T with R = H D / sqrt(k), the rotation the activations get
+    online, quantised per output channel by the same symmetric INT4 rule ("SpinQuant
+    Guide", "Production Engineering and Cluster Deployment Best Practices": compute
+    W R^T offline, quantise it and pack INT4 nibbles). Returns (codes [n_out, k/2],
+    scales [n_out])."""
+    return r4_rows(w_bits, clip, signs=signs, threads=threads)
+
+
+def w4a4_gemm(xq, xs, wq, ws, threads=1) -> np.ndarray:
+    """y [tokens, n_out] = (s_x q_x)(s_w q_w)^T from packed INT4 codes ("SpinQuant Guide",
+    "End-to-End Implementation": the quantised output is the product of the dequantised
+    activations and weights), exact integer sums scaled once in fp64."""
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    xs = np.ascontiguousarray(xs, dtype=np.float32)
+    ws = np.ascontiguousarray(ws, dtype=np.float32)
+    T, kh = xq.shape
+    N = wq.shape[0]
+    if wq.shape[1] != kh or xs.shape != (T,) or ws.shape != (N,):
+        raise ValueError("w4a4_gemm: shapes do not match")
+    y = np.empty((T, N), dtype=np.float64)
+    if lib().orc_w4a4_gemm(xq, xs, T, wq, ws, N, 2 * kh, y, int(threads)):
+        raise ValueError("orc_w4a4_gemm failed")
+    return y
 
 
 # ---------------------------------------------------------------- R3

@@ -25,8 +25,11 @@
  *        [-8, 7], step = max|x| / (2^(b-1) - 1); at b = 8 the per-token INT8
  *        activations of W4A8), section "End-to-End
  *        Implementation" (scale clamped below at 1e-8, x_dequant = x_quant *
- *        scale), section "RoPE Compatibility with 4-Bit KV Caching" (RoPE
- *        rotates 2-D coordinate pairs; KV cache stored as 4-bit).
+ *        scale; the quantised layer output is the product of the quantised
+ *        activations and weights), section "RoPE Compatibility with 4-Bit KV
+ *        Caching" (RoPE rotates 2-D coordinate pairs; KV cache stored as 4-bit),
+ *        section "Production Engineering and Cluster Deployment Best Practices"
+ *        (W R^T baked offline into packed INT4 weights for an INT4 GEMM).
  *  [SW]  "SpinQuant, when rotations are worth learning", section "Four
  *        rotation sites, two of them free" (R3: Hadamard on Q and K after
  *        RoPE; R4: Hadamard on the down-projection input), section "Paper vs.
@@ -41,7 +44,9 @@
  * fp16-rounded scale; for n = m 2^k that is not a power of two, the small factor
  * H_m is Paley's (type I or II, a named published construction: the pages give
  * none), the product is H_m (x) H_{2^k} with the H_m index as the high part of
- * the element index, and the diagonal again comes first.
+ * the element index, and the diagonal again comes first; the W4A4 GEMM's weights
+ * are quantised per output channel by the activations' symmetric INT4 rule (the
+ * pages' listing uses one scale per tensor), each row first rotated by the same R.
  */
 #include <fenv.h>
 #include <math.h>
@@ -554,6 +559,47 @@ int orc_max_threads(void) {
 #else
   return 1;
 #endif
+}
+
+/* ------------------------------------------------------------------ */
+/* W4A4 GEMM on the codes                                               */
+/* ------------------------------------------------------------------ */
+
+/* [SG] "End-to-End Implementation": the quantised layer output is the matrix product of
+ * the quantised activations and the quantised (rotated) weights, each dequantised as
+ * code * scale; "Production Engineering and Cluster Deployment Best Practices": the
+ * rotated weights W R^T are quantised offline and stored as packed INT4 nibbles, and
+ * the product runs on INT4 tensor cores.
+ *   y[t][o] = sum_k (s_x[t] q_x[t][k]) (s_w[o] q_w[o][k]) = s_x[t] s_w[o] sum_k q_x q_w
+ * The integer sum is exact (int64); the scales multiply it once, in binary64. Codes are
+ * 4-bit two's complement, element 2j in the low nibble of byte j: x [tokens, k/2],
+ * w [n_out, k/2] (one row per output channel), y [tokens, n_out]. Rows of y are
+ * independent; `threads` spreads them over OpenMP threads. */
+int orc_w4a4_gemm(const uint8_t *xq, const float *xs, int64_t tokens, const uint8_t *wq, const float *ws,
+                  int n_out, int k, double *y, int threads) {
+  if (tokens < 0 || n_out <= 0 || k <= 0 || (k & 1)) return -1;
+  int32_t *w = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_out * (size_t)k);
+  if (!w) return -1;
+  for (int o = 0; o < n_out; o++) orc_unpack_nibbles(wq + (size_t)o * (k / 2), k, 1, w + (size_t)o * k);
+  int rc = 0;
+#pragma omp parallel for schedule(dynamic, 4) num_threads(threads > 0 ? threads : 1) reduction(| : rc)
+  for (int64_t t = 0; t < tokens; t++) {
+    int32_t *x = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
+    if (!x) {
+      rc |= 1;
+      continue;
+    }
+    orc_unpack_nibbles(xq + (size_t)t * (k / 2), k, 1, x);
+    for (int o = 0; o < n_out; o++) {
+      const int32_t *wo = w + (size_t)o * k;
+      int64_t acc = 0;
+      for (int j = 0; j < k; j++) acc += (int64_t)x[j] * wo[j];
+      y[(size_t)t * n_out + o] = (double)xs[t] * (double)ws[o] * (double)acc;
+    }
+    free(x);
+  }
+  free(w);
+  return rc ? -1 : 0;
 }
 
 /* ------------------------------------------------------------------ */
