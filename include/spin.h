@@ -319,6 +319,37 @@ spin_status_t spin_decode_attention_int4kv(const void *q, const uint8_t *k_cache
  * ceil(cache_len / 256) partials of head_dim + 2 fp32 values); 0 for sizes <= 0. */
 size_t spin_decode_attention_workspace_bytes(int32_t batch, int32_t n_q_heads, int32_t cache_len);
 
+/*
+ * W4A4 GEMM on packed INT4 codes ("SpinQuant Guide: Learned Rotations for 4-Bit
+ * LLMs", section "End-to-End Implementation": the quantised layer output is the
+ * product of the quantised activations and the quantised weights, each dequantised as
+ * code x scale; section "Production Engineering and Cluster Deployment Best
+ * Practices": the rotated weights W R^T are baked offline into packed INT4 nibbles and
+ * multiplied on INT4 tensor cores):
+ *   out[t][o] = x_scales[t] w_scales[o] sum_k q_x[t][k] q_w[o][k]
+ * The activations are what spin_hadamard_quant_int4_ex / _kron write (per-token codes
+ * and fp32 steps); the weights are packed the same way, one row and one fp32 step per
+ * output channel (rows of W R^T quantised by the same symmetric INT4 rule: run the
+ * weight rows through spin_hadamard_quant_int4_ex with the activations' diagonal at
+ * clip 1.0). The integer sum is exact (int32 accumulation on the tensor cores); the
+ * product of the two steps and the sum are rounded once each to fp32, then to bf16
+ * when out_dtype is SPIN_BF16.
+ *  x_codes   [tokens, k/2] packed 4-bit two's-complement codes, element 2j in the low
+ *            nibble of byte j, 16-byte aligned
+ *  x_scales  [tokens] fp32, 4-byte aligned
+ *  w_codes   [n_out, k/2] packed codes of the weight rows, 16-byte aligned
+ *  w_scales  [n_out] fp32, 16-byte aligned
+ *  n_out     a multiple of 256; k a multiple of 128, 128 .. 65536
+ *  out       [tokens, n_out] fp32 or bf16 (out_dtype), 16-byte aligned
+ * One kernel on `stream`; tokens == 0 is a no-op.
+ * Errors: SPIN_ERR_INVALID_ARG (tokens < 0, a NULL pointer, out_dtype),
+ * SPIN_ERR_UNSUPPORTED_SIZE (n_out, k or tokens outside the ranges above),
+ * SPIN_ERR_MISALIGNED, SPIN_ERR_DEVICE, SPIN_ERR_CUDA.
+ */
+spin_status_t spin_w4a4_gemm(const uint8_t *x_codes, const float *x_scales, int64_t tokens, const uint8_t *w_codes,
+                             const float *w_scales, int32_t n_out, int32_t k, void *out, int32_t out_dtype,
+                             spin_stream_t stream);
+
 /* Bytes of the scratch array built into the library for
  * spin_decode_attention_int4kv_noalloc (held by every GPU that loads the library). */
 #define SPIN_NOALLOC_SCRATCH_BYTES (4u << 20)

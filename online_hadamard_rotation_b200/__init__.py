@@ -73,11 +73,12 @@ def lib() -> C.CDLL:
     L.spin_hadamard_quant_kron.argtypes = [vp, i64, i32, i32, f32, vp, u32, i32, vp, vp, vp]
     L.spin_decode_attention_int4kv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32,
                                                vp, C.c_size_t, vp]
+    L.spin_w4a4_gemm.argtypes = [vp, vp, i64, vp, vp, i32, i32, vp, i32, vp]
     L.spin_decode_attention_workspace_bytes.argtypes = [i32, i32, i32]
     L.spin_decode_attention_workspace_bytes.restype = C.c_size_t
     for name in ("spin_hadamard_quant_int4", "spin_hadamard_quant_int4_ex", "spin_hadamard_quant_int8",
                  "spin_rope_hadamard_kvquant", "spin_dequant_hadamard_inverse", "spin_hadamard_quant_kron",
-                 "spin_decode_attention_int4kv"):
+                 "spin_decode_attention_int4kv", "spin_w4a4_gemm"):
         getattr(L, name).restype = C.c_int
     L.spin_uses_tensor_cores.argtypes = [i32, i64, i32, u32, i32]
     L.spin_uses_tensor_cores.restype = C.c_int
@@ -126,6 +127,10 @@ def spin_hadamard_quant_kron(x_bf16, tokens, m, n, clip, sign_bits, flags, bits,
 
 def spin_decode_attention_int4kv(*args) -> int:
     return lib().spin_decode_attention_int4kv(*args)
+
+
+def spin_w4a4_gemm(*args) -> int:
+    return lib().spin_w4a4_gemm(*args)
 
 
 def spin_rope_hadamard_kvquant(*args) -> int:
@@ -261,6 +266,33 @@ def hadamard_quant_kron(x: torch.Tensor, m: int, clip: float = 1.0, signs: torch
                                   _ptr(scales), _stream(stream))
     _check("spin_hadamard_quant_kron", st)
     return out, scales
+
+
+def w4a4_gemm(x_codes: torch.Tensor, x_scales: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor,
+              out_dtype=torch.float32, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """W4A4 GEMM on packed INT4 codes: x_codes [tokens, k/2] uint8 and x_scales [tokens]
+    fp32 (as hadamard_quant_int4 / hadamard_quant_kron return them), w_codes [n_out, k/2]
+    uint8 and w_scales [n_out] fp32 (weight rows packed the same way) -> out [tokens, n_out]
+    = x_scales[t] w_scales[o] sum_k q_x q_w, fp32 or bf16."""
+    _need(x_codes, "x_codes", torch.uint8)
+    if x_codes.dim() != 2 or w_codes.dim() != 2:
+        raise ValueError("x_codes and w_codes must be 2-D [rows, k/2]")
+    tokens, kh = x_codes.shape
+    n_out = w_codes.shape[0]
+    _need(w_codes, "w_codes", torch.uint8, x_codes.device, (n_out, kh))
+    _need(x_scales, "x_scales", torch.float32, x_codes.device, (tokens,))
+    _need(w_scales, "w_scales", torch.float32, x_codes.device, (n_out,))
+    if out is None:
+        if out_dtype not in (torch.float32, torch.bfloat16):
+            raise TypeError(f"out_dtype: expected torch.float32 or torch.bfloat16, got {out_dtype}")
+        out = torch.empty((tokens, n_out), dtype=out_dtype, device=x_codes.device)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"out: expected torch.float32 or torch.bfloat16, got {out.dtype}")
+    _need(out, "out", out.dtype, x_codes.device, (tokens, n_out))
+    st = spin_w4a4_gemm(_ptr(x_codes), _ptr(x_scales), tokens, _ptr(w_codes), _ptr(w_scales), n_out, 2 * kh,
+                        _ptr(out), F32 if out.dtype == torch.float32 else BF16, _stream(stream))
+    _check("spin_w4a4_gemm", st)
+    return out
 
 
 def hadamard_quant_host(x_host: torch.Tensor, clip: float = 1.0, signs: torch.Tensor | None = None, bits: int = 4,

@@ -162,6 +162,22 @@ spin_status_t spin_hadamard_quant_kron(const void *x_bf16, int64_t tokens, int32
                                               scales_f32, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+spin_status_t spin_w4a4_gemm(const uint8_t *x_codes, const float *x_scales, int64_t tokens, const uint8_t *w_codes,
+                             const float *w_scales, int32_t n_out, int32_t k, void *out, int32_t out_dtype,
+                             spin_stream_t stream) {
+  if (tokens < 0 || (out_dtype != SPIN_BF16 && out_dtype != SPIN_F32)) return SPIN_ERR_INVALID_ARG;
+  if (!w4a4_shape_supported(tokens, n_out, k)) return SPIN_ERR_UNSUPPORTED_SIZE;
+  if (tokens == 0) return SPIN_OK;
+  if (!x_codes || !x_scales || !w_codes || !w_scales || !out) return SPIN_ERR_INVALID_ARG;
+  if (!aligned(x_codes, 16) || !aligned(w_codes, 16) || !aligned(out, 16) || !aligned(w_scales, 16) ||
+      !aligned(x_scales, 4))
+    return SPIN_ERR_MISALIGNED;
+  spin_status_t st = check_device();
+  if (st != SPIN_OK) return st;
+  return cuda_status(launch_w4a4_gemm(x_codes, x_scales, tokens, w_codes, w_scales, n_out, k, out,
+                                      out_dtype == SPIN_F32, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 spin_status_t spin_rope_hadamard_kvquant(const void *q, const void *k, const void *v, const int32_t *pos,
                                          float theta, int32_t head_dim, int32_t batch, int32_t seq,
                                          int32_t n_q_heads, int32_t n_kv_heads, float clip, void *q_out,
@@ -264,11 +280,12 @@ int spin_last_cuda_error(void) { return g_last_cuda_error; }
 
 spin_status_t spin_device_status(uint32_t *status, int reset) {
   if (!status) return SPIN_ERR_INVALID_ARG;
-  unsigned int v = 0, w = 0, u = 0;
+  unsigned int v = 0, w = 0, u = 0, g = 0;
   spin_status_t st = cuda_status(read_device_status(&v, reset != 0));
   if (st == SPIN_OK) st = cuda_status(read_rope_status(&w, reset != 0));
   if (st == SPIN_OK) st = cuda_status(read_dequant_status(&u, reset != 0));
-  *status = v | w | u;
+  if (st == SPIN_OK) st = cuda_status(read_gemm_status(&g, reset != 0));
+  *status = v | w | u | g;
   return st;
 }
 

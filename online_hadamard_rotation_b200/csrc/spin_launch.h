@@ -48,6 +48,12 @@ cudaError_t launch_decode_attention(const void *q, const uint8_t *k_cache, const
                                     const void *v_zero, const int32_t *lens, int batch, int n_q_heads,
                                     int n_kv_heads, int cache_len, float softmax_scale, void *out, bool out_f32,
                                     float *workspace, cudaStream_t stream);
+// W4A4 GEMM on packed INT4 codes (k5_w4a4_gemm.cu): shapes it takes (n_out a multiple
+// of 256, k a multiple of 128 up to 65536), the launch, and its status word.
+bool w4a4_shape_supported(int64_t tokens, int n_out, int k);
+cudaError_t launch_w4a4_gemm(const uint8_t *xq, const float *xs, int64_t tokens, const uint8_t *wq, const float *ws,
+                             int n_out, int k, void *out, bool out_f32, cudaStream_t stream);
+cudaError_t read_gemm_status(unsigned int *status, bool reset);
 cudaError_t launch_rotate_quant_tc(int log_n, int bits, const void *x, int64_t tokens, float clip,
                                    const uint32_t *signs, uint8_t *q, float *scales, cudaStream_t stream);
 

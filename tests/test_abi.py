@@ -207,6 +207,27 @@ def test_kron_size_rules(L):
     assert f(None, 4, 28, 14336, 1.0, None, 0, 4, None, None, None) == BAD      # null pointers
 
 
+def test_w4a4_gemm_host_rules(L):
+    """spin_w4a4_gemm takes n_out a multiple of 256 and k a multiple of 128 in
+    [128, 65536]; tokens = 0 and every rejected argument return before any device
+    access, so the rules are checked here without a GPU."""
+    f = L.spin_w4a4_gemm
+    f.argtypes = [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_void_p,
+                  C.c_int32, C.c_void_p]
+    f.restype = C.c_int
+    OK, BAD, SIZE, MIS = 0, 1, 2, 3
+    for n_out, k in ((256, 128), (4096, 14336), (14336, 4096), (11008, 4096), (256, 65536)):
+        assert f(None, None, 0, None, None, n_out, k, None, 1, None) == OK, (n_out, k)
+    for n_out, k in ((128, 4096), (4000, 4096), (4096, 64), (4096, 4000), (4096, 65536 + 128), (0, 128),
+                     (256, 0), (-256, 128)):
+        assert f(None, None, 0, None, None, n_out, k, None, 1, None) == SIZE, (n_out, k)
+    assert f(None, None, -1, None, None, 256, 128, None, 1, None) == BAD      # tokens < 0
+    assert f(None, None, 0, None, None, 256, 128, None, 2, None) == BAD       # out_dtype
+    assert f(None, None, 4, None, None, 256, 128, None, 1, None) == BAD       # null pointers
+    assert f(FAKE, FAKE + 4, 4, FAKE, FAKE + 4, 256, 128, FAKE, 1, None) == MIS   # w_scales not 16-byte aligned
+    assert f(FAKE + 8, FAKE, 4, FAKE, FAKE, 256, 128, FAKE, 1, None) == MIS      # x_codes
+
+
 def test_decode_attention_host_rules(L):
     """Workspace size and argument rules of the decode-attention entry point; batch = 0
     and every rejected argument return before any device access."""
