@@ -51,6 +51,10 @@ def metric_for(wl) -> str:
     if wl.get("kind") == "r3":
         return ("fused RoPE + Hadamard (R3) on Q/K + asymmetric INT4 KV-cache quant: HBM GB/s (% of B200 peak) "
                 "and tokens/s at head_dim=128")
+    if wl.get("kind") == "gemm":
+        T, K = wl["bits"].shape
+        return (f"W4A4 GEMM on the R4 kernel's INT4 codes (tcgen05 kind::i8): TOPS (% of int8 tensor peak) at "
+                f"{T} x {wl['n_out']} x k={K}")
     m = METRIC.replace("INT4", "INT8") if wl.get("code_bits", 4) == 8 else METRIC
     n = int(wl["bits"].shape[1]) if "bits" in wl else 16384
     if wl.get("kron_m"):
@@ -105,6 +109,19 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def int8_peak_tops():
+    """Dense int8 tensor peak for a kernel timed inside a sustained loop: the measured
+    sustained bf16 GEMM throughput times the nominal int8 : bf16 dense ratio (4.5 : 2.25
+    PFLOP/s on B200)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        if "bf16_tflops_sustained" in d:
+            return 2.0 * float(d["bf16_tflops_sustained"]), "2 x measured bf16_tflops_sustained (int8 : bf16 = 2)"
+    return 2.0 * 1400.0, "2 x fallback sustained bf16 1.4 PFLOP/s (int8 : bf16 = 2)"
 
 
 def kernel_source_digest(kernel: str) -> str:
@@ -229,6 +246,17 @@ def make_workload(name: str, rank: int, tokens: int | None = None):
                     desc={"workload": f"decode attention over the INT4 KV cache: batch {batch} x 4096 cached slots "
                                       "(the R3+KV workload's cache, written by the R3 kernel), 32 q / 8 kv heads, "
                                       "head_dim 128, one query token per row", "tokens": batch})
+    if name == "w4a4_gemm":
+        T = tokens or 8192
+        bits, signs, _ = synthetic.r4_prefill(tokens=T, n=14336, seed=1 + rank)
+        return dict(kind="gemm", bits=bits, w_bits=synthetic.weights(4096, 14336, seed=7 + rank), signs=signs,
+                    kron_m=28, clip=0.9, n_out=4096,
+                    desc={"workload": f"W4A4 GEMM at the LLaMA-3 8B down-projection shape: {T} tokens x k = 14336 "
+                                      "(the R4 kernel's codes of the n = 14336 prefill: H_28 Paley (x) H_512, seeded "
+                                      "+-1 diagonal, clip 0.9) against 4096 output channels (N(0, 1/k) bf16 weight "
+                                      "rows baked by the same kernel, clip 1.0); bf16 output",
+                          "tokens": T, "n_out": 4096, "k": 14336,
+                          "l2": "operands (88 MB of codes) stay L2-resident across steps, as for any GEMM"})
     if name.startswith("kron"):
         n = int(name[len("kron"):] or 14336)
         m = {14336: 28, 6144: 12, 10240: 20, 12288: 12}[n]
@@ -260,9 +288,9 @@ def make_workload(name: str, rank: int, tokens: int | None = None):
 
 def config_for(wl, world: int, workload: str) -> dict:
     """The `config` object both arms print (same workload, same keys)."""
-    return dict(wl["desc"], parallelism=f"dp{world}" if world > 1 else "single GPU",
-                l2="inputs larger than L2 (268 MB bf16 input vs 126 MB L2); two buffer sets alternate"
-                if workload.startswith("r4_prefill") else "two buffer sets alternate")
+    l2 = ("inputs larger than L2 (268 MB bf16 input vs 126 MB L2); two buffer sets alternate"
+          if workload.startswith("r4_prefill") else "two buffer sets alternate")
+    return dict(wl["desc"], parallelism=f"dp{world}" if world > 1 else "single GPU", l2=wl["desc"].get("l2", l2))
 
 
 def r3_bytes(tokens, hq=32, hkv=8, d=128):
@@ -309,11 +337,42 @@ def run_reference_attn(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_gemm(args, wl):
+    """The oracle's pipeline on a bounded sample: the first 16 token rows through the R4
+    rows and all weight rows baked once, then the GEMM of those rows against every output
+    channel, all host cores; TOPS of the GEMM part."""
+    import oracle
+    oracle.lib()
+    threads = oracle.max_threads()
+    rows = 16
+    xq, xs = oracle.r4_rows_kron(wl["bits"][:rows], wl["kron_m"], wl["clip"], wl["signs"], threads=threads)
+    wq, ws = oracle.r4_rows_kron(wl["w_bits"], wl["kron_m"], 1.0, wl["signs"], threads=threads)
+    for _ in range(args.warmup):
+        oracle.w4a4_gemm(xq[:1], xs[:1], wq, ws, threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.w4a4_gemm(xq, xs, wq, ws, threads=threads)
+    dt = time.perf_counter() - t0
+    tops = 2 * rows * wq.shape[0] * 2 * wq.shape[1] * args.steps / dt / 1e12
+    line = {"impl": "reference", "metric": metric_for(wl), "value": tops, "unit": "TOPS",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int64", "data": "synthetic",
+            "config": config_for(wl, args.gpus, args.workload),
+            "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                             "sample": f"{rows} of {wl['bits'].shape[0]} token rows per step against all "
+                                       f"{wq.shape[0]} outputs, exact int64 sums, {threads} host thread(s)"},
+            "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args, wl):
     import oracle
     oracle.lib()
     if wl["kind"] == "attn":
         return run_reference_attn(args, wl)
+    if wl["kind"] == "gemm":
+        return run_reference_gemm(args, wl)
     if wl["kind"] != "r4":
         raise SystemExit("the reference arm times the R4 and decode-attention workloads")
     bits, n = wl["bits"], wl["bits"].shape[1]
@@ -372,6 +431,32 @@ def cpu_baseline_leg(wl):
     cpu["all_cores"] = {"value": cpu_bytes / dt / 1e9, "unit": "GB/s", "cores": used, "tokens_per_s": sample / dt,
                         "sample": "the same rows, spread over the host's cores"}
     return cpu, ref
+
+
+def cpu_baseline_gemm(xq, xs, wq, ws, out_dev, rows: int = 8):
+    """The fp64 oracle GEMM on a bounded sample (the first `rows` token rows against every
+    output channel), one thread and all host cores; the same rows of the GPU's last timed
+    step must match it within the bf16 output tolerance."""
+    import oracle
+    oracle.lib()
+    xq_h, xs_h = xq[:rows].cpu().numpy(), xs[:rows].cpu().numpy()
+    wq_h, ws_h = wq.cpu().numpy(), ws.cpu().numpy()
+    ops = 2 * rows * wq_h.shape[0] * 2 * wq_h.shape[1]
+    t0 = time.perf_counter()
+    oracle.w4a4_gemm(xq_h, xs_h, wq_h, ws_h, threads=1)
+    dt1 = time.perf_counter() - t0
+    used = oracle.max_threads()
+    t0 = time.perf_counter()
+    ref = oracle.w4a4_gemm(xq_h, xs_h, wq_h, ws_h, threads=used)
+    dtn = time.perf_counter() - t0
+    got = out_dev[:rows].float().cpu().numpy().astype(np.float64)
+    lim = np.maximum(2e-2, np.abs(ref) * 2.0 ** -8)  # bf16 rounding of the output (round to nearest)
+    bad = int(np.sum(np.abs(got - ref) > lim))
+    return {"value": ops / dt1 / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} token rows x {wq_h.shape[0]} outputs x k = {2 * wq_h.shape[1]}, exact int64 sums, "
+                      "1 thread",
+            "all_cores": {"value": ops / dtn / 1e12, "unit": "TOPS", "cores": used, "sample": "the same rows"},
+            "spot_check": {"rows": rows, "outputs_off": bad, "ok": bad == 0}}
 
 
 # ---------------------------------------------------------------------------
@@ -576,6 +661,22 @@ def main():
         def step(i, cores_only=False):
             b = sets[i & 1]
             quant(b["x"], wl["clip"], signs, out=b["q"], scales=b["s"], stream=stream, cuda_cores_only=cores_only)
+    elif wl["kind"] == "gemm":
+        # activations through the R4 kernel, weight rows baked by the same kernel (same diagonal)
+        T, K = wl["bits"].shape
+        N = wl["n_out"]
+        tokens = T
+        signs = torch.from_numpy(wl["signs"].view(np.int32)).to(dev)
+        to_dev = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
+        xq, xs = spin.hadamard_quant_kron(to_dev(wl["bits"]), wl["kron_m"], wl["clip"], signs)
+        wq, ws = spin.hadamard_quant_kron(to_dev(wl["w_bits"]), wl["kron_m"], 1.0, signs)
+        sets = [dict(out=torch.empty((T, N), dtype=torch.bfloat16, device=dev)) for _ in range(2)]
+        torch.cuda.synchronize()
+        step_ops = 2 * T * N * K
+        step_bytes = T * (K // 2 + 4) + N * (K // 2 + 4) + 2 * T * N  # codes, steps, bf16 output
+
+        def step(i, cores_only=False):
+            spin.w4a4_gemm(xq, xs, wq, ws, out=sets[i & 1]["out"], stream=stream)
     elif wl["kind"] == "attn":
         # the cache as the R3 kernel writes it from the workload's Q, K, V; one query per row
         q, k, v, pos = wl["q"], wl["k"], wl["v"], wl["pos"]
@@ -633,7 +734,8 @@ def main():
     require_clean_status(spin, "timed region")
     ms_per_step, window_info = window_stats(windows, args.steps)
     last = sets[(args.steps * len(windows) - 1) & 1]  # buffers of the last timed step, kept for the spot check
-    last = {"q": last["q"].clone(), "s": last["s"].clone()} if wl["kind"] == "r4" else None
+    last = ({"q": last["q"].clone(), "s": last["s"].clone()} if wl["kind"] == "r4"
+            else {"out": last["out"].clone()} if wl["kind"] == "gemm" else None)
     if wl["kind"] == "attn":  # per-call latency: the cache of the R3 + KV workload is L2-resident
         latency = {"us_per_call": ms_per_step * 1e3, "launches_per_call": 2}
     if world > 1:
@@ -753,6 +855,8 @@ def main():
     peak, peak_kind = measured_peaks()
     if wl["kind"] == "attn":
         kname = "k4_attn_partial"
+    elif wl["kind"] == "gemm":
+        kname = "k5_w4a4_gemm"
     elif wl["kind"] == "r4" and "kron_m" in wl:
         kname = "k1_tc_rotate_quant"
     elif wl["kind"] == "r4":
@@ -765,12 +869,25 @@ def main():
                 "frac": per_gpu_gbs / peak, "traffic": traffic, "kernel": kname,
                 "algorithmic_bytes_per_launch": step_bytes,
                 "peak_source": f"{peak_kind} hbm_gbs (STREAM-style copy)"}
+    value, unit = gbs, "GB/s"
+    if wl["kind"] == "gemm":
+        tops_peak, tops_src = int8_peak_tops()
+        per_gpu_tops = step_ops / (ms_per_step / 1e3) / 1e12
+        value, unit = per_gpu_tops * world, "TOPS"
+        roofline = {"bound": "tensor", "achieved": per_gpu_tops, "peak": tops_peak, "unit": "TOPS",
+                    "frac": per_gpu_tops / tops_peak, "traffic": traffic, "kernel": kname,
+                    "algorithmic_ops_per_launch": step_ops, "peak_source": tops_src,
+                    "operand_and_output_gbs": per_gpu_gbs}
 
     extras = None
     if args.workload == "r4_prefill" and not args.no_extras and args.tokens is None:
         extras = extra_workloads(spin, dev, world, rank, stream, args, peak)
 
     cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and wl["kind"] == "gemm":
+        cpu = cpu_baseline_gemm(xq, xs, wq, ws, last["out"])
+        if not cpu["spot_check"]["ok"]:
+            raise SystemExit(f"the last timed step disagrees with the oracle: {cpu['spot_check']}")
     if rank == 0 and world == 1 and not args.no_cpu_baseline and wl["kind"] == "r4":
         cpu, ref_out = cpu_baseline_leg(wl)
         cpu["spot_check"] = (spot_check(ref_out[0], wl, ref_out[1], ref_out[2], last["q"], last["s"], ref_out[3])
@@ -779,10 +896,10 @@ def main():
             raise SystemExit(f"the last timed step disagrees with the oracle: {cpu['spot_check']}")
 
     if rank == 0:
-        line = {"metric": metric_for(wl), "value": gbs, "unit": "GB/s", "tokens_per_s": tok_s,
+        line = {"metric": metric_for(wl), "value": value, "unit": unit, "tokens_per_s": tok_s,
                 "pct_of_hbm_peak": 100.0 * per_gpu_gbs / peak, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "vs_baseline": None, "dtype": "s8" if wl["kind"] == "gemm" else "f32", "data": "synthetic",
                 "config": config_for(wl, world, args.workload),
                 "gpu_launches": args.steps * (2 if wl["kind"] == "attn" else 1), "timed_windows": window_info, "e2e": e2e, "roofline": roofline,
                 "cpu_baseline": cpu, "cuda_core_kernel": cores, "decode_latency": latency,

@@ -131,3 +131,15 @@ def sweep(k: int, tokens: int | None = None, seed: int | None = None, block_elem
         x[:, channels] *= np.float32(100.0)
         out[t0:t1] = to_bf16_bits(x)
     return out
+
+
+def weights(n_out: int = 4096, k: int = 14336, seed: int = 7, block_rows: int = 512) -> np.ndarray:
+    """A linear layer's weight rows [n_out, k] as bf16 bits: N(0, 1/k) (random-init scale),
+    drawn in blocks of rows from the seeded generator."""
+    rng = _rng(seed)
+    out = np.empty((n_out, k), dtype=np.uint16)
+    for r0 in range(0, n_out, block_rows):
+        r1 = min(n_out, r0 + block_rows)
+        w = rng.standard_normal((r1 - r0, k), dtype=np.float32) * np.float32(1.0 / np.sqrt(k))
+        out[r0:r1] = to_bf16_bits(w)
+    return out
