@@ -48,7 +48,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kConv = 192;                      // converter threads (warps 2-7)
 constexpr int BM = 128, BN = 256, BK = 128;     // tokens x output channels x codes per chunk
-constexpr int kPS = 4, kOS = 2;                 // packed and operand ring stages
+constexpr int kPS = 3, kOS = 3;                 // packed and operand ring stages
 constexpr uint32_t kPackA = BM * BK / 2;        // 8 KiB of packed x codes per chunk
 constexpr uint32_t kPackStage = kPackA + BN * BK / 2;  // + 16 KiB of packed w codes
 constexpr uint32_t kOpA = BM * BK;              // 16 KiB of int8 x operand
@@ -58,9 +58,11 @@ constexpr uint32_t kOffO = kOffP + kPS * kPackStage;  // operand ring (1024-byte
 constexpr uint32_t kOffBar = kOffO + kOS * kOpStage;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 256;
+constexpr int kQPT = (BM + BN) * 4 / kConv;     // packed quads per converter thread and chunk
 constexpr long long kTimeoutCycles = 4000000000LL;     // about two seconds
 static_assert(kOffO % 1024 == 0 && kOpStage % 1024 == 0 && kOpA % 1024 == 0, "swizzled operand alignment");
 static_assert(kSmemBytes <= 232448, "shared memory per block");
+static_assert(kQPT * kConv == (BM + BN) * 4, "the quads of a chunk divide evenly among the converters");
 
 struct Shared {
   uint64_t pfull[kPS], pempty[kPS], ofull[kOS], oempty[kOS], tfull, drain;
@@ -194,14 +196,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (c >= kOS && !wait_bounded(&S.oempty[os], (uint32_t)((c / kOS - 1) & 1), S, true)) break;
       const uint8_t *pk = smem + kOffP + ps * kPackStage;
       uint8_t *op = smem + kOffO + os * kOpStage;
-#pragma unroll 2
-      for (uint32_t qd = cid; qd < (uint32_t)(BM + BN) * 4u; qd += kConv) {
-        const uint32_t row = qd >> 2, qi = qd & 3u;  // four 16-byte quads of packed codes per row
-        const uint4 w = *reinterpret_cast<const uint4 *>(pk + row * 64u + qi * 16u);
+      // all of a thread's loads first, then its stores (four 16-byte quads per packed row)
+      uint4 wv[kQPT];
+#pragma unroll
+      for (int j = 0; j < kQPT; ++j) {
+        const uint32_t qd = cid + (uint32_t)j * kConv;
+        wv[j] = *reinterpret_cast<const uint4 *>(pk + (qd >> 2) * 64u + (qd & 3u) * 16u);
+      }
+#pragma unroll
+      for (int j = 0; j < kQPT; ++j) {
+        const uint32_t qd = cid + (uint32_t)j * kConv;
+        const uint32_t row = qd >> 2, qi = qd & 3u, sw = row & 7u;
         uint8_t *orow = op + row * 128u;
-        const uint32_t sw = row & 7u;
-        *reinterpret_cast<uint4 *>(orow + (((2u * qi) ^ sw) << 4)) = widen2(w.x, w.y);
-        *reinterpret_cast<uint4 *>(orow + (((2u * qi + 1u) ^ sw) << 4)) = widen2(w.z, w.w);
+        *reinterpret_cast<uint4 *>(orow + (((2u * qi) ^ sw) << 4)) = widen2(wv[j].x, wv[j].y);
+        *reinterpret_cast<uint4 *>(orow + (((2u * qi + 1u) ^ sw) << 4)) = widen2(wv[j].z, wv[j].w);
       }
       tc::fence_proxy_async_smem();
       tc::named_sync(1, kConv);
@@ -210,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_arrive(&S.pempty[ps]);
       }
     }
-    if (warp >= 4 && wait_bounded(&S.tfull, 0, S, true)) {
+    if (warp >= 4 && warp < 8 && wait_bounded(&S.tfull, 0, S, true)) {
       // epilogue: TMEM lane = token row of the tile, columns = output channels
       tc::tc_fence_after();
       const uint32_t q4 = warp & 3u;
