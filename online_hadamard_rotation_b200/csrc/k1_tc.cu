@@ -290,6 +290,22 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 
 
+// Named barrier that also ANDs a predicate over the participating threads: every
+// thread leaves with the same answer, so a decision taken on it stays uniform.
+// Not .aligned: threads of a warp may reach it on different paths.
+__device__ __forceinline__ bool bar_red_and(uint32_t id, uint32_t threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
+
 // byte offset of 16-byte chunk `ch` (0..7) of row `r` in a 128-byte-swizzled [rows][128 B] tile
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t ch) { return r * 128u + ((ch ^ (r & 7u)) << 4); }
 
@@ -638,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The warpgroup (both, for one n = 32768 token) meets here on every step; with
       // their own waits, its threads all leave when any of them has no group to finish.
       if constexpr (kOwnWaits) {
-        if (!(SH::SPLIT ? tc::bar_red_and(4, 256, have) : tc::bar_red_and(1 + g, 128, have))) break;
+        if (!(SH::SPLIT ? bar_red_and(4, 256, have) : bar_red_and(1 + g, 128, have))) break;
       } else if constexpr (SH::SPLIT) {
         tc::named_sync(4, 256);
       } else {
