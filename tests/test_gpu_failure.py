@@ -1,7 +1,10 @@
 """Failure detection without a GPU fault: the tensor-core kernel's bounded waits
 run out when one internal signal is withheld (test hook), the kernel returns
 through its abort path, the device status word reports it, and the context
-stays usable."""
+stays usable. Sizes cover both ways the epilogue leaves on an abort: one thread
+deciding for its warpgroup (n = 4096) and every thread waiting itself, with the
+warpgroup's reducing barrier making the decision uniform (n = 16384; n = 32768,
+whose token spans both warpgroups)."""
 import numpy as np
 import pytest
 import torch
@@ -13,9 +16,10 @@ from tests.gpu_util import to_dev_bf16
 pytestmark = pytest.mark.gpu
 
 
-def test_bounded_wait_expiry_sets_status_and_context_survives(spin_gpu, orc):
-    n, tokens = 4096, 64
-    bits = synthetic.sweep(12, tokens=tokens, seed=31)
+@pytest.mark.parametrize("k", [12, 14, 15])
+def test_bounded_wait_expiry_sets_status_and_context_survives(spin_gpu, orc, k):
+    n, tokens = 1 << k, 64
+    bits = synthetic.sweep(k, tokens=tokens, seed=31)
     x = to_dev_bf16(bits)
     spin_gpu.device_status(reset=True)
     assert spin_gpu.device_status() == 0
